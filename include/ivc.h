@@ -1,0 +1,210 @@
+/*
+ * ivc.h — C ABI of libivc.so: InternVL visual-token compression on B200.
+ *
+ * The library implements, for one GPU, the data-parallel hot path that the
+ * InternVL pages describe between the vision encoder and the language model:
+ *
+ *   - pixel_shuffle (space-to-depth, ps_version v2) of each 32x32xC tile grid
+ *     at factor 0.5 (1024 -> 256 tokens of 4C channels) and at factor 0.25
+ *     (1024 -> 64 tokens of 16C channels), followed by the connector MLP
+ *     (mlp1 = LayerNorm -> Linear -> GELU -> Linear; mlp2 = LayerNorm ->
+ *     Linear -> GELU -> Linear -> GELU -> Linear);
+ *   - the Flash Visual Resolution Router (ViR): CrossAttentionPooling (a
+ *     learnable query refined by 4 masked multi-head cross-attention layers
+ *     over each tile's tokens), Gating (4 residual MLP blocks, Linear(D,2),
+ *     softmax), the double threshold gate > quantile_0.1(gate of the image)
+ *     AND gate >= 0.5, and compaction of every tile to 64 or 256 rows.
+ *
+ * Sources, by page title and section:
+ *   [PS]  InternVL3-14B-Instruct, "Pixel Shuffle + MLP connector, line by line":
+ *         "Pixel Shuffle 源码逐行解析", "ps_version v1 与 v2",
+ *         "MLP 连接器源码逐行解析", "extract_feature() 完整调用链".
+ *   [DP]  InternVL3_5-2B-Flash, "1024->256->64 dual-path compression pipeline":
+ *         table "三档 Token 规模", "双路压缩管线全流程拆解",
+ *         "路由决策：相对 + 绝对双阈值判定", table "核心配置参数速查".
+ *   [VIR] InternVL3_5-4B-Flash, "Gating and CrossAttentionPooling":
+ *         section 2 (pooling), section 3 (Gating), section 4 (thresholds),
+ *         section 5 (data flow).
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument named as device memory must point to memory the
+ *     caller allocated on the current CUDA device (e.g. by PyTorch). The
+ *     library never allocates, frees or retains caller memory. Each call
+ *     only enqueues work on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and returns; results are ready when the stream reaches them.
+ *   - Tensors are dense and row-major. bf16 is IEEE bfloat16 stored in
+ *     uint16_t. Weights use the nn.Linear layout [out, in]; biases, LayerNorm
+ *     gamma/beta and the pooling query are bf16 vectors.
+ *   - Device pointers must be 16-byte aligned (the TMA and vector paths need
+ *     it); otherwise IVC_EALIGN.
+ *   - Scratch memory is the caller's `workspace` of at least
+ *     ivc_workspace_size() bytes, 256-byte aligned. Its first 256 bytes hold a
+ *     sticky device status word that kernels set when they detect bad device
+ *     data (a valid length or image offset out of range) or a bounded wait
+ *     that ran out; read and clear it with ivc_device_status().
+ *   - Return value: IVC_OK (0) or a negative IVC_E* code; on error nothing was
+ *     enqueued unless the code is IVC_ECUDA.
+ *   - Calls on different streams with the same workspace race.
+ */
+#ifndef IVC_H_
+#define IVC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* ivc_stream_t; /* cudaStream_t */
+
+enum ivc_status {
+  IVC_OK = 0,
+  IVC_EINVAL = -1,       /* null pointer, negative count, bad flag or enum */
+  IVC_EUNSUPPORTED = -2, /* shape the kernels do not handle (see each call) */
+  IVC_EWORKSPACE = -3,   /* workspace smaller than ivc_workspace_size() */
+  IVC_ECUDA = -4,        /* a CUDA runtime or driver call failed */
+  IVC_EDEVICE = -5,      /* the device status word is set (ivc_device_status) */
+  IVC_EALIGN = -6        /* a pointer is not 16-byte aligned */
+};
+
+/* Bits of the device status word. */
+enum ivc_device_bits {
+  IVC_DEV_BAD_VALID_LEN = 1,  /* valid_len[t] outside [1, 1024]; clamped */
+  IVC_DEV_BAD_OFFSETS = 2,    /* image_offsets not 0 = o0 <= o1 <= ... = T */
+  IVC_DEV_WAIT_TIMEOUT = 4,   /* a pipeline barrier wait ran out; outputs invalid */
+  IVC_DEV_GROUP_TOO_LARGE = 8 /* a quantile group above IVC_MAX_QUANTILE_GROUP */
+};
+
+#define IVC_MAX_QUANTILE_GROUP 8192
+
+/* pixel_shuffle flags ([PS] "ps_version v1 与 v2"; [DP] table). */
+enum ivc_ps_flags {
+  IVC_PS_V1 = 1,            /* ps_version "v1": output token grid transposed */
+  IVC_PS_QUARTER_TWICE = 2  /* factor 0.25 as two factor-0.5 calls (channel order) */
+};
+
+/* Connector MLP ([PS] "MLP 连接器源码逐行解析"; [DP] table "三档 Token 规模").
+ * n_linear = 2: LN(dims[0]) -> W0 [dims[1],dims[0]] -> GELU -> W1 [dims[2],dims[1]].
+ * n_linear = 3: LN(dims[0]) -> W0 -> GELU -> W1 -> GELU -> W2 [dims[3],dims[2]].
+ * LayerNorm: biased variance, eps 1e-5; GELU: exact (erf).
+ * The `fold_*` fields are optional device pointers written by ivc_mlp_fold()
+ * (LayerNorm's affine part folded into W0); when fold_colsum is NULL every call
+ * recomputes the fold into its workspace. */
+typedef struct ivc_mlp {
+  int n_linear;
+  int dims[4];
+  const void* ln_gamma;      /* bf16 [dims[0]] */
+  const void* ln_beta;       /* bf16 [dims[0]] */
+  const void* W[3];          /* bf16 [dims[i+1], dims[i]] */
+  const void* b[3];          /* bf16 [dims[i+1]] */
+  const void* fold_W0;       /* bf16 [dims[1], dims[0]] = W0 * gamma (per input column) */
+  const float* fold_colsum;  /* fp32 [dims[1]]: row sums of fold_W0 */
+  const float* fold_bias;    /* fp32 [dims[1]]: b0 + W0 beta */
+} ivc_mlp;
+
+/* ViR router ([VIR] sections 2-4; [DP] "双路压缩管线全流程拆解" step 3).
+ * Pooling: 4 layers, each with its own Wq, Wk, Wv, Wo [D,D] and biases [D];
+ * `heads` heads of width D/heads (must be 64); scale 1/sqrt(64); q_0 = query;
+ * q_l = Wo_l attn(Wq_l q_{l-1} + bq_l, K_l, V_l) + bo_l; pooled = q_4.
+ * Gating: 4 blocks h <- h + LN_b(W2_b GELU(W1_b h + b1_b) + b2_b) with
+ * W1 [gate_hidden, D], W2 [D, gate_hidden]; then softmax(Wout h + bout),
+ * Wout [2, D]. Routing: tile t is compressed iff
+ * gate[t,0] > quantile(gate[.,0] over its group, rel_q) and gate[t,0] >= abs_t,
+ * quantile by linear interpolation in fp64; group = image (scope 0) or the
+ * whole batch (scope 1). */
+typedef struct ivc_router {
+  int D;
+  int heads;
+  int gate_hidden;
+  const void* query;  /* bf16 [D] */
+  const void *Wq[4], *bq[4], *Wk[4], *bk[4], *Wv[4], *bv[4], *Wo[4], *bo[4];
+  const void *gW1[4], *gb1[4], *gW2[4], *gb2[4], *gln_g[4], *gln_b[4];
+  const void *gWout, *gbout;
+  double rel_q;       /* flash_relative_threshold, 0.1 */
+  double abs_t;       /* flash_absolute_threshold, 0.5 */
+  int quantile_scope; /* 0 = per image, 1 = whole batch */
+} ivc_router;
+
+enum ivc_op {
+  IVC_OP_PS_PROJECT_HALF = 1,    /* ivc_ps_project at factor 0.5 */
+  IVC_OP_PS_PROJECT_QUARTER = 2, /* ivc_ps_project at factor 0.25 */
+  IVC_OP_VIR_ROUTE = 3,
+  IVC_OP_FLASH_COMPRESS = 4
+};
+
+/* Text for a status code (static storage). */
+const char* ivc_strerror(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int ivc_version(void);
+
+/* Workspace bytes that `op` needs for T tiles of width C. `m` is the MLP of
+ * ps_project (factor 0.5 or 0.25) or mlp1 of flash_compress, `m2` is mlp2 of
+ * flash_compress, `r` the router (NULL where the op has none). Returns 0 for
+ * invalid arguments. */
+size_t ivc_workspace_size(int op, int T, int C, const ivc_mlp* m, const ivc_mlp* m2,
+                          const ivc_router* r);
+
+/* Fold LayerNorm's gamma and beta into the first Linear of `m`, once per set
+ * of weights: fold_W0 = W0 * gamma, fold_colsum[n] = sum_k fold_W0[n,k],
+ * fold_bias = b0 + W0 beta. The connector then computes
+ * LN(P) W0^T + b0 = rstd (P fold_W0^T - mean * fold_colsum) + fold_bias
+ * inside the GEMM epilogue (an exact rewrite of the LayerNorm of [PS]).
+ * `dst` (device, >= ivc_mlp_fold_size(m) bytes) receives the three arrays;
+ * on success m->fold_* point into it. */
+size_t ivc_mlp_fold_size(const ivc_mlp* m);
+int ivc_mlp_fold(ivc_mlp* m, void* dst, size_t dst_bytes, ivc_stream_t stream);
+
+/* pixel_shuffle + connector MLP ([PS] "extract_feature() 完整调用链" steps 5-8;
+ * [DP] table "三档 Token 规模").
+ *   x      device bf16 [T, 32, 32, C]: ViT features, CLS dropped.
+ *   scale  0.5 (256 tokens of 4C per tile; m->dims[0] must be 4C) or
+ *          0.25 (64 tokens of 16C; m->dims[0] must be 16C).
+ *   flags  IVC_PS_* bits.
+ *   y      device bf16 [T * tokens, m->dims[n_linear]]; token order within a
+ *          tile is row-major over the output grid (transposed for IVC_PS_V1).
+ * Unsupported (IVC_EUNSUPPORTED): C % 64 != 0, any Linear width % 64 != 0,
+ * n_linear not 2 or 3. T == 0 enqueues nothing. */
+int ivc_ps_project(const void* x, int T, int C, float scale, int flags, const ivc_mlp* m,
+                   void* y, void* workspace, size_t ws_bytes, ivc_stream_t stream);
+
+/* ViR routing ([VIR] sections 2-4).
+ *   x              device bf16 [T, 32, 32, D] (tokens row-major over the grid).
+ *   valid_len      device int32 [T] (tokens t >= valid_len are padding), or
+ *                  NULL for all 1024; values outside [1,1024] set
+ *                  IVC_DEV_BAD_VALID_LEN.
+ *   image_offsets  device int32 [I+1], 0 = o_0 <= ... <= o_I = T; image i owns
+ *                  tiles [o_i, o_{i+1}). Ignored for quantile_scope 1.
+ *   gate           device fp32 [T, 2] softmax probabilities; column 0 means
+ *                  "compress to 64 tokens".
+ *   mask           device uint8 [T]: 1 = compressed (64 rows), 0 = 256 rows.
+ *   offsets        device int32 [T+1]: exclusive scan of the row counts;
+ *                  offsets[T] = total rows = 256 (T - k) + 64 k.
+ * Unsupported: D != C, D % 256 != 0, heads * 64 != D, gate_hidden % 256 != 0. */
+int ivc_vir_route(const void* x, const int32_t* valid_len, int T, int C,
+                  const int32_t* image_offsets, int I, const ivc_router* r, float* gate,
+                  uint8_t* mask, int32_t* offsets, void* workspace, size_t ws_bytes,
+                  ivc_stream_t stream);
+
+/* The Flash dual path ([DP] "双路压缩管线全流程拆解"; [VIR] section 5):
+ * ivc_ps_project at 0.5 with mlp1 and at 0.25 with mlp2, ivc_vir_route, then
+ * compaction: out rows [offsets[t], offsets[t+1]) = the 64 mlp2 rows of tile t
+ * if mask[t] else its 256 mlp1 rows, tiles in order.
+ *   out    device bf16 [T * 256, H] capacity (H = output width of both MLPs).
+ *   total  device int32 [1]: rows written (= offsets[T]).
+ * gate, mask, offsets as in ivc_vir_route. */
+int ivc_flash_compress(const void* x, const int32_t* valid_len, int T, int C,
+                       const int32_t* image_offsets, int I, const ivc_mlp* mlp1,
+                       const ivc_mlp* mlp2, const ivc_router* r, void* out, float* gate,
+                       uint8_t* mask, int32_t* offsets, int32_t* total, void* workspace,
+                       size_t ws_bytes, ivc_stream_t stream);
+
+/* Synchronise `stream`, copy the workspace's device status word to *bits and
+ * clear it. Returns IVC_OK when no bit was set, IVC_EDEVICE otherwise. */
+int ivc_device_status(void* workspace, int* bits, ivc_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* IVC_H_ */

@@ -1,0 +1,97 @@
+"""The C ABI loads and exports what include/ivc.h declares; host-side argument
+checks return their codes before any GPU work (runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "ivc.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ivc_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_three_calls():
+    names = _declared()
+    for n in ("ivc_ps_project", "ivc_vir_route", "ivc_flash_compress", "ivc_workspace_size"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    import vlm_visual_token_b200 as ivc
+    L = ivc.lib()
+    for n in _declared():
+        assert hasattr(L, n), n
+    assert L.ivc_version() >= 100
+
+
+def test_status_strings():
+    import vlm_visual_token_b200 as ivc
+    L = ivc.lib()
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert L.ivc_strerror(code).decode() not in ("", "unknown status")
+
+
+def _mlp(dims):
+    import vlm_visual_token_b200 as ivc
+    c = ivc._CMlp()
+    c.n_linear = len(dims) - 1
+    for i, d in enumerate(dims):
+        c.dims[i] = d
+    c.ln_gamma = c.ln_beta = 256
+    for i in range(c.n_linear):
+        c.W[i] = 256 * (i + 2)
+        c.b[i] = 256
+    return c
+
+
+def test_workspace_size_and_shape_checks():
+    import vlm_visual_token_b200 as ivc
+    L = ivc.lib()
+    m1 = _mlp([4096, 2048, 2048])
+    m2 = _mlp([16384, 4096, 2048, 2048])
+    n1 = L.ivc_workspace_size(ivc.OP_PS_HALF, 13, 1024, ctypes.byref(m1), None, None)
+    n2 = L.ivc_workspace_size(ivc.OP_PS_HALF, 26, 1024, ctypes.byref(m1), None, None)
+    assert n1 > 0 and n2 > n1
+    # at least the hidden activations [T*256, H] bf16 and the row statistics
+    assert n1 >= 13 * 256 * 2048 * 2 + 2 * 13 * 256 * 4
+    assert L.ivc_workspace_size(ivc.OP_PS_QUARTER, 13, 1024, ctypes.byref(m2), None, None) > 0
+    bad = _mlp([4096, 2000, 2048])   # width not a multiple of 64
+    assert L.ivc_workspace_size(ivc.OP_PS_HALF, 1, 1024, ctypes.byref(bad), None, None) == 0
+    assert L.ivc_workspace_size(99, 1, 1024, ctypes.byref(m1), None, None) == 0
+    assert L.ivc_workspace_size(ivc.OP_PS_HALF, -1, 1024, ctypes.byref(m1), None, None) == 0
+
+
+def test_entry_points_reject_bad_arguments_without_touching_the_gpu():
+    import vlm_visual_token_b200 as ivc
+    L = ivc.lib()
+    m1 = _mlp([4096, 2048, 2048])
+    ws = ctypes.c_void_p(1 << 20)
+    x = ctypes.c_void_p(1 << 24)
+    y = ctypes.c_void_p(1 << 26)
+    P = ctypes.byref
+    # bad scale, bad flags
+    assert L.ivc_ps_project(x, 1, 1024, ctypes.c_float(0.3), 0, P(m1), y, ws, 1 << 40, None) == -1
+    assert L.ivc_ps_project(x, 1, 1024, ctypes.c_float(0.5), 8, P(m1), y, ws, 1 << 40, None) == -1
+    # C not a multiple of 64; dims[0] != 4C
+    assert L.ivc_ps_project(x, 1, 1000, ctypes.c_float(0.5), 0, P(m1), y, ws, 1 << 40, None) == -2
+    assert L.ivc_ps_project(x, 1, 512, ctypes.c_float(0.5), 0, P(m1), y, ws, 1 << 40, None) == -2
+    # null input, misaligned input, small workspace
+    assert L.ivc_ps_project(None, 1, 1024, ctypes.c_float(0.5), 0, P(m1), y, ws, 1 << 40, None) == -1
+    assert L.ivc_ps_project(ctypes.c_void_p((1 << 24) + 8), 1, 1024, ctypes.c_float(0.5), 0, P(m1),
+                            y, ws, 1 << 40, None) == -6
+    assert L.ivc_ps_project(x, 1, 1024, ctypes.c_float(0.5), 0, P(m1), y, ws, 16, None) == -3
+    # negative tile count
+    assert L.ivc_ps_project(x, -2, 1024, ctypes.c_float(0.5), 0, P(m1), y, ws, 1 << 40, None) == -1
+    # router: D must equal C and be 64 x heads
+    r = ivc._CRouter()
+    r.D, r.heads, r.gate_hidden = 1024, 8, 1024
+    assert L.ivc_vir_route(x, None, 1, 1024, x, 1, P(r), y, y, y, ws, 1 << 40, None) == -2
+    r.heads = 16
+    assert L.ivc_vir_route(x, None, 1, 512, x, 1, P(r), y, y, y, ws, 1 << 40, None) == -2
+    r.quantile_scope = 3
+    assert L.ivc_vir_route(x, None, 1, 1024, x, 1, P(r), y, y, y, ws, 1 << 40, None) == -1

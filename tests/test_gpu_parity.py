@@ -1,0 +1,270 @@
+"""GPU (libivc.so through its C ABI) against the fp64 oracle on the same
+seeded bf16 inputs.
+
+Bars: pixel_shuffle, the routing mask and the compaction offsets bit-exact
+(the mask given the same fp32 gate vector), gate probabilities within 1e-3
+absolute, connector outputs within relative Frobenius 1e-2 and max-abs 3e-2
+(plus half a bf16 ulp where |y| >= 4, see tests/_parity.py).
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+from tests._parity import GATE_ABS, assert_connector_close, connector_errors, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _ivc():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import vlm_visual_token_b200 as ivc
+    return ivc
+
+
+def small_workload(C=128, H=192, mid=320, tiles=(3, 4), var=0.0, gate_hidden=256, name="small"):
+    return W.Workload(name, "flash", C=C, H=H, tiles_per_image=tuple(tiles), n_images=len(tiles),
+                      mlp2_mid=mid, D=C, gate_hidden=gate_hidden, var_len_frac=var,
+                      seed_base=90)
+
+
+# ------------------------------------------------------------------ connector
+@pytest.mark.parametrize("flags", [0, 1])
+def test_ps_project_half_small_ragged(flags):
+    ivc = _ivc()
+    inp = W.make(small_workload(C=128, H=192), affine="random")
+    x = inp["x"].cuda()
+    m = ivc.Mlp(inp["mlp1"])
+    y = ivc.ps_project(x, 0.5, m, flags=flags)
+    torch.cuda.synchronize()
+    ref = O.ps_project(O.to64(inp["x"]), 0.5, O.to64(inp["mlp1"]),
+                       ps_version="v1" if flags & 1 else "v2")
+    assert_connector_close(y, ref.reshape(-1, ref.shape[-1]), f"half flags={flags}")
+
+
+@pytest.mark.parametrize("flags", [0, 1, 2])
+def test_ps_project_quarter_small_ragged(flags):
+    ivc = _ivc()
+    inp = W.make(small_workload(C=128, H=192, tiles=(3,)), affine="random")  # 3*64 rows: ragged
+    x = inp["x"].cuda()
+    m = ivc.Mlp(inp["mlp2"])
+    y = ivc.ps_project(x, 0.25, m, flags=flags)
+    torch.cuda.synchronize()
+    x64 = O.to64(inp["x"])
+    if flags == 2:
+        ref = O.ps_project(x64, 0.25, O.to64(inp["mlp2"]), quarter_order="twice")
+    else:
+        ref = O.ps_project(x64, 0.25, O.to64(inp["mlp2"]), ps_version="v1" if flags else "v2")
+        if flags == 1:  # v1 transposes the 8x8 token grid
+            ref = ref.reshape(3, 8, 8, -1).transpose(0, 2, 1, 3).reshape(3, 64, -1)
+    assert_connector_close(y, ref.reshape(-1, ref.shape[-1]), f"quarter flags={flags}")
+
+
+def test_prefolded_equals_per_call_fold():
+    ivc = _ivc()
+    inp = W.make(small_workload(C=64, H=128, tiles=(2,)), affine="random")
+    x = inp["x"].cuda()
+    a = ivc.ps_project(x, 0.5, ivc.Mlp(inp["mlp1"]))
+    b = ivc.ps_project(x, 0.5, ivc.Mlp(inp["mlp1"]).fold())
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_ps_project_deterministic():
+    ivc = _ivc()
+    inp = W.make(small_workload(C=256, H=256, tiles=(5,)), affine="random")
+    x = inp["x"].cuda()
+    m = ivc.Mlp(inp["mlp2"]).fold()
+    a = ivc.ps_project(x, 0.25, m)
+    b = ivc.ps_project(x, 0.25, m)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_single_tile_2b_connector_full():
+    ivc = _ivc()
+    inp = W.make("single_tile_2b")
+    m = ivc.Mlp(inp["mlp1"]).fold()
+    y = ivc.ps_project(inp["x"].cuda(), 0.5, m)
+    torch.cuda.synchronize()
+    assert y.shape == (256, 2048)
+    ref = O.ps_project(O.to64(inp["x"]), 0.5, O.to64(inp["mlp1"]))
+    e = assert_connector_close(y, ref.reshape(256, 2048), "single tile")
+    assert e["max_abs"] <= 3e-2, e  # literal bound holds at these magnitudes
+
+
+def test_ps_project_empty_batch():
+    ivc = _ivc()
+    inp = W.make(small_workload(C=64, H=128, tiles=(1,)))
+    m = ivc.Mlp(inp["mlp1"])
+    x = torch.empty(0, 32, 32, 64, dtype=torch.bfloat16, device="cuda")
+    y = ivc.ps_project(x, 0.5, m, out=torch.empty(0, 128, dtype=torch.bfloat16, device="cuda"))
+    torch.cuda.synchronize()
+    assert y.numel() == 0
+
+
+@pytest.mark.parametrize("name", ["connector_14b_832tiles", "connector_38b_416tiles"])
+def test_large_connector_sampled_tiles(name):
+    """Full-size launch (the sizes the benchmark times); the oracle checks a
+    seeded sample of tiles spread over the batch, row by row."""
+    ivc = _ivc()
+    inp = W.make(name)
+    T, C, H = inp["T"], inp["C"], inp["H"]
+    x = inp["x"].cuda()
+    m = ivc.Mlp(inp["mlp1"]).fold()
+    y = ivc.ps_project(x, 0.5, m)
+    torch.cuda.synchronize()
+    del x
+    rng = np.random.default_rng(7)
+    tiles = sorted(set([0, T - 1] + rng.choice(T, 4, replace=False).tolist()))
+    xs = O.to64(inp["x"][tiles])
+    ref = O.ps_project(xs, 0.5, O.to64(inp["mlp1"]))
+    got = y.view(T, 256, H)[tiles]
+    assert_connector_close(got, ref, name)
+
+
+# ------------------------------------------------------------------ router
+def _route_check(ivc, inp, gate, mask, offsets, sample=None, scope=0):
+    x64 = O.to64(inp["x"])
+    T = inp["T"]
+    tiles = list(range(T)) if sample is None else sample
+    r64 = O.to64(inp["router"])
+    ref_gate = O.vir_gate(x64[tiles], inp["valid_len"].numpy()[tiles], r64)
+    g = to_np(gate)
+    assert np.all(np.isfinite(g))
+    np.testing.assert_allclose(g[:, 0] + g[:, 1], 1.0, atol=1e-6)
+    err = np.abs(g[tiles] - ref_gate).max()
+    assert err <= GATE_ABS, err
+    # routing and offsets: bit-exact given the GPU's own fp32 gate vector
+    ref_mask = O.route(g[:, 0].astype(np.float32).astype(np.float64), inp["image_offsets"].numpy(),
+                       0.1, 0.5, scope="batch" if scope else "image")
+    np.testing.assert_array_equal(to_np(mask), ref_mask)
+    np.testing.assert_array_equal(to_np(offsets), O.compaction_offsets(ref_mask))
+    return err
+
+
+def test_vir_route_small_with_padding():
+    ivc = _ivc()
+    w = small_workload(C=256, H=128, tiles=(3, 1, 5), var=0.6)
+    inp = W.make(w, affine="random")
+    vl = inp["valid_len"].clone()
+    vl[1] = 1   # a single valid token
+    inp["valid_len"] = vl
+    inp["x"] = W.features(inp["T"], 256, 1234 + 90, vl)
+    r = ivc.Router(inp["router"])
+    ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_VIR_ROUTE, inp["T"], 256, r=r))
+    gate, mask, offsets = ivc.vir_route(inp["x"].cuda(), vl.cuda(), inp["image_offsets"].cuda(), r,
+                                        workspace=ws)
+    torch.cuda.synchronize()
+    assert ivc.device_status(ws) == 0
+    _route_check(ivc, inp, gate, mask, offsets)
+    assert to_np(mask)[3] == 0  # the one-tile image is never compressed
+
+
+def test_vir_route_batch_scope():
+    ivc = _ivc()
+    inp = W.make(small_workload(C=256, H=128, tiles=(4, 4)), affine="random")
+    r = ivc.Router(inp["router"], scope=1)
+    gate, mask, offsets = ivc.vir_route(inp["x"].cuda(), None, inp["image_offsets"].cuda(), r)
+    torch.cuda.synchronize()
+    _route_check(ivc, inp, gate, mask, offsets, scope=1)
+
+
+def test_bad_valid_len_sets_status_bit():
+    ivc = _ivc()
+    inp = W.make(small_workload(C=256, H=128, tiles=(2,)))
+    r = ivc.Router(inp["router"])
+    ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_VIR_ROUTE, 2, 256, r=r))
+    vl = torch.tensor([0, 1024], dtype=torch.int32, device="cuda")
+    ivc.vir_route(inp["x"].cuda(), vl, inp["image_offsets"].cuda(), r, workspace=ws)
+    assert ivc.device_status(ws) & 1
+    assert ivc.device_status(ws) == 0  # cleared by the read
+
+
+def test_bad_image_offsets_sets_status_bit():
+    ivc = _ivc()
+    inp = W.make(small_workload(C=256, H=128, tiles=(2, 2)))
+    r = ivc.Router(inp["router"])
+    ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_VIR_ROUTE, 4, 256, r=r))
+    offs = torch.tensor([0, 3, 2], dtype=torch.int32, device="cuda")  # ends at 2 != T
+    _, mask, offsets = ivc.vir_route(inp["x"].cuda(), None, offs, r, workspace=ws)
+    assert ivc.device_status(ws) & 2
+    assert to_np(mask).sum() == 0 and to_np(offsets)[-1] == 4 * 256
+
+
+# ------------------------------------------------------------------ whole path
+def _flash_check(ivc, inp, res, tiles=None):
+    T, H = inp["T"], inp["H"]
+    x64 = O.to64(inp["x"])
+    sel = list(range(T)) if tiles is None else tiles
+    Y256 = O.ps_project(x64[sel], 0.5, O.to64(inp["mlp1"]))
+    Y64 = O.ps_project(x64[sel], 0.25, O.to64(inp["mlp2"]))
+    gate, mask, offsets = res["gate"], res["mask"], res["offsets"]
+    _route_check(ivc, inp, gate, mask, offsets, sample=tiles)
+    offs = to_np(offsets)
+    m = to_np(mask)
+    assert int(to_np(res["total"])[0]) == offs[-1] == 256 * (T - m.sum()) + 64 * m.sum()
+    out = res["out"]
+    stats = []
+    for i, t in enumerate(sel):
+        rows = out[offs[t]:offs[t + 1]]
+        ref = Y64[i] if m[t] else Y256[i]
+        stats.append(assert_connector_close(rows, ref, f"tile {t}"))
+    return stats
+
+
+def test_flash_compress_small():
+    ivc = _ivc()
+    inp = W.make(small_workload(C=256, H=192, tiles=(3, 1, 4), var=0.3), affine="random")
+    m1, m2, r = ivc.Mlp(inp["mlp1"]), ivc.Mlp(inp["mlp2"]).fold(), ivc.Router(inp["router"])
+    ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_FLASH, inp["T"], 256, m1, m2, r))
+    res = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(), inp["image_offsets"].cuda(),
+                             m1, m2, r, workspace=ws)
+    torch.cuda.synchronize()
+    assert ivc.device_status(ws) == 0
+    _flash_check(ivc, inp, res)
+
+
+def test_flash_compress_empty():
+    ivc = _ivc()
+    inp = W.make(small_workload(C=256, H=128, tiles=(1,)))
+    m1, m2, r = ivc.Mlp(inp["mlp1"]), ivc.Mlp(inp["mlp2"]), ivc.Router(inp["router"])
+    x = torch.empty(0, 32, 32, 256, dtype=torch.bfloat16, device="cuda")
+    res = ivc.flash_compress(x, None, torch.zeros(1, dtype=torch.int32, device="cuda"), m1, m2, r)
+    torch.cuda.synchronize()
+    assert int(res["total"].item()) == 0 and int(res["offsets"][0].item()) == 0
+
+
+def test_flash_2b_13tiles_full():
+    """The benchmark workload, every output checked against the oracle."""
+    ivc = _ivc()
+    inp = W.make("flash_2b_13tiles")
+    m1, m2, r = ivc.Mlp(inp["mlp1"]).fold(), ivc.Mlp(inp["mlp2"]).fold(), ivc.Router(inp["router"])
+    res = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(), inp["image_offsets"].cuda(),
+                             m1, m2, r)
+    torch.cuda.synchronize()
+    stats = _flash_check(ivc, inp, res)
+    assert max(s["max_abs"] for s in stats) <= 3e-2, stats
+
+
+def test_flash_4b_batched_sampled():
+    """16 images with drawn tile counts and 10% padded tiles; the oracle checks
+    a seeded sample of tiles (including padded ones); routing and offsets are
+    checked for every tile."""
+    ivc = _ivc()
+    inp = W.make("flash_4b_batched")
+    T = inp["T"]
+    m1, m2, r = ivc.Mlp(inp["mlp1"]).fold(), ivc.Mlp(inp["mlp2"]).fold(), ivc.Router(inp["router"])
+    ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_FLASH, T, 1024, m1, m2, r))
+    res = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(), inp["image_offsets"].cuda(),
+                             m1, m2, r, workspace=ws)
+    torch.cuda.synchronize()
+    assert ivc.device_status(ws) == 0
+    padded = np.nonzero(inp["valid_len"].numpy() < 1024)[0].tolist()
+    rng = np.random.default_rng(11)
+    tiles = sorted(set(padded[:4] + rng.choice(T, 6, replace=False).tolist() + [T - 1]))
+    _flash_check(ivc, inp, res, tiles=tiles)

@@ -1,0 +1,447 @@
+// ivc_api.cu — the C ABI of libivc.so (declared in include/ivc.h).
+//
+// Each entry point validates its arguments on the host, carves its scratch
+// buffers out of the caller's workspace and enqueues the kernels of the hot
+// path on the caller's stream. Nothing here computes on the host and nothing
+// allocates device memory.
+#include <cuda_runtime.h>
+#include <cstring>
+
+#include "ivc_gemm.cuh"
+#include "ivc_internal.h"
+
+using namespace ivc;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kHeader = 256;  // status word lives at offset 0
+
+inline size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
+
+// Sequential carve-out of workspace buffers (sizes only when base == nullptr).
+struct Carver {
+  char* base;
+  size_t off = kHeader;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <typename T>
+  T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += align_up(count * sizeof(T));
+    return p;
+  }
+};
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool mlp_shape_ok(const ivc_mlp* m) {
+  if (!m || (m->n_linear != 2 && m->n_linear != 3)) return false;
+  for (int i = 0; i <= m->n_linear; ++i)
+    if (m->dims[i] <= 0 || m->dims[i] % 64 != 0) return false;
+  return true;
+}
+
+int mlp_ptrs_ok(const ivc_mlp* m) {
+  if (!m->ln_gamma || !m->ln_beta) return IVC_EINVAL;
+  for (int i = 0; i < m->n_linear; ++i) {
+    if (!m->W[i]) return IVC_EINVAL;
+    if (!aligned16(m->W[i])) return IVC_EALIGN;
+  }
+  if (m->fold_colsum && (!m->fold_W0 || !m->fold_bias)) return IVC_EINVAL;
+  if (m->fold_W0 && !aligned16(m->fold_W0)) return IVC_EALIGN;
+  return IVC_OK;
+}
+
+int router_shape_ok(const ivc_router* r, int C) {
+  if (!r) return IVC_EINVAL;
+  if (r->D != C || r->heads * 64 != r->D) return IVC_EUNSUPPORTED;
+  const int okK[4] = {256, 512, 1024, 2048};
+  bool d_ok = false, g_ok = false;
+  for (int k : okK) {
+    d_ok |= r->D == k;
+    g_ok |= r->gate_hidden == k;
+  }
+  if (!d_ok || !g_ok) return IVC_EUNSUPPORTED;
+  if (r->quantile_scope != 0 && r->quantile_scope != 1) return IVC_EINVAL;
+  if (!r->query || !r->gWout) return IVC_EINVAL;
+  for (int l = 0; l < 4; ++l) {
+    const void* ws[4] = {r->Wq[l], r->Wk[l], r->Wv[l], r->Wo[l]};
+    for (const void* w : ws) {
+      if (!w) return IVC_EINVAL;
+      if (!aligned16(w)) return IVC_EALIGN;
+    }
+    if (!r->gW1[l] || !r->gW2[l] || !r->gln_g[l] || !r->gln_b[l]) return IVC_EINVAL;
+  }
+  return IVC_OK;
+}
+
+// Buffers one ps_project needs (given rows and the MLP).
+struct PsBufs {
+  float* mean = nullptr;
+  float* rstd = nullptr;
+  bf16* fold_W0 = nullptr;
+  float* fold_cs = nullptr;
+  float* fold_b = nullptr;
+  bf16* h1 = nullptr;
+  bf16* h2 = nullptr;
+};
+
+void carve_ps(Carver& cv, const ivc_mlp* m, long long rows, bool need_stats, PsBufs& b) {
+  if (need_stats) {
+    b.mean = cv.take<float>(rows);
+    b.rstd = cv.take<float>(rows);
+  }
+  if (!m->fold_colsum) {
+    b.fold_W0 = cv.take<bf16>(static_cast<size_t>(m->dims[1]) * m->dims[0]);
+    b.fold_cs = cv.take<float>(m->dims[1]);
+    b.fold_b = cv.take<float>(m->dims[1]);
+  }
+  b.h1 = cv.take<bf16>(rows * m->dims[1]);
+  if (m->n_linear == 3) b.h2 = cv.take<bf16>(rows * m->dims[2]);
+}
+
+struct RouteBufs {
+  bf16* KV;
+  float* Q1;
+  float* Q;
+  float* O;
+  float* q;
+  float* u1;
+  float* u2;
+};
+
+void carve_route(Carver& cv, const ivc_router* r, int T, RouteBufs& b) {
+  const long long D = r->D;
+  b.KV = cv.take<bf16>(static_cast<size_t>(T) * 1024 * 8 * D);
+  b.Q1 = cv.take<float>(D);
+  b.Q = cv.take<float>(static_cast<size_t>(T) * D);
+  b.O = cv.take<float>(static_cast<size_t>(T) * D);
+  b.q = cv.take<float>(static_cast<size_t>(T) * D);
+  b.u1 = cv.take<float>(static_cast<size_t>(T) * r->gate_hidden);
+  b.u2 = cv.take<float>(static_cast<size_t>(T) * D);
+}
+
+#define IVC_TRY(expr)          \
+  do {                         \
+    const int _rc = (expr);    \
+    if (_rc != IVC_OK) return _rc; \
+  } while (0)
+
+// pixel_shuffle + MLP with the statistics already in b.mean / b.rstd.
+int ps_mlp(const void* x, int T, int C, bool half, int flags, const ivc_mlp* m, bf16* y,
+           const PsBufs& b, const Launch& L) {
+  const long long rows = static_cast<long long>(T) * (half ? 256 : 64);
+  const bf16* W0 = static_cast<const bf16*>(m->fold_W0);
+  const float* cs = m->fold_colsum;
+  const float* fb = m->fold_bias;
+  if (!cs) {
+    IVC_TRY(launch_fold(static_cast<const bf16*>(m->W[0]), static_cast<const bf16*>(m->b[0]),
+                        static_cast<const bf16*>(m->ln_gamma),
+                        static_cast<const bf16*>(m->ln_beta), m->dims[1], m->dims[0],
+                        b.fold_W0, b.fold_cs, b.fold_b, L));
+    W0 = b.fold_W0;
+    cs = b.fold_cs;
+    fb = b.fold_b;
+  }
+  const int remap = (flags & IVC_PS_V1) ? (half ? 1 : 2) : 0;
+  GemmCall c{};
+  c.a_mode = half ? A_PS_HALF : ((flags & IVC_PS_QUARTER_TWICE) ? A_PS_QUARTER_TWICE : A_PS_QUARTER);
+  c.a = x;
+  c.T = T;
+  c.C = C;
+  c.M = static_cast<int>(rows);
+  c.N = m->dims[1];
+  c.K = m->dims[0];
+  c.groups = 1;
+  c.B[0] = W0;
+  c.epi_mode = EPI_LNFOLD;
+  c.gelu = 1;
+  c.colsum = cs;
+  c.fbias = fb;
+  c.row_mean = b.mean;
+  c.row_rstd = b.rstd;
+  c.out = b.h1;
+  c.ldo = m->dims[1];
+  IVC_TRY(launch_gemm(c, L));
+  const bf16* a = b.h1;
+  for (int i = 1; i < m->n_linear; ++i) {
+    const bool last = i + 1 == m->n_linear;
+    GemmCall d{};
+    d.a_mode = A_PLAIN;
+    d.a = a;
+    d.M = static_cast<int>(rows);
+    d.N = m->dims[i + 1];
+    d.K = m->dims[i];
+    d.groups = 1;
+    d.B[0] = m->W[i];
+    d.bias[0] = static_cast<const bf16*>(m->b[i]);
+    d.epi_mode = EPI_BIAS;
+    d.gelu = last ? 0 : 1;
+    d.remap = last ? remap : 0;
+    d.out = last ? y : b.h2;
+    d.ldo = m->dims[i + 1];
+    IVC_TRY(launch_gemm(d, L));
+    a = b.h2;
+  }
+  return IVC_OK;
+}
+
+int route_impl(const void* x, const int32_t* valid_len, int T, const int32_t* image_offsets,
+               int I, const ivc_router* r, float* gate, uint8_t* mask, int32_t* offsets,
+               int32_t* total, const RouteBufs& b, const Launch& L) {
+  const int D = r->D;
+  // K/V projections of the four layers: one grouped GEMM, X [T*1024, D].
+  GemmCall c{};
+  c.a_mode = A_PLAIN;
+  c.a = x;
+  c.M = T * 1024;
+  c.N = D;
+  c.K = D;
+  c.groups = 8;
+  for (int l = 0; l < 4; ++l) {
+    c.B[2 * l] = r->Wk[l];
+    c.B[2 * l + 1] = r->Wv[l];
+    c.bias[2 * l] = static_cast<const bf16*>(r->bk[l]);
+    c.bias[2 * l + 1] = static_cast<const bf16*>(r->bv[l]);
+  }
+  c.epi_mode = EPI_BIAS;
+  c.out = b.KV;
+  c.ldo = 8LL * D;
+  IVC_TRY(launch_gemm(c, L));
+  const long long ldkv = 8LL * D;
+  // layer 1: the query is the same for every tile.
+  IVC_TRY(launch_gemv_bf16x(static_cast<const bf16*>(r->query), D,
+                            static_cast<const bf16*>(r->Wq[0]),
+                            static_cast<const bf16*>(r->bq[0]), D, b.Q1, L));
+  for (int l = 0; l < 4; ++l) {
+    const float* Q = b.Q1;
+    long long ldq = 0;
+    if (l > 0) {
+      IVC_TRY(launch_gemv(b.q, D, T, D, static_cast<const bf16*>(r->Wq[l]),
+                          static_cast<const bf16*>(r->bq[l]), D, b.Q, D, 0, L));
+      Q = b.Q;
+      ldq = D;
+    }
+    IVC_TRY(launch_pool_attention(Q, ldq, b.KV, ldkv, 2 * l * D, (2 * l + 1) * D, valid_len, T, D,
+                                  r->heads, b.O, L));
+    IVC_TRY(launch_gemv(b.O, D, T, D, static_cast<const bf16*>(r->Wo[l]),
+                        static_cast<const bf16*>(r->bo[l]), D, b.q, D, 0, L));
+  }
+  // Gating: h = pooled (in b.q), 4 residual blocks, 2-way head.
+  const int G = r->gate_hidden;
+  for (int k = 0; k < 4; ++k) {
+    IVC_TRY(launch_gemv(b.q, D, T, D, static_cast<const bf16*>(r->gW1[k]),
+                        static_cast<const bf16*>(r->gb1[k]), G, b.u1, G, 1, L));
+    IVC_TRY(launch_gemv(b.u1, G, T, G, static_cast<const bf16*>(r->gW2[k]),
+                        static_cast<const bf16*>(r->gb2[k]), D, b.u2, D, 0, L));
+    IVC_TRY(launch_residual_ln(b.q, b.u2, static_cast<const bf16*>(r->gln_g[k]),
+                               static_cast<const bf16*>(r->gln_b[k]), T, D, L));
+  }
+  IVC_TRY(launch_gate_head(b.q, static_cast<const bf16*>(r->gWout),
+                           static_cast<const bf16*>(r->gbout), T, D, gate, L));
+  return launch_route(gate, T, image_offsets, I, r->rel_q, r->abs_t, r->quantile_scope, mask,
+                      offsets, total, L);
+}
+
+int check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (!ws) return IVC_EINVAL;
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign) return IVC_EALIGN;
+  if (ws_bytes < need) return IVC_EWORKSPACE;
+  return IVC_OK;
+}
+
+size_t ps_ws(int T, const ivc_mlp* m, bool half) {
+  Carver cv(nullptr);
+  PsBufs b;
+  carve_ps(cv, m, static_cast<long long>(T) * (half ? 256 : 64), true, b);
+  return cv.off;
+}
+
+size_t route_ws(int T, const ivc_router* r) {
+  Carver cv(nullptr);
+  RouteBufs b;
+  carve_route(cv, r, T, b);
+  return cv.off;
+}
+
+size_t flash_ws(int T, const ivc_mlp* m1, const ivc_mlp* m2, const ivc_router* r) {
+  Carver cv(nullptr);
+  PsBufs b1, b2;
+  RouteBufs br;
+  carve_ps(cv, m1, static_cast<long long>(T) * 256, true, b1);
+  carve_ps(cv, m2, static_cast<long long>(T) * 64, true, b2);
+  cv.take<bf16>(static_cast<size_t>(T) * 256 * m1->dims[m1->n_linear]);
+  cv.take<bf16>(static_cast<size_t>(T) * 64 * m2->dims[m2->n_linear]);
+  carve_route(cv, r, T, br);
+  return cv.off;
+}
+
+int ps_args_ok(const void* x, int T, int C, const ivc_mlp* m, bool half) {
+  if (T < 0 || C <= 0) return IVC_EINVAL;
+  if (!m) return IVC_EINVAL;
+  if (C % 64 != 0 || !mlp_shape_ok(m)) return IVC_EUNSUPPORTED;
+  if (m->dims[0] != (half ? 4 : 16) * C) return IVC_EUNSUPPORTED;
+  if (static_cast<long long>(T) * 256 > 0x7fffffffLL) return IVC_EUNSUPPORTED;
+  if (T > 0 && !x) return IVC_EINVAL;
+  if (!aligned16(x)) return IVC_EALIGN;
+  return mlp_ptrs_ok(m);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ivc_strerror(int status) {
+  switch (status) {
+    case IVC_OK: return "ok";
+    case IVC_EINVAL: return "invalid argument";
+    case IVC_EUNSUPPORTED: return "unsupported shape";
+    case IVC_EWORKSPACE: return "workspace too small";
+    case IVC_ECUDA: return "CUDA call failed";
+    case IVC_EDEVICE: return "device status word set";
+    case IVC_EALIGN: return "pointer not 16-byte aligned";
+    default: return "unknown status";
+  }
+}
+
+int ivc_version(void) { return 100; }
+
+size_t ivc_workspace_size(int op, int T, int C, const ivc_mlp* m, const ivc_mlp* m2,
+                          const ivc_router* r) {
+  if (T < 0 || C <= 0) return 0;
+  switch (op) {
+    case IVC_OP_PS_PROJECT_HALF:
+      return mlp_shape_ok(m) ? ps_ws(T, m, true) : 0;
+    case IVC_OP_PS_PROJECT_QUARTER:
+      return mlp_shape_ok(m) ? ps_ws(T, m, false) : 0;
+    case IVC_OP_VIR_ROUTE:
+      return router_shape_ok(r, C) == IVC_OK ? route_ws(T, r) : 0;
+    case IVC_OP_FLASH_COMPRESS:
+      if (!mlp_shape_ok(m) || !mlp_shape_ok(m2) || router_shape_ok(r, C) != IVC_OK) return 0;
+      return flash_ws(T, m, m2, r);
+    default:
+      return 0;
+  }
+}
+
+size_t ivc_mlp_fold_size(const ivc_mlp* m) {
+  if (!mlp_shape_ok(m)) return 0;
+  return align_up(static_cast<size_t>(m->dims[1]) * m->dims[0] * sizeof(bf16)) +
+         2 * align_up(static_cast<size_t>(m->dims[1]) * sizeof(float));
+}
+
+int ivc_mlp_fold(ivc_mlp* m, void* dst, size_t dst_bytes, ivc_stream_t stream) {
+  if (!m || !dst) return IVC_EINVAL;
+  if (!mlp_shape_ok(m)) return IVC_EUNSUPPORTED;
+  if (!m->ln_gamma || !m->ln_beta || !m->W[0]) return IVC_EINVAL;
+  if (reinterpret_cast<uintptr_t>(dst) % kAlign) return IVC_EALIGN;
+  if (dst_bytes < ivc_mlp_fold_size(m)) return IVC_EWORKSPACE;
+  char* p = static_cast<char*>(dst);
+  bf16* W0 = reinterpret_cast<bf16*>(p);
+  p += align_up(static_cast<size_t>(m->dims[1]) * m->dims[0] * sizeof(bf16));
+  float* cs = reinterpret_cast<float*>(p);
+  p += align_up(static_cast<size_t>(m->dims[1]) * sizeof(float));
+  float* fb = reinterpret_cast<float*>(p);
+  Launch L{static_cast<cudaStream_t>(stream), nullptr};
+  IVC_TRY(launch_fold(static_cast<const bf16*>(m->W[0]), static_cast<const bf16*>(m->b[0]),
+                      static_cast<const bf16*>(m->ln_gamma), static_cast<const bf16*>(m->ln_beta),
+                      m->dims[1], m->dims[0], W0, cs, fb, L));
+  m->fold_W0 = W0;
+  m->fold_colsum = cs;
+  m->fold_bias = fb;
+  return IVC_OK;
+}
+
+int ivc_ps_project(const void* x, int T, int C, float scale, int flags, const ivc_mlp* m,
+                   void* y, void* workspace, size_t ws_bytes, ivc_stream_t stream) {
+  const bool half = scale == 0.5f;
+  if (!half && scale != 0.25f) return IVC_EINVAL;
+  if (flags & ~(IVC_PS_V1 | IVC_PS_QUARTER_TWICE)) return IVC_EINVAL;
+  IVC_TRY(ps_args_ok(x, T, C, m, half));
+  if (T > 0 && !y) return IVC_EINVAL;
+  if (!aligned16(y)) return IVC_EALIGN;
+  IVC_TRY(check_ws(workspace, ws_bytes, ps_ws(T, m, half)));
+  if (T == 0) return IVC_OK;
+  Launch L{static_cast<cudaStream_t>(stream), static_cast<int*>(workspace)};
+  Carver cv(workspace);
+  PsBufs b;
+  const long long rows = static_cast<long long>(T) * (half ? 256 : 64);
+  carve_ps(cv, m, rows, true, b);
+  IVC_TRY(launch_ps_stats(static_cast<const bf16*>(x), T, C, half ? b.mean : nullptr,
+                          half ? b.rstd : nullptr, half ? nullptr : b.mean,
+                          half ? nullptr : b.rstd, L));
+  return ps_mlp(x, T, C, half, flags, m, static_cast<bf16*>(y), b, L);
+}
+
+int ivc_vir_route(const void* x, const int32_t* valid_len, int T, int C,
+                  const int32_t* image_offsets, int I, const ivc_router* r, float* gate,
+                  uint8_t* mask, int32_t* offsets, void* workspace, size_t ws_bytes,
+                  ivc_stream_t stream) {
+  if (T < 0 || C <= 0 || I < 0) return IVC_EINVAL;
+  IVC_TRY(router_shape_ok(r, C));
+  if (!offsets || (T > 0 && (!x || !gate || !mask))) return IVC_EINVAL;
+  if (T > 0 && r->quantile_scope == 0 && !image_offsets) return IVC_EINVAL;
+  if (!aligned16(x)) return IVC_EALIGN;
+  IVC_TRY(check_ws(workspace, ws_bytes, route_ws(T, r)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (T == 0) return cu_check(cudaMemsetAsync(offsets, 0, sizeof(int32_t), s));
+  Launch L{s, static_cast<int*>(workspace)};
+  Carver cv(workspace);
+  RouteBufs b;
+  carve_route(cv, r, T, b);
+  return route_impl(x, valid_len, T, image_offsets, I, r, gate, mask, offsets, nullptr, b, L);
+}
+
+int ivc_flash_compress(const void* x, const int32_t* valid_len, int T, int C,
+                       const int32_t* image_offsets, int I, const ivc_mlp* mlp1,
+                       const ivc_mlp* mlp2, const ivc_router* r, void* out, float* gate,
+                       uint8_t* mask, int32_t* offsets, int32_t* total, void* workspace,
+                       size_t ws_bytes, ivc_stream_t stream) {
+  if (T < 0 || C <= 0 || I < 0) return IVC_EINVAL;
+  IVC_TRY(ps_args_ok(x, T, C, mlp1, true));
+  IVC_TRY(ps_args_ok(x, T, C, mlp2, false));
+  const int H = mlp1->dims[mlp1->n_linear];
+  if (mlp2->dims[mlp2->n_linear] != H) return IVC_EUNSUPPORTED;
+  IVC_TRY(router_shape_ok(r, C));
+  if (!offsets || !total || (T > 0 && (!out || !gate || !mask))) return IVC_EINVAL;
+  if (T > 0 && r->quantile_scope == 0 && !image_offsets) return IVC_EINVAL;
+  if (!aligned16(out)) return IVC_EALIGN;
+  IVC_TRY(check_ws(workspace, ws_bytes, flash_ws(T, mlp1, mlp2, r)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    IVC_TRY(cu_check(cudaMemsetAsync(offsets, 0, sizeof(int32_t), s)));
+    return cu_check(cudaMemsetAsync(total, 0, sizeof(int32_t), s));
+  }
+  Launch L{s, static_cast<int*>(workspace)};
+  Carver cv(workspace);
+  PsBufs b1, b2;
+  RouteBufs br;
+  carve_ps(cv, mlp1, static_cast<long long>(T) * 256, true, b1);
+  carve_ps(cv, mlp2, static_cast<long long>(T) * 64, true, b2);
+  bf16* Y256 = cv.take<bf16>(static_cast<size_t>(T) * 256 * H);
+  bf16* Y64 = cv.take<bf16>(static_cast<size_t>(T) * 64 * H);
+  carve_route(cv, r, T, br);
+  IVC_TRY(launch_ps_stats(static_cast<const bf16*>(x), T, C, b1.mean, b1.rstd, b2.mean, b2.rstd,
+                          L));
+  IVC_TRY(ps_mlp(x, T, C, true, 0, mlp1, Y256, b1, L));
+  IVC_TRY(ps_mlp(x, T, C, false, 0, mlp2, Y64, b2, L));
+  IVC_TRY(route_impl(x, valid_len, T, image_offsets, I, r, gate, mask, offsets, total, br, L));
+  return launch_compact(Y256, Y64, mask, offsets, T, H, static_cast<bf16*>(out), L);
+}
+
+int ivc_device_status(void* workspace, int* bits, ivc_stream_t stream) {
+  if (!workspace || !bits) return IVC_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return IVC_ECUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return IVC_ECUDA;
+  if (v != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(int), s) != cudaSuccess) return IVC_ECUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return IVC_ECUDA;
+  }
+  *bits = v;
+  return v ? IVC_EDEVICE : IVC_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,267 @@
+// ivc_connector.cu — pixel_shuffle + connector MLP kernels for sm_100a.
+//
+// LayerNorm ("MLP 连接器源码逐行解析" of the InternVL3-14B-Instruct connector
+// article: LayerNorm(4C) -> Linear -> GELU -> Linear) is applied without ever
+// writing the normalised rows: with mean mu and rstd of row P,
+//   LN(P) W0^T + b0 = rstd * (P (W0*gamma)^T - mu * colsum(W0*gamma)) + (b0 + W0 beta),
+// so the first GEMM multiplies the raw pixel-shuffled features (read through
+// the 5-D TMA map, see ivc_gemm.cuh) and its epilogue applies rstd, mu and the
+// two folded column vectors. ps_stats_kernel computes mu and rstd of every
+// shuffled row in one pass over the features.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <mutex>
+
+#include "ivc_gemm.cuh"
+#include "ivc_internal.h"
+
+namespace ivc {
+
+// ---------------------------------------------------------------- LN statistics
+// One CTA per 4x4 block of ViT tokens = one factor-0.25 row; its four 2x2
+// sub-blocks are four factor-0.5 rows. Warp w = 4q + r reduces token
+// (4a+q, 4b+r) over C channels (sums shifted by the token's first value to
+// keep the one-pass variance well conditioned); the token statistics are
+// then merged per row with the pairwise (Chan) update in fp64.
+__global__ void __launch_bounds__(512) ps_stats_kernel(const bf16* __restrict__ x, int C,
+                                                       float* __restrict__ mean_half,
+                                                       float* __restrict__ rstd_half,
+                                                       float* __restrict__ mean_quarter,
+                                                       float* __restrict__ rstd_quarter) {
+  __shared__ double s_mean[16], s_m2[16];
+  const int cell = blockIdx.x;  // tile * 64 + a * 8 + b
+  const int tile = cell >> 6, a = (cell >> 3) & 7, b = cell & 7;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q = warp >> 2, r = warp & 3;
+  const bf16* tok = x + ((static_cast<long long>(tile) * 32 + 4 * a + q) * 32 + 4 * b + r) * C;
+  const float shift = __bfloat162float(tok[0]);
+  float s1 = 0.f, s2 = 0.f;
+  const uint4* v = reinterpret_cast<const uint4*>(tok);
+  for (int i = lane; i < C / 8; i += 32) {
+    const uint4 u = v[i];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float lo = __uint_as_float(w[j] << 16) - shift;
+      const float hi = __uint_as_float(w[j] & 0xffff0000u) - shift;
+      s1 += lo + hi;
+      s2 = fmaf(lo, lo, fmaf(hi, hi, s2));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+    s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+  }
+  if (lane == 0) {
+    const double n = C;
+    s_mean[warp] = shift + s1 / n;
+    s_m2[warp] = fmax(static_cast<double>(s2) - static_cast<double>(s1) * s1 / n, 0.0);
+  }
+  __syncthreads();
+  const double eps = 1e-5;
+  if (threadIdx.x < 4 && mean_half != nullptr) {
+    const int sa = threadIdx.x >> 1, sb = threadIdx.x & 1;
+    const int w0 = 4 * (2 * sa) + 2 * sb;  // tokens (2sa+di, 2sb+dj)
+    const int ids[4] = {w0, w0 + 1, w0 + 4, w0 + 5};
+    double mu = 0.0;
+    for (int i = 0; i < 4; ++i) mu += s_mean[ids[i]];
+    mu *= 0.25;
+    double m2 = 0.0;
+    for (int i = 0; i < 4; ++i) {
+      const double d = s_mean[ids[i]] - mu;
+      m2 += s_m2[ids[i]] + C * d * d;
+    }
+    const double var = m2 / (4.0 * C);
+    const long long row = static_cast<long long>(tile) * 256 + (2 * a + sa) * 16 + (2 * b + sb);
+    mean_half[row] = static_cast<float>(mu);
+    rstd_half[row] = static_cast<float>(1.0 / sqrt(var + eps));
+  }
+  if (threadIdx.x == 32 && mean_quarter != nullptr) {
+    double mu = 0.0;
+    for (int i = 0; i < 16; ++i) mu += s_mean[i];
+    mu *= 1.0 / 16.0;
+    double m2 = 0.0;
+    for (int i = 0; i < 16; ++i) {
+      const double d = s_mean[i] - mu;
+      m2 += s_m2[i] + C * d * d;
+    }
+    const double var = m2 / (16.0 * C);
+    mean_quarter[cell] = static_cast<float>(mu);
+    rstd_quarter[cell] = static_cast<float>(1.0 / sqrt(var + eps));
+  }
+}
+
+int launch_ps_stats(const bf16* x, int T, int C, float* mean_half, float* rstd_half,
+                    float* mean_quarter, float* rstd_quarter, const Launch& L) {
+  if (T == 0) return IVC_OK;
+  ps_stats_kernel<<<T * 64, 512, 0, L.stream>>>(x, C, mean_half, rstd_half, mean_quarter,
+                                                rstd_quarter);
+  return cu_check(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------- LN fold
+// One warp per output feature n: W_out[n,k] = bf16(W[n,k] * gamma[k]),
+// colsum[n] = sum_k W_out[n,k], fbias[n] = b[n] + sum_k W[n,k] * beta[k].
+__global__ void __launch_bounds__(256) fold_kernel(const bf16* __restrict__ W,
+                                                   const bf16* __restrict__ b,
+                                                   const bf16* __restrict__ gamma,
+                                                   const bf16* __restrict__ beta, int N, int K,
+                                                   bf16* __restrict__ W_out,
+                                                   float* __restrict__ colsum,
+                                                   float* __restrict__ fbias) {
+  const int n = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (n >= N) return;
+  const bf16* w = W + static_cast<long long>(n) * K;
+  bf16* wo = W_out + static_cast<long long>(n) * K;
+  double cs = 0.0, fb = 0.0;
+  for (int k = lane; k < K; k += 32) {
+    const float wv = __bfloat162float(w[k]);
+    const bf16 scaled = __float2bfloat16_rn(wv * __bfloat162float(gamma[k]));
+    wo[k] = scaled;
+    cs += static_cast<double>(__bfloat162float(scaled));
+    fb += static_cast<double>(wv) * static_cast<double>(__bfloat162float(beta[k]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    cs += __shfl_xor_sync(0xffffffffu, cs, o);
+    fb += __shfl_xor_sync(0xffffffffu, fb, o);
+  }
+  if (lane == 0) {
+    colsum[n] = static_cast<float>(cs);
+    fbias[n] = static_cast<float>(fb + (b ? static_cast<double>(__bfloat162float(b[n])) : 0.0));
+  }
+}
+
+int launch_fold(const bf16* W, const bf16* b, const bf16* gamma, const bf16* beta, int N, int K,
+                bf16* W_out, float* colsum, float* fbias, const Launch& L) {
+  fold_kernel<<<(N + 7) / 8, 256, 0, L.stream>>>(W, b, gamma, beta, N, K, W_out, colsum, fbias);
+  return cu_check(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+static int encode(CUtensorMap* m, int rank, const void* base, const cuuint64_t* dims,
+                  const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return IVC_ECUDA;
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
+                  strides_bytes, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? IVC_OK : IVC_ECUDA;
+}
+
+// Row-major [rows, cols] bf16 matrix, box 64 columns x box_rows rows.
+static int map_2d(CUtensorMap* m, const void* base, long long rows, long long cols,
+                  int box_rows) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {GEMM_BK, static_cast<cuuint32_t>(box_rows)};
+  return encode(m, 2, base, dims, strides, box);
+}
+
+// The [T,32,32,C] features seen as the pixel-shuffled [T*tokens, f*f*C] matrix.
+static int map_ps(CUtensorMap* m, const void* x, int T, int C, int f) {
+  const cuuint64_t Cu = static_cast<cuuint64_t>(C);
+  const int g = 32 / f;  // output grid side
+  cuuint64_t dims[5] = {Cu, static_cast<cuuint64_t>(f), static_cast<cuuint64_t>(g),
+                        static_cast<cuuint64_t>(f), static_cast<cuuint64_t>(T) * g};
+  // strides (bytes) of dims 1..4: next column in the block, next output
+  // column b, next row in the block, next output row (a) / tile.
+  cuuint64_t strides[4] = {Cu * 2, Cu * f * 2, Cu * 32 * 2, Cu * 32 * f * 2};
+  cuuint32_t box[5] = {GEMM_BK, 1, static_cast<cuuint32_t>(g), 1,
+                       static_cast<cuuint32_t>(GEMM_BM / g)};
+  return encode(m, 5, x, dims, strides, box);
+}
+
+int num_sms() {
+  static int n = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  });
+  return n;
+}
+
+template <int BN, int STAGES>
+static int run_gemm(const GemmMaps& maps, const GemmArgs& args, int groups, const Launch& L) {
+  using S = GemmSmem<BN, STAGES>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_sm100_kernel<BN, STAGES>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL);
+    if (e != cudaSuccess) return IVC_ECUDA;
+    attr_set = true;
+  }
+  dim3 grid((args.N + BN - 1) / BN, (args.M + GEMM_BM - 1) / GEMM_BM, groups);
+  gemm_sm100_kernel<BN, STAGES><<<grid, GEMM_THREADS, S::TOTAL, L.stream>>>(maps, args, L.status);
+  return cu_check(cudaGetLastError());
+}
+
+int launch_gemm(const GemmCall& c, const Launch& L) {
+  if (c.M == 0 || c.N == 0) return IVC_OK;
+  if (c.K % GEMM_BK != 0 || c.N % 32 != 0 || c.groups < 1 || c.groups > GEMM_MAX_GROUPS)
+    return IVC_EUNSUPPORTED;
+  // Tile width: 256 columns unless that leaves most SMs idle.
+  const int m_tiles = (c.M + GEMM_BM - 1) / GEMM_BM;
+  const long long tiles256 = static_cast<long long>(m_tiles) * ((c.N + 255) / 256) * c.groups;
+  const int bn = (tiles256 * 2 <= num_sms() && c.N > 128) || c.N <= 128 ? 128 : 256;
+
+  GemmMaps maps;
+  int rc;
+  switch (c.a_mode) {
+    case A_PLAIN: rc = map_2d(&maps.a, c.a, c.M, c.K, GEMM_BM); break;
+    case A_PS_HALF: rc = map_ps(&maps.a, c.a, c.T, c.C, 2); break;
+    default: rc = map_ps(&maps.a, c.a, c.T, c.C, 4); break;
+  }
+  if (rc) return rc;
+  for (int g = 0; g < c.groups; ++g) {
+    rc = map_2d(&maps.b[g], c.B[g], c.N, c.K, bn);
+    if (rc) return rc;
+  }
+  GemmArgs a{};
+  a.M = c.M;
+  a.N = c.N;
+  a.K = c.K;
+  a.a_mode = c.a_mode;
+  a.c_blocks = c.C / GEMM_BK;
+  a.epi_mode = c.epi_mode;
+  a.gelu = c.gelu;
+  a.remap = c.remap;
+  a.out = c.out;
+  a.ldo = c.ldo;
+  a.group_col_stride = c.N;
+  for (int g = 0; g < c.groups; ++g) a.bias[g] = c.bias[g];
+  a.colsum = c.colsum;
+  a.fbias = c.fbias;
+  a.row_mean = c.row_mean;
+  a.row_rstd = c.row_rstd;
+  return bn == 256 ? run_gemm<256, 4>(maps, a, c.groups, L)
+                   : run_gemm<128, 6>(maps, a, c.groups, L);
+}
+
+}  // namespace ivc

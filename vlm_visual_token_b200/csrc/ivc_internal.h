@@ -1,0 +1,88 @@
+// ivc_internal.h — host-side launchers shared by the library's translation units.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "ivc.h"
+
+namespace ivc {
+
+typedef __nv_bfloat16 bf16;
+
+// Status word bits (mirror enum ivc_device_bits).
+constexpr int DEV_BAD_VALID_LEN = IVC_DEV_BAD_VALID_LEN;
+constexpr int DEV_BAD_OFFSETS = IVC_DEV_BAD_OFFSETS;
+constexpr int DEV_WAIT_TIMEOUT = IVC_DEV_WAIT_TIMEOUT;
+constexpr int DEV_GROUP_TOO_LARGE = IVC_DEV_GROUP_TOO_LARGE;
+
+struct Launch {
+  cudaStream_t stream;
+  int* status;  // device status word (workspace header)
+};
+
+// Converts a CUDA error into IVC_ECUDA (and remembers nothing else).
+inline int cu_check(cudaError_t e) { return e == cudaSuccess ? IVC_OK : IVC_ECUDA; }
+
+// -------------------------------------------------------------- connector
+// Per-row LayerNorm statistics of the pixel-shuffled rows, read straight
+// from the [T,32,32,C] features: mean/rstd of every factor-0.5 row
+// (T*256 rows of 4C values) and/or every factor-0.25 row (T*64 rows of 16C).
+int launch_ps_stats(const bf16* x, int T, int C, float* mean_half, float* rstd_half,
+                    float* mean_quarter, float* rstd_quarter, const Launch& L);
+
+// LayerNorm affine fold into the first Linear (see ivc_mlp_fold).
+int launch_fold(const bf16* W, const bf16* b, const bf16* gamma, const bf16* beta, int N, int K,
+                bf16* W_out, float* colsum, float* fbias, const Launch& L);
+
+// One GEMM of the connector or of the pooling projections.
+struct GemmCall {
+  int a_mode;          // AMode
+  const void* a;       // A base (features for the pixel_shuffle modes)
+  int T, C;            // pixel_shuffle modes
+  int M, N, K;
+  int groups;          // >1: blockIdx.z selects B[g], bias[g], column offset g*N
+  const void* B[8];
+  const bf16* bias[8];
+  int epi_mode;        // EpiMode
+  int gelu;
+  int remap;
+  const float* colsum;
+  const float* fbias;
+  const float* row_mean;
+  const float* row_rstd;
+  bf16* out;
+  long long ldo;
+};
+int launch_gemm(const GemmCall& c, const Launch& L);
+
+// -------------------------------------------------------------- router
+// Y[m, n] = act(sum_k X[m, k] W[n, k] + b[n]); X fp32 [M, ldx], W bf16 [N, K].
+int launch_gemv(const float* X, long long ldx, int M, int K, const bf16* W, const bf16* b, int N,
+                float* Y, long long ldy, int gelu, const Launch& L);
+// Same with a bf16 input vector broadcast (M = 1).
+int launch_gemv_bf16x(const bf16* x, int K, const bf16* W, const bf16* b, int N, float* Y,
+                      const Launch& L);
+// Masked single-query multi-head attention of one pooling layer.
+int launch_pool_attention(const float* Q, long long ldq, const bf16* KV, long long ldkv,
+                          int koff, int voff, const int32_t* valid_len, int T, int D, int heads,
+                          float* O, const Launch& L);
+// h[t] += LN(u[t]) * gamma + beta over D.
+int launch_residual_ln(float* h, const float* u, const bf16* gamma, const bf16* beta, int T,
+                       int D, const Launch& L);
+// gate[t] = softmax(Wout h[t] + bout), Wout [2, D].
+int launch_gate_head(const float* h, const bf16* Wout, const bf16* bout, int T, int D,
+                     float* gate, const Launch& L);
+// Quantile + double threshold + row-count scan.
+int launch_route(const float* gate, int T, const int32_t* image_offsets, int I, double rel_q,
+                 double abs_t, int scope, uint8_t* mask, int32_t* offsets, int32_t* total,
+                 const Launch& L);
+// out[offsets[t] + j] = mask[t] ? Y64[t*64 + j] : Y256[t*256 + j].
+int launch_compact(const bf16* Y256, const bf16* Y64, const uint8_t* mask,
+                   const int32_t* offsets, int T, int H, bf16* out, const Launch& L);
+
+int num_sms();
+
+}  // namespace ivc

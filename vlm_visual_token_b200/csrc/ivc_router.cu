@@ -1,0 +1,485 @@
+// ivc_router.cu — the Flash Visual Resolution Router (ViR) kernels for sm_100a.
+//
+// InternVL3_5-4B-Flash "Gating and CrossAttentionPooling" article:
+//   section 2  CrossAttentionPooling — a learnable query refined by 4
+//              multi-head cross-attention layers over a tile's tokens, pad
+//              tokens masked out;
+//   section 3  Gating — 4 residual blocks Linear -> GELU -> Dropout -> Linear
+//              -> Dropout -> LayerNorm, then Linear(hidden, 2) and softmax;
+//   section 4  gate > quantile(gate, 0.1) and gate >= 0.5 per image;
+// InternVL3_5-2B-Flash dual-path article, "路由决策" (operators of the double
+// threshold) and section 5 of the 4B-Flash article (tiles spliced back in
+// order, 64 or 256 rows each).
+//
+// The K and V projections of all four pooling layers are one grouped
+// tensor-core GEMM (ivc_gemm.cuh); what remains per layer is a skinny
+// projection of the query (M = tiles), the masked softmax-weighted sum over
+// the tile's tokens, and the output projection. All router activations stay
+// fp32; only K/V (GEMM outputs) are bf16.
+#include <cuda_runtime.h>
+
+#include "ivc_internal.h"
+
+namespace ivc {
+
+__device__ __forceinline__ float gelu_f(float y) {
+  return 0.5f * y * (1.0f + erff(y * 0.70710678118654752f));
+}
+
+// ---------------------------------------------------------------- skinny GEMV
+// One warp per output column n, all rows m. Lane l owns k = 128 j + 4 l .. +3
+// of the weight row (kept in registers); input rows are staged 8 at a time in
+// shared memory as fp32.
+constexpr int GEMV_WARPS = 8;
+constexpr int GEMV_ROWS = 8;
+
+template <typename XT>
+__device__ __forceinline__ float4 load4(const XT* p);
+template <>
+__device__ __forceinline__ float4 load4<float>(const float* p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+template <>
+__device__ __forceinline__ float4 load4<bf16>(const bf16* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                     __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+}
+
+template <typename XT, int J>
+__global__ void __launch_bounds__(GEMV_WARPS * 32)
+    gemv_kernel(const XT* __restrict__ X, long long ldx, int M,
+                const bf16* __restrict__ W, const bf16* __restrict__ b, int N,
+                float* __restrict__ Y, long long ldy, int gelu) {
+  extern __shared__ float sx[];  // [GEMV_ROWS][K]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int K = J * 128;
+  const int n = blockIdx.x * GEMV_WARPS + warp;
+  float4 w[J];
+  if (n < N) {
+    const bf16* wr = W + static_cast<long long>(n) * K;
+#pragma unroll
+    for (int j = 0; j < J; ++j) w[j] = load4<bf16>(wr + j * 128 + lane * 4);
+  }
+  const float bias = (n < N && b != nullptr) ? __bfloat162float(b[n]) : 0.f;
+  for (int m0 = 0; m0 < M; m0 += GEMV_ROWS) {
+    const int rows = min(GEMV_ROWS, M - m0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < rows * (K / 4); i += blockDim.x) {
+      const int r = i / (K / 4), c = (i - r * (K / 4)) * 4;
+      *reinterpret_cast<float4*>(sx + r * K + c) = load4<XT>(X + (m0 + r) * ldx + c);
+    }
+    __syncthreads();
+    if (n >= N) continue;
+    for (int r = 0; r < rows; ++r) {
+      float acc = 0.f;
+#pragma unroll
+      for (int j = 0; j < J; ++j) {
+        const float4 xv = *reinterpret_cast<const float4*>(sx + r * K + j * 128 + lane * 4);
+        acc = fmaf(w[j].x, xv.x, acc);
+        acc = fmaf(w[j].y, xv.y, acc);
+        acc = fmaf(w[j].z, xv.z, acc);
+        acc = fmaf(w[j].w, xv.w, acc);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) {
+        float y = acc + bias;
+        if (gelu) y = gelu_f(y);
+        Y[(m0 + r) * ldy + n] = y;
+      }
+    }
+  }
+}
+
+template <typename XT, int J>
+static int run_gemv(const XT* X, long long ldx, int M, const bf16* W, const bf16* b, int N,
+                    float* Y, long long ldy, int gelu, const Launch& L) {
+  const int smem = GEMV_ROWS * J * 128 * static_cast<int>(sizeof(float));
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(gemv_kernel<XT, J>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return IVC_ECUDA;
+    attr = true;
+  }
+  gemv_kernel<XT, J><<<(N + GEMV_WARPS - 1) / GEMV_WARPS, GEMV_WARPS * 32, smem, L.stream>>>(
+      X, ldx, M, W, b, N, Y, ldy, gelu);
+  return cu_check(cudaGetLastError());
+}
+
+template <typename XT>
+static int dispatch_gemv(const XT* X, long long ldx, int M, int K, const bf16* W, const bf16* b,
+                         int N, float* Y, long long ldy, int gelu, const Launch& L) {
+  if (M == 0 || N == 0) return IVC_OK;
+  switch (K) {
+    case 256: return run_gemv<XT, 2>(X, ldx, M, W, b, N, Y, ldy, gelu, L);
+    case 512: return run_gemv<XT, 4>(X, ldx, M, W, b, N, Y, ldy, gelu, L);
+    case 1024: return run_gemv<XT, 8>(X, ldx, M, W, b, N, Y, ldy, gelu, L);
+    case 2048: return run_gemv<XT, 16>(X, ldx, M, W, b, N, Y, ldy, gelu, L);
+    default: return IVC_EUNSUPPORTED;
+  }
+}
+
+int launch_gemv(const float* X, long long ldx, int M, int K, const bf16* W, const bf16* b, int N,
+                float* Y, long long ldy, int gelu, const Launch& L) {
+  return dispatch_gemv<float>(X, ldx, M, K, W, b, N, Y, ldy, gelu, L);
+}
+
+int launch_gemv_bf16x(const bf16* x, int K, const bf16* W, const bf16* b, int N, float* Y,
+                      const Launch& L) {
+  return dispatch_gemv<bf16>(x, 0, 1, K, W, b, N, Y, 0, 0, L);
+}
+
+// ---------------------------------------------------------------- pooling attention
+// One CTA per (head, tile). Scores s_t = (Q_h . K_h[t]) / sqrt(64) for the
+// valid prefix t < len; softmax in fp32; o_h = sum_t p_t V_h[t] / sum_t p_t.
+constexpr int ATT_THREADS = 256;
+constexpr int TILE_TOKENS = 1024;
+constexpr int HEAD_DIM = 64;
+
+__global__ void __launch_bounds__(ATT_THREADS)
+    pool_attention_kernel(const float* __restrict__ Q, long long ldq,
+                          const bf16* __restrict__ KV, long long ldkv, int koff, int voff,
+                          const int32_t* __restrict__ valid_len, float* __restrict__ O, int D,
+                          int* __restrict__ status) {
+  __shared__ float s_q[HEAD_DIM];
+  __shared__ float s_p[TILE_TOKENS];
+  __shared__ float s_red[ATT_THREADS / 32][HEAD_DIM];
+  __shared__ float s_scalar[ATT_THREADS / 32];
+  const int h = blockIdx.x, tile = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int n = TILE_TOKENS;
+  if (valid_len != nullptr) {
+    n = valid_len[tile];
+    if (n < 1 || n > TILE_TOKENS) {
+      if (threadIdx.x == 0) atomicOr(status, DEV_BAD_VALID_LEN);
+      n = n < 1 ? 1 : TILE_TOKENS;
+    }
+  }
+  if (threadIdx.x < HEAD_DIM)
+    s_q[threadIdx.x] = Q[tile * ldq + h * HEAD_DIM + threadIdx.x] * 0.125f;  // 1/sqrt(64)
+  __syncthreads();
+  const bf16* kbase = KV + static_cast<long long>(tile) * TILE_TOKENS * ldkv + koff + h * HEAD_DIM;
+  float mx = -INFINITY;
+  for (int t = threadIdx.x; t < n; t += ATT_THREADS) {
+    const uint4* kr = reinterpret_cast<const uint4*>(kbase + t * ldkv);
+    float s = 0.f;
+#pragma unroll
+    for (int c = 0; c < HEAD_DIM / 8; ++c) {
+      const uint4 u = kr[c];
+      const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        s = fmaf(__uint_as_float(wv[j] << 16), s_q[c * 8 + 2 * j], s);
+        s = fmaf(__uint_as_float(wv[j] & 0xffff0000u), s_q[c * 8 + 2 * j + 1], s);
+      }
+    }
+    s_p[t] = s;
+    mx = fmaxf(mx, s);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) s_scalar[warp] = mx;
+  __syncthreads();
+  mx = s_scalar[0];
+#pragma unroll
+  for (int i = 1; i < ATT_THREADS / 32; ++i) mx = fmaxf(mx, s_scalar[i]);
+  __syncthreads();
+  float sum = 0.f;
+  for (int t = threadIdx.x; t < n; t += ATT_THREADS) {
+    const float e = expf(s_p[t] - mx);
+    s_p[t] = e;
+    sum += e;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) s_scalar[warp] = sum;
+  __syncthreads();
+  sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < ATT_THREADS / 32; ++i) sum += s_scalar[i];
+  // weighted V: warp w takes tokens w, w+8, ...; lane l owns dims 2l, 2l+1
+  const bf16* vbase = KV + static_cast<long long>(tile) * TILE_TOKENS * ldkv + voff + h * HEAD_DIM;
+  float a0 = 0.f, a1 = 0.f;
+  for (int t = warp; t < n; t += ATT_THREADS / 32) {
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(vbase + t * ldkv + 2 * lane);
+    const float p = s_p[t];
+    a0 = fmaf(p, __uint_as_float(u << 16), a0);
+    a1 = fmaf(p, __uint_as_float(u & 0xffff0000u), a1);
+  }
+  s_red[warp][2 * lane] = a0;
+  s_red[warp][2 * lane + 1] = a1;
+  __syncthreads();
+  if (threadIdx.x < HEAD_DIM) {
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < ATT_THREADS / 32; ++i) acc += s_red[i][threadIdx.x];
+    O[static_cast<long long>(tile) * D + h * HEAD_DIM + threadIdx.x] = acc / sum;
+  }
+}
+
+int launch_pool_attention(const float* Q, long long ldq, const bf16* KV, long long ldkv,
+                          int koff, int voff, const int32_t* valid_len, int T, int D, int heads,
+                          float* O, const Launch& L) {
+  if (T == 0) return IVC_OK;
+  if (heads * HEAD_DIM != D) return IVC_EUNSUPPORTED;
+  pool_attention_kernel<<<dim3(heads, T), ATT_THREADS, 0, L.stream>>>(Q, ldq, KV, ldkv, koff,
+                                                                     voff, valid_len, O, D,
+                                                                     L.status);
+  return cu_check(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------- residual + LayerNorm
+// h[t] += (u[t] - mean) * rstd * gamma + beta (biased variance, eps 1e-5).
+__global__ void __launch_bounds__(256) residual_ln_kernel(float* __restrict__ h,
+                                                          const float* __restrict__ u,
+                                                          const bf16* __restrict__ gamma,
+                                                          const bf16* __restrict__ beta, int D) {
+  __shared__ float s_red[8];
+  const int t = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float* ur = u + static_cast<long long>(t) * D;
+  float s = 0.f;
+  for (int i = threadIdx.x; i < D; i += 256) s += ur[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) s_red[warp] = s;
+  __syncthreads();
+  float mean = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mean += s_red[i];
+  mean /= D;
+  __syncthreads();
+  float v = 0.f;
+  for (int i = threadIdx.x; i < D; i += 256) {
+    const float d = ur[i] - mean;
+    v = fmaf(d, d, v);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) s_red[warp] = v;
+  __syncthreads();
+  float var = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) var += s_red[i];
+  var /= D;
+  const float rstd = 1.0f / sqrtf(var + 1e-5f);
+  float* hr = h + static_cast<long long>(t) * D;
+  for (int i = threadIdx.x; i < D; i += 256)
+    hr[i] += (ur[i] - mean) * rstd * __bfloat162float(gamma[i]) + __bfloat162float(beta[i]);
+}
+
+int launch_residual_ln(float* h, const float* u, const bf16* gamma, const bf16* beta, int T,
+                       int D, const Launch& L) {
+  if (T == 0) return IVC_OK;
+  residual_ln_kernel<<<T, 256, 0, L.stream>>>(h, u, gamma, beta, D);
+  return cu_check(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------- gate head
+// One warp per tile: two dot products of length D, then a 2-way softmax.
+__global__ void __launch_bounds__(256) gate_head_kernel(const float* __restrict__ h,
+                                                        const bf16* __restrict__ Wout,
+                                                        const bf16* __restrict__ bout, int T,
+                                                        int D, float* __restrict__ gate) {
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const float* hr = h + static_cast<long long>(t) * D;
+  float l0 = 0.f, l1 = 0.f;
+  for (int i = lane; i < D; i += 32) {
+    const float v = hr[i];
+    l0 = fmaf(__bfloat162float(Wout[i]), v, l0);
+    l1 = fmaf(__bfloat162float(Wout[D + i]), v, l1);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+  }
+  if (lane == 0) {
+    if (bout) {
+      l0 += __bfloat162float(bout[0]);
+      l1 += __bfloat162float(bout[1]);
+    }
+    const float m = fmaxf(l0, l1);
+    const float e0 = expf(l0 - m), e1 = expf(l1 - m);
+    const float s = e0 + e1;
+    gate[2 * t] = e0 / s;
+    gate[2 * t + 1] = e1 / s;
+  }
+}
+
+int launch_gate_head(const float* h, const bf16* Wout, const bf16* bout, int T, int D,
+                     float* gate, const Launch& L) {
+  if (T == 0) return IVC_OK;
+  gate_head_kernel<<<(T + 7) / 8, 256, 0, L.stream>>>(h, Wout, bout, T, D, gate);
+  return cu_check(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------- routing
+// Single CTA. For each group (image, or the whole batch): the group's gate
+// column 0 values are placed in ascending order by rank (ties broken by tile
+// index), the linear-interpolation quantile is taken in fp64 with each
+// operation rounded on its own (no fused multiply-add), and tile t is marked
+// compressed iff gate > quantile and gate >= abs_t. Then the 64/256 row
+// counts are prefix-summed into offsets[0..T] and total.
+constexpr int ROUTE_THREADS = 1024;
+
+__global__ void __launch_bounds__(ROUTE_THREADS)
+    route_kernel(const float* __restrict__ gate, int T, const int32_t* __restrict__ offs, int I,
+                 double rel_q, double abs_t, int scope, uint8_t* __restrict__ mask,
+                 int32_t* __restrict__ offsets, int32_t* __restrict__ total,
+                 int* __restrict__ status) {
+  extern __shared__ double s_dyn[];  // values then sorted values, IVC_MAX_QUANTILE_GROUP each
+  double* s_vals = s_dyn;
+  double* s_sorted = s_dyn + IVC_MAX_QUANTILE_GROUP;
+  __shared__ double s_qv;
+  __shared__ int s_bad;
+  __shared__ int s_warp[ROUTE_THREADS / 32];
+  __shared__ int s_carry;
+  if (threadIdx.x == 0) {
+    int bad = 0;
+    if (scope == 0) {
+      if (offs[0] != 0 || offs[I] != T) bad = 1;
+      for (int i = 0; i < I && !bad; ++i)
+        if (offs[i + 1] < offs[i]) bad = 1;
+      if (bad) atomicOr(status, DEV_BAD_OFFSETS);
+    }
+    s_bad = bad;
+  }
+  __syncthreads();
+  const int groups = scope == 0 ? I : 1;
+  for (int gi = 0; gi < groups; ++gi) {
+    int s = 0, e = T;
+    if (scope == 0) {
+      if (s_bad) break;
+      s = offs[gi];
+      e = offs[gi + 1];
+    }
+    const int n = e - s;
+    if (n <= 0) continue;
+    if (n > IVC_MAX_QUANTILE_GROUP) {
+      if (threadIdx.x == 0) atomicOr(status, DEV_GROUP_TOO_LARGE);
+      for (int i = threadIdx.x; i < n; i += ROUTE_THREADS) mask[s + i] = 0;
+      __syncthreads();
+      continue;
+    }
+    for (int i = threadIdx.x; i < n; i += ROUTE_THREADS)
+      s_vals[i] = static_cast<double>(gate[2 * (s + i)]);
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += ROUTE_THREADS) {
+      const double v = s_vals[i];
+      int rank = 0;
+      for (int j = 0; j < n; ++j) {
+        const double u = s_vals[j];
+        rank += (u < v) || (u == v && j < i);
+      }
+      s_sorted[rank] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const double pos = __dmul_rn(rel_q, static_cast<double>(n - 1));
+      const double flo = floor(pos);
+      const int lo = static_cast<int>(flo);
+      const int hi = static_cast<int>(ceil(pos));
+      const double w = __dsub_rn(pos, flo);
+      const double diff = __dsub_rn(s_sorted[hi], s_sorted[lo]);
+      s_qv = __dadd_rn(s_sorted[lo], __dmul_rn(w, diff));
+    }
+    __syncthreads();
+    const double qv = s_qv;
+    for (int i = threadIdx.x; i < n; i += ROUTE_THREADS) {
+      const double v = s_vals[i];
+      mask[s + i] = (v > qv && v >= abs_t) ? 1 : 0;
+    }
+    __syncthreads();
+  }
+  if (scope == 0 && s_bad) {
+    for (int i = threadIdx.x; i < T; i += ROUTE_THREADS) mask[i] = 0;
+  }
+  __syncthreads();
+  // exclusive scan of the row counts
+  if (threadIdx.x == 0) s_carry = 0;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int base = 0; base < T; base += ROUTE_THREADS) {
+    const int i = base + threadIdx.x;
+    const int cnt = i < T ? (mask[i] ? 64 : 256) : 0;
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int w = s_warp[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += v;
+      }
+      s_warp[lane] = w;
+    }
+    __syncthreads();
+    const int before = (warp > 0 ? s_warp[warp - 1] : 0) + s_carry;
+    if (i < T) offsets[i] = before + incl - cnt;
+    __syncthreads();
+    if (threadIdx.x == ROUTE_THREADS - 1) s_carry = before + incl;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    offsets[T] = s_carry;
+    if (total) *total = s_carry;
+  }
+}
+
+int launch_route(const float* gate, int T, const int32_t* image_offsets, int I, double rel_q,
+                 double abs_t, int scope, uint8_t* mask, int32_t* offsets, int32_t* total,
+                 const Launch& L) {
+  const size_t smem = 2 * IVC_MAX_QUANTILE_GROUP * sizeof(double);
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return IVC_ECUDA;
+    attr = true;
+  }
+  route_kernel<<<1, ROUTE_THREADS, smem, L.stream>>>(gate, T, image_offsets, I, rel_q, abs_t,
+                                                     scope, mask, offsets, total, L.status);
+  return cu_check(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------- compaction
+// Grid (T, 8): CTA (t, y) copies rows 32y..32y+31 of tile t when they exist
+// (64 rows for a compressed tile, 256 otherwise), 16 bytes per thread-step.
+__global__ void __launch_bounds__(256) compact_kernel(const bf16* __restrict__ Y256,
+                                                      const bf16* __restrict__ Y64,
+                                                      const uint8_t* __restrict__ mask,
+                                                      const int32_t* __restrict__ offsets, int H,
+                                                      bf16* __restrict__ out) {
+  const int t = blockIdx.x;
+  const int r0 = blockIdx.y * 32;
+  const bool comp = mask[t] != 0;
+  const int rows = comp ? 64 : 256;
+  if (r0 >= rows) return;
+  const bf16* src = comp ? Y64 + (static_cast<long long>(t) * 64 + r0) * H
+                         : Y256 + (static_cast<long long>(t) * 256 + r0) * H;
+  bf16* dst = out + (static_cast<long long>(offsets[t]) + r0) * H;
+  const int per_row = H / 8;
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+  for (int i = threadIdx.x; i < 32 * per_row; i += 256) d4[i] = s4[i];
+}
+
+int launch_compact(const bf16* Y256, const bf16* Y64, const uint8_t* mask,
+                   const int32_t* offsets, int T, int H, bf16* out, const Launch& L) {
+  if (T == 0) return IVC_OK;
+  compact_kernel<<<dim3(T, 8), 256, 0, L.stream>>>(Y256, Y64, mask, offsets, H, out);
+  return cu_check(cudaGetLastError());
+}
+
+}  // namespace ivc

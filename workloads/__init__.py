@@ -192,5 +192,6 @@ def make(name_or_w, affine: str = "config", n_images: Optional[int] = None,
            "mlp1": mlp_params([4 * w.C, w.H, w.H], wseed, affine)}
     if w.path == "flash":
         out["mlp2"] = mlp_params([16 * w.C, w.mlp2_mid, w.H, w.H], wseed + 1000, affine)
-        out["router"] = router_params(w.D, w.gate_hidden, wseed + 2000, affine)
+        out["router"] = router_params(w.D, w.gate_hidden, wseed + 2000, affine,
+                                      heads=w.D // 64)
     return out
