@@ -1,0 +1,434 @@
+"""Throughput of the InternVL visual-token compression hot path on B200.
+
+One step = one ivc_flash_compress over one image of 12 tiles + thumbnail
+(T = 13 tiles of [32, 32, 1024] bf16, InternVL3.5-2B-Flash dims): pixel_shuffle
+0.5 -> mlp1 and 0.25 -> mlp2 for every tile, the ViR router (CrossAttentionPooling,
+Gating, quantile + absolute threshold) and compaction to 64/256 rows per tile.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ivc|reference]
+
+Prints one JSON line (rank 0). Metric: tiles per second (whole job). Inputs
+are resident in HBM; L2 is flushed (512 MiB write) between timed steps, each
+step timed with CUDA events on the launching stream; max over ranks. With
+N > 1 every rank processes its own image (weights replicated, no data-path
+collective): weak scaling. ``--impl reference`` times the fp64 CPU oracle on
+a bounded per-step sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "ViT tiles/sec through ps+MLP connector & ViR router; % of bf16 tensor/HBM peak"
+UNIT = "tiles/s"
+WORKLOAD = "flash_2b_13tiles"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------- helpers (CPU-testable)
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max of a float over all ranks (identity when world == 1)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic(w, T):
+    """Algorithmic FLOPs / bytes of each kernel role for T tiles of workload w.
+
+    FLOPs count 2 per multiply-add of the literal method; bytes count each
+    operand read once and each result written once."""
+    C, H, M2, D, G = w.C, w.H, w.mlp2_mid, w.D, w.gate_hidden
+    r256, r64, tok = T * 256, T * 64, T * 1024
+    bf, f32 = 2, 4
+    f = {
+        "mlp1.fc1": (2.0 * r256 * 4 * C * H, bf * (tok * C + 4 * C * H + r256 * H)),
+        "mlp1.fc2": (2.0 * r256 * H * H, bf * (r256 * H + H * H + r256 * H)),
+        "mlp2.fc1": (2.0 * r64 * 16 * C * M2, bf * (tok * C + 16 * C * M2 + r64 * M2)),
+        "mlp2.fc2": (2.0 * r64 * M2 * H, bf * (r64 * M2 + M2 * H + r64 * H)),
+        "mlp2.fc3": (2.0 * r64 * H * H, bf * (r64 * H + H * H + r64 * H)),
+        "pool.kv": (2.0 * tok * D * 8 * D, bf * (tok * D + 8 * D * D) + f32 * tok * 8 * D),
+        "pool.attention": (4.0 * tok * D, f32 * tok * 2 * D),          # per layer launch
+        "ps_stats": (3.0 * tok * C, bf * tok * C + f32 * 2 * (r256 + r64)),
+        "compact": (0.0, bf * 2 * r256 * H),
+        "route": (0.0, f32 * 2 * T),
+    }
+    return f
+
+
+def image_gen(rank: int):
+    import workloads as W
+    return W.make(WORKLOAD, seed_offset=1000 * rank)
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 100 ms while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                p = [v.strip() for v in line.split(",")]
+                if len(p) >= 9 and p[1].replace(".", "").isdigit():
+                    rows.append(p)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+def thread_count() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+# ----------------------------------------------------------------- oracle (CPU) legs
+def oracle_sample(inp, tile: int, frac: float):
+    """The oracle's whole path for `frac` of one tile: mlp1 on the first
+    256*frac shuffled rows, mlp2 on the first 64*frac, pooling over the first
+    1024*frac tokens (fewer K/V rows), gating, routing of the one-tile group
+    and the compaction offsets. Returns the tiles processed (= frac)."""
+    import numpy as np
+
+    import oracle as O
+    x = O.to64(inp["x"][tile:tile + 1])
+    n256, n64, ntok = max(1, round(256 * frac)), max(1, round(64 * frac)), max(1, round(1024 * frac))
+    P = O.pixel_shuffle(x, 0.5)[0, :n256]
+    m1 = inp["_m1_64"]
+    O.mlp(P, m1["ln_g"], m1["ln_b"], m1["W"], m1["b"])
+    Q = O.pixel_shuffle_quarter(x)[0, :n64]
+    m2 = inp["_m2_64"]
+    O.mlp(Q, m2["ln_g"], m2["ln_b"], m2["W"], m2["b"])
+    X = x.reshape(1, 1024, -1)[:, :ntok]
+    pooled = O.cross_attention_pooling(X, np.array([ntok]), inp["_r_64"])
+    gate = O.gating(pooled, inp["_r_64"])
+    mask = O.route(gate[:, 0], np.array([0, 1]))
+    O.compaction_offsets(mask)
+    return frac
+
+
+def cpu_baseline(inp):
+    """The oracle, as it stands, over the whole 13-tile image once."""
+    import oracle as O
+    t0 = time.perf_counter()
+    O.flash_compress(O.to64(inp["x"]), inp["valid_len"].numpy(), inp["image_offsets"].numpy(),
+                     inp["_m1_64"], inp["_m2_64"], inp["_r_64"])
+    dt = time.perf_counter() - t0
+    return {"value": inp["T"] / dt, "unit": UNIT, "cores": thread_count(), "kind": "oracle",
+            "sample": f"one full image of {inp['T']} tiles (whole path, fp64), {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle as O
+    inp = image_gen(0)
+    inp["_m1_64"], inp["_m2_64"], inp["_r_64"] = (O.to64(inp["mlp1"]), O.to64(inp["mlp2"]),
+                                                   O.to64(inp["router"]))
+    T = inp["T"]
+    t0 = time.perf_counter()
+    oracle_sample(inp, 0, 1.0)
+    t_tile = time.perf_counter() - t0
+    budget = 150.0
+    frac = 1.0
+    while frac > 1.0 / 256 and (args.steps + args.warmup) * t_tile * frac > budget:
+        frac /= 2
+    for i in range(args.warmup):
+        oracle_sample(inp, i % T, frac)
+    units, dt = 0.0, 0.0
+    for i in range(args.steps):
+        t0 = time.perf_counter()
+        units += oracle_sample(inp, i % T, frac)
+        dt += time.perf_counter() - t0
+    value = units / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "tiles": T, "C": 1024, "H": 2048},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": thread_count(), "kind": "oracle",
+                             "sample": f"per step {frac:g} of one tile (rows/tokens subsampled), "
+                                       f"whole path in fp64"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- GPU leg
+def run_ivc(args):
+    import ctypes
+
+    import torch
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    import vlm_visual_token_b200 as ivc
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    inp = image_gen(rank)
+    w, T = inp["workload"], inp["T"]
+    x = inp["x"].to(dev)
+    vl = inp["valid_len"].to(dev)
+    offs = inp["image_offsets"].to(dev)
+    m1 = ivc.Mlp(inp["mlp1"], dev).fold()
+    m2 = ivc.Mlp(inp["mlp2"], dev).fold()
+    r = ivc.Router(inp["router"], device=dev)
+    ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_FLASH, T, w.C, m1, m2, r), dev)
+    bufs = {"gate": torch.empty(T, 2, dtype=torch.float32, device=dev),
+            "mask": torch.empty(T, dtype=torch.uint8, device=dev),
+            "offsets": torch.empty(T + 1, dtype=torch.int32, device=dev),
+            "total": torch.empty(1, dtype=torch.int32, device=dev)}
+    out = torch.empty(T * 256, w.H, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ivc.flash_compress(x, vl, offs, m1, m2, r, out=out, workspace=ws, bufs=bufs)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    assert ivc.device_status(ws) == 0
+    graph = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        graph = g
+    except Exception:
+        graph = None
+    run = graph.replay if graph is not None else step
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        run()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        t_wall = time.perf_counter()
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            run()
+            b.record(stream)
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    barrier()
+    torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = reduce_max(sum(step_ms), world, dev)
+    value = world * T * args.steps / (total_ms / 1e3)
+    clocks = clk.summary()
+    if ivc.device_status(ws) != 0:
+        raise RuntimeError("device status word set during the timed steps")
+
+    # ---- traced pass: per-kernel device time of the same steps (eager launches)
+    L = ivc.lib()
+    L.ivc_trace_enable.argtypes = [ctypes.c_int]
+    L.ivc_trace_report.argtypes = [ctypes.c_char_p, ctypes.c_size_t]
+    n_trace = min(args.steps, 50)
+    L.ivc_trace_reset()
+    L.ivc_trace_enable(1)
+    for _ in range(n_trace):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    L.ivc_trace_enable(0)
+    buf = ctypes.create_string_buffer(1 << 16)
+    L.ivc_trace_report(buf, len(buf))
+    trace = json.loads(buf.value.decode())
+    L.ivc_trace_reset()
+    launches_per_step = sum(v["launches"] for v in trace.values()) / n_trace
+    per_step_ms = {k: v["ms"] / n_trace for k, v in trace.items()}
+    trace_total = sum(per_step_ms.values())
+    dom = max(per_step_ms, key=per_step_ms.get)
+    alg = algorithmic(w, T)
+    peaks, src = load_peaks()
+    fl, by = alg.get(dom, (0.0, 0.0))
+    per_launch_ms = trace[dom]["ms"] / trace[dom]["launches"]
+    launches_dom = trace[dom]["launches"] / n_trace
+    if fl / max(by, 1) > peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9):
+        ach = fl / launches_dom / (per_launch_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": ach / peak, "traffic": None,
+                "kernel": dom, "peak_source": f"{src} bf16_tflops_sustained"}
+    else:
+        ach = by / launches_dom / (per_launch_ms / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                "traffic": None, "kernel": dom, "peak_source": f"{src} hbm_gbs"}
+    # whole-step roofline: algorithmic FLOPs at the dense bf16 peak vs bytes at HBM peak
+    F = sum(v[0] for k, v in alg.items() if k not in ("pool.attention",)) + 4 * alg["pool.attention"][0]
+    B_alg = 2 * (T * 1024 * w.C) + 2 * (4 * w.C * w.H + w.H * w.H + 16 * w.C * w.mlp2_mid +
+                                        w.mlp2_mid * w.H + w.H * w.H + 16 * w.D * w.D +
+                                        8 * w.D * w.gate_hidden) + 2 * T * 256 * w.H
+    t_roof = max(F / (peaks["bf16_tflops"] * 1e12), B_alg / (peaks["hbm_gbs"] * 1e9))
+    step_roofline = {"flops": F, "bytes": B_alg, "roofline_us": t_roof * 1e6,
+                     "measured_us": total_ms / args.steps * 1e3,
+                     "frac": t_roof / (total_ms / args.steps / 1e3),
+                     "peak_source": f"{src} bf16_tflops (burst), hbm_gbs"}
+
+    # ---- end to end through the public API with host buffers
+    e2e_steps = min(args.steps, 100)
+    hx = inp["x"].pin_memory()
+    hvl = inp["valid_len"].pin_memory()
+    hoffs = inp["image_offsets"].pin_memory()
+    hout = torch.empty(T * 256, w.H, dtype=torch.bfloat16).pin_memory()
+    hsmall = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in bufs.items()}
+    h2d = hx.numel() * 2 + hvl.numel() * 4 + hoffs.numel() * 4
+    d2h_small = sum(v.numel() * v.element_size() for v in bufs.values())
+    d2h_rows = 0
+    torch.cuda.synchronize()
+    barrier()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        x.copy_(hx, non_blocking=True)
+        vl.copy_(hvl, non_blocking=True)
+        offs.copy_(hoffs, non_blocking=True)
+        run()
+        for k in bufs:
+            hsmall[k].copy_(bufs[k], non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        rows = int(hsmall["total"][0])
+        hout[:rows].copy_(out[:rows], non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        d2h_rows += rows * w.H * 2
+    e2e_s = reduce_max(time.perf_counter() - t0, world, dev)
+    e2e = {"value": world * T * e2e_steps / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h_small + d2h_rows // e2e_steps, "steps": e2e_steps,
+           "timing": "wall clock, host sync per step (needs the row count before the row copy)"}
+
+    if graph is not None:
+        del graph
+    barrier()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "tiles_per_step": T, "C": w.C, "H": w.H,
+                       "mlp2_mid": w.mlp2_mid, "pool_heads": 16, "gate_hidden": w.gate_hidden,
+                       "l2": "flushed between steps (512 MiB write, outside the timed events)",
+                       "launch": "CUDA graph of one ivc_flash_compress" if graph is not None
+                                 else "eager ivc_flash_compress",
+                       "parallelism": f"replicas x{world}, one image per GPU, no collective"},
+            "roofline": roof, "step_roofline": step_roofline,
+            "kernels_ms_per_step": {k: round(v, 5) for k, v in per_step_ms.items()},
+            "traced_ms_per_step": trace_total,
+            "clocks": clocks, "e2e": e2e, "gpu_launches": int(round(launches_per_step * args.steps)),
+            "wall_s_timed": t_wall}
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle as O
+        inp["_m1_64"], inp["_m2_64"], inp["_r_64"] = (O.to64(inp["mlp1"]), O.to64(inp["mlp2"]),
+                                                       O.to64(inp["router"]))
+        line["cpu_baseline"] = cpu_baseline(inp)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ivc", "reference"], default="ivc")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ivc(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

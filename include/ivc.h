@@ -204,6 +204,17 @@ int ivc_flash_compress(const void* x, const int32_t* valid_len, int T, int C,
  * clear it. Returns IVC_OK when no bit was set, IVC_EDEVICE otherwise. */
 int ivc_device_status(void* workspace, int* bits, ivc_stream_t stream);
 
+/* Per-kernel device timing (diagnostics; off by default). While enabled,
+ * every kernel launch is bracketed by two CUDA events on its stream and filed
+ * under its role (e.g. "mlp1.fc1", "pool.kv", "pool.attention", "route").
+ * ivc_trace_report() waits for the recorded events and writes a JSON object
+ * {role: {"launches": n, "ms": total}} into buf (n bytes); IVC_EINVAL if buf
+ * is too small. ivc_trace_reset() forgets the records. Not for use while a
+ * stream is being captured into a CUDA graph. */
+int ivc_trace_enable(int on);
+int ivc_trace_reset(void);
+int ivc_trace_report(char* buf, size_t n);
+
 #ifdef __cplusplus
 }
 #endif

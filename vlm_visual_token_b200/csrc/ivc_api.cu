@@ -101,7 +101,7 @@ void carve_ps(Carver& cv, const ivc_mlp* m, long long rows, bool need_stats, PsB
 }
 
 struct RouteBufs {
-  bf16* KV;
+  float* KV;
   float* Q1;
   float* Q;
   float* O;
@@ -112,7 +112,7 @@ struct RouteBufs {
 
 void carve_route(Carver& cv, const ivc_router* r, int T, RouteBufs& b) {
   const long long D = r->D;
-  b.KV = cv.take<bf16>(static_cast<size_t>(T) * 1024 * 8 * D);
+  b.KV = cv.take<float>(static_cast<size_t>(T) * 1024 * 8 * D);
   b.Q1 = cv.take<float>(D);
   b.Q = cv.take<float>(static_cast<size_t>(T) * D);
   b.O = cv.take<float>(static_cast<size_t>(T) * D);
@@ -130,6 +130,8 @@ void carve_route(Carver& cv, const ivc_router* r, int T, RouteBufs& b) {
 // pixel_shuffle + MLP with the statistics already in b.mean / b.rstd.
 int ps_mlp(const void* x, int T, int C, bool half, int flags, const ivc_mlp* m, bf16* y,
            const PsBufs& b, const Launch& L) {
+  static const char* const kTags[2][3] = {{"mlp2.fc1", "mlp2.fc2", "mlp2.fc3"},
+                                          {"mlp1.fc1", "mlp1.fc2", "mlp1.fc3"}};
   const long long rows = static_cast<long long>(T) * (half ? 256 : 64);
   const bf16* W0 = static_cast<const bf16*>(m->fold_W0);
   const float* cs = m->fold_colsum;
@@ -145,6 +147,7 @@ int ps_mlp(const void* x, int T, int C, bool half, int flags, const ivc_mlp* m, 
   }
   const int remap = (flags & IVC_PS_V1) ? (half ? 1 : 2) : 0;
   GemmCall c{};
+  c.tag = kTags[half][0];
   c.a_mode = half ? A_PS_HALF : ((flags & IVC_PS_QUARTER_TWICE) ? A_PS_QUARTER_TWICE : A_PS_QUARTER);
   c.a = x;
   c.T = T;
@@ -167,6 +170,7 @@ int ps_mlp(const void* x, int T, int C, bool half, int flags, const ivc_mlp* m, 
   for (int i = 1; i < m->n_linear; ++i) {
     const bool last = i + 1 == m->n_linear;
     GemmCall d{};
+    d.tag = kTags[half][i];
     d.a_mode = A_PLAIN;
     d.a = a;
     d.M = static_cast<int>(rows);
@@ -192,6 +196,7 @@ int route_impl(const void* x, const int32_t* valid_len, int T, const int32_t* im
   const int D = r->D;
   // K/V projections of the four layers: one grouped GEMM, X [T*1024, D].
   GemmCall c{};
+  c.tag = "pool.kv";
   c.a_mode = A_PLAIN;
   c.a = x;
   c.M = T * 1024;
@@ -206,6 +211,7 @@ int route_impl(const void* x, const int32_t* valid_len, int T, const int32_t* im
   }
   c.epi_mode = EPI_BIAS;
   c.out = b.KV;
+  c.out_f32 = 1;  // K/V kept in fp32: bf16 K/V alone moves the gates by ~1e-3
   c.ldo = 8LL * D;
   IVC_TRY(launch_gemm(c, L));
   const long long ldkv = 8LL * D;

@@ -95,6 +95,7 @@ __global__ void __launch_bounds__(512) ps_stats_kernel(const bf16* __restrict__ 
 int launch_ps_stats(const bf16* x, int T, int C, float* mean_half, float* rstd_half,
                     float* mean_quarter, float* rstd_quarter, const Launch& L) {
   if (T == 0) return IVC_OK;
+  TraceScope ts("ps_stats", L.stream);
   ps_stats_kernel<<<T * 64, 512, 0, L.stream>>>(x, C, mean_half, rstd_half, mean_quarter,
                                                 rstd_quarter);
   return cu_check(cudaGetLastError());
@@ -136,6 +137,7 @@ __global__ void __launch_bounds__(256) fold_kernel(const bf16* __restrict__ W,
 
 int launch_fold(const bf16* W, const bf16* b, const bf16* gamma, const bf16* beta, int N, int K,
                 bf16* W_out, float* colsum, float* fbias, const Launch& L) {
+  TraceScope ts("ln_fold", L.stream);
   fold_kernel<<<(N + 7) / 8, 256, 0, L.stream>>>(W, b, gamma, beta, N, K, W_out, colsum, fbias);
   return cu_check(cudaGetLastError());
 }
@@ -208,7 +210,8 @@ int num_sms() {
 }
 
 template <int BN, int STAGES>
-static int run_gemm(const GemmMaps& maps, const GemmArgs& args, int groups, const Launch& L) {
+static int run_gemm(const GemmMaps& maps, const GemmArgs& args, int groups, const char* tag,
+                    const Launch& L) {
   using S = GemmSmem<BN, STAGES>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -218,6 +221,7 @@ static int run_gemm(const GemmMaps& maps, const GemmArgs& args, int groups, cons
     attr_set = true;
   }
   dim3 grid((args.N + BN - 1) / BN, (args.M + GEMM_BM - 1) / GEMM_BM, groups);
+  TraceScope ts(tag ? tag : "gemm", L.stream);
   gemm_sm100_kernel<BN, STAGES><<<grid, GEMM_THREADS, S::TOTAL, L.stream>>>(maps, args, L.status);
   return cu_check(cudaGetLastError());
 }
@@ -253,6 +257,7 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
   a.gelu = c.gelu;
   a.remap = c.remap;
   a.out = c.out;
+  a.out_f32 = c.out_f32;
   a.ldo = c.ldo;
   a.group_col_stride = c.N;
   for (int g = 0; g < c.groups; ++g) a.bias[g] = c.bias[g];
@@ -260,8 +265,8 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
   a.fbias = c.fbias;
   a.row_mean = c.row_mean;
   a.row_rstd = c.row_rstd;
-  return bn == 256 ? run_gemm<256, 4>(maps, a, c.groups, L)
-                   : run_gemm<128, 6>(maps, a, c.groups, L);
+  return bn == 256 ? run_gemm<256, 4>(maps, a, c.groups, c.tag, L)
+                   : run_gemm<128, 6>(maps, a, c.groups, c.tag, L);
 }
 
 }  // namespace ivc

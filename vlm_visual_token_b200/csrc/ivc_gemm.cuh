@@ -52,7 +52,8 @@ struct GemmArgs {
   int epi_mode;
   int gelu;
   int remap;                     // 0: none; 1: transpose 16x16 token grid; 2: 8x8
-  __nv_bfloat16* out;
+  int out_f32;                   // 1: store fp32 instead of bf16
+  void* out;
   long long ldo;                 // elements
   int group_col_stride;          // output column offset per group (blockIdx.z)
   const __nv_bfloat16* bias[GEMM_MAX_GROUPS];  // EPI_BIAS, per group (may be null)
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int t = row & 63;
       out_row = (row & ~63) | ((t & 7) << 3) | (t >> 3);
     }
-    __nv_bfloat16* orow = args.out + out_row * args.ldo + (long long)g * args.group_col_stride + n0;
+    const long long out_off = out_row * args.ldo + (long long)g * args.group_col_stride + n0;
     const bool ok_any = __all_sync(0xffffffffu, ok);
     if (ok_any) {
 #pragma unroll 1
@@ -223,28 +224,31 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + c, r);
         tmem_ld_wait();
         if (row < args.M && n0 + c < args.N) {
-          uint32_t pk[16];
+          float v[32];
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float v0 = __uint_as_float(r[i]);
-            float v1 = __uint_as_float(r[i + 1]);
-            if (args.epi_mode == EPI_LNFOLD) {
-              v0 = fmaf(rstd, v0, nms * s_col0[c + i]) + s_col1[c + i];
-              v1 = fmaf(rstd, v1, nms * s_col0[c + i + 1]) + s_col1[c + i + 1];
-            } else {
-              v0 += s_col1[c + i];
-              v1 += s_col1[c + i + 1];
-            }
-            if (args.gelu) {
-              v0 = gelu_erf(v0);
-              v1 = gelu_erf(v1);
-            }
-            pk[i >> 1] = pack_bf16x2(v0, v1);
+          for (int i = 0; i < 32; ++i) {
+            float t = __uint_as_float(r[i]);
+            if (args.epi_mode == EPI_LNFOLD)
+              t = fmaf(rstd, t, nms * s_col0[c + i]) + s_col1[c + i];
+            else
+              t += s_col1[c + i];
+            v[i] = args.gelu ? gelu_erf(t) : t;
           }
-          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+          if (args.out_f32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + out_off + c);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            for (int j = 0; j < 8; ++j)
+              dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+          } else {
+            uint4* dst =
+                reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) + out_off + c);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]),
+                                  pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                                  pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
+                                  pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+          }
         }
       }
     }

@@ -23,6 +23,20 @@ struct Launch {
   int* status;  // device status word (workspace header)
 };
 
+// Brackets one kernel launch with CUDA events when tracing is on (ivc_trace.cu).
+class TraceScope {
+ public:
+  TraceScope(const char* name, cudaStream_t s);
+  ~TraceScope();
+  TraceScope(const TraceScope&) = delete;
+  TraceScope& operator=(const TraceScope&) = delete;
+
+ private:
+  cudaStream_t stream_;
+  bool active_;
+  size_t idx_ = 0;
+};
+
 // Converts a CUDA error into IVC_ECUDA (and remembers nothing else).
 inline int cu_check(cudaError_t e) { return e == cudaSuccess ? IVC_OK : IVC_ECUDA; }
 
@@ -39,6 +53,7 @@ int launch_fold(const bf16* W, const bf16* b, const bf16* gamma, const bf16* bet
 
 // One GEMM of the connector or of the pooling projections.
 struct GemmCall {
+  const char* tag;     // role, for tracing ("mlp1.fc1", "pool.kv", ...)
   int a_mode;          // AMode
   const void* a;       // A base (features for the pixel_shuffle modes)
   int T, C;            // pixel_shuffle modes
@@ -53,7 +68,8 @@ struct GemmCall {
   const float* fbias;
   const float* row_mean;
   const float* row_rstd;
-  bf16* out;
+  void* out;
+  int out_f32;         // store fp32 (pooling K/V) instead of bf16
   long long ldo;
 };
 int launch_gemm(const GemmCall& c, const Launch& L);
@@ -66,7 +82,7 @@ int launch_gemv(const float* X, long long ldx, int M, int K, const bf16* W, cons
 int launch_gemv_bf16x(const bf16* x, int K, const bf16* W, const bf16* b, int N, float* Y,
                       const Launch& L);
 // Masked single-query multi-head attention of one pooling layer.
-int launch_pool_attention(const float* Q, long long ldq, const bf16* KV, long long ldkv,
+int launch_pool_attention(const float* Q, long long ldq, const float* KV, long long ldkv,
                           int koff, int voff, const int32_t* valid_len, int T, int D, int heads,
                           float* O, const Launch& L);
 // h[t] += LN(u[t]) * gamma + beta over D.

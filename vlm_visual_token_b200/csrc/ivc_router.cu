@@ -14,8 +14,9 @@
 // The K and V projections of all four pooling layers are one grouped
 // tensor-core GEMM (ivc_gemm.cuh); what remains per layer is a skinny
 // projection of the query (M = tiles), the masked softmax-weighted sum over
-// the tile's tokens, and the output projection. All router activations stay
-// fp32; only K/V (GEMM outputs) are bf16.
+// the tile's tokens, and the output projection. All router activations,
+// K/V included, are fp32 (rounding K/V to bf16 alone moves the gate
+// probabilities by about 1e-3 on the 13-tile workload).
 #include <cuda_runtime.h>
 
 #include "ivc_internal.h"
@@ -103,6 +104,7 @@ static int run_gemv(const XT* X, long long ldx, int M, const bf16* W, const bf16
       return IVC_ECUDA;
     attr = true;
   }
+  TraceScope ts(gelu ? "router.gemv_gelu" : "router.gemv", L.stream);
   gemv_kernel<XT, J><<<(N + GEMV_WARPS - 1) / GEMV_WARPS, GEMV_WARPS * 32, smem, L.stream>>>(
       X, ldx, M, W, b, N, Y, ldy, gelu);
   return cu_check(cudaGetLastError());
@@ -140,7 +142,7 @@ constexpr int HEAD_DIM = 64;
 
 __global__ void __launch_bounds__(ATT_THREADS)
     pool_attention_kernel(const float* __restrict__ Q, long long ldq,
-                          const bf16* __restrict__ KV, long long ldkv, int koff, int voff,
+                          const float* __restrict__ KV, long long ldkv, int koff, int voff,
                           const int32_t* __restrict__ valid_len, float* __restrict__ O, int D,
                           int* __restrict__ status) {
   __shared__ float s_q[HEAD_DIM];
@@ -160,20 +162,18 @@ __global__ void __launch_bounds__(ATT_THREADS)
   if (threadIdx.x < HEAD_DIM)
     s_q[threadIdx.x] = Q[tile * ldq + h * HEAD_DIM + threadIdx.x] * 0.125f;  // 1/sqrt(64)
   __syncthreads();
-  const bf16* kbase = KV + static_cast<long long>(tile) * TILE_TOKENS * ldkv + koff + h * HEAD_DIM;
+  const float* kbase = KV + static_cast<long long>(tile) * TILE_TOKENS * ldkv + koff + h * HEAD_DIM;
   float mx = -INFINITY;
   for (int t = threadIdx.x; t < n; t += ATT_THREADS) {
-    const uint4* kr = reinterpret_cast<const uint4*>(kbase + t * ldkv);
+    const float4* kr = reinterpret_cast<const float4*>(kbase + t * ldkv);
     float s = 0.f;
 #pragma unroll
-    for (int c = 0; c < HEAD_DIM / 8; ++c) {
-      const uint4 u = kr[c];
-      const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        s = fmaf(__uint_as_float(wv[j] << 16), s_q[c * 8 + 2 * j], s);
-        s = fmaf(__uint_as_float(wv[j] & 0xffff0000u), s_q[c * 8 + 2 * j + 1], s);
-      }
+    for (int c = 0; c < HEAD_DIM / 4; ++c) {
+      const float4 k4 = kr[c];
+      s = fmaf(k4.x, s_q[4 * c], s);
+      s = fmaf(k4.y, s_q[4 * c + 1], s);
+      s = fmaf(k4.z, s_q[4 * c + 2], s);
+      s = fmaf(k4.w, s_q[4 * c + 3], s);
     }
     s_p[t] = s;
     mx = fmaxf(mx, s);
@@ -200,13 +200,13 @@ __global__ void __launch_bounds__(ATT_THREADS)
 #pragma unroll
   for (int i = 0; i < ATT_THREADS / 32; ++i) sum += s_scalar[i];
   // weighted V: warp w takes tokens w, w+8, ...; lane l owns dims 2l, 2l+1
-  const bf16* vbase = KV + static_cast<long long>(tile) * TILE_TOKENS * ldkv + voff + h * HEAD_DIM;
+  const float* vbase = KV + static_cast<long long>(tile) * TILE_TOKENS * ldkv + voff + h * HEAD_DIM;
   float a0 = 0.f, a1 = 0.f;
   for (int t = warp; t < n; t += ATT_THREADS / 32) {
-    const uint32_t u = *reinterpret_cast<const uint32_t*>(vbase + t * ldkv + 2 * lane);
+    const float2 v2 = *reinterpret_cast<const float2*>(vbase + t * ldkv + 2 * lane);
     const float p = s_p[t];
-    a0 = fmaf(p, __uint_as_float(u << 16), a0);
-    a1 = fmaf(p, __uint_as_float(u & 0xffff0000u), a1);
+    a0 = fmaf(p, v2.x, a0);
+    a1 = fmaf(p, v2.y, a1);
   }
   s_red[warp][2 * lane] = a0;
   s_red[warp][2 * lane + 1] = a1;
@@ -219,11 +219,12 @@ __global__ void __launch_bounds__(ATT_THREADS)
   }
 }
 
-int launch_pool_attention(const float* Q, long long ldq, const bf16* KV, long long ldkv,
+int launch_pool_attention(const float* Q, long long ldq, const float* KV, long long ldkv,
                           int koff, int voff, const int32_t* valid_len, int T, int D, int heads,
                           float* O, const Launch& L) {
   if (T == 0) return IVC_OK;
   if (heads * HEAD_DIM != D) return IVC_EUNSUPPORTED;
+  TraceScope ts("pool.attention", L.stream);
   pool_attention_kernel<<<dim3(heads, T), ATT_THREADS, 0, L.stream>>>(Q, ldq, KV, ldkv, koff,
                                                                      voff, valid_len, O, D,
                                                                      L.status);
@@ -273,6 +274,7 @@ __global__ void __launch_bounds__(256) residual_ln_kernel(float* __restrict__ h,
 int launch_residual_ln(float* h, const float* u, const bf16* gamma, const bf16* beta, int T,
                        int D, const Launch& L) {
   if (T == 0) return IVC_OK;
+  TraceScope ts("gate.residual_ln", L.stream);
   residual_ln_kernel<<<T, 256, 0, L.stream>>>(h, u, gamma, beta, D);
   return cu_check(cudaGetLastError());
 }
@@ -314,6 +316,7 @@ __global__ void __launch_bounds__(256) gate_head_kernel(const float* __restrict_
 int launch_gate_head(const float* h, const bf16* Wout, const bf16* bout, int T, int D,
                      float* gate, const Launch& L) {
   if (T == 0) return IVC_OK;
+  TraceScope ts("gate.head", L.stream);
   gate_head_kernel<<<(T + 7) / 8, 256, 0, L.stream>>>(h, Wout, bout, T, D, gate);
   return cu_check(cudaGetLastError());
 }
@@ -448,6 +451,7 @@ int launch_route(const float* gate, int T, const int32_t* image_offsets, int I, 
       return IVC_ECUDA;
     attr = true;
   }
+  TraceScope ts("route", L.stream);
   route_kernel<<<1, ROUTE_THREADS, smem, L.stream>>>(gate, T, image_offsets, I, rel_q, abs_t,
                                                      scope, mask, offsets, total, L.status);
   return cu_check(cudaGetLastError());
@@ -478,6 +482,7 @@ __global__ void __launch_bounds__(256) compact_kernel(const bf16* __restrict__ Y
 int launch_compact(const bf16* Y256, const bf16* Y64, const uint8_t* mask,
                    const int32_t* offsets, int T, int H, bf16* out, const Launch& L) {
   if (T == 0) return IVC_OK;
+  TraceScope ts("compact", L.stream);
   compact_kernel<<<dim3(T, 8), 256, 0, L.stream>>>(Y256, Y64, mask, offsets, H, out);
   return cu_check(cudaGetLastError());
 }
