@@ -384,8 +384,10 @@ def run_ivc(args):
            "d2h_bytes_per_step": d2h_small + d2h_rows // e2e_steps, "steps": e2e_steps,
            "timing": "wall clock, host sync per step (needs the row count before the row copy)"}
 
-    if graph is not None:
-        del graph
+    launch_desc = ("CUDA graph of one ivc_flash_compress" if graph is not None
+                   else "eager ivc_flash_compress")
+    run = None
+    graph = None
     barrier()
     if world > 1:
         import torch.distributed as dist
@@ -398,8 +400,7 @@ def run_ivc(args):
             "config": {"workload": WORKLOAD, "tiles_per_step": T, "C": w.C, "H": w.H,
                        "mlp2_mid": w.mlp2_mid, "pool_heads": 16, "gate_hidden": w.gate_hidden,
                        "l2": "flushed between steps (512 MiB write, outside the timed events)",
-                       "launch": "CUDA graph of one ivc_flash_compress" if graph is not None
-                                 else "eager ivc_flash_compress",
+                       "launch": launch_desc,
                        "parallelism": f"replicas x{world}, one image per GPU, no collective"},
             "roofline": roof, "step_roofline": step_roofline,
             "kernels_ms_per_step": {k: round(v, 5) for k, v in per_step_ms.items()},
