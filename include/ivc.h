@@ -204,6 +204,29 @@ int ivc_flash_compress(const void* x, const int32_t* valid_len, int T, int C,
  * clear it. Returns IVC_OK when no bit was set, IVC_EDEVICE otherwise. */
 int ivc_device_status(void* workspace, int* bits, ivc_stream_t stream);
 
+/* ivc_ps_project for callers that cannot allocate device memory.
+ * No counterpart on the pages: this is a deployment variant of the call above.
+ * Callers such as an inference-engine plugin whose device memory is planned
+ * ahead, or a latency-critical loop that cannot afford the synchronisation an
+ * allocation may cause, cannot call cudaMalloc to create a workspace. This
+ * entry point instead uses a fixed scratch array of IVC_NOALLOC_SCRATCH_BYTES
+ * that the library holds in device memory on every GPU that loads it, until
+ * the process exits. It allocates nothing itself.
+ *   Arguments and results are those of ivc_ps_project, without the workspace.
+ *   `m` must already be folded (ivc_mlp_fold); otherwise IVC_EINVAL.
+ *   Calls needing more scratch than IVC_NOALLOC_SCRATCH_BYTES (the
+ *   ivc_workspace_size of the same op) return IVC_EWORKSPACE and enqueue
+ *   nothing: e.g. up to 15 tiles of mlp1 4096->2048->2048 fit.
+ *   The first call on a device looks up the array's device address (with that
+ *   device current); make that first call before any stream capture.
+ *   All calls share the one array and it keeps the last call's contents:
+ *   calls whose GPU work can overlap (other streams, other host threads on
+ *   the same device) race on it. The device status word inside the array is
+ *   cleared at the start of every call and cannot be read by the caller. */
+#define IVC_NOALLOC_SCRATCH_BYTES (16u << 20)
+int ivc_ps_project_noalloc(const void* x, int T, int C, float scale, int flags,
+                           const ivc_mlp* m, void* y, ivc_stream_t stream);
+
 /* Per-kernel device timing (diagnostics; off by default). While enabled,
  * every kernel launch is bracketed by two CUDA events on its stream and filed
  * under its role (e.g. "mlp1.fc1", "pool.kv", "pool.attention", "route").
