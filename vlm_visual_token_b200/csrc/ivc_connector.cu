@@ -183,6 +183,17 @@ static int map_2d(CUtensorMap* m, const void* base, long long rows, long long co
   return encode(m, 2, base, dims, strides, box);
 }
 
+// Batched [batches][rows][inner] bf16 (row stride ld, batch stride bs elements),
+// box {box_inner, box_rows, 1}.
+static int map_3d(CUtensorMap* m, const void* base, long long batches, long long rows,
+                  long long inner, long long ld, long long bs, int box_inner, int box_rows) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(batches)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld) * 2, static_cast<cuuint64_t>(bs) * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows), 1};
+  return encode(m, 3, base, dims, strides, box);
+}
+
 // The [T,32,32,C] features seen as the pixel-shuffled [T*tokens, f*f*C] matrix.
 static int map_ps(CUtensorMap* m, const void* x, int T, int C, int f) {
   const cuuint64_t Cu = static_cast<cuuint64_t>(C);
@@ -210,7 +221,7 @@ int num_sms() {
 }
 
 template <int BN, int STAGES>
-static int run_gemm(const GemmMaps& maps, const GemmArgs& args, int groups, const char* tag,
+static int run_gemm(const GemmMaps& maps, const GemmArgs& args, const char* tag,
                     const Launch& L) {
   using S = GemmSmem<BN, STAGES>;
   static bool attr_set = false;
@@ -220,20 +231,38 @@ static int run_gemm(const GemmMaps& maps, const GemmArgs& args, int groups, cons
     if (e != cudaSuccess) return IVC_ECUDA;
     attr_set = true;
   }
-  dim3 grid((args.N + BN - 1) / BN, (args.M + GEMM_BM - 1) / GEMM_BM, groups);
+  const long long tiles = static_cast<long long>((args.M + GEMM_BM - 1) / GEMM_BM) *
+                          ((args.N + BN - 1) / BN) * args.groups;
+  const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
   TraceScope ts(tag ? tag : "gemm", L.stream);
   gemm_sm100_kernel<BN, STAGES><<<grid, GEMM_THREADS, S::TOTAL, L.stream>>>(maps, args, L.status);
   return cu_check(cudaGetLastError());
+}
+
+// Output tile width: the one that finishes the tile set soonest on the SMs
+// (persistent CTAs; narrower tiles pay ~15% more per flop in operand traffic).
+static int pick_bn(const GemmCall& c) {
+  if (c.N <= 32) return 32;
+  if (c.N <= 64) return 64;
+  const long long mt = (c.M + GEMM_BM - 1) / GEMM_BM;
+  const long long sms = num_sms();
+  auto cost = [&](int bn, double eff) {
+    const long long tiles = mt * ((c.N + bn - 1) / bn) * c.groups;
+    return static_cast<double>((tiles + sms - 1) / sms) * bn * eff;
+  };
+  if (c.b_mode == B_MN3D) return cost(128, 1.15) < cost(256, 1.0) ? 128 : 256;
+  if (c.N <= 128) return 128;
+  return cost(128, 1.15) < cost(256, 1.0) ? 128 : 256;
 }
 
 int launch_gemm(const GemmCall& c, const Launch& L) {
   if (c.M == 0 || c.N == 0) return IVC_OK;
   if (c.K % GEMM_BK != 0 || c.N % 32 != 0 || c.groups < 1 || c.groups > GEMM_MAX_GROUPS)
     return IVC_EUNSUPPORTED;
-  // Tile width: 256 columns unless that leaves most SMs idle.
-  const int m_tiles = (c.M + GEMM_BM - 1) / GEMM_BM;
-  const long long tiles256 = static_cast<long long>(m_tiles) * ((c.N + 255) / 256) * c.groups;
-  const int bn = (tiles256 * 2 <= num_sms() && c.N > 128) || c.N <= 128 ? 128 : 256;
+  if (c.b_mode != B_K2D && (c.b_batch_rows <= 0 || c.b_batch_rows % GEMM_BM != 0))
+    return IVC_EUNSUPPORTED;
+  if (c.b_mode == B_MN3D && c.N % 64 != 0) return IVC_EUNSUPPORTED;
+  const int bn = pick_bn(c);
 
   GemmMaps maps;
   int rc;
@@ -244,14 +273,24 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
   }
   if (rc) return rc;
   for (int g = 0; g < c.groups; ++g) {
-    rc = map_2d(&maps.b[g], c.B[g], c.N, c.K, bn);
+    if (c.b_mode == B_K2D)
+      rc = map_2d(&maps.b[g], c.B[g], c.N, c.K, bn);
+    else if (c.b_mode == B_K3D)
+      rc = map_3d(&maps.b[g], c.B[g], c.b_batches, c.N, c.K, c.b_ld, c.b_batch_stride, GEMM_BK,
+                  bn);
+    else
+      rc = map_3d(&maps.b[g], c.B[g], c.b_batches, c.K, c.N, c.b_ld, c.b_batch_stride, 64,
+                  GEMM_BK);
     if (rc) return rc;
   }
   GemmArgs a{};
   a.M = c.M;
   a.N = c.N;
   a.K = c.K;
+  a.groups = c.groups;
   a.a_mode = c.a_mode;
+  a.b_mode = c.b_mode;
+  a.b_batch_rows = c.b_mode == B_K2D ? 0 : c.b_batch_rows;
   a.c_blocks = c.C / GEMM_BK;
   a.epi_mode = c.epi_mode;
   a.gelu = c.gelu;
@@ -265,8 +304,12 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
   a.fbias = c.fbias;
   a.row_mean = c.row_mean;
   a.row_rstd = c.row_rstd;
-  return bn == 256 ? run_gemm<256, 4>(maps, a, c.groups, c.tag, L)
-                   : run_gemm<128, 6>(maps, a, c.groups, c.tag, L);
+  switch (bn) {
+    case 256: return run_gemm<256, 4>(maps, a, c.tag, L);
+    case 128: return run_gemm<128, 6>(maps, a, c.tag, L);
+    case 64: return run_gemm<64, 8>(maps, a, c.tag, L);
+    default: return run_gemm<32, 8>(maps, a, c.tag, L);
+  }
 }
 
 }  // namespace ivc

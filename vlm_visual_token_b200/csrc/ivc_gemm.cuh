@@ -2,17 +2,19 @@
 //
 //   out[m, n] = epilogue( sum_k A[m, k] * B[n, k] )      (B = nn.Linear weight [N, K])
 //
-// One CTA computes one 128 x BN output tile with the 5th-generation tensor
-// cores: TMA streams 128 x 64 A tiles and BN x 64 B tiles (128-byte swizzle)
-// through a STAGES-deep shared-memory ring, one thread issues
-// tcgen05.mma (M=128, N=BN, K=16) into a TMEM accumulator, and four epilogue
-// warps read the accumulator back with tcgen05.ld and apply the fused
-// epilogue (LayerNorm fold or bias, then optional GELU) before storing bf16.
+// Persistent, warp-specialised tcgen05 kernel. Each CTA loops over output
+// tiles of 128 x BN (static round-robin over tile index, n fastest). TMA
+// streams 128 x 64 A tiles and BN x 64 B tiles (128-byte swizzle) through a
+// STAGES-deep shared-memory ring; one thread issues tcgen05.mma (M=128, N=BN,
+// K=16) into one of two TMEM accumulators; four epilogue warps drain the other
+// accumulator with tcgen05.ld, apply the fused epilogue (LayerNorm fold or
+// bias, optional GELU) and store bf16 or fp32, so a tile's epilogue overlaps
+// the next tile's mainloop.
 //
 // Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM owner and
 // MMA issuer, warps 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
 //
-// A-operand modes. pixel_shuffle ("Pixel Shuffle 源码逐行解析" of the
+// A operand. pixel_shuffle ("Pixel Shuffle 源码逐行解析" of the
 // InternVL3-14B-Instruct connector article; table "三档 Token 规模" of the
 // InternVL3_5-2B-Flash article) is not materialised: the GEMM row of
 // token (tile, a, b) and the column block of grid offset (di, dj) are
@@ -23,6 +25,12 @@
 // Column m of the shuffled row is (block*C + c) with block = 2di+dj
 // (4q+r for the quarter), so k-step kk loads block kk/(C/64), channels
 // 64*(kk%(C/64)).. of each of the 128 tokens of the tile.
+//
+// B operand. K-major (nn.Linear weights, 2-D or batched 3-D with the batch
+// chosen by the tile's row: batch = m0 / b_batch_rows), or MN-major batched
+// 3-D (B[n, k] stored with n contiguous, e.g. a [tokens, channels] feature
+// block used as B = X^T): then each stage holds BN/64 boxes of 64 k-rows x
+// 64 n-columns and the UMMA descriptor walks them MN-major.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -33,12 +41,14 @@
 namespace ivc {
 
 enum AMode : int { A_PLAIN = 0, A_PS_HALF = 1, A_PS_QUARTER = 2, A_PS_QUARTER_TWICE = 3 };
+enum BMode : int { B_K2D = 0, B_K3D = 1, B_MN3D = 2 };
 enum EpiMode : int { EPI_BIAS = 0, EPI_LNFOLD = 1 };
 
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 64;
 constexpr int GEMM_MAX_GROUPS = 8;
 constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_EPI_BAR = 1;  // named barrier of the 4 epilogue warps
 
 struct alignas(64) GemmMaps {
   CUtensorMap a;
@@ -47,7 +57,10 @@ struct alignas(64) GemmMaps {
 
 struct GemmArgs {
   int M, N, K;
+  int groups;                    // blockIdx-independent group count (tile index space)
   int a_mode;
+  int b_mode;
+  int b_batch_rows;              // B_K3D / B_MN3D: rows of A per B batch
   int c_blocks;                  // C / 64 for the pixel_shuffle modes
   int epi_mode;
   int gelu;
@@ -55,7 +68,7 @@ struct GemmArgs {
   int out_f32;                   // 1: store fp32 instead of bf16
   void* out;
   long long ldo;                 // elements
-  int group_col_stride;          // output column offset per group (blockIdx.z)
+  int group_col_stride;          // output column offset per group
   const __nv_bfloat16* bias[GEMM_MAX_GROUPS];  // EPI_BIAS, per group (may be null)
   const float* colsum;           // EPI_LNFOLD
   const float* fbias;            // EPI_LNFOLD
@@ -67,10 +80,12 @@ template <int BN, int STAGES>
 struct GemmSmem {
   static constexpr uint32_t A_BYTES = GEMM_BM * GEMM_BK * 2;
   static constexpr uint32_t B_BYTES = BN * GEMM_BK * 2;
-  static constexpr uint32_t RING = STAGES * (A_BYTES + B_BYTES);
-  static constexpr uint32_t BARS = (2 * STAGES + 1) * 8 + 16;
+  static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
+  static constexpr uint32_t RING = STAGES * STAGE;
+  static constexpr uint32_t BARS = (2 * STAGES + 4) * 8 + 16;
   static constexpr uint32_t COLS = 2 * BN * 4;
   static constexpr uint32_t TOTAL = 1024 + RING + BARS + COLS;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;  // double-buffered accumulator
 };
 
 __device__ __forceinline__ float gelu_erf(float y) {
@@ -82,28 +97,44 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+__device__ __forceinline__ void epi_bar_sync() {
+  asm volatile("bar.sync %0, 128;" ::"n"(GEMM_EPI_BAR) : "memory");
+}
+
+// Tile index -> (group, m-tile, n-tile), n fastest.
+struct TileCoord {
+  int g, m0, n0;
+};
+__device__ __forceinline__ TileCoord tile_coord(int idx, int m_tiles, int n_tiles, int BN) {
+  const int n = idx % n_tiles;
+  const int rest = idx / n_tiles;
+  const int m = rest % m_tiles;
+  return {rest / m_tiles, m * GEMM_BM, n * BN};
+}
+
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_sm100_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs args,
                       int* __restrict__ status) {
   using L = GemmSmem<BN, STAGES>;
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * L::A_BYTES;
+  uint8_t* ring = smem;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + L::RING);
   uint64_t* empty_bar = full_bar + STAGES;
-  uint64_t* accum_bar = empty_bar + STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum_bar + 1);
+  uint64_t* tfull_bar = empty_bar + STAGES;   // [2] accumulator ready
+  uint64_t* tempty_bar = tfull_bar + 2;       // [2] accumulator drained
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 2);
   float* s_col0 = reinterpret_cast<float*>(smem + L::RING + L::BARS);
   float* s_col1 = s_col0 + BN;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int g = blockIdx.z;
-  const int m0 = blockIdx.y * GEMM_BM;
-  const int n0 = blockIdx.x * BN;
+  const int m_tiles = (args.M + GEMM_BM - 1) / GEMM_BM;
+  const int n_tiles = (args.N + BN - 1) / BN;
+  const int n_total = m_tiles * n_tiles * args.groups;
   const int KT = args.K / GEMM_BK;
 
   if (warp == 0 && lane == 0) {
@@ -111,31 +142,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    mbar_init(accum_bar, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 4);  // one arrival per epilogue warp
+    }
     fence_mbar_init();
     tma_prefetch_desc(&maps.a);
-    tma_prefetch_desc(&maps.b[g]);
+    for (int g = 0; g < args.groups; ++g) tma_prefetch_desc(&maps.b[g]);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, BN);
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
     tmem_relinquish();
-  }
-  if (warp >= 2) {
-    // Per-column epilogue vectors for this tile, staged once in shared memory.
-    for (int i = threadIdx.x - 64; i < BN; i += 128) {
-      const int n = n0 + i;
-      float c0 = 0.f, c1 = 0.f;
-      if (n < args.N) {
-        if (args.epi_mode == EPI_LNFOLD) {
-          c0 = args.colsum[n];
-          c1 = args.fbias[n];
-        } else if (args.bias[g] != nullptr) {
-          c1 = __bfloat162float(args.bias[g][n]);
-        }
-      }
-      s_col0[i] = c0;
-      s_col1[i] = c1;
-    }
   }
   tc_fence_before();
   __syncthreads();
@@ -146,84 +163,147 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
-      for (int kk = 0; kk < KT; ++kk) {
-        const int s = kk % STAGES;
-        const uint32_t ph = (kk / STAGES) & 1;
-        if (!mbar_wait(&empty_bar[s], ph ^ 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(&full_bar[s], L::A_BYTES + L::B_BYTES);
-        uint8_t* a_dst = sA + s * L::A_BYTES;
-        if (args.a_mode == A_PLAIN) {
-          tma_load_2d(a_dst, &maps.a, &full_bar[s], kk * GEMM_BK, m0);
-        } else {
-          const int blk = kk / args.c_blocks;
-          const int c0 = (kk - blk * args.c_blocks) * GEMM_BK;
-          if (args.a_mode == A_PS_HALF) {
-            tma_load_5d(a_dst, &maps.a, &full_bar[s], c0, blk & 1, 0, blk >> 1, m0 >> 4);
+      int it = 0;
+      for (int idx = blockIdx.x; idx < n_total && ok; idx += gridDim.x) {
+        const TileCoord tc = tile_coord(idx, m_tiles, n_tiles, BN);
+        const int bb = args.b_batch_rows > 0 ? tc.m0 / args.b_batch_rows : 0;
+        for (int kk = 0; kk < KT; ++kk, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(&empty_bar[s], ph ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full_bar[s], L::STAGE);
+          uint8_t* a_dst = ring + s * L::STAGE;
+          uint8_t* b_dst = a_dst + L::A_BYTES;
+          if (args.a_mode == A_PLAIN) {
+            tma_load_2d(a_dst, &maps.a, &full_bar[s], kk * GEMM_BK, tc.m0);
           } else {
-            int q, r;
-            if (args.a_mode == A_PS_QUARTER) {
-              q = blk >> 2;
-              r = blk & 3;
-            } else {  // two successive factor-0.5 shuffles: blk = 8ei + 4ej + 2di + dj
-              q = 2 * (blk >> 3) + ((blk >> 1) & 1);
-              r = 2 * ((blk >> 2) & 1) + (blk & 1);
+            const int blk = kk / args.c_blocks;
+            const int c0 = (kk - blk * args.c_blocks) * GEMM_BK;
+            if (args.a_mode == A_PS_HALF) {
+              tma_load_5d(a_dst, &maps.a, &full_bar[s], c0, blk & 1, 0, blk >> 1, tc.m0 >> 4);
+            } else {
+              int q, r;
+              if (args.a_mode == A_PS_QUARTER) {
+                q = blk >> 2;
+                r = blk & 3;
+              } else {  // two successive factor-0.5 shuffles: blk = 8ei + 4ej + 2di + dj
+                q = 2 * (blk >> 3) + ((blk >> 1) & 1);
+                r = 2 * ((blk >> 2) & 1) + (blk & 1);
+              }
+              tma_load_5d(a_dst, &maps.a, &full_bar[s], c0, r, 0, q, tc.m0 >> 3);
             }
-            tma_load_5d(a_dst, &maps.a, &full_bar[s], c0, r, 0, q, m0 >> 3);
+          }
+          const CUtensorMap* bm = &maps.b[tc.g];
+          if (args.b_mode == B_K2D) {
+            tma_load_2d(b_dst, bm, &full_bar[s], kk * GEMM_BK, tc.n0);
+          } else if (args.b_mode == B_K3D) {
+            tma_load_3d(b_dst, bm, &full_bar[s], kk * GEMM_BK, tc.n0, bb);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_3d(b_dst + j * (64 * GEMM_BK * 2), bm, &full_bar[s], tc.n0 + 64 * j,
+                          kk * GEMM_BK, bb);
           }
         }
-        tma_load_2d(sB + s * L::B_BYTES, &maps.b[g], &full_bar[s], kk * GEMM_BK, n0);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc = idesc_bf16_f32(GEMM_BM, BN);
-      for (int kk = 0; kk < KT; ++kk) {
-        const int s = kk % STAGES;
-        const uint32_t ph = (kk / STAGES) & 1;
-        if (!mbar_wait(&full_bar[s], ph)) { ok = false; break; }
+      const uint32_t idesc = idesc_bf16_f32(GEMM_BM, BN) |
+                             (args.b_mode == B_MN3D ? (1u << 16) : 0u);  // B MN-major
+      int it = 0, local = 0;
+      for (int idx = blockIdx.x; idx < n_total && ok; idx += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t use = static_cast<uint32_t>(local >> 1);
+        if (!mbar_wait(&tempty_bar[acc], (use & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
-        const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * L::A_BYTES));
-        const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * L::B_BYTES));
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kk = 0; kk < KT; ++kk, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(&full_bar[s], ph)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(ring + s * L::STAGE);
+          const uint64_t ad = sw128_kmajor_desc(a_addr);
+          const uint64_t bd = args.b_mode == B_MN3D
+                                  ? sw128_mnmajor_desc(a_addr + L::A_BYTES, 64 * GEMM_BK * 2)
+                                  : sw128_kmajor_desc(a_addr + L::A_BYTES);
+          const uint64_t bstep = args.b_mode == B_MN3D ? (16 * 128) >> 4 : 2;
 #pragma unroll
-        for (int k = 0; k < GEMM_BK / 16; ++k) {
-          // advance 16 bf16 = 32 bytes (2 x 16 B) along K inside the swizzle atom
-          umma_bf16(tmem_base, ad + 2 * k, bd + 2 * k, idesc, (kk | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < GEMM_BK / 16; ++k) {
+            // K-major: advance 16 bf16 = 32 bytes inside the swizzle atom;
+            // MN-major: advance 16 k-rows of 128 bytes.
+            umma_bf16(d_tmem, ad + 2 * k, bd + bstep * k, idesc, (kk | k) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty_bar[s]);
         }
-        umma_commit(&empty_bar[s]);
+        if (!ok) break;
+        umma_commit(&tfull_bar[acc]);
       }
-      umma_commit(accum_bar);
     }
   } else {
     // -------------------------------------------------------------- epilogue
     const int quad = warp & 3;
-    const int row = m0 + quad * 32 + lane;
-    if (!mbar_wait(accum_bar, 0)) ok = false;
-    __syncwarp();
-    tc_fence_after();
-    float mean = 0.f, rstd = 1.f;
-    if (args.epi_mode == EPI_LNFOLD && row < args.M) {
-      mean = args.row_mean[row];
-      rstd = args.row_rstd[row];
-    }
-    const float nms = -mean * rstd;
-    long long out_row = row;
-    if (args.remap == 1) {
-      const int t = row & 255;
-      out_row = (row & ~255) | ((t & 15) << 4) | (t >> 4);
-    } else if (args.remap == 2) {
-      const int t = row & 63;
-      out_row = (row & ~63) | ((t & 7) << 3) | (t >> 3);
-    }
-    const long long out_off = out_row * args.ldo + (long long)g * args.group_col_stride + n0;
-    const bool ok_any = __all_sync(0xffffffffu, ok);
-    if (ok_any) {
+    const int et = threadIdx.x - 64;  // 0..127
+    int local = 0;
+    for (int idx = blockIdx.x; idx < n_total; idx += gridDim.x, ++local) {
+      const TileCoord tc = tile_coord(idx, m_tiles, n_tiles, BN);
+      const int acc = local & 1;
+      const uint32_t use = static_cast<uint32_t>(local >> 1);
+      // per-column epilogue vectors of this tile
+      epi_bar_sync();
+      for (int i = et; i < BN; i += 128) {
+        const int n = tc.n0 + i;
+        float c0 = 0.f, c1 = 0.f;
+        if (n < args.N) {
+          if (args.epi_mode == EPI_LNFOLD) {
+            c0 = args.colsum[n];
+            c1 = args.fbias[n];
+          } else if (args.bias[tc.g] != nullptr) {
+            c1 = __bfloat162float(args.bias[tc.g][n]);
+          }
+        }
+        s_col0[i] = c0;
+        s_col1[i] = c1;
+      }
+      epi_bar_sync();
+      // After a timed-out wait the warp keeps looping (the named barrier above
+      // counts all four epilogue warps every tile) but does no more work.
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], use & 1));
+      if (!ok) continue;
+      tc_fence_after();
+      const int row = tc.m0 + quad * 32 + lane;
+      float mean = 0.f, rstd = 1.f;
+      if (args.epi_mode == EPI_LNFOLD && row < args.M) {
+        mean = args.row_mean[row];
+        rstd = args.row_rstd[row];
+      }
+      const float nms = -mean * rstd;
+      long long out_row = row;
+      if (args.remap == 1) {
+        const int t = row & 255;
+        out_row = (row & ~255) | ((t & 15) << 4) | (t >> 4);
+      } else if (args.remap == 2) {
+        const int t = row & 63;
+        out_row = (row & ~63) | ((t & 7) << 3) | (t >> 3);
+      }
+      const long long out_off =
+          out_row * args.ldo + static_cast<long long>(tc.g) * args.group_col_stride + tc.n0;
+      const uint32_t t_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                              static_cast<uint32_t>(acc * BN);
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
         uint32_t r[32];
-        tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + c, r);
+        tmem_ld32(t_base + c, r);
         tmem_ld_wait();
-        if (row < args.M && n0 + c < args.N) {
+        if (c + 32 == BN) {
+          // accumulator fully read: hand it back to the MMA warp
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+        }
+        if (row < args.M && tc.n0 + c < args.N) {
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
@@ -259,7 +339,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, BN);
+    tmem_dealloc(tmem_base, L::TMEM_COLS);
   }
 }
 

@@ -58,8 +58,13 @@ struct GemmCall {
   const void* a;       // A base (features for the pixel_shuffle modes)
   int T, C;            // pixel_shuffle modes
   int M, N, K;
-  int groups;          // >1: blockIdx.z selects B[g], bias[g], column offset g*N
+  int groups;          // >1: group g uses B[g], bias[g], output column offset g*N
   const void* B[8];
+  int b_mode;          // BMode: K-major 2-D (default), K-major 3-D batched, MN-major 3-D
+  int b_batch_rows;    // 3-D modes: rows of A (multiple of 128) per B batch
+  int b_batches;       // 3-D modes: number of batches
+  long long b_ld;      // 3-D modes: elements between consecutive rows (K-major: n; MN: k)
+  long long b_batch_stride;  // 3-D modes: elements between batches
   const bf16* bias[8];
   int epi_mode;        // EpiMode
   int gelu;
