@@ -124,7 +124,17 @@ typedef struct ivc_router {
   double rel_q;       /* flash_relative_threshold, 0.1 */
   double abs_t;       /* flash_absolute_threshold, 0.5 */
   int quantile_scope; /* 0 = per image, 1 = whole batch */
+  int pool_mode;      /* IVC_POOL_FOLDED (0) or IVC_POOL_LITERAL (1) */
 } ivc_router;
+
+/* How CrossAttentionPooling is evaluated; both compute the same function.
+ * LITERAL: K_l = X Wk_l^T + bk_l and V_l = X Wv_l^T + bv_l for all tokens (one
+ *   grouped tensor-core GEMM, fp32 K/V), then per head softmax(Q.K/8) V.
+ * FOLDED: with one query per tile the projections are reassociated exactly:
+ *   scores = X (Wk_h^T Q_h / 8) + bk_h.Q_h / 8 and o_h = Wv_h (sum_t p_t x_t) + bv_h,
+ *   two thin tensor-core GEMMs over the raw features per layer (~60x fewer
+ *   FLOPs, no K/V tensor). */
+enum ivc_pool_mode { IVC_POOL_FOLDED = 0, IVC_POOL_LITERAL = 1 };
 
 enum ivc_op {
   IVC_OP_PS_PROJECT_HALF = 1,    /* ivc_ps_project at factor 0.5 */

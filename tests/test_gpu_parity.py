@@ -147,7 +147,8 @@ def _route_check(ivc, inp, gate, mask, offsets, sample=None, scope=0):
     return err
 
 
-def test_vir_route_small_with_padding():
+@pytest.mark.parametrize("pool_mode", [0, 1])
+def test_vir_route_small_with_padding(pool_mode):
     ivc = _ivc()
     w = small_workload(C=256, H=128, tiles=(3, 1, 5), var=0.6)
     inp = W.make(w, affine="random")
@@ -155,7 +156,7 @@ def test_vir_route_small_with_padding():
     vl[1] = 1   # a single valid token
     inp["valid_len"] = vl
     inp["x"] = W.features(inp["T"], 256, 1234 + 90, vl)
-    r = ivc.Router(inp["router"])
+    r = ivc.Router(inp["router"], pool_mode=pool_mode)
     ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_VIR_ROUTE, inp["T"], 256, r=r))
     gate, mask, offsets = ivc.vir_route(inp["x"].cuda(), vl.cuda(), inp["image_offsets"].cuda(), r,
                                         workspace=ws)
@@ -165,10 +166,11 @@ def test_vir_route_small_with_padding():
     assert to_np(mask)[3] == 0  # the one-tile image is never compressed
 
 
-def test_vir_route_batch_scope():
+@pytest.mark.parametrize("pool_mode", [0, 1])
+def test_vir_route_batch_scope(pool_mode):
     ivc = _ivc()
     inp = W.make(small_workload(C=256, H=128, tiles=(4, 4)), affine="random")
-    r = ivc.Router(inp["router"], scope=1)
+    r = ivc.Router(inp["router"], scope=1, pool_mode=pool_mode)
     gate, mask, offsets = ivc.vir_route(inp["x"].cuda(), None, inp["image_offsets"].cuda(), r)
     torch.cuda.synchronize()
     _route_check(ivc, inp, gate, mask, offsets, scope=1)
@@ -217,10 +219,12 @@ def _flash_check(ivc, inp, res, tiles=None):
     return stats
 
 
-def test_flash_compress_small():
+@pytest.mark.parametrize("pool_mode", [0, 1])
+def test_flash_compress_small(pool_mode):
     ivc = _ivc()
     inp = W.make(small_workload(C=256, H=192, tiles=(3, 1, 4), var=0.3), affine="random")
-    m1, m2, r = ivc.Mlp(inp["mlp1"]), ivc.Mlp(inp["mlp2"]).fold(), ivc.Router(inp["router"])
+    m1, m2 = ivc.Mlp(inp["mlp1"]), ivc.Mlp(inp["mlp2"]).fold()
+    r = ivc.Router(inp["router"], pool_mode=pool_mode)
     ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_FLASH, inp["T"], 256, m1, m2, r))
     res = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(), inp["image_offsets"].cuda(),
                              m1, m2, r, workspace=ws)
@@ -239,11 +243,13 @@ def test_flash_compress_empty():
     assert int(res["total"].item()) == 0 and int(res["offsets"][0].item()) == 0
 
 
-def test_flash_2b_13tiles_full():
+@pytest.mark.parametrize("pool_mode", [0, 1])
+def test_flash_2b_13tiles_full(pool_mode):
     """The benchmark workload, every output checked against the oracle."""
     ivc = _ivc()
     inp = W.make("flash_2b_13tiles")
-    m1, m2, r = ivc.Mlp(inp["mlp1"]).fold(), ivc.Mlp(inp["mlp2"]).fold(), ivc.Router(inp["router"])
+    m1, m2 = ivc.Mlp(inp["mlp1"]).fold(), ivc.Mlp(inp["mlp2"]).fold()
+    r = ivc.Router(inp["router"], pool_mode=pool_mode)
     res = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(), inp["image_offsets"].cuda(),
                              m1, m2, r)
     torch.cuda.synchronize()
@@ -251,14 +257,16 @@ def test_flash_2b_13tiles_full():
     assert max(s["max_abs"] for s in stats) <= 3e-2, stats
 
 
-def test_flash_4b_batched_sampled():
+@pytest.mark.parametrize("pool_mode", [0, 1])
+def test_flash_4b_batched_sampled(pool_mode):
     """16 images with drawn tile counts and 10% padded tiles; the oracle checks
     a seeded sample of tiles (including padded ones); routing and offsets are
     checked for every tile."""
     ivc = _ivc()
     inp = W.make("flash_4b_batched")
     T = inp["T"]
-    m1, m2, r = ivc.Mlp(inp["mlp1"]).fold(), ivc.Mlp(inp["mlp2"]).fold(), ivc.Router(inp["router"])
+    m1, m2 = ivc.Mlp(inp["mlp1"]).fold(), ivc.Mlp(inp["mlp2"]).fold()
+    r = ivc.Router(inp["router"], pool_mode=pool_mode)
     ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_FLASH, T, 1024, m1, m2, r))
     res = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(), inp["image_offsets"].cuda(),
                              m1, m2, r, workspace=ws)

@@ -19,7 +19,9 @@ from typing import Optional, Sequence
 
 import torch
 
-__all__ = ["Mlp", "Router", "ps_project", "vir_route", "flash_compress", "workspace_size",
+POOL_FOLDED, POOL_LITERAL = 0, 1
+
+__all__ = ["Mlp", "Router", "POOL_FOLDED", "POOL_LITERAL", "ps_project", "vir_route", "flash_compress", "workspace_size",
            "device_status", "IvcError", "lib", "LIB_PATH", "PS_V1", "PS_QUARTER_TWICE",
            "OP_PS_HALF", "OP_PS_QUARTER", "OP_VIR_ROUTE", "OP_FLASH"]
 
@@ -46,7 +48,7 @@ class _CRouter(ctypes.Structure):
                 ("gW1", _vp * 4), ("gb1", _vp * 4), ("gW2", _vp * 4), ("gb2", _vp * 4),
                 ("gln_g", _vp * 4), ("gln_b", _vp * 4), ("gWout", _vp), ("gbout", _vp),
                 ("rel_q", ctypes.c_double), ("abs_t", ctypes.c_double),
-                ("quantile_scope", ctypes.c_int)]
+                ("quantile_scope", ctypes.c_int), ("pool_mode", ctypes.c_int)]
 
 
 class IvcError(RuntimeError):
@@ -152,7 +154,7 @@ class Router:
     """ViR router weights (CrossAttentionPooling + Gating) and thresholds."""
 
     def __init__(self, params: dict, rel_q: float = 0.1, abs_t: float = 0.5, scope: int = 0,
-                 device="cuda"):
+                 device="cuda", pool_mode: int = 0):
         def dev(t):
             return t.to(device=device, dtype=torch.bfloat16).contiguous()
         self.t = {}
@@ -175,6 +177,7 @@ class Router:
         c.rel_q = float(rel_q)
         c.abs_t = float(abs_t)
         c.quantile_scope = int(scope)
+        c.pool_mode = int(pool_mode)
         self.c = c
 
 

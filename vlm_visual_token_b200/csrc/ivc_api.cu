@@ -63,6 +63,9 @@ int router_shape_ok(const ivc_router* r, int C) {
   }
   if (!d_ok || !g_ok) return IVC_EUNSUPPORTED;
   if (r->quantile_scope != 0 && r->quantile_scope != 1) return IVC_EINVAL;
+  if (r->pool_mode != IVC_POOL_FOLDED && r->pool_mode != IVC_POOL_LITERAL) return IVC_EINVAL;
+  if (r->pool_mode == IVC_POOL_FOLDED && (r->heads > 16 || r->D % 128 != 0))
+    return IVC_EUNSUPPORTED;
   if (!r->query || !r->gWout) return IVC_EINVAL;
   for (int l = 0; l < 4; ++l) {
     const void* ws[4] = {r->Wq[l], r->Wk[l], r->Wv[l], r->Wo[l]};
@@ -101,7 +104,12 @@ void carve_ps(Carver& cv, const ivc_mlp* m, long long rows, bool need_stats, PsB
 }
 
 struct RouteBufs {
-  float* KV;
+  float* KV = nullptr;   // literal pooling: K/V of the 4 layers
+  bf16* U2 = nullptr;    // folded pooling: split u of one layer [T][32][D]
+  float* cb = nullptr;   //   c [T][16]
+  float* S = nullptr;    //   split scores [T*1024][32]
+  bf16* P2 = nullptr;    //   split softmax weights [T*128][1024]
+  float* Z = nullptr;    //   split weighted sums [T*128][D]
   float* Q1;
   float* Q;
   float* O;
@@ -112,7 +120,15 @@ struct RouteBufs {
 
 void carve_route(Carver& cv, const ivc_router* r, int T, RouteBufs& b) {
   const long long D = r->D;
-  b.KV = cv.take<float>(static_cast<size_t>(T) * 1024 * 8 * D);
+  if (r->pool_mode == IVC_POOL_LITERAL) {
+    b.KV = cv.take<float>(static_cast<size_t>(T) * 1024 * 8 * D);
+  } else {
+    b.U2 = cv.take<bf16>(static_cast<size_t>(T) * 32 * D);
+    b.cb = cv.take<float>(static_cast<size_t>(T) * 16);
+    b.S = cv.take<float>(static_cast<size_t>(T) * 1024 * 32);
+    b.P2 = cv.take<bf16>(static_cast<size_t>(T) * 128 * 1024);
+    b.Z = cv.take<float>(static_cast<size_t>(T) * 128 * D);
+  }
   b.Q1 = cv.take<float>(D);
   b.Q = cv.take<float>(static_cast<size_t>(T) * D);
   b.O = cv.take<float>(static_cast<size_t>(T) * D);
@@ -190,10 +206,84 @@ int ps_mlp(const void* x, int T, int C, bool half, int flags, const ivc_mlp* m, 
   return IVC_OK;
 }
 
+int gating_and_route(int T, const int32_t* image_offsets, int I, const ivc_router* r, float* gate,
+                     uint8_t* mask, int32_t* offsets, int32_t* total, const RouteBufs& b,
+                     const Launch& L);
+
+// One folded pooling layer (see ivc_router.cu): u/c from the layer's query,
+// scores = X u^T on the tensor cores, masked softmax, z = p X on the tensor
+// cores, o = Wv z + bv. Q is [T, D], or the shared query (ldq = 0, Tq = 1).
+int folded_layer(const void* x, const int32_t* valid_len, int T, const ivc_router* r, int l,
+                 const float* Q, long long ldq, const RouteBufs& b, const Launch& L) {
+  const int D = r->D;
+  const int Tq = ldq == 0 ? 1 : T;
+  IVC_TRY(launch_pool_fold_query(Q, ldq, Tq, static_cast<const bf16*>(r->Wk[l]),
+                                 static_cast<const bf16*>(r->bk[l]), D, b.U2, b.cb, L));
+  GemmCall s{};
+  s.tag = "pool.scores";
+  s.a_mode = A_PLAIN;
+  s.a = x;
+  s.M = T * 1024;
+  s.N = 32;
+  s.K = D;
+  s.groups = 1;
+  s.B[0] = b.U2;
+  s.b_mode = B_K3D;
+  s.b_batches = Tq;
+  s.b_batch_rows = Tq == 1 ? T * 1024 : 1024;
+  s.b_ld = D;
+  s.b_batch_stride = 32LL * D;
+  s.epi_mode = EPI_BIAS;
+  s.out = b.S;
+  s.out_f32 = 1;
+  s.ldo = 32;
+  IVC_TRY(launch_gemm(s, L));
+  IVC_TRY(launch_pool_softmax(b.S, b.cb, Tq == 1 ? 0 : 16, valid_len, T, r->heads, b.P2, L));
+  GemmCall z{};
+  z.tag = "pool.wsum";
+  z.a_mode = A_PLAIN;
+  z.a = b.P2;
+  z.M = T * 128;
+  z.N = D;
+  z.K = 1024;
+  z.groups = 1;
+  z.B[0] = x;
+  z.b_mode = B_MN3D;
+  z.b_batches = T;
+  z.b_batch_rows = 128;
+  z.b_ld = D;
+  z.b_batch_stride = 1024LL * D;
+  z.epi_mode = EPI_BIAS;
+  z.out = b.Z;
+  z.out_f32 = 1;
+  z.m_valid = 32;
+  z.ldo = D;
+  IVC_TRY(launch_gemm(z, L));
+  return launch_pool_vproj(b.Z, T, D, static_cast<const bf16*>(r->Wv[l]),
+                           static_cast<const bf16*>(r->bv[l]), b.O, L);
+}
+
 int route_impl(const void* x, const int32_t* valid_len, int T, const int32_t* image_offsets,
                int I, const ivc_router* r, float* gate, uint8_t* mask, int32_t* offsets,
                int32_t* total, const RouteBufs& b, const Launch& L) {
   const int D = r->D;
+  if (r->pool_mode == IVC_POOL_FOLDED) {
+    IVC_TRY(launch_gemv_bf16x(static_cast<const bf16*>(r->query), D,
+                              static_cast<const bf16*>(r->Wq[0]),
+                              static_cast<const bf16*>(r->bq[0]), D, b.Q1, L));
+    for (int l = 0; l < 4; ++l) {
+      if (l == 0) {
+        IVC_TRY(folded_layer(x, valid_len, T, r, 0, b.Q1, 0, b, L));
+      } else {
+        IVC_TRY(launch_gemv(b.q, D, T, D, static_cast<const bf16*>(r->Wq[l]),
+                            static_cast<const bf16*>(r->bq[l]), D, b.Q, D, 0, L));
+        IVC_TRY(folded_layer(x, valid_len, T, r, l, b.Q, D, b, L));
+      }
+      IVC_TRY(launch_gemv(b.O, D, T, D, static_cast<const bf16*>(r->Wo[l]),
+                          static_cast<const bf16*>(r->bo[l]), D, b.q, D, 0, L));
+    }
+    return gating_and_route(T, image_offsets, I, r, gate, mask, offsets, total, b, L);
+  }
   // K/V projections of the four layers: one grouped GEMM, X [T*1024, D].
   GemmCall c{};
   c.tag = "pool.kv";
@@ -233,7 +323,14 @@ int route_impl(const void* x, const int32_t* valid_len, int T, const int32_t* im
     IVC_TRY(launch_gemv(b.O, D, T, D, static_cast<const bf16*>(r->Wo[l]),
                         static_cast<const bf16*>(r->bo[l]), D, b.q, D, 0, L));
   }
-  // Gating: h = pooled (in b.q), 4 residual blocks, 2-way head.
+  return gating_and_route(T, image_offsets, I, r, gate, mask, offsets, total, b, L);
+}
+
+// Gating on the pooled vectors (in b.q), the 2-way head, then routing.
+int gating_and_route(int T, const int32_t* image_offsets, int I, const ivc_router* r, float* gate,
+                     uint8_t* mask, int32_t* offsets, int32_t* total, const RouteBufs& b,
+                     const Launch& L) {
+  const int D = r->D;
   const int G = r->gate_hidden;
   for (int k = 0; k < 4; ++k) {
     IVC_TRY(launch_gemv(b.q, D, T, D, static_cast<const bf16*>(r->gW1[k]),

@@ -10,6 +10,7 @@
 // shuffled row in one pass over the features.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cstdlib>
 #include <mutex>
 
 #include "ivc_gemm.cuh"
@@ -220,39 +221,58 @@ int num_sms() {
   return n;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int CG>
 static int run_gemm(const GemmMaps& maps, const GemmArgs& args, const char* tag,
                     const Launch& L) {
-  using S = GemmSmem<BN, STAGES>;
+  using S = GemmSmem<BN, STAGES, CG>;
+  auto kern = gemm_sm100_kernel<BN, STAGES, CG>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_sm100_kernel<BN, STAGES>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL);
-    if (e != cudaSuccess) return IVC_ECUDA;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL) !=
+        cudaSuccess)
+      return IVC_ECUDA;
     attr_set = true;
   }
-  const long long tiles = static_cast<long long>((args.M + GEMM_BM - 1) / GEMM_BM) *
+  const long long tiles = static_cast<long long>((args.M + GEMM_BM * CG - 1) / (GEMM_BM * CG)) *
                           ((args.N + BN - 1) / BN) * args.groups;
-  const int grid = static_cast<int>(tiles < num_sms() ? tiles : num_sms());
+  const long long units = num_sms() / CG;
+  const int grid = CG * static_cast<int>(tiles < units ? tiles : units);
   TraceScope ts(tag ? tag : "gemm", L.stream);
-  gemm_sm100_kernel<BN, STAGES><<<grid, GEMM_THREADS, S::TOTAL, L.stream>>>(maps, args, L.status);
-  return cu_check(cudaGetLastError());
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(GEMM_THREADS);
+  cfg.dynamicSmemBytes = S::TOTAL;
+  cfg.stream = L.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = CG == 2 ? 1 : 0;
+  return cu_check(cudaLaunchKernelEx(&cfg, kern, maps, args, L.status));
 }
 
-// Output tile width: the one that finishes the tile set soonest on the SMs
-// (persistent CTAs; narrower tiles pay ~15% more per flop in operand traffic).
+// 256-wide tiles run on CTA pairs unless IVC_GEMM_PAIRS=0 (kept for
+// comparing the two variants on the same build).
+static bool pairs_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* e = std::getenv("IVC_GEMM_PAIRS");
+    on = (e && e[0] == '0') ? 0 : 1;
+  }
+  return on == 1;
+}
+
+// Output tile width. Measured on B200 (tcgen05 M=128, TMA-fed ring with
+// L2-resident operands): N=256 tiles run at ~1.8-2.2 PFLOP/s, N=128 tiles at
+// ~1.08 PFLOP/s, i.e. an N=128 tile takes as long as an N=256 one. So 256 is
+// used whenever N > 128, even when it leaves SMs idle.
 static int pick_bn(const GemmCall& c) {
   if (c.N <= 32) return 32;
   if (c.N <= 64) return 64;
-  const long long mt = (c.M + GEMM_BM - 1) / GEMM_BM;
-  const long long sms = num_sms();
-  auto cost = [&](int bn, double eff) {
-    const long long tiles = mt * ((c.N + bn - 1) / bn) * c.groups;
-    return static_cast<double>((tiles + sms - 1) / sms) * bn * eff;
-  };
-  if (c.b_mode == B_MN3D) return cost(128, 1.15) < cost(256, 1.0) ? 128 : 256;
   if (c.N <= 128) return 128;
-  return cost(128, 1.15) < cost(256, 1.0) ? 128 : 256;
+  return 256;
 }
 
 int launch_gemm(const GemmCall& c, const Launch& L) {
@@ -263,6 +283,8 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
     return IVC_EUNSUPPORTED;
   if (c.b_mode == B_MN3D && c.N % 64 != 0) return IVC_EUNSUPPORTED;
   const int bn = pick_bn(c);
+  // CTA pairs (cta_group::2) for 256-wide tiles of plain K-major weights.
+  const int cg = (bn == 256 && c.b_mode == B_K2D && pairs_enabled()) ? 2 : 1;
 
   GemmMaps maps;
   int rc;
@@ -274,7 +296,7 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
   if (rc) return rc;
   for (int g = 0; g < c.groups; ++g) {
     if (c.b_mode == B_K2D)
-      rc = map_2d(&maps.b[g], c.B[g], c.N, c.K, bn);
+      rc = map_2d(&maps.b[g], c.B[g], c.N, c.K, bn / cg);
     else if (c.b_mode == B_K3D)
       rc = map_3d(&maps.b[g], c.B[g], c.b_batches, c.N, c.K, c.b_ld, c.b_batch_stride, GEMM_BK,
                   bn);
@@ -297,6 +319,7 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
   a.remap = c.remap;
   a.out = c.out;
   a.out_f32 = c.out_f32;
+  a.m_valid = c.m_valid;
   a.ldo = c.ldo;
   a.group_col_stride = c.N;
   for (int g = 0; g < c.groups; ++g) a.bias[g] = c.bias[g];
@@ -305,10 +328,11 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
   a.row_mean = c.row_mean;
   a.row_rstd = c.row_rstd;
   switch (bn) {
-    case 256: return run_gemm<256, 4>(maps, a, c.tag, L);
-    case 128: return run_gemm<128, 6>(maps, a, c.tag, L);
-    case 64: return run_gemm<64, 8>(maps, a, c.tag, L);
-    default: return run_gemm<32, 8>(maps, a, c.tag, L);
+    case 256: return cg == 2 ? run_gemm<256, 6, 2>(maps, a, c.tag, L)
+                             : run_gemm<256, 4, 1>(maps, a, c.tag, L);
+    case 128: return run_gemm<128, 6, 1>(maps, a, c.tag, L);
+    case 64: return run_gemm<64, 8, 1>(maps, a, c.tag, L);
+    default: return run_gemm<32, 8, 1>(maps, a, c.tag, L);
   }
 }
 

@@ -14,6 +14,14 @@
 // Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM owner and
 // MMA issuer, warps 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
 //
+// CG = 2 runs the same roles on a CTA pair (a cluster of 2) with
+// tcgen05.mma.cta_group::2: the pair computes 256 x BN tiles, each CTA loads
+// its own 128 rows of A and BN/2 rows of B into its own shared memory (TMA
+// transaction bytes complete on the leader's barrier), the leader issues the
+// MMAs and commits them to both CTAs' barriers, and each CTA drains its own
+// 128 accumulator rows from its TMEM. Per SM this halves the B traffic into
+// shared memory. No load uses cluster multicast.
+//
 // A operand. pixel_shuffle ("Pixel Shuffle 源码逐行解析" of the
 // InternVL3-14B-Instruct connector article; table "三档 Token 规模" of the
 // InternVL3_5-2B-Flash article) is not materialised: the GEMM row of
@@ -66,6 +74,7 @@ struct GemmArgs {
   int gelu;
   int remap;                     // 0: none; 1: transpose 16x16 token grid; 2: 8x8
   int out_f32;                   // 1: store fp32 instead of bf16
+  int m_valid;                   // >0: store only rows with (row % 128) < m_valid
   void* out;
   long long ldo;                 // elements
   int group_col_stride;          // output column offset per group
@@ -76,10 +85,11 @@ struct GemmArgs {
   const float* row_rstd;         // EPI_LNFOLD
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int CG = 1>
 struct GemmSmem {
   static constexpr uint32_t A_BYTES = GEMM_BM * GEMM_BK * 2;
-  static constexpr uint32_t B_BYTES = BN * GEMM_BK * 2;
+  static constexpr uint32_t B_ROWS = BN / CG;  // rows of B this CTA loads
+  static constexpr uint32_t B_BYTES = B_ROWS * GEMM_BK * 2;
   static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
   static constexpr uint32_t RING = STAGES * STAGE;
   static constexpr uint32_t BARS = (2 * STAGES + 4) * 8 + 16;
@@ -105,19 +115,22 @@ __device__ __forceinline__ void epi_bar_sync() {
 struct TileCoord {
   int g, m0, n0;
 };
-__device__ __forceinline__ TileCoord tile_coord(int idx, int m_tiles, int n_tiles, int BN) {
+__device__ __forceinline__ TileCoord tile_coord(int idx, int m_tiles, int n_tiles, int tile_m,
+                                                int BN) {
   const int n = idx % n_tiles;
   const int rest = idx / n_tiles;
   const int m = rest % m_tiles;
-  return {rest / m_tiles, m * GEMM_BM, n * BN};
+  return {rest / m_tiles, m * tile_m, n * BN};
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int CG>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_sm100_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs args,
                       int* __restrict__ status) {
-  using L = GemmSmem<BN, STAGES>;
+  using L = GemmSmem<BN, STAGES, CG>;
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+  static_assert(CG == 1 || (CG == 2 && BN == 256), "CTA pairs use 256-wide tiles");
+  constexpr int TILE_M = GEMM_BM * CG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -132,7 +145,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m_tiles = (args.M + GEMM_BM - 1) / GEMM_BM;
+  const int rank = CG == 2 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int unit = blockIdx.x / CG;     // this CTA (pair) in the persistent grid
+  const int n_units = gridDim.x / CG;
+  const int m_tiles = (args.M + TILE_M - 1) / TILE_M;
   const int n_tiles = (args.N + BN - 1) / BN;
   const int n_total = m_tiles * n_tiles * args.groups;
   const int KT = args.K / GEMM_BK;
@@ -144,15 +160,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], 4);  // one arrival per epilogue warp
+      mbar_init(&tempty_bar[a], 4 * CG);  // one arrival per epilogue warp of the group
     }
     fence_mbar_init();
     tma_prefetch_desc(&maps.a);
     for (int g = 0; g < args.groups; ++g) tma_prefetch_desc(&maps.b[g]);
   }
+  if constexpr (CG == 2) cluster_sync();  // peer barriers initialised before any remote use
   if (warp == 1) {
-    tmem_alloc(tmem_slot, L::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (CG == 2) {
+      tmem_alloc_pair(tmem_slot, L::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, L::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -164,23 +186,30 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     if (lane == 0) {
       // ------------------------------------------------------------ producer
       int it = 0;
-      for (int idx = blockIdx.x; idx < n_total && ok; idx += gridDim.x) {
-        const TileCoord tc = tile_coord(idx, m_tiles, n_tiles, BN);
+      for (int idx = unit; idx < n_total && ok; idx += n_units) {
+        const TileCoord tc = tile_coord(idx, m_tiles, n_tiles, TILE_M, BN);
+        const int my_m0 = tc.m0 + GEMM_BM * rank;
+        const int my_n0 = tc.n0 + static_cast<int>(L::B_ROWS) * rank;
         const int bb = args.b_batch_rows > 0 ? tc.m0 / args.b_batch_rows : 0;
         for (int kk = 0; kk < KT; ++kk, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
           if (!mbar_wait(&empty_bar[s], ph ^ 1)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full_bar[s], L::STAGE);
+          // the leader's barrier counts the bytes of both CTAs of a pair
+          if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], L::STAGE * CG);
           uint8_t* a_dst = ring + s * L::STAGE;
           uint8_t* b_dst = a_dst + L::A_BYTES;
+          int ac[5];
+          int a_rank = 2;
           if (args.a_mode == A_PLAIN) {
-            tma_load_2d(a_dst, &maps.a, &full_bar[s], kk * GEMM_BK, tc.m0);
+            ac[0] = kk * GEMM_BK;
+            ac[1] = my_m0;
           } else {
             const int blk = kk / args.c_blocks;
             const int c0 = (kk - blk * args.c_blocks) * GEMM_BK;
+            a_rank = 5;
             if (args.a_mode == A_PS_HALF) {
-              tma_load_5d(a_dst, &maps.a, &full_bar[s], c0, blk & 1, 0, blk >> 1, tc.m0 >> 4);
+              ac[0] = c0; ac[1] = blk & 1; ac[2] = 0; ac[3] = blk >> 1; ac[4] = my_m0 >> 4;
             } else {
               int q, r;
               if (args.a_mode == A_PS_QUARTER) {
@@ -190,9 +219,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 q = 2 * (blk >> 3) + ((blk >> 1) & 1);
                 r = 2 * ((blk >> 2) & 1) + (blk & 1);
               }
-              tma_load_5d(a_dst, &maps.a, &full_bar[s], c0, r, 0, q, tc.m0 >> 3);
+              ac[0] = c0; ac[1] = r; ac[2] = 0; ac[3] = q; ac[4] = my_m0 >> 3;
             }
           }
+          if constexpr (CG == 2) {
+            const uint32_t lb = pair_leader_addr(&full_bar[s]);
+            if (a_rank == 2)
+              tma_load_2d_pair(a_dst, &maps.a, lb, ac[0], ac[1]);
+            else
+              tma_load_5d_pair(a_dst, &maps.a, lb, ac[0], ac[1], ac[2], ac[3], ac[4]);
+            tma_load_2d_pair(b_dst, &maps.b[tc.g], lb, kk * GEMM_BK, my_n0);
+            continue;
+          }
+          if (a_rank == 2)
+            tma_load_2d(a_dst, &maps.a, &full_bar[s], ac[0], ac[1]);
+          else
+            tma_load_5d(a_dst, &maps.a, &full_bar[s], ac[0], ac[1], ac[2], ac[3], ac[4]);
           const CUtensorMap* bm = &maps.b[tc.g];
           if (args.b_mode == B_K2D) {
             tma_load_2d(b_dst, bm, &full_bar[s], kk * GEMM_BK, tc.n0);
@@ -208,12 +250,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       // ------------------------------------------------------------ MMA issuer
-      const uint32_t idesc = idesc_bf16_f32(GEMM_BM, BN) |
+      const uint32_t idesc = idesc_bf16_f32(TILE_M, BN) |
                              (args.b_mode == B_MN3D ? (1u << 16) : 0u);  // B MN-major
       int it = 0, local = 0;
-      for (int idx = blockIdx.x; idx < n_total && ok; idx += gridDim.x, ++local) {
+      for (int idx = unit; idx < n_total && ok; idx += n_units, ++local) {
         const int acc = local & 1;
         const uint32_t use = static_cast<uint32_t>(local >> 1);
         if (!mbar_wait(&tempty_bar[acc], (use & 1) ^ 1)) { ok = false; break; }
@@ -234,12 +276,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           for (int k = 0; k < GEMM_BK / 16; ++k) {
             // K-major: advance 16 bf16 = 32 bytes inside the swizzle atom;
             // MN-major: advance 16 k-rows of 128 bytes.
-            umma_bf16(d_tmem, ad + 2 * k, bd + bstep * k, idesc, (kk | k) != 0 ? 1u : 0u);
+            if constexpr (CG == 2)
+              umma_bf16_pair(d_tmem, ad + 2 * k, bd + bstep * k, idesc, (kk | k) != 0 ? 1u : 0u);
+            else
+              umma_bf16(d_tmem, ad + 2 * k, bd + bstep * k, idesc, (kk | k) != 0 ? 1u : 0u);
           }
-          umma_commit(&empty_bar[s]);
+          if constexpr (CG == 2)
+            umma_commit_pair(&empty_bar[s]);
+          else
+            umma_commit(&empty_bar[s]);
         }
         if (!ok) break;
-        umma_commit(&tfull_bar[acc]);
+        if constexpr (CG == 2)
+          umma_commit_pair(&tfull_bar[acc]);
+        else
+          umma_commit(&tfull_bar[acc]);
       }
     }
   } else {
@@ -247,8 +298,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const int quad = warp & 3;
     const int et = threadIdx.x - 64;  // 0..127
     int local = 0;
-    for (int idx = blockIdx.x; idx < n_total; idx += gridDim.x, ++local) {
-      const TileCoord tc = tile_coord(idx, m_tiles, n_tiles, BN);
+    for (int idx = unit; idx < n_total; idx += n_units, ++local) {
+      const TileCoord tc = tile_coord(idx, m_tiles, n_tiles, TILE_M, BN);
       const int acc = local & 1;
       const uint32_t use = static_cast<uint32_t>(local >> 1);
       // per-column epilogue vectors of this tile
@@ -273,7 +324,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], use & 1));
       if (!ok) continue;
       tc_fence_after();
-      const int row = tc.m0 + quad * 32 + lane;
+      const int row = tc.m0 + GEMM_BM * rank + quad * 32 + lane;
       float mean = 0.f, rstd = 1.f;
       if (args.epi_mode == EPI_LNFOLD && row < args.M) {
         mean = args.row_mean[row];
@@ -301,9 +352,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           // accumulator fully read: hand it back to the MMA warp
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+          if (lane == 0) {
+            if constexpr (CG == 2)
+              mbar_arrive_cluster(pair_leader_addr(&tempty_bar[acc]));
+            else
+              mbar_arrive(&tempty_bar[acc]);
+          }
         }
-        if (row < args.M && tc.n0 + c < args.N) {
+        if (row < args.M && tc.n0 + c < args.N && (args.m_valid == 0 || (row & 127) < args.m_valid)) {
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
@@ -337,9 +393,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   if (!ok && status != nullptr) atomicOr(status, 4 /* IVC_DEV_WAIT_TIMEOUT */);
   tc_fence_before();
   __syncthreads();
+  // a pair stays resident until neither CTA touches the other's barriers
+  if constexpr (CG == 2) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, L::TMEM_COLS);
+    if constexpr (CG == 2)
+      tmem_dealloc_pair(tmem_base, L::TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, L::TMEM_COLS);
   }
 }
 

@@ -75,6 +75,7 @@ struct GemmCall {
   const float* row_rstd;
   void* out;
   int out_f32;         // store fp32 (pooling K/V) instead of bf16
+  int m_valid;         // >0: store only rows with (row % 128) < m_valid
   long long ldo;
 };
 int launch_gemm(const GemmCall& c, const Launch& L);
@@ -90,6 +91,15 @@ int launch_gemv_bf16x(const bf16* x, int K, const bf16* W, const bf16* b, int N,
 int launch_pool_attention(const float* Q, long long ldq, const float* KV, long long ldkv,
                           int koff, int voff, const int32_t* valid_len, int T, int D, int heads,
                           float* O, const Launch& L);
+// Folded pooling (up to 16 heads of 64): u/c of one layer from Q [Tq, D] (Tq = 1:
+// the same query for every tile), scores' softmax into the split P2 operand,
+// and o = Wv z + bv from the split weighted sums Z [T*128, D].
+int launch_pool_fold_query(const float* Q, long long ldq, int Tq, const bf16* Wk, const bf16* bk,
+                           int D, bf16* U2, float* cb, const Launch& L);
+int launch_pool_softmax(const float* S, const float* cb, int cb_stride, const int32_t* valid_len,
+                        int T, int heads, bf16* P2, const Launch& L);
+int launch_pool_vproj(const float* Z, int T, int D, const bf16* Wv, const bf16* bv, float* O,
+                      const Launch& L);
 // h[t] += LN(u[t]) * gamma + beta over D.
 int launch_residual_ln(float* h, const float* u, const bf16* gamma, const bf16* beta, int T,
                        int D, const Launch& L);

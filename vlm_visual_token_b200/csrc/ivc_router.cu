@@ -47,7 +47,9 @@ __device__ __forceinline__ float4 load4<bf16>(const bf16* p) {
                      __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
 }
 
-template <typename XT, int J>
+// PAIRED: the input row m of output column n is Z[m*128 + h] + Z[m*128 + 16 + h]
+// with h = n / 64 (the folded pooling's split weighted sums, ldx = row length).
+template <typename XT, int J, bool PAIRED = false>
 __global__ void __launch_bounds__(GEMV_WARPS * 32)
     gemv_kernel(const XT* __restrict__ X, long long ldx, int M,
                 const bf16* __restrict__ W, const bf16* __restrict__ b, int N,
@@ -68,7 +70,15 @@ __global__ void __launch_bounds__(GEMV_WARPS * 32)
     __syncthreads();
     for (int i = threadIdx.x; i < rows * (K / 4); i += blockDim.x) {
       const int r = i / (K / 4), c = (i - r * (K / 4)) * 4;
-      *reinterpret_cast<float4*>(sx + r * K + c) = load4<XT>(X + (m0 + r) * ldx + c);
+      if constexpr (PAIRED) {
+        const int h = (blockIdx.x * GEMV_WARPS) / 64;
+        const XT* zr = X + (static_cast<long long>(m0 + r) * 128 + h) * ldx + c;
+        const float4 a = load4<XT>(zr), bb = load4<XT>(zr + 16 * ldx);
+        *reinterpret_cast<float4*>(sx + r * K + c) =
+            make_float4(a.x + bb.x, a.y + bb.y, a.z + bb.z, a.w + bb.w);
+      } else {
+        *reinterpret_cast<float4*>(sx + r * K + c) = load4<XT>(X + (m0 + r) * ldx + c);
+      }
     }
     __syncthreads();
     if (n >= N) continue;
@@ -93,34 +103,40 @@ __global__ void __launch_bounds__(GEMV_WARPS * 32)
   }
 }
 
-template <typename XT, int J>
+template <typename XT, int J, bool PAIRED = false>
 static int run_gemv(const XT* X, long long ldx, int M, const bf16* W, const bf16* b, int N,
                     float* Y, long long ldy, int gelu, const Launch& L) {
   const int smem = GEMV_ROWS * J * 128 * static_cast<int>(sizeof(float));
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(gemv_kernel<XT, J>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(gemv_kernel<XT, J, PAIRED>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return IVC_ECUDA;
     attr = true;
   }
-  TraceScope ts(gelu ? "router.gemv_gelu" : "router.gemv", L.stream);
-  gemv_kernel<XT, J><<<(N + GEMV_WARPS - 1) / GEMV_WARPS, GEMV_WARPS * 32, smem, L.stream>>>(
-      X, ldx, M, W, b, N, Y, ldy, gelu);
+  TraceScope ts(PAIRED ? "pool.vproj" : (gelu ? "router.gemv_gelu" : "router.gemv"), L.stream);
+  gemv_kernel<XT, J, PAIRED>
+      <<<(N + GEMV_WARPS - 1) / GEMV_WARPS, GEMV_WARPS * 32, smem, L.stream>>>(X, ldx, M, W, b, N,
+                                                                               Y, ldy, gelu);
   return cu_check(cudaGetLastError());
 }
 
-template <typename XT>
+template <typename XT, bool PAIRED = false>
 static int dispatch_gemv(const XT* X, long long ldx, int M, int K, const bf16* W, const bf16* b,
                          int N, float* Y, long long ldy, int gelu, const Launch& L) {
   if (M == 0 || N == 0) return IVC_OK;
   switch (K) {
-    case 256: return run_gemv<XT, 2>(X, ldx, M, W, b, N, Y, ldy, gelu, L);
-    case 512: return run_gemv<XT, 4>(X, ldx, M, W, b, N, Y, ldy, gelu, L);
-    case 1024: return run_gemv<XT, 8>(X, ldx, M, W, b, N, Y, ldy, gelu, L);
-    case 2048: return run_gemv<XT, 16>(X, ldx, M, W, b, N, Y, ldy, gelu, L);
+    case 256: return run_gemv<XT, 2, PAIRED>(X, ldx, M, W, b, N, Y, ldy, gelu, L);
+    case 512: return run_gemv<XT, 4, PAIRED>(X, ldx, M, W, b, N, Y, ldy, gelu, L);
+    case 1024: return run_gemv<XT, 8, PAIRED>(X, ldx, M, W, b, N, Y, ldy, gelu, L);
+    case 2048: return run_gemv<XT, 16, PAIRED>(X, ldx, M, W, b, N, Y, ldy, gelu, L);
     default: return IVC_EUNSUPPORTED;
   }
+}
+
+int launch_pool_vproj(const float* Z, int T, int D, const bf16* Wv, const bf16* bv, float* O,
+                      const Launch& L) {
+  return dispatch_gemv<float, true>(Z, D, T, D, Wv, bv, D, O, D, 0, L);
 }
 
 int launch_gemv(const float* X, long long ldx, int M, int K, const bf16* W, const bf16* b, int N,
@@ -228,6 +244,141 @@ int launch_pool_attention(const float* Q, long long ldq, const float* KV, long l
   pool_attention_kernel<<<dim3(heads, T), ATT_THREADS, 0, L.stream>>>(Q, ldq, KV, ldkv, koff,
                                                                      voff, valid_len, O, D,
                                                                      L.status);
+  return cu_check(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------- folded pooling
+// The single query of each pooling layer lets the K and V projections be
+// reassociated (exactly, in real arithmetic):
+//   score_t = Q_h . (Wk_h x_t + bk_h) / 8 = x_t . u_h + c_h,
+//       u_h = Wk_h^T Q_h / 8,  c_h = bk_h . Q_h / 8;
+//   o_h = sum_t p_t (Wv_h x_t + bv_h) = Wv_h z_h + bv_h,  z_h = sum_t p_t x_t,
+// since the softmax weights of the valid tokens sum to 1. The two
+// contractions with the raw features x (scores: x u^T, sums: p x) run on the
+// tensor cores; their fp32 right-hand sides u and p are fed as bf16 pairs
+// hi + lo (hi = bf16(v), lo = bf16(v - hi)), keeping ~16 significant bits.
+
+// u/c of one layer. Grid (D/128, heads <= 16); thread = feature column c.
+// U2[t][j][c]: j < 16 hi part of u_j, j >= 16 lo part of u_{j-16}; rows of
+// heads that do not exist are left as they are (their score columns and
+// weighted-sum rows are never read).
+__global__ void __launch_bounds__(128) pool_fold_query_kernel(
+    const float* __restrict__ Q, long long ldq, int Tq, const bf16* __restrict__ Wk,
+    const bf16* __restrict__ bk, int D, bf16* __restrict__ U2, float* __restrict__ cb) {
+  __shared__ float s_q[64][HEAD_DIM];  // 64 tiles x head slice of Q
+  const int h = blockIdx.y;
+  const int c = blockIdx.x * 128 + threadIdx.x;
+  float w[HEAD_DIM];
+#pragma unroll
+  for (int d = 0; d < HEAD_DIM; ++d)
+    w[d] = __bfloat162float(Wk[static_cast<long long>(h * HEAD_DIM + d) * D + c]);
+  for (int t0 = 0; t0 < Tq; t0 += 64) {
+    const int nt = min(64, Tq - t0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < nt * HEAD_DIM; i += 128)
+      s_q[i / HEAD_DIM][i % HEAD_DIM] =
+          Q[(t0 + i / HEAD_DIM) * ldq + h * HEAD_DIM + i % HEAD_DIM] * 0.125f;
+    __syncthreads();
+    for (int t = 0; t < nt; ++t) {
+      float u = 0.f;
+#pragma unroll
+      for (int d = 0; d < HEAD_DIM; ++d) u = fmaf(w[d], s_q[t][d], u);
+      const bf16 hi = __float2bfloat16_rn(u);
+      const bf16 lo = __float2bfloat16_rn(u - __bfloat162float(hi));
+      bf16* base = U2 + static_cast<long long>(t0 + t) * 32 * D;
+      base[static_cast<long long>(h) * D + c] = hi;
+      base[static_cast<long long>(16 + h) * D + c] = lo;
+    }
+    if (blockIdx.x == 0 && threadIdx.x < nt) {
+      float acc = 0.f;
+      for (int d = 0; d < HEAD_DIM; ++d)
+        acc = fmaf(bk ? __bfloat162float(bk[h * HEAD_DIM + d]) : 0.f, s_q[threadIdx.x][d], acc);
+      cb[(t0 + threadIdx.x) * 16 + h] = acc;
+    }
+  }
+}
+
+int launch_pool_fold_query(const float* Q, long long ldq, int Tq, const bf16* Wk, const bf16* bk,
+                           int D, bf16* U2, float* cb, const Launch& L) {
+  if (Tq == 0) return IVC_OK;
+  const int heads = D / HEAD_DIM;
+  if (D % 128 != 0 || heads > 16) return IVC_EUNSUPPORTED;
+  TraceScope ts("pool.fold_query", L.stream);
+  pool_fold_query_kernel<<<dim3(D / 128, heads), 128, 0, L.stream>>>(Q, ldq, Tq, Wk, bk, D, U2,
+                                                                     cb);
+  return cu_check(cudaGetLastError());
+}
+
+// Masked softmax of one (head, tile) from the split scores; writes the
+// weights as a bf16 hi/lo pair into rows h and 16+h of the tile's 128-row
+// block of P2 (rows 32..127 zero), the A operand of the weighted-sum GEMM.
+__global__ void __launch_bounds__(ATT_THREADS)
+    pool_softmax_kernel(const float* __restrict__ S, const float* __restrict__ cb, int cb_stride,
+                        const int32_t* __restrict__ valid_len, bf16* __restrict__ P2,
+                        int* __restrict__ status) {
+  __shared__ float s_p[TILE_TOKENS];
+  __shared__ float s_scalar[ATT_THREADS / 32];
+  const int h = blockIdx.x, tile = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int n = TILE_TOKENS;
+  if (valid_len != nullptr) {
+    n = valid_len[tile];
+    if (n < 1 || n > TILE_TOKENS) {
+      if (threadIdx.x == 0) atomicOr(status, DEV_BAD_VALID_LEN);
+      n = n < 1 ? 1 : TILE_TOKENS;
+    }
+  }
+  const float c = cb[tile * cb_stride + h];
+  const float* srow = S + static_cast<long long>(tile) * TILE_TOKENS * 32;
+  float mx = -INFINITY;
+  for (int t = threadIdx.x; t < n; t += ATT_THREADS) {
+    const float v = srow[t * 32 + h] + srow[t * 32 + 16 + h] + c;
+    s_p[t] = v;
+    mx = fmaxf(mx, v);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) s_scalar[warp] = mx;
+  __syncthreads();
+  mx = s_scalar[0];
+#pragma unroll
+  for (int i = 1; i < ATT_THREADS / 32; ++i) mx = fmaxf(mx, s_scalar[i]);
+  __syncthreads();
+  float sum = 0.f;
+  for (int t = threadIdx.x; t < n; t += ATT_THREADS) {
+    const float e = expf(s_p[t] - mx);
+    s_p[t] = e;
+    sum += e;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) s_scalar[warp] = sum;
+  __syncthreads();
+  sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < ATT_THREADS / 32; ++i) sum += s_scalar[i];
+  const float inv = 1.0f / sum;
+  bf16* blk = P2 + static_cast<long long>(tile) * 128 * TILE_TOKENS;
+  for (int t = threadIdx.x; t < TILE_TOKENS; t += ATT_THREADS) {
+    const float p = t < n ? s_p[t] * inv : 0.f;
+    const bf16 hi = __float2bfloat16_rn(p);
+    blk[h * TILE_TOKENS + t] = hi;
+    blk[(16 + h) * TILE_TOKENS + t] = __float2bfloat16_rn(p - __bfloat162float(hi));
+  }
+  // rows 32..127 of the block stay zero, shared out over the heads' CTAs
+  const bf16 z = __float2bfloat16_rn(0.f);
+  const int per = (96 + gridDim.x - 1) / gridDim.x;
+  for (int r = 32 + per * h; r < min(128, 32 + per * (h + 1)); ++r)
+    for (int t = threadIdx.x; t < TILE_TOKENS; t += ATT_THREADS) blk[r * TILE_TOKENS + t] = z;
+}
+
+int launch_pool_softmax(const float* S, const float* cb, int cb_stride, const int32_t* valid_len,
+                        int T, int heads, bf16* P2, const Launch& L) {
+  if (T == 0) return IVC_OK;
+  if (heads < 1 || heads > 16) return IVC_EUNSUPPORTED;
+  TraceScope ts("pool.softmax", L.stream);
+  pool_softmax_kernel<<<dim3(heads, T), ATT_THREADS, 0, L.stream>>>(S, cb, cb_stride, valid_len,
+                                                                   P2, L.status);
   return cu_check(cudaGetLastError());
 }
 
