@@ -203,7 +203,10 @@ int ivc_vir_route(const void* x, const int32_t* valid_len, int T, int C,
  * if mask[t] else its 256 mlp1 rows, tiles in order.
  *   out    device bf16 [T * 256, H] capacity (H = output width of both MLPs).
  *   total  device int32 [1]: rows written (= offsets[T]).
- * gate, mask, offsets as in ivc_vir_route. */
+ * gate, mask, offsets as in ivc_vir_route.
+ * The router part runs on a library-owned high-priority stream of the current
+ * device (created on the first call, with two events), forked from and joined
+ * back into `stream`: to the caller the call is ordered on `stream` alone. */
 int ivc_flash_compress(const void* x, const int32_t* valid_len, int T, int C,
                        const int32_t* image_offsets, int I, const ivc_mlp* mlp1,
                        const ivc_mlp* mlp2, const ivc_router* r, void* out, float* gate,

@@ -6,6 +6,7 @@
 // allocates device memory.
 #include <cuda_runtime.h>
 #include <cstring>
+#include <mutex>
 
 #include "ivc_gemm.cuh"
 #include "ivc_internal.h"
@@ -346,6 +347,35 @@ int gating_and_route(int T, const int32_t* image_offsets, int I, const ivc_route
                       offsets, total, L);
 }
 
+// Side stream (highest priority) and fork/join events used by
+// ivc_flash_compress to run the router next to the connector, created once
+// per device. The router's kernels are small and latency-bound; at high
+// priority they take SMs as soon as connector GEMM CTAs retire.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+int side_stream(SideStream** out) {
+  static std::mutex mu;
+  static SideStream per_dev[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return IVC_ECUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  SideStream& s = per_dev[dev];
+  if (!s.stream) {
+    int lo = 0, hi = 0;
+    if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) return IVC_ECUDA;
+    if (cudaStreamCreateWithPriority(&s.stream, cudaStreamNonBlocking, hi) != cudaSuccess)
+      return IVC_ECUDA;
+    if (cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming) != cudaSuccess)
+      return IVC_ECUDA;
+  }
+  *out = &s;
+  return IVC_OK;
+}
+
 int check_ws(void* ws, size_t ws_bytes, size_t need) {
   if (!ws) return IVC_EINVAL;
   if (reinterpret_cast<uintptr_t>(ws) % kAlign) return IVC_EALIGN;
@@ -524,11 +554,25 @@ int ivc_flash_compress(const void* x, const int32_t* valid_len, int T, int C,
   bf16* Y256 = cv.take<bf16>(static_cast<size_t>(T) * 256 * H);
   bf16* Y64 = cv.take<bf16>(static_cast<size_t>(T) * 64 * H);
   carve_route(cv, r, T, br);
-  IVC_TRY(launch_ps_stats(static_cast<const bf16*>(x), T, C, b1.mean, b1.rstd, b2.mean, b2.rstd,
-                          L));
-  IVC_TRY(ps_mlp(x, T, C, true, 0, mlp1, Y256, b1, L));
-  IVC_TRY(ps_mlp(x, T, C, false, 0, mlp2, Y64, b2, L));
-  IVC_TRY(route_impl(x, valid_len, T, image_offsets, I, r, gate, mask, offsets, total, br, L));
+  // The router (own buffers) runs on the side stream while the connector runs
+  // on the caller's stream; they meet before compaction.
+  SideStream* side = nullptr;
+  IVC_TRY(side_stream(&side));
+  Launch R{side->stream, L.status};
+  IVC_TRY(cu_check(cudaEventRecord(side->fork, s)));
+  IVC_TRY(cu_check(cudaStreamWaitEvent(side->stream, side->fork, 0)));
+  int rc = route_impl(x, valid_len, T, image_offsets, I, r, gate, mask, offsets, total, br, R);
+  // join even on failure so that the caller's stream never runs ahead of work
+  // already enqueued on the side stream
+  const int rc_rec = cu_check(cudaEventRecord(side->join, side->stream));
+  if (rc == IVC_OK) rc = rc_rec;
+  if (rc == IVC_OK)
+    rc = launch_ps_stats(static_cast<const bf16*>(x), T, C, b1.mean, b1.rstd, b2.mean, b2.rstd, L);
+  if (rc == IVC_OK) rc = ps_mlp(x, T, C, true, 0, mlp1, Y256, b1, L);
+  if (rc == IVC_OK) rc = ps_mlp(x, T, C, false, 0, mlp2, Y64, b2, L);
+  const int rc_wait = rc_rec == IVC_OK ? cu_check(cudaStreamWaitEvent(s, side->join, 0)) : rc_rec;
+  if (rc != IVC_OK) return rc;
+  if (rc_wait != IVC_OK) return rc_wait;
   return launch_compact(Y256, Y64, mask, offsets, T, H, static_cast<bf16*>(out), L);
 }
 

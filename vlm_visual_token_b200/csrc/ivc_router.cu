@@ -28,11 +28,20 @@ __device__ __forceinline__ float gelu_f(float y) {
 }
 
 // ---------------------------------------------------------------- skinny GEMV
-// One warp per output column n, all rows m. Lane l owns k = 128 j + 4 l .. +3
-// of the weight row (kept in registers); input rows are staged 8 at a time in
-// shared memory as fp32.
-constexpr int GEMV_WARPS = 8;
-constexpr int GEMV_ROWS = 8;
+// Y[m, n] = act(sum_k X[m, k] W[n, k] + b[n]) for few rows m (router vectors).
+// A CTA of GEMV_WARPS warps owns GEMV_WARPS*GEMV_COLS consecutive columns;
+// warp w keeps its GEMV_COLS weight rows in registers (packed bf16, lane l
+// holds k = 128 j + 4 l .. +3) and reads each staged input row once for all
+// of them. Input rows are staged in shared memory as fp32, GEMV_ROWS(J) at a
+// time, with every load of a thread issued before its stores.
+constexpr int GEMV_WARPS = 4;
+constexpr int GEMV_COLS = 4;
+constexpr int GEMV_CTA_COLS = GEMV_WARPS * GEMV_COLS;  // 16: one head of 64 spans 4 CTAs
+
+template <int J>
+struct GemvRows {
+  static constexpr int value = J <= 8 ? 16 : 8;  // staged rows: 64 KB of fp32 at most
+};
 
 template <typename XT>
 __device__ __forceinline__ float4 load4(const XT* p);
@@ -47,57 +56,87 @@ __device__ __forceinline__ float4 load4<bf16>(const bf16* p) {
                      __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
 }
 
-// PAIRED: the input row m of output column n is Z[m*128 + h] + Z[m*128 + 16 + h]
-// with h = n / 64 (the folded pooling's split weighted sums, ldx = row length).
+__device__ __forceinline__ float dot4(uint2 w, float4 x, float acc) {
+  acc = fmaf(__uint_as_float(w.x << 16), x.x, acc);
+  acc = fmaf(__uint_as_float(w.x & 0xffff0000u), x.y, acc);
+  acc = fmaf(__uint_as_float(w.y << 16), x.z, acc);
+  return fmaf(__uint_as_float(w.y & 0xffff0000u), x.w, acc);
+}
+
+// PAIRED: the input row m of the CTA's columns is Z[m*128 + h] + Z[m*128 + 16 + h]
+// with h = (first column) / 64 (the folded pooling's split weighted sums; ldx
+// is then the row length of Z).
 template <typename XT, int J, bool PAIRED = false>
 __global__ void __launch_bounds__(GEMV_WARPS * 32)
     gemv_kernel(const XT* __restrict__ X, long long ldx, int M,
                 const bf16* __restrict__ W, const bf16* __restrict__ b, int N,
                 float* __restrict__ Y, long long ldy, int gelu) {
-  extern __shared__ float sx[];  // [GEMV_ROWS][K]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int K = J * 128;
-  const int n = blockIdx.x * GEMV_WARPS + warp;
-  float4 w[J];
-  if (n < N) {
-    const bf16* wr = W + static_cast<long long>(n) * K;
+  constexpr int ROWS = GemvRows<J>::value;
+  constexpr int F4_ROW = K / 4;
+  constexpr int PER_THREAD = ROWS * F4_ROW / (GEMV_WARPS * 32);
+  extern __shared__ float sx[];  // [ROWS][K]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * GEMV_CTA_COLS + warp * GEMV_COLS;
+  uint2 w[GEMV_COLS][J];
+  float bias[GEMV_COLS];
 #pragma unroll
-    for (int j = 0; j < J; ++j) w[j] = load4<bf16>(wr + j * 128 + lane * 4);
+  for (int c = 0; c < GEMV_COLS; ++c) {
+    const int n = n0 + c;
+    const bf16* wr = W + static_cast<long long>(n < N ? n : 0) * K;
+#pragma unroll
+    for (int j = 0; j < J; ++j) w[c][j] = *reinterpret_cast<const uint2*>(wr + j * 128 + lane * 4);
+    bias[c] = (n < N && b != nullptr) ? __bfloat162float(b[n]) : 0.f;
   }
-  const float bias = (n < N && b != nullptr) ? __bfloat162float(b[n]) : 0.f;
-  for (int m0 = 0; m0 < M; m0 += GEMV_ROWS) {
-    const int rows = min(GEMV_ROWS, M - m0);
+  const int h = PAIRED ? (blockIdx.x * GEMV_CTA_COLS) / 64 : 0;
+  for (int m0 = 0; m0 < M; m0 += ROWS) {
+    const int rows = min(ROWS, M - m0);
     __syncthreads();
-    for (int i = threadIdx.x; i < rows * (K / 4); i += blockDim.x) {
-      const int r = i / (K / 4), c = (i - r * (K / 4)) * 4;
-      if constexpr (PAIRED) {
-        const int h = (blockIdx.x * GEMV_WARPS) / 64;
-        const XT* zr = X + (static_cast<long long>(m0 + r) * 128 + h) * ldx + c;
-        const float4 a = load4<XT>(zr), bb = load4<XT>(zr + 16 * ldx);
-        *reinterpret_cast<float4*>(sx + r * K + c) =
-            make_float4(a.x + bb.x, a.y + bb.y, a.z + bb.z, a.w + bb.w);
-      } else {
-        *reinterpret_cast<float4*>(sx + r * K + c) = load4<XT>(X + (m0 + r) * ldx + c);
+    constexpr int BATCH = PER_THREAD < 8 ? PER_THREAD : 8;  // loads in flight per thread
+#pragma unroll 1
+    for (int u0 = 0; u0 < PER_THREAD; u0 += BATCH) {
+      float4 v[BATCH];
+#pragma unroll
+      for (int u = 0; u < BATCH; ++u) {
+        const int i = threadIdx.x + (u0 + u) * GEMV_WARPS * 32;
+        const int r = i / F4_ROW, c = (i - r * F4_ROW) * 4;
+        if (r < rows) {
+          if constexpr (PAIRED) {
+            const XT* zr = X + (static_cast<long long>(m0 + r) * 128 + h) * ldx + c;
+            const float4 a = load4<XT>(zr), bb = load4<XT>(zr + 16 * ldx);
+            v[u] = make_float4(a.x + bb.x, a.y + bb.y, a.z + bb.z, a.w + bb.w);
+          } else {
+            v[u] = load4<XT>(X + static_cast<long long>(m0 + r) * ldx + c);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < BATCH; ++u) {
+        const int i = threadIdx.x + (u0 + u) * GEMV_WARPS * 32;
+        if (i / F4_ROW < rows) *reinterpret_cast<float4*>(sx + i * 4) = v[u];
       }
     }
     __syncthreads();
-    if (n >= N) continue;
     for (int r = 0; r < rows; ++r) {
-      float acc = 0.f;
+      float acc[GEMV_COLS] = {};
 #pragma unroll
       for (int j = 0; j < J; ++j) {
         const float4 xv = *reinterpret_cast<const float4*>(sx + r * K + j * 128 + lane * 4);
-        acc = fmaf(w[j].x, xv.x, acc);
-        acc = fmaf(w[j].y, xv.y, acc);
-        acc = fmaf(w[j].z, xv.z, acc);
-        acc = fmaf(w[j].w, xv.w, acc);
+#pragma unroll
+        for (int c = 0; c < GEMV_COLS; ++c) acc[c] = dot4(w[c][j], xv, acc[c]);
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) {
-        float y = acc + bias;
+      for (int c = 0; c < GEMV_COLS; ++c) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], o);
+      }
+      if (lane < GEMV_COLS) {
+        float y = 0.f;
+#pragma unroll
+        for (int c = 0; c < GEMV_COLS; ++c)
+          if (c == lane) y = acc[c] + bias[c];
         if (gelu) y = gelu_f(y);
-        Y[(m0 + r) * ldy + n] = y;
+        if (n0 + lane < N) Y[static_cast<long long>(m0 + r) * ldy + n0 + lane] = y;
       }
     }
   }
@@ -106,7 +145,7 @@ __global__ void __launch_bounds__(GEMV_WARPS * 32)
 template <typename XT, int J, bool PAIRED = false>
 static int run_gemv(const XT* X, long long ldx, int M, const bf16* W, const bf16* b, int N,
                     float* Y, long long ldy, int gelu, const Launch& L) {
-  const int smem = GEMV_ROWS * J * 128 * static_cast<int>(sizeof(float));
+  const int smem = GemvRows<J>::value * J * 128 * static_cast<int>(sizeof(float));
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(gemv_kernel<XT, J, PAIRED>,
@@ -116,8 +155,8 @@ static int run_gemv(const XT* X, long long ldx, int M, const bf16* W, const bf16
   }
   TraceScope ts(PAIRED ? "pool.vproj" : (gelu ? "router.gemv_gelu" : "router.gemv"), L.stream);
   gemv_kernel<XT, J, PAIRED>
-      <<<(N + GEMV_WARPS - 1) / GEMV_WARPS, GEMV_WARPS * 32, smem, L.stream>>>(X, ldx, M, W, b, N,
-                                                                               Y, ldy, gelu);
+      <<<(N + GEMV_CTA_COLS - 1) / GEMV_CTA_COLS, GEMV_WARPS * 32, smem, L.stream>>>(
+          X, ldx, M, W, b, N, Y, ldy, gelu);
   return cu_check(cudaGetLastError());
 }
 
@@ -134,11 +173,6 @@ static int dispatch_gemv(const XT* X, long long ldx, int M, int K, const bf16* W
   }
 }
 
-int launch_pool_vproj(const float* Z, int T, int D, const bf16* Wv, const bf16* bv, float* O,
-                      const Launch& L) {
-  return dispatch_gemv<float, true>(Z, D, T, D, Wv, bv, D, O, D, 0, L);
-}
-
 int launch_gemv(const float* X, long long ldx, int M, int K, const bf16* W, const bf16* b, int N,
                 float* Y, long long ldy, int gelu, const Launch& L) {
   return dispatch_gemv<float>(X, ldx, M, K, W, b, N, Y, ldy, gelu, L);
@@ -147,6 +181,11 @@ int launch_gemv(const float* X, long long ldx, int M, int K, const bf16* W, cons
 int launch_gemv_bf16x(const bf16* x, int K, const bf16* W, const bf16* b, int N, float* Y,
                       const Launch& L) {
   return dispatch_gemv<bf16>(x, 0, 1, K, W, b, N, Y, 0, 0, L);
+}
+
+int launch_pool_vproj(const float* Z, int T, int D, const bf16* Wv, const bf16* bv, float* O,
+                      const Launch& L) {
+  return dispatch_gemv<float, true>(Z, D, T, D, Wv, bv, D, O, D, 0, L);
 }
 
 // ---------------------------------------------------------------- pooling attention
