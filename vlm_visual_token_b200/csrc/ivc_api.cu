@@ -68,13 +68,14 @@ int router_shape_ok(const ivc_router* r, int C) {
   if (r->pool_mode == IVC_POOL_FOLDED && (r->heads > 16 || r->D % 128 != 0))
     return IVC_EUNSUPPORTED;
   if (!r->query || !r->gWout) return IVC_EINVAL;
+  if (!aligned16(r->query)) return IVC_EALIGN;
   for (int l = 0; l < 4; ++l) {
-    const void* ws[4] = {r->Wq[l], r->Wk[l], r->Wv[l], r->Wo[l]};
+    const void* ws[6] = {r->Wq[l], r->Wk[l], r->Wv[l], r->Wo[l], r->gW1[l], r->gW2[l]};
     for (const void* w : ws) {
       if (!w) return IVC_EINVAL;
       if (!aligned16(w)) return IVC_EALIGN;
     }
-    if (!r->gW1[l] || !r->gW2[l] || !r->gln_g[l] || !r->gln_b[l]) return IVC_EINVAL;
+    if (!r->gln_g[l] || !r->gln_b[l]) return IVC_EINVAL;
   }
   return IVC_OK;
 }

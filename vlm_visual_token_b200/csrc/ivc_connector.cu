@@ -34,6 +34,8 @@ __global__ void __launch_bounds__(512) ps_stats_kernel(const bf16* __restrict__ 
   const int tile = cell >> 6, a = (cell >> 3) & 7, b = cell & 7;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = warp >> 2, r = warp & 3;
+  pdl_wait();
+  pdl_trigger();
   const bf16* tok = x + ((static_cast<long long>(tile) * 32 + 4 * a + q) * 32 + 4 * b + r) * C;
   const float shift = __bfloat162float(tok[0]);
   float s1 = 0.f, s2 = 0.f;
@@ -97,9 +99,8 @@ int launch_ps_stats(const bf16* x, int T, int C, float* mean_half, float* rstd_h
                     float* mean_quarter, float* rstd_quarter, const Launch& L) {
   if (T == 0) return IVC_OK;
   TraceScope ts("ps_stats", L.stream);
-  ps_stats_kernel<<<T * 64, 512, 0, L.stream>>>(x, C, mean_half, rstd_half, mean_quarter,
-                                                rstd_quarter);
-  return cu_check(cudaGetLastError());
+  return launch_k(ps_stats_kernel, dim3(T * 64), dim3(512), 0, L.stream, 1, x, C, mean_half,
+                  rstd_half, mean_quarter, rstd_quarter);
 }
 
 // ---------------------------------------------------------------- LN fold
@@ -114,6 +115,8 @@ __global__ void __launch_bounds__(256) fold_kernel(const bf16* __restrict__ W,
                                                    float* __restrict__ fbias) {
   const int n = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
   if (n >= N) return;
   const bf16* w = W + static_cast<long long>(n) * K;
   bf16* wo = W_out + static_cast<long long>(n) * K;
@@ -139,8 +142,8 @@ __global__ void __launch_bounds__(256) fold_kernel(const bf16* __restrict__ W,
 int launch_fold(const bf16* W, const bf16* b, const bf16* gamma, const bf16* beta, int N, int K,
                 bf16* W_out, float* colsum, float* fbias, const Launch& L) {
   TraceScope ts("ln_fold", L.stream);
-  fold_kernel<<<(N + 7) / 8, 256, 0, L.stream>>>(W, b, gamma, beta, N, K, W_out, colsum, fbias);
-  return cu_check(cudaGetLastError());
+  return launch_k(fold_kernel, dim3((N + 7) / 8), dim3(256), 0, L.stream, 1, W, b, gamma, beta,
+                  N, K, W_out, colsum, fbias);
 }
 
 // ---------------------------------------------------------------- tensor maps
@@ -238,19 +241,8 @@ static int run_gemm(const GemmMaps& maps, const GemmArgs& args, const char* tag,
   const long long units = num_sms() / CG;
   const int grid = CG * static_cast<int>(tiles < units ? tiles : units);
   TraceScope ts(tag ? tag : "gemm", L.stream);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(GEMM_THREADS);
-  cfg.dynamicSmemBytes = S::TOTAL;
-  cfg.stream = L.stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CG;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = CG == 2 ? 1 : 0;
-  return cu_check(cudaLaunchKernelEx(&cfg, kern, maps, args, L.status));
+  return launch_k(kern, dim3(grid), dim3(GEMM_THREADS), S::TOTAL, L.stream, CG, maps, args,
+                  L.status);
 }
 
 // 256-wide tiles run on CTA pairs unless IVC_GEMM_PAIRS=0 (kept for

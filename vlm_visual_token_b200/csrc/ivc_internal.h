@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 
 #include "ivc.h"
 
@@ -39,6 +40,33 @@ class TraceScope {
 
 // Converts a CUDA error into IVC_ECUDA (and remembers nothing else).
 inline int cu_check(cudaError_t e) { return e == cudaSuccess ? IVC_OK : IVC_ECUDA; }
+
+// Launches `kern` with programmatic stream serialisation (see pdl_wait in
+// ivc_ptx.cuh) and, when cluster_x > 1, thread-block clusters of cluster_x.
+template <typename... KArgs, typename... Args>
+inline int launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                    int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cu_check(cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...));
+}
 
 // -------------------------------------------------------------- connector
 // Per-row LayerNorm statistics of the pixel-shuffled rows, read straight

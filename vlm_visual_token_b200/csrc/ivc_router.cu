@@ -20,6 +20,7 @@
 #include <cuda_runtime.h>
 
 #include "ivc_internal.h"
+#include "ivc_ptx.cuh"
 
 namespace ivc {
 
@@ -29,18 +30,29 @@ __device__ __forceinline__ float gelu_f(float y) {
 
 // ---------------------------------------------------------------- skinny GEMV
 // Y[m, n] = act(sum_k X[m, k] W[n, k] + b[n]) for few rows m (router vectors).
-// A CTA of GEMV_WARPS warps owns GEMV_WARPS*GEMV_COLS consecutive columns;
-// warp w keeps its GEMV_COLS weight rows in registers (packed bf16, lane l
-// holds k = 128 j + 4 l .. +3) and reads each staged input row once for all
-// of them. Input rows are staged in shared memory as fp32, GEMV_ROWS(J) at a
-// time, with every load of a thread issued before its stores.
+// A CTA of GEMV_WARPS warps owns GEMV_CTA_COLS consecutive columns. One
+// thread brings the CTA's weight block (GEMV_CTA_COLS contiguous rows of W)
+// and up to GEMV_ROWS input rows into shared memory with bulk copies on one
+// mbarrier (the weight copy is issued before waiting for the previous
+// kernel), so the load latency is paid once. Warp w then keeps its
+// GEMV_COLS weight rows in registers (packed bf16, lane l holds
+// k = 128 j + 4 l .. +3) and reads each staged input row once for all of them.
 constexpr int GEMV_WARPS = 4;
 constexpr int GEMV_COLS = 4;
 constexpr int GEMV_CTA_COLS = GEMV_WARPS * GEMV_COLS;  // 16: one head of 64 spans 4 CTAs
 
 template <int J>
 struct GemvRows {
-  static constexpr int value = J <= 8 ? 16 : 8;  // staged rows: 64 KB of fp32 at most
+  static constexpr int value = J <= 8 ? 16 : 8;  // staged rows per round
+};
+
+template <typename XT, int J, bool PAIRED>
+struct GemvSmem {
+  static constexpr int K = J * 128;
+  static constexpr int ROWS = GemvRows<J>::value;
+  static constexpr size_t W_BYTES = static_cast<size_t>(GEMV_CTA_COLS) * K * 2;
+  static constexpr size_t X_BYTES = static_cast<size_t>(ROWS) * K * sizeof(XT) * (PAIRED ? 2 : 1);
+  static constexpr size_t TOTAL = 16 + W_BYTES + X_BYTES;
 };
 
 template <typename XT>
@@ -70,58 +82,73 @@ template <typename XT, int J, bool PAIRED = false>
 __global__ void __launch_bounds__(GEMV_WARPS * 32)
     gemv_kernel(const XT* __restrict__ X, long long ldx, int M,
                 const bf16* __restrict__ W, const bf16* __restrict__ b, int N,
-                float* __restrict__ Y, long long ldy, int gelu) {
-  constexpr int K = J * 128;
-  constexpr int ROWS = GemvRows<J>::value;
-  constexpr int F4_ROW = K / 4;
-  constexpr int PER_THREAD = ROWS * F4_ROW / (GEMV_WARPS * 32);
-  extern __shared__ float sx[];  // [ROWS][K]
+                float* __restrict__ Y, long long ldy, int gelu, int* __restrict__ status) {
+  using S = GemvSmem<XT, J, PAIRED>;
+  constexpr int K = S::K;
+  constexpr int ROWS = S::ROWS;
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
+  bf16* sw = reinterpret_cast<bf16*>(smem + 16);
+  XT* sx = reinterpret_cast<XT*>(smem + 16 + S::W_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * GEMV_CTA_COLS + warp * GEMV_COLS;
-  uint2 w[GEMV_COLS][J];
+  const int cta_n0 = blockIdx.x * GEMV_CTA_COLS;
+  const int n0 = cta_n0 + warp * GEMV_COLS;
+  const int w_rows = min(GEMV_CTA_COLS, N - cta_n0);
+  const int h = PAIRED ? cta_n0 / 64 : 0;
+  const int rows0 = min(ROWS, M);
+  const uint32_t x_row_bytes = K * sizeof(XT);
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar, w_rows * K * 2 + rows0 * x_row_bytes * (PAIRED ? 2 : 1));
+    bulk_load(sw, W + static_cast<long long>(cta_n0) * K, w_rows * K * 2, bar);
+  }
+  __syncthreads();  // barrier initialised before anyone waits on it
   float bias[GEMV_COLS];
 #pragma unroll
-  for (int c = 0; c < GEMV_COLS; ++c) {
-    const int n = n0 + c;
-    const bf16* wr = W + static_cast<long long>(n < N ? n : 0) * K;
-#pragma unroll
-    for (int j = 0; j < J; ++j) w[c][j] = *reinterpret_cast<const uint2*>(wr + j * 128 + lane * 4);
-    bias[c] = (n < N && b != nullptr) ? __bfloat162float(b[n]) : 0.f;
-  }
-  const int h = PAIRED ? (blockIdx.x * GEMV_CTA_COLS) / 64 : 0;
-  for (int m0 = 0; m0 < M; m0 += ROWS) {
+  for (int c = 0; c < GEMV_COLS; ++c)
+    bias[c] = (n0 + c < N && b != nullptr) ? __bfloat162float(b[n0 + c]) : 0.f;
+  pdl_wait();
+  pdl_trigger();
+  bool ok = true;
+  uint2 w[GEMV_COLS][J];
+  for (int m0 = 0, round = 0; m0 < M; m0 += ROWS, ++round) {
     const int rows = min(ROWS, M - m0);
-    __syncthreads();
-    constexpr int BATCH = PER_THREAD < 8 ? PER_THREAD : 8;  // loads in flight per thread
-#pragma unroll 1
-    for (int u0 = 0; u0 < PER_THREAD; u0 += BATCH) {
-      float4 v[BATCH];
-#pragma unroll
-      for (int u = 0; u < BATCH; ++u) {
-        const int i = threadIdx.x + (u0 + u) * GEMV_WARPS * 32;
-        const int r = i / F4_ROW, c = (i - r * F4_ROW) * 4;
-        if (r < rows) {
-          if constexpr (PAIRED) {
-            const XT* zr = X + (static_cast<long long>(m0 + r) * 128 + h) * ldx + c;
-            const float4 a = load4<XT>(zr), bb = load4<XT>(zr + 16 * ldx);
-            v[u] = make_float4(a.x + bb.x, a.y + bb.y, a.z + bb.z, a.w + bb.w);
-          } else {
-            v[u] = load4<XT>(X + static_cast<long long>(m0 + r) * ldx + c);
-          }
+    if (threadIdx.x == 0) {
+      if (round > 0) mbar_arrive_expect_tx(bar, rows * x_row_bytes * (PAIRED ? 2 : 1));
+      for (int r = 0; r < rows; ++r) {
+        if constexpr (PAIRED) {
+          const XT* zr = X + (static_cast<long long>(m0 + r) * 128 + h) * ldx;
+          bulk_load(sx + r * K, zr, x_row_bytes, bar);
+          bulk_load(sx + (ROWS + r) * K, zr + 16 * ldx, x_row_bytes, bar);
+        } else {
+          bulk_load(sx + r * K, X + static_cast<long long>(m0 + r) * ldx, x_row_bytes, bar);
         }
       }
+    }
+    ok = __syncthreads_and(ok && mbar_wait(bar, round & 1)) != 0;  // uniform decision
+    if (!ok) {
+      if (threadIdx.x == 0) atomicOr(status, DEV_WAIT_TIMEOUT);
+      break;
+    }
+    if (round == 0) {
 #pragma unroll
-      for (int u = 0; u < BATCH; ++u) {
-        const int i = threadIdx.x + (u0 + u) * GEMV_WARPS * 32;
-        if (i / F4_ROW < rows) *reinterpret_cast<float4*>(sx + i * 4) = v[u];
+      for (int c = 0; c < GEMV_COLS; ++c) {
+        const int wr = warp * GEMV_COLS + c < w_rows ? warp * GEMV_COLS + c : 0;
+#pragma unroll
+        for (int j = 0; j < J; ++j)
+          w[c][j] = *reinterpret_cast<const uint2*>(sw + wr * K + j * 128 + lane * 4);
       }
     }
-    __syncthreads();
     for (int r = 0; r < rows; ++r) {
       float acc[GEMV_COLS] = {};
 #pragma unroll
       for (int j = 0; j < J; ++j) {
-        const float4 xv = *reinterpret_cast<const float4*>(sx + r * K + j * 128 + lane * 4);
+        float4 xv = load4<XT>(sx + r * K + j * 128 + lane * 4);
+        if constexpr (PAIRED) {
+          const float4 x2 = load4<XT>(sx + (ROWS + r) * K + j * 128 + lane * 4);
+          xv = make_float4(xv.x + x2.x, xv.y + x2.y, xv.z + x2.z, xv.w + x2.w);
+        }
 #pragma unroll
         for (int c = 0; c < GEMV_COLS; ++c) acc[c] = dot4(w[c][j], xv, acc[c]);
       }
@@ -139,13 +166,14 @@ __global__ void __launch_bounds__(GEMV_WARPS * 32)
         if (n0 + lane < N) Y[static_cast<long long>(m0 + r) * ldy + n0 + lane] = y;
       }
     }
+    __syncthreads();  // staged rows consumed before the next round overwrites them
   }
 }
 
 template <typename XT, int J, bool PAIRED = false>
 static int run_gemv(const XT* X, long long ldx, int M, const bf16* W, const bf16* b, int N,
                     float* Y, long long ldy, int gelu, const Launch& L) {
-  const int smem = GemvRows<J>::value * J * 128 * static_cast<int>(sizeof(float));
+  const int smem = static_cast<int>(GemvSmem<XT, J, PAIRED>::TOTAL);
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(gemv_kernel<XT, J, PAIRED>,
@@ -154,10 +182,9 @@ static int run_gemv(const XT* X, long long ldx, int M, const bf16* W, const bf16
     attr = true;
   }
   TraceScope ts(PAIRED ? "pool.vproj" : (gelu ? "router.gemv_gelu" : "router.gemv"), L.stream);
-  gemv_kernel<XT, J, PAIRED>
-      <<<(N + GEMV_CTA_COLS - 1) / GEMV_CTA_COLS, GEMV_WARPS * 32, smem, L.stream>>>(
-          X, ldx, M, W, b, N, Y, ldy, gelu);
-  return cu_check(cudaGetLastError());
+  return launch_k(gemv_kernel<XT, J, PAIRED>, dim3((N + GEMV_CTA_COLS - 1) / GEMV_CTA_COLS),
+                  dim3(GEMV_WARPS * 32), smem, L.stream, 1, X, ldx, M, W, b, N, Y, ldy, gelu,
+                  L.status);
 }
 
 template <typename XT, bool PAIRED = false>
@@ -206,6 +233,8 @@ __global__ void __launch_bounds__(ATT_THREADS)
   __shared__ float s_scalar[ATT_THREADS / 32];
   const int h = blockIdx.x, tile = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
   int n = TILE_TOKENS;
   if (valid_len != nullptr) {
     n = valid_len[tile];
@@ -280,10 +309,8 @@ int launch_pool_attention(const float* Q, long long ldq, const float* KV, long l
   if (T == 0) return IVC_OK;
   if (heads * HEAD_DIM != D) return IVC_EUNSUPPORTED;
   TraceScope ts("pool.attention", L.stream);
-  pool_attention_kernel<<<dim3(heads, T), ATT_THREADS, 0, L.stream>>>(Q, ldq, KV, ldkv, koff,
-                                                                     voff, valid_len, O, D,
-                                                                     L.status);
-  return cu_check(cudaGetLastError());
+  return launch_k(pool_attention_kernel, dim3(heads, T), dim3(ATT_THREADS), 0, L.stream, 1, Q,
+                  ldq, KV, ldkv, koff, voff, valid_len, O, D, L.status);
 }
 
 // ---------------------------------------------------------------- folded pooling
@@ -311,6 +338,8 @@ __global__ void __launch_bounds__(128) pool_fold_query_kernel(
 #pragma unroll
   for (int d = 0; d < HEAD_DIM; ++d)
     w[d] = __bfloat162float(Wk[static_cast<long long>(h * HEAD_DIM + d) * D + c]);
+  pdl_wait();
+  pdl_trigger();
   for (int t0 = 0; t0 < Tq; t0 += 64) {
     const int nt = min(64, Tq - t0);
     __syncthreads();
@@ -343,9 +372,8 @@ int launch_pool_fold_query(const float* Q, long long ldq, int Tq, const bf16* Wk
   const int heads = D / HEAD_DIM;
   if (D % 128 != 0 || heads > 16) return IVC_EUNSUPPORTED;
   TraceScope ts("pool.fold_query", L.stream);
-  pool_fold_query_kernel<<<dim3(D / 128, heads), 128, 0, L.stream>>>(Q, ldq, Tq, Wk, bk, D, U2,
-                                                                     cb);
-  return cu_check(cudaGetLastError());
+  return launch_k(pool_fold_query_kernel, dim3(D / 128, heads), dim3(128), 0, L.stream, 1, Q, ldq,
+                  Tq, Wk, bk, D, U2, cb);
 }
 
 // Masked softmax of one (head, tile) from the split scores; writes the
@@ -359,6 +387,8 @@ __global__ void __launch_bounds__(ATT_THREADS)
   __shared__ float s_scalar[ATT_THREADS / 32];
   const int h = blockIdx.x, tile = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
   int n = TILE_TOKENS;
   if (valid_len != nullptr) {
     n = valid_len[tile];
@@ -416,9 +446,8 @@ int launch_pool_softmax(const float* S, const float* cb, int cb_stride, const in
   if (T == 0) return IVC_OK;
   if (heads < 1 || heads > 16) return IVC_EUNSUPPORTED;
   TraceScope ts("pool.softmax", L.stream);
-  pool_softmax_kernel<<<dim3(heads, T), ATT_THREADS, 0, L.stream>>>(S, cb, cb_stride, valid_len,
-                                                                   P2, L.status);
-  return cu_check(cudaGetLastError());
+  return launch_k(pool_softmax_kernel, dim3(heads, T), dim3(ATT_THREADS), 0, L.stream, 1, S, cb,
+                  cb_stride, valid_len, P2, L.status);
 }
 
 // ---------------------------------------------------------------- residual + LayerNorm
@@ -430,6 +459,8 @@ __global__ void __launch_bounds__(256) residual_ln_kernel(float* __restrict__ h,
   __shared__ float s_red[8];
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
   const float* ur = u + static_cast<long long>(t) * D;
   float s = 0.f;
   for (int i = threadIdx.x; i < D; i += 256) s += ur[i];
@@ -465,8 +496,7 @@ int launch_residual_ln(float* h, const float* u, const bf16* gamma, const bf16* 
                        int D, const Launch& L) {
   if (T == 0) return IVC_OK;
   TraceScope ts("gate.residual_ln", L.stream);
-  residual_ln_kernel<<<T, 256, 0, L.stream>>>(h, u, gamma, beta, D);
-  return cu_check(cudaGetLastError());
+  return launch_k(residual_ln_kernel, dim3(T), dim3(256), 0, L.stream, 1, h, u, gamma, beta, D);
 }
 
 // ---------------------------------------------------------------- gate head
@@ -477,6 +507,8 @@ __global__ void __launch_bounds__(256) gate_head_kernel(const float* __restrict_
                                                         int D, float* __restrict__ gate) {
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
   if (t >= T) return;
   const float* hr = h + static_cast<long long>(t) * D;
   float l0 = 0.f, l1 = 0.f;
@@ -507,8 +539,8 @@ int launch_gate_head(const float* h, const bf16* Wout, const bf16* bout, int T, 
                      float* gate, const Launch& L) {
   if (T == 0) return IVC_OK;
   TraceScope ts("gate.head", L.stream);
-  gate_head_kernel<<<(T + 7) / 8, 256, 0, L.stream>>>(h, Wout, bout, T, D, gate);
-  return cu_check(cudaGetLastError());
+  return launch_k(gate_head_kernel, dim3((T + 7) / 8), dim3(256), 0, L.stream, 1, h, Wout, bout,
+                  T, D, gate);
 }
 
 // ---------------------------------------------------------------- routing
@@ -532,6 +564,8 @@ __global__ void __launch_bounds__(ROUTE_THREADS)
   __shared__ int s_bad;
   __shared__ int s_warp[ROUTE_THREADS / 32];
   __shared__ int s_carry;
+  pdl_wait();
+  pdl_trigger();
   if (threadIdx.x == 0) {
     int bad = 0;
     if (scope == 0) {
@@ -642,9 +676,8 @@ int launch_route(const float* gate, int T, const int32_t* image_offsets, int I, 
     attr = true;
   }
   TraceScope ts("route", L.stream);
-  route_kernel<<<1, ROUTE_THREADS, smem, L.stream>>>(gate, T, image_offsets, I, rel_q, abs_t,
-                                                     scope, mask, offsets, total, L.status);
-  return cu_check(cudaGetLastError());
+  return launch_k(route_kernel, dim3(1), dim3(ROUTE_THREADS), smem, L.stream, 1, gate, T,
+                  image_offsets, I, rel_q, abs_t, scope, mask, offsets, total, L.status);
 }
 
 // ---------------------------------------------------------------- compaction
@@ -657,6 +690,8 @@ __global__ void __launch_bounds__(256) compact_kernel(const bf16* __restrict__ Y
                                                       bf16* __restrict__ out) {
   const int t = blockIdx.x;
   const int r0 = blockIdx.y * 32;
+  pdl_wait();
+  pdl_trigger();
   const bool comp = mask[t] != 0;
   const int rows = comp ? 64 : 256;
   if (r0 >= rows) return;
@@ -673,8 +708,8 @@ int launch_compact(const bf16* Y256, const bf16* Y64, const uint8_t* mask,
                    const int32_t* offsets, int T, int H, bf16* out, const Launch& L) {
   if (T == 0) return IVC_OK;
   TraceScope ts("compact", L.stream);
-  compact_kernel<<<dim3(T, 8), 256, 0, L.stream>>>(Y256, Y64, mask, offsets, H, out);
-  return cu_check(cudaGetLastError());
+  return launch_k(compact_kernel, dim3(T, 8), dim3(256), 0, L.stream, 1, Y256, Y64, mask, offsets,
+                  H, out);
 }
 
 }  // namespace ivc
