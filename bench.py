@@ -463,6 +463,39 @@ def run_ivc(args):
     return 0
 
 
+def run_op(args):
+    """One entry point alone on the bench image (profiling aid: a short,
+    eager run whose kernels ncu can pick out by launch index)."""
+    import torch
+
+    import vlm_visual_token_b200 as ivc
+    torch.cuda.set_device(0)
+    inp = image_gen(0)
+    w, T = inp["workload"], inp["T"]
+    x = inp["x"].cuda()
+    vl, offs = inp["valid_len"].cuda(), inp["image_offsets"].cuda()
+    if args.op in ("ps_half", "ps_quarter"):
+        m = ivc.Mlp(inp["mlp1" if args.op == "ps_half" else "mlp2"]).fold()
+        scale = 0.5 if args.op == "ps_half" else 0.25
+        fn = lambda: ivc.ps_project(x, scale, m)
+    else:
+        r = ivc.Router(inp["router"], pool_mode=1 if args.op == "route_literal" else 0)
+        fn = lambda: ivc.vir_route(x, vl, offs, r)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        fn()
+    b.record()
+    b.synchronize()
+    ms = a.elapsed_time(b) / args.steps
+    print(json.dumps({"op": args.op, "workload": WORKLOAD, "tiles": T, "ms_per_call": ms,
+                      "tiles_per_s": T / (ms / 1e3), "timing": "eager, back to back, no L2 flush"}))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -470,11 +503,15 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ivc", "reference"], default="ivc")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", choices=["flash", "ps_half", "ps_quarter", "route", "route_literal"],
+                    default="flash", help="profiling aid: time one entry point alone")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.op != "flash":
+        return run_op(args)
     return run_ivc(args)
 
 

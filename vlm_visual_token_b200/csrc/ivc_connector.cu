@@ -256,6 +256,17 @@ static bool pairs_enabled() {
   return on == 1;
 }
 
+// L2 prefetch distance of streamed weights in k-steps (IVC_GEMM_PREFETCH, default 16).
+static int prefetch_depth() {
+  static int d = -1;
+  if (d < 0) {
+    const char* e = std::getenv("IVC_GEMM_PREFETCH");
+    d = e ? std::atoi(e) : 16;
+    if (d < 0) d = 0;
+  }
+  return d;
+}
+
 // Output tile width. Measured on B200 (tcgen05 M=128, TMA-fed ring with
 // L2-resident operands): N=256 tiles run at ~1.8-2.2 PFLOP/s, N=128 tiles at
 // ~1.08 PFLOP/s, i.e. an N=128 tile takes as long as an N=256 one. So 256 is
@@ -306,6 +317,9 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
   a.b_mode = c.b_mode;
   a.b_batch_rows = c.b_mode == B_K2D ? 0 : c.b_batch_rows;
   a.c_blocks = c.C / GEMM_BK;
+  // Weights that stream from HBM once per M-tile row (long K): prefetch the
+  // B operand ~16 k-steps ahead into L2 so TMA loads see L2 latency.
+  a.b_prefetch = (c.b_mode == B_K2D && c.K >= 2048) ? prefetch_depth() : 0;
   a.epi_mode = c.epi_mode;
   a.gelu = c.gelu;
   a.remap = c.remap;

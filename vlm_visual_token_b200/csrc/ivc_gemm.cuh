@@ -70,6 +70,7 @@ struct GemmArgs {
   int b_mode;
   int b_batch_rows;              // B_K3D / B_MN3D: rows of A per B batch
   int c_blocks;                  // C / 64 for the pixel_shuffle modes
+  int b_prefetch;                // >0: prefetch B (K2D) this many k-steps ahead into L2
   int epi_mode;
   int gelu;
   int remap;                     // 0: none; 1: transpose 16x16 token grid; 2: 8x8
@@ -194,9 +195,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const int my_m0 = tc.m0 + GEMM_BM * rank;
         const int my_n0 = tc.n0 + static_cast<int>(L::B_ROWS) * rank;
         const int bb = args.b_batch_rows > 0 ? tc.m0 / args.b_batch_rows : 0;
+        if (args.b_prefetch > 0 && args.b_mode == B_K2D) {
+          for (int kk = 0; kk < args.b_prefetch && kk < KT; ++kk)
+            tma_prefetch_2d(&maps.b[tc.g], kk * GEMM_BK, my_n0);
+        }
         for (int kk = 0; kk < KT; ++kk, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
+          if (args.b_prefetch > 0 && args.b_mode == B_K2D && kk + args.b_prefetch < KT)
+            tma_prefetch_2d(&maps.b[tc.g], (kk + args.b_prefetch) * GEMM_BK, my_n0);
           if (!mbar_wait(&empty_bar[s], ph ^ 1)) { ok = false; break; }
           // the leader's barrier counts the bytes of both CTAs of a pair
           if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], L::STAGE * CG);

@@ -116,6 +116,16 @@ __device__ __forceinline__ void tma_load_5d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// Ask TMA to pull a box into L2 (no shared memory, no barrier): lets a
+// producer run further ahead of its shared-memory ring on operands that
+// stream from HBM.
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
+
 // Plain bulk copy global -> this CTA's shared memory (16-byte aligned
 // addresses, size a multiple of 16), completing `bytes` on `bar`.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
