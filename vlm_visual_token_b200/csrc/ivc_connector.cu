@@ -256,12 +256,12 @@ static bool pairs_enabled() {
   return on == 1;
 }
 
-// L2 prefetch distance of streamed weights in k-steps (IVC_GEMM_PREFETCH, default 16).
+// L2 prefetch distance of streamed weights in k-steps (IVC_GEMM_PREFETCH, default 0: measured no gain).
 static int prefetch_depth() {
   static int d = -1;
   if (d < 0) {
     const char* e = std::getenv("IVC_GEMM_PREFETCH");
-    d = e ? std::atoi(e) : 16;
+    d = e ? std::atoi(e) : 0;
     if (d < 0) d = 0;
   }
   return d;
