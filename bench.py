@@ -484,15 +484,36 @@ def run_op(args):
     for _ in range(args.warmup):
         fn()
     torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     for _ in range(args.steps):
-        fn()
+        g.replay()
     b.record()
     b.synchronize()
     ms = a.elapsed_time(b) / args.steps
-    print(json.dumps({"op": args.op, "workload": WORKLOAD, "tiles": T, "ms_per_call": ms,
-                      "tiles_per_s": T / (ms / 1e3), "timing": "eager, back to back, no L2 flush"}))
+    line = {"op": args.op, "workload": WORKLOAD, "tiles": T, "ms_per_call": ms,
+            "tiles_per_s": T / (ms / 1e3), "timing": "CUDA graph, back to back, no L2 flush"}
+    if args.trace:
+        import ctypes
+        L = ivc.lib()
+        L.ivc_trace_enable.argtypes = [ctypes.c_int]
+        L.ivc_trace_report.argtypes = [ctypes.c_char_p, ctypes.c_size_t]
+        L.ivc_trace_reset()
+        L.ivc_trace_enable(1)
+        for _ in range(args.steps):
+            fn()
+        torch.cuda.synchronize()
+        L.ivc_trace_enable(0)
+        buf = ctypes.create_string_buffer(1 << 16)
+        L.ivc_trace_report(buf, len(buf))
+        tr = json.loads(buf.value.decode())
+        line["traced_us_per_launch"] = {k: round(1e3 * v["ms"] / v["launches"], 2)
+                                        for k, v in tr.items()}
+        line["traced_launches_per_call"] = {k: v["launches"] // args.steps for k, v in tr.items()}
+    print(json.dumps(line))
     return 0
 
 
@@ -505,6 +526,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", choices=["flash", "ps_half", "ps_quarter", "route", "route_literal"],
                     default="flash", help="profiling aid: time one entry point alone")
+    ap.add_argument("--trace", action="store_true",
+                    help="with --op: also report per-kernel device times (event-bracketed)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
