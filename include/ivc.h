@@ -125,6 +125,8 @@ typedef struct ivc_router {
   double abs_t;       /* flash_absolute_threshold, 0.5 */
   int quantile_scope; /* 0 = per image, 1 = whole batch */
   int pool_mode;      /* IVC_POOL_FOLDED (0) or IVC_POOL_LITERAL (1) */
+  int gate_residual;  /* 0: h <- h + LN(u) (the listed block inside the residual);
+                         1: h <- LN(h + u) (residual inside the LayerNorm) */
 } ivc_router;
 
 /* How CrossAttentionPooling is evaluated; both compute the same function.

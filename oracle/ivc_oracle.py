@@ -268,11 +268,11 @@ def compact(Y256: np.ndarray, Y64: np.ndarray, mask: np.ndarray) -> np.ndarray:
 # ----------------------------------------------------------------------------
 # Whole path
 # ----------------------------------------------------------------------------
-def vir_gate(x: np.ndarray, valid_len: np.ndarray, r: dict) -> np.ndarray:
+def vir_gate(x: np.ndarray, valid_len: np.ndarray, r: dict, residual: str = "outside") -> np.ndarray:
     """Gate probabilities [T, 2] of the router for features x [T, 32, 32, D]."""
     T, G, _, D = x.shape
     pooled = cross_attention_pooling(x.reshape(T, G * G, D), valid_len, r)
-    return gating(pooled, r)
+    return gating(pooled, r, residual)
 
 
 def flash_compress(x, valid_len, image_offsets, mlp1, mlp2, r, rel_q=0.1, abs_t=0.5,

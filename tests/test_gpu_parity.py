@@ -176,6 +176,21 @@ def test_vir_route_batch_scope(pool_mode):
     _route_check(ivc, inp, gate, mask, offsets, scope=1)
 
 
+@pytest.mark.parametrize("pool_mode", [0, 1])
+def test_vir_route_gating_residual_inside(pool_mode):
+    """Reading variant: h <- LN(h + u) in the gating blocks."""
+    ivc = _ivc()
+    inp = W.make(small_workload(C=256, H=128, tiles=(3, 2)), affine="random")
+    r = ivc.Router(inp["router"], pool_mode=pool_mode, gate_residual=1)
+    gate, mask, offsets = ivc.vir_route(inp["x"].cuda(), None, inp["image_offsets"].cuda(), r)
+    torch.cuda.synchronize()
+    ref = O.vir_gate(O.to64(inp["x"]), inp["valid_len"].numpy(), O.to64(inp["router"]),
+                     residual="inside")
+    assert np.abs(to_np(gate) - ref).max() <= GATE_ABS
+    outside = O.vir_gate(O.to64(inp["x"]), inp["valid_len"].numpy(), O.to64(inp["router"]))
+    assert np.abs(ref - outside).max() > 10 * GATE_ABS  # the variant really differs
+
+
 def test_bad_valid_len_sets_status_bit():
     ivc = _ivc()
     inp = W.make(small_workload(C=256, H=128, tiles=(2,)))

@@ -48,7 +48,8 @@ class _CRouter(ctypes.Structure):
                 ("gW1", _vp * 4), ("gb1", _vp * 4), ("gW2", _vp * 4), ("gb2", _vp * 4),
                 ("gln_g", _vp * 4), ("gln_b", _vp * 4), ("gWout", _vp), ("gbout", _vp),
                 ("rel_q", ctypes.c_double), ("abs_t", ctypes.c_double),
-                ("quantile_scope", ctypes.c_int), ("pool_mode", ctypes.c_int)]
+                ("quantile_scope", ctypes.c_int), ("pool_mode", ctypes.c_int),
+                ("gate_residual", ctypes.c_int)]
 
 
 class IvcError(RuntimeError):
@@ -154,7 +155,7 @@ class Router:
     """ViR router weights (CrossAttentionPooling + Gating) and thresholds."""
 
     def __init__(self, params: dict, rel_q: float = 0.1, abs_t: float = 0.5, scope: int = 0,
-                 device="cuda", pool_mode: int = 0):
+                 device="cuda", pool_mode: int = 0, gate_residual: int = 0):
         def dev(t):
             return t.to(device=device, dtype=torch.bfloat16).contiguous()
         self.t = {}
@@ -178,6 +179,7 @@ class Router:
         c.abs_t = float(abs_t)
         c.quantile_scope = int(scope)
         c.pool_mode = int(pool_mode)
+        c.gate_residual = int(gate_residual)
         self.c = c
 
 

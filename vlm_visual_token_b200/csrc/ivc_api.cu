@@ -65,6 +65,7 @@ int router_shape_ok(const ivc_router* r, int C) {
   if (!d_ok || !g_ok) return IVC_EUNSUPPORTED;
   if (r->quantile_scope != 0 && r->quantile_scope != 1) return IVC_EINVAL;
   if (r->pool_mode != IVC_POOL_FOLDED && r->pool_mode != IVC_POOL_LITERAL) return IVC_EINVAL;
+  if (r->gate_residual != 0 && r->gate_residual != 1) return IVC_EINVAL;
   if (r->pool_mode == IVC_POOL_FOLDED && (r->heads > 16 || r->D % 128 != 0))
     return IVC_EUNSUPPORTED;
   if (!r->query || !r->gWout) return IVC_EINVAL;
@@ -110,8 +111,11 @@ struct RouteBufs {
   bf16* U2 = nullptr;    // folded pooling: split u of one layer [T][32][D]
   float* cb = nullptr;   //   c [T][16]
   float* S = nullptr;    //   split scores [T*1024][32]
-  bf16* P2 = nullptr;    //   split softmax weights [T*128][1024]
-  float* Z = nullptr;    //   split weighted sums [T*128][D]
+  bf16* P2 = nullptr;    //   split softmax weights [T*128][1024] (multi-kernel form)
+  float* Z = nullptr;    //   split weighted sums [T*128][D] (multi-kernel form)
+  float* z = nullptr;    //   fused router: weighted sums [T][16][D]
+  float* h = nullptr;    //   fused router: gating state [T][D]
+  unsigned* bar = nullptr;  // fused router: grid barrier words
   float* Q1;
   float* Q;
   float* O;
@@ -128,8 +132,13 @@ void carve_route(Carver& cv, const ivc_router* r, int T, RouteBufs& b) {
     b.U2 = cv.take<bf16>(static_cast<size_t>(T) * 32 * D);
     b.cb = cv.take<float>(static_cast<size_t>(T) * 16);
     b.S = cv.take<float>(static_cast<size_t>(T) * 1024 * 32);
+    // P2 in the multi-kernel form [T*128][1024]; the persistent kernel uses
+    // its first T*32*1024 entries as [T][32][1024]
     b.P2 = cv.take<bf16>(static_cast<size_t>(T) * 128 * 1024);
     b.Z = cv.take<float>(static_cast<size_t>(T) * 128 * D);
+    b.z = cv.take<float>(static_cast<size_t>(T) * 16 * D);
+    b.h = cv.take<float>(static_cast<size_t>(T) * D);
+    b.bar = cv.take<unsigned>(2);
   }
   b.Q1 = cv.take<float>(D);
   b.Q = cv.take<float>(static_cast<size_t>(T) * D);
@@ -269,6 +278,11 @@ int route_impl(const void* x, const int32_t* valid_len, int T, const int32_t* im
                int I, const ivc_router* r, float* gate, uint8_t* mask, int32_t* offsets,
                int32_t* total, const RouteBufs& b, const Launch& L) {
   const int D = r->D;
+  if (r->pool_mode == IVC_POOL_FOLDED && router_fused_enabled()) {
+    FusedRouterBufs f{b.Q, b.U2, b.cb, b.S, b.P2, b.z, b.O, b.q, b.h, b.u1, b.u2, b.bar};
+    return launch_router_fused(r, x, valid_len, T, image_offsets, I, gate, mask, offsets, total,
+                               f, L);
+  }
   if (r->pool_mode == IVC_POOL_FOLDED) {
     IVC_TRY(launch_gemv_bf16x(static_cast<const bf16*>(r->query), D,
                               static_cast<const bf16*>(r->Wq[0]),
@@ -340,7 +354,7 @@ int gating_and_route(int T, const int32_t* image_offsets, int I, const ivc_route
     IVC_TRY(launch_gemv(b.u1, G, T, G, static_cast<const bf16*>(r->gW2[k]),
                         static_cast<const bf16*>(r->gb2[k]), D, b.u2, D, 0, L));
     IVC_TRY(launch_residual_ln(b.q, b.u2, static_cast<const bf16*>(r->gln_g[k]),
-                               static_cast<const bf16*>(r->gln_b[k]), T, D, L));
+                               static_cast<const bf16*>(r->gln_b[k]), T, D, r->gate_residual, L));
   }
   IVC_TRY(launch_gate_head(b.q, static_cast<const bf16*>(r->gWout),
                            static_cast<const bf16*>(r->gbout), T, D, gate, L));

@@ -128,9 +128,32 @@ int launch_pool_softmax(const float* S, const float* cb, int cb_stride, const in
                         int T, int heads, bf16* P2, const Launch& L);
 int launch_pool_vproj(const float* Z, int T, int D, const bf16* Wv, const bf16* bv, float* O,
                       const Launch& L);
-// h[t] += LN(u[t]) * gamma + beta over D.
+// The whole folded router (pooling, gating, routing) as one cooperative
+// persistent kernel (ivc_router_fused.cu).
+struct FusedRouterBufs {
+  float* Q;
+  bf16* U2;
+  float* cb;
+  float* S;
+  bf16* P2;
+  float* z;
+  float* O;
+  float* q;
+  float* h;
+  float* u1;
+  float* u2;
+  unsigned* bar;
+};
+// Folded pooling runs as one persistent cooperative kernel (grid barriers
+// between its phases) when IVC_ROUTER_FUSED=1; otherwise as separate kernels.
+bool router_fused_enabled();
+int launch_router_fused(const ivc_router* r, const void* x, const int32_t* valid_len, int T,
+                        const int32_t* image_offsets, int I, float* gate, uint8_t* mask,
+                        int32_t* offsets, int32_t* total, const FusedRouterBufs& b,
+                        const Launch& L);
+// h[t] += LN(u[t]) * gamma + beta over D (inside = 1: h[t] = LN(h[t] + u[t]) ...).
 int launch_residual_ln(float* h, const float* u, const bf16* gamma, const bf16* beta, int T,
-                       int D, const Launch& L);
+                       int D, int inside, const Launch& L);
 // gate[t] = softmax(Wout h[t] + bout), Wout [2, D].
 int launch_gate_head(const float* h, const bf16* Wout, const bf16* bout, int T, int D,
                      float* gate, const Launch& L);

@@ -451,17 +451,25 @@ int launch_pool_softmax(const float* S, const float* cb, int cb_stride, const in
 }
 
 // ---------------------------------------------------------------- residual + LayerNorm
-// h[t] += (u[t] - mean) * rstd * gamma + beta (biased variance, eps 1e-5).
+// inside = 0: h[t] += (u[t] - mean) * rstd * gamma + beta;
+// inside = 1: v = h[t] + u[t], h[t] = (v - mean) * rstd * gamma + beta
+// (biased variance, eps 1e-5; D <= 2048).
 __global__ void __launch_bounds__(256) residual_ln_kernel(float* __restrict__ h,
                                                           const float* __restrict__ u,
                                                           const bf16* __restrict__ gamma,
-                                                          const bf16* __restrict__ beta, int D) {
+                                                          const bf16* __restrict__ beta, int D,
+                                                          int inside) {
   __shared__ float s_red[8];
+  __shared__ float s_v[2048];
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_wait();
   pdl_trigger();
-  const float* ur = u + static_cast<long long>(t) * D;
+  const float* u0 = u + static_cast<long long>(t) * D;
+  const float* hr0 = h + static_cast<long long>(t) * D;
+  for (int i = threadIdx.x; i < D; i += 256) s_v[i] = inside ? hr0[i] + u0[i] : u0[i];
+  __syncthreads();
+  const float* ur = s_v;
   float s = 0.f;
   for (int i = threadIdx.x; i < D; i += 256) s += ur[i];
 #pragma unroll
@@ -488,15 +496,19 @@ __global__ void __launch_bounds__(256) residual_ln_kernel(float* __restrict__ h,
   var /= D;
   const float rstd = 1.0f / sqrtf(var + 1e-5f);
   float* hr = h + static_cast<long long>(t) * D;
-  for (int i = threadIdx.x; i < D; i += 256)
-    hr[i] += (ur[i] - mean) * rstd * __bfloat162float(gamma[i]) + __bfloat162float(beta[i]);
+  for (int i = threadIdx.x; i < D; i += 256) {
+    const float n = (ur[i] - mean) * rstd * __bfloat162float(gamma[i]) + __bfloat162float(beta[i]);
+    hr[i] = inside ? n : hr[i] + n;
+  }
 }
 
 int launch_residual_ln(float* h, const float* u, const bf16* gamma, const bf16* beta, int T,
-                       int D, const Launch& L) {
+                       int D, int inside, const Launch& L) {
   if (T == 0) return IVC_OK;
+  if (D > 2048) return IVC_EUNSUPPORTED;
   TraceScope ts("gate.residual_ln", L.stream);
-  return launch_k(residual_ln_kernel, dim3(T), dim3(256), 0, L.stream, 1, h, u, gamma, beta, D);
+  return launch_k(residual_ln_kernel, dim3(T), dim3(256), 0, L.stream, 1, h, u, gamma, beta, D,
+                  inside);
 }
 
 // ---------------------------------------------------------------- gate head
