@@ -325,6 +325,32 @@ def test_gating_matches_torch_modules():
     np.testing.assert_allclose(O.gating(h0, r), ref, rtol=1e-12, atol=1e-14)
 
 
+def test_gating_inside_variant_matches_torch_modules():
+    """The other reading of a Gating block: LayerNorm applied to the residual
+    sum, h <- LN(h + W2 GELU(W1 h + b1) + b2), checked against torch modules."""
+    D, hid = 32, 24
+    r = _router(D=D, hid=hid)
+    h0 = RNG.standard_normal((5, D))
+    h = torch.from_numpy(h0)
+    for b in range(4):
+        l1 = torch.nn.Linear(D, hid).double()
+        l2 = torch.nn.Linear(hid, D).double()
+        ln = torch.nn.LayerNorm(D).double()
+        with torch.no_grad():
+            l1.weight.copy_(torch.from_numpy(r["gW1"][b])); l1.bias.copy_(torch.from_numpy(r["gb1"][b]))
+            l2.weight.copy_(torch.from_numpy(r["gW2"][b])); l2.bias.copy_(torch.from_numpy(r["gb2"][b]))
+            ln.weight.copy_(torch.from_numpy(r["gln_g"][b])); ln.bias.copy_(torch.from_numpy(r["gln_b"][b]))
+            h = ln(h + l2(torch.nn.functional.gelu(l1(h))))
+    out = torch.nn.Linear(D, 2).double()
+    with torch.no_grad():
+        out.weight.copy_(torch.from_numpy(r["gWout"])); out.bias.copy_(torch.from_numpy(r["gbout"]))
+    ref = torch.softmax(out(h), dim=-1).detach().numpy()
+    got = O.gating(h0, r, residual="inside")
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-14)
+    # the two readings differ (a swapped branch would pass one test, not both)
+    assert np.abs(got - O.gating(h0, r)).max() > 1e-3
+
+
 # ------------------------------------------------------------------ quantile / routing
 @pytest.mark.parametrize("n", [1, 2, 3, 5, 11, 13, 64, 257])
 def test_quantile_matches_numpy_and_torch(n):
