@@ -11,12 +11,17 @@
 // threshold) and section 5 of the 4B-Flash article (tiles spliced back in
 // order, 64 or 256 rows each).
 //
-// The K and V projections of all four pooling layers are one grouped
-// tensor-core GEMM (ivc_gemm.cuh); what remains per layer is a skinny
-// projection of the query (M = tiles), the masked softmax-weighted sum over
-// the tile's tokens, and the output projection. All router activations,
-// K/V included, are fp32 (rounding K/V to bf16 alone moves the gate
-// probabilities by about 1e-3 on the 13-tile workload).
+// Two forms of the pooling, chosen by ivc_router.pool_mode:
+//  * folded (default): the single query lets each layer's K and V
+//    projections be reassociated onto the query (see "folded pooling"
+//    below); per layer two thin tensor-core contractions with the raw
+//    features, a masked softmax and skinny projections remain;
+//  * literal: the K and V projections of all four layers are one grouped
+//    tensor-core GEMM (ivc_gemm.cuh) with fp32 output, then a masked
+//    softmax-weighted sum per (head, tile) over fp32 K/V (rounding K/V to
+//    bf16 alone moves the gate probabilities by about 1e-3 on the 13-tile
+//    workload).
+// All router vectors between steps are fp32.
 #include <cuda_runtime.h>
 
 #include "ivc_internal.h"
