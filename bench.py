@@ -268,8 +268,10 @@ def run_ivc(args):
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
+    routed = args.flow == "routed"
+
     def step():
-        ivc.flash_compress(x, vl, offs, m1, m2, r, out=out, workspace=ws, bufs=bufs)
+        ivc.flash_compress(x, vl, offs, m1, m2, r, out=out, workspace=ws, bufs=bufs, routed=routed)
 
     for _ in range(3):
         step()
@@ -400,6 +402,17 @@ def run_ivc(args):
                      "measured_us": meas * 1e6, "frac_vs_literal": t_roof / meas,
                      "frac_vs_folded": t_roof_f / meas,
                      "peak_source": f"{src} bf16_tflops (burst), hbm_gbs"}
+    if routed:
+        # router-first: only the selected path of each tile is computed
+        k = int(bufs["mask"].sum().item())
+        m1f = (alg["mlp1.fc1"][0] + alg["mlp1.fc2"][0]) * (T - k) / T
+        m2f = (alg["mlp2.fc1"][0] + alg["mlp2.fc2"][0] + alg["mlp2.fc3"][0]) * k / T
+        F_routed = F_folded - conn + m1f + m2f
+        B_routed = B_alg - 2 * T * 256 * w.H + 2 * (256 * (T - k) + 64 * k) * w.H
+        t_roof_r = max(F_routed / (peaks["bf16_tflops"] * 1e12), B_routed / (peaks["hbm_gbs"] * 1e9))
+        step_roofline.update({"compressed_tiles": k, "flops_routed": F_routed,
+                              "bytes_routed": B_routed, "roofline_us_routed": t_roof_r * 1e6,
+                              "frac_vs_routed": t_roof_r / meas})
 
     # ---- end to end through the public API with host buffers
     e2e_steps = min(args.steps, 100)
@@ -431,8 +444,8 @@ def run_ivc(args):
            "d2h_bytes_per_step": d2h_small + d2h_rows // e2e_steps, "steps": e2e_steps,
            "timing": "wall clock, host sync per step (needs the row count before the row copy)"}
 
-    launch_desc = ("CUDA graph of one ivc_flash_compress" if graph is not None
-                   else "eager ivc_flash_compress")
+    fn_name = "ivc_flash_compress_routed" if routed else "ivc_flash_compress"
+    launch_desc = (f"CUDA graph of one {fn_name}" if graph is not None else f"eager {fn_name}")
     run = None
     graph = None
     barrier()
@@ -448,6 +461,8 @@ def run_ivc(args):
                        "mlp2_mid": w.mlp2_mid, "pool_heads": 16, "gate_hidden": w.gate_hidden,
                        "l2": "flushed between steps (512 MiB write, outside the timed events)",
                        "launch": launch_desc,
+                       "flow": ("router first, each tile through its selected path" if routed
+                                else "both paths for every tile, then compaction"),
                        "parallelism": f"replicas x{world}, one image per GPU, no collective"},
             "roofline": roof, "step_roofline": step_roofline,
             "kernels_ms_per_step": {k: round(v, 5) for k, v in per_step_ms.items()},
@@ -474,7 +489,11 @@ def run_op(args):
     w, T = inp["workload"], inp["T"]
     x = inp["x"].cuda()
     vl, offs = inp["valid_len"].cuda(), inp["image_offsets"].cuda()
-    if args.op in ("ps_half", "ps_quarter"):
+    if args.op in ("flash_dual", "flash_routed"):
+        m1, m2 = ivc.Mlp(inp["mlp1"]).fold(), ivc.Mlp(inp["mlp2"]).fold()
+        r = ivc.Router(inp["router"])
+        fn = lambda: ivc.flash_compress(x, vl, offs, m1, m2, r, routed=args.op == "flash_routed")
+    elif args.op in ("ps_half", "ps_quarter"):
         m = ivc.Mlp(inp["mlp1" if args.op == "ps_half" else "mlp2"]).fold()
         scale = 0.5 if args.op == "ps_half" else 0.25
         fn = lambda: ivc.ps_project(x, scale, m)
@@ -524,8 +543,13 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ivc", "reference"], default="ivc")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["flash", "ps_half", "ps_quarter", "route", "route_literal"],
-                    default="flash", help="profiling aid: time one entry point alone")
+    ap.add_argument("--flow", choices=["dual", "routed"], default="dual",
+                    help="dual: ivc_flash_compress (both paths, then compaction); "
+                         "routed: ivc_flash_compress_routed (router first)")
+    ap.add_argument("--op", choices=["flash", "flash_dual", "flash_routed", "ps_half",
+                                     "ps_quarter", "route", "route_literal"],
+                    default="flash", help="profiling aid: time one entry point alone "
+                                          "(flash = the full benchmark)")
     ap.add_argument("--trace", action="store_true",
                     help="with --op: also report per-kernel device times (event-bracketed)")
     args = ap.parse_args(argv)

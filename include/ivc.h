@@ -193,7 +193,10 @@ int ivc_ps_project(const void* x, int T, int C, float scale, int flags, const iv
  *   mask           device uint8 [T]: 1 = compressed (64 rows), 0 = 256 rows.
  *   offsets        device int32 [T+1]: exclusive scan of the row counts;
  *                  offsets[T] = total rows = 256 (T - k) + 64 k.
- * Unsupported: D != C, D % 256 != 0, heads * 64 != D, gate_hidden % 256 != 0. */
+ * Unsupported: D != C, D % 256 != 0, heads * 64 != D, gate_hidden % 256 != 0.
+ * With folded pooling, D <= 1024 and at most 16 heads, the router runs as one
+ * cooperative persistent kernel that holds every SM until it ends (the
+ * environment variable IVC_ROUTER_FUSED=0 selects separate kernels instead). */
 int ivc_vir_route(const void* x, const int32_t* valid_len, int T, int C,
                   const int32_t* image_offsets, int I, const ivc_router* r, float* gate,
                   uint8_t* mask, int32_t* offsets, void* workspace, size_t ws_bytes,
@@ -214,6 +217,21 @@ int ivc_flash_compress(const void* x, const int32_t* valid_len, int T, int C,
                        const ivc_mlp* mlp2, const ivc_router* r, void* out, float* gate,
                        uint8_t* mask, int32_t* offsets, int32_t* total, void* workspace,
                        size_t ws_bytes, ivc_stream_t stream);
+
+/* The Flash dual path computed router-first: ivc_vir_route, then each tile
+ * only through the path it was routed to (mlp2 at 0.25 for mask[t] = 1, mlp1
+ * at 0.5 otherwise), the last Linear of each MLP storing the tile's rows
+ * straight at out rows [offsets[t], offsets[t+1]). The pages compute both
+ * paths for every tile and then keep one ([DP] "双路压缩管线全流程拆解");
+ * the kept rows are the same, the discarded path is never computed.
+ * Arguments, results, workspace size (IVC_OP_FLASH_COMPRESS) and errors are
+ * those of ivc_flash_compress; every step runs on `stream`, and the router
+ * runs as in ivc_vir_route. */
+int ivc_flash_compress_routed(const void* x, const int32_t* valid_len, int T, int C,
+                              const int32_t* image_offsets, int I, const ivc_mlp* mlp1,
+                              const ivc_mlp* mlp2, const ivc_router* r, void* out, float* gate,
+                              uint8_t* mask, int32_t* offsets, int32_t* total, void* workspace,
+                              size_t ws_bytes, ivc_stream_t stream);
 
 /* Synchronise `stream`, copy the workspace's device status word to *bits and
  * clear it. Returns IVC_OK when no bit was set, IVC_EDEVICE otherwise. */

@@ -95,3 +95,36 @@ def test_entry_points_reject_bad_arguments_without_touching_the_gpu():
     assert L.ivc_vir_route(x, None, 1, 512, x, 1, P(r), y, y, y, ws, 1 << 40, None) == -2
     r.quantile_scope = 3
     assert L.ivc_vir_route(x, None, 1, 1024, x, 1, P(r), y, y, y, ws, 1 << 40, None) == -1
+
+
+@pytest.mark.parametrize("name", ["ivc_flash_compress", "ivc_flash_compress_routed"])
+def test_flash_entry_points_reject_bad_arguments(name):
+    """Both flash flows share their argument checks; none reaches the GPU."""
+    import vlm_visual_token_b200 as ivc
+    L = ivc.lib()
+    fn = getattr(L, name)
+    m1 = _mlp([4096, 2048, 2048])
+    m2 = _mlp([16384, 4096, 2048, 2048])
+    m2_bad = _mlp([16384, 4096, 2048, 1024])  # output width differs from mlp1's
+    r = ivc._CRouter()
+    r.D, r.heads, r.gate_hidden = 1024, 16, 1024
+    r.query = r.gWout = 1 << 28
+    for k in ("Wq", "Wk", "Wv", "Wo", "gW1", "gW2", "gln_g", "gln_b"):
+        arr = getattr(r, k)
+        for l in range(4):
+            arr[l] = 1 << 28
+    ws = ctypes.c_void_p(1 << 20)
+    x = ctypes.c_void_p(1 << 24)
+    y = ctypes.c_void_p(1 << 26)
+    P = ctypes.byref
+
+    def call(T=1, C=1024, mlp2=m2, out=y, nbytes=1 << 40, xx=x):
+        return fn(xx, None, T, C, x, 1, P(m1), P(mlp2), P(r), out, y, y, y, y, ws, nbytes, None)
+
+    assert call(T=-1) == -1
+    assert call(mlp2=m2_bad) == -2
+    assert call(C=512) == -2
+    assert call(out=None) == -1
+    assert call(out=ctypes.c_void_p((1 << 26) + 4)) == -6
+    assert call(nbytes=64) == -3
+    assert call(xx=ctypes.c_void_p((1 << 24) + 2)) == -6

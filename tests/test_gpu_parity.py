@@ -128,7 +128,7 @@ def test_large_connector_sampled_tiles(name):
 
 
 # ------------------------------------------------------------------ router
-def _route_check(ivc, inp, gate, mask, offsets, sample=None, scope=0):
+def _route_check(ivc, inp, gate, mask, offsets, sample=None, scope=0, rel_q=0.1, abs_t=0.5):
     x64 = O.to64(inp["x"])
     T = inp["T"]
     tiles = list(range(T)) if sample is None else sample
@@ -141,7 +141,7 @@ def _route_check(ivc, inp, gate, mask, offsets, sample=None, scope=0):
     assert err <= GATE_ABS, err
     # routing and offsets: bit-exact given the GPU's own fp32 gate vector
     ref_mask = O.route(g[:, 0].astype(np.float32).astype(np.float64), inp["image_offsets"].numpy(),
-                       0.1, 0.5, scope="batch" if scope else "image")
+                       rel_q, abs_t, scope="batch" if scope else "image")
     np.testing.assert_array_equal(to_np(mask), ref_mask)
     np.testing.assert_array_equal(to_np(offsets), O.compaction_offsets(ref_mask))
     return err
@@ -214,14 +214,14 @@ def test_bad_image_offsets_sets_status_bit():
 
 
 # ------------------------------------------------------------------ whole path
-def _flash_check(ivc, inp, res, tiles=None):
+def _flash_check(ivc, inp, res, tiles=None, rel_q=0.1, abs_t=0.5):
     T, H = inp["T"], inp["H"]
     x64 = O.to64(inp["x"])
     sel = list(range(T)) if tiles is None else tiles
     Y256 = O.ps_project(x64[sel], 0.5, O.to64(inp["mlp1"]))
     Y64 = O.ps_project(x64[sel], 0.25, O.to64(inp["mlp2"]))
     gate, mask, offsets = res["gate"], res["mask"], res["offsets"]
-    _route_check(ivc, inp, gate, mask, offsets, sample=tiles)
+    _route_check(ivc, inp, gate, mask, offsets, sample=tiles, rel_q=rel_q, abs_t=abs_t)
     offs = to_np(offsets)
     m = to_np(mask)
     assert int(to_np(res["total"])[0]) == offs[-1] == 256 * (T - m.sum()) + 64 * m.sum()
@@ -291,3 +291,103 @@ def test_flash_4b_batched_sampled(pool_mode):
     rng = np.random.default_rng(11)
     tiles = sorted(set(padded[:4] + rng.choice(T, 6, replace=False).tolist() + [T - 1]))
     _flash_check(ivc, inp, res, tiles=tiles)
+
+
+# ---------------------------------------------------------------- router-first flow
+def _routed_vs_dual(ivc, inp, m1, m2, r, routed_res):
+    """Rows of tiles routed alike in both flows are bit-identical: each output
+    row of a GEMM depends only on its own input row."""
+    dual = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(), inp["image_offsets"].cuda(),
+                              m1, m2, r)
+    torch.cuda.synchronize()
+    md, mr = to_np(dual["mask"]), to_np(routed_res["mask"])
+    od, orr = to_np(dual["offsets"]), to_np(routed_res["offsets"])
+    same = 0
+    for t in range(inp["T"]):
+        if md[t] != mr[t]:
+            continue
+        a = dual["out"][od[t]:od[t + 1]]
+        b = routed_res["out"][orr[t]:orr[t + 1]]
+        assert torch.equal(a, b), f"tile {t}: routed rows differ from the dual-path rows"
+        same += 1
+    assert same > 0
+
+
+@pytest.mark.parametrize("pool_mode", [0, 1])
+def test_flash_routed_small(pool_mode):
+    ivc = _ivc()
+    inp = W.make(small_workload(C=256, H=192, tiles=(3, 1, 4), var=0.3), affine="random")
+    m1, m2 = ivc.Mlp(inp["mlp1"]), ivc.Mlp(inp["mlp2"]).fold()
+    r = ivc.Router(inp["router"], pool_mode=pool_mode)
+    ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_FLASH, inp["T"], 256, m1, m2, r))
+    res = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(), inp["image_offsets"].cuda(),
+                             m1, m2, r, workspace=ws, routed=True)
+    torch.cuda.synchronize()
+    assert ivc.device_status(ws) == 0
+    _flash_check(ivc, inp, res)
+    _routed_vs_dual(ivc, inp, m1, m2, r, res)
+
+
+@pytest.mark.parametrize("abs_t,rel_q", [(1.5, 0.1), (0.0, 0.0)])
+def test_flash_routed_one_path_only(abs_t, rel_q):
+    """abs_t 1.5: no tile is compressed (the mlp2 launches see zero rows);
+    abs_t 0 with rel_q 0: every tile but each image's lowest gate is."""
+    ivc = _ivc()
+    inp = W.make(small_workload(C=256, H=128, tiles=(5, 2), var=0.0))
+    m1, m2 = ivc.Mlp(inp["mlp1"]).fold(), ivc.Mlp(inp["mlp2"]).fold()
+    r = ivc.Router(inp["router"], rel_q=rel_q, abs_t=abs_t)
+    res = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(), inp["image_offsets"].cuda(),
+                             m1, m2, r, routed=True)
+    torch.cuda.synchronize()
+    m = to_np(res["mask"])
+    if abs_t > 1:
+        assert m.sum() == 0
+    else:
+        assert m.sum() == inp["T"] - 2
+    _flash_check(ivc, inp, res, rel_q=rel_q, abs_t=abs_t)
+
+
+def test_flash_routed_empty():
+    ivc = _ivc()
+    inp = W.make(small_workload(C=256, H=128, tiles=(1,)))
+    m1, m2, r = ivc.Mlp(inp["mlp1"]), ivc.Mlp(inp["mlp2"]), ivc.Router(inp["router"])
+    x = torch.empty(0, 32, 32, 256, dtype=torch.bfloat16, device="cuda")
+    res = ivc.flash_compress(x, None, torch.zeros(1, dtype=torch.int32, device="cuda"), m1, m2, r,
+                             routed=True)
+    torch.cuda.synchronize()
+    assert int(res["total"].item()) == 0 and int(res["offsets"][0].item()) == 0
+
+
+def test_flash_routed_2b_13tiles_full():
+    """The benchmark workload through the router-first flow, every output
+    row checked against the oracle and against the dual-path flow."""
+    ivc = _ivc()
+    inp = W.make("flash_2b_13tiles")
+    m1, m2 = ivc.Mlp(inp["mlp1"]).fold(), ivc.Mlp(inp["mlp2"]).fold()
+    r = ivc.Router(inp["router"])
+    res = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(), inp["image_offsets"].cuda(),
+                             m1, m2, r, routed=True)
+    torch.cuda.synchronize()
+    stats = _flash_check(ivc, inp, res)
+    assert max(s["max_abs"] for s in stats) <= 3e-2, stats
+    _routed_vs_dual(ivc, inp, m1, m2, r, res)
+
+
+def test_flash_routed_4b_batched_sampled():
+    """97 tiles in 16 images: odd per-path tile counts, many m-tiles and CTA
+    pairs spanning two listed tiles of the factor-0.25 path."""
+    ivc = _ivc()
+    inp = W.make("flash_4b_batched")
+    T = inp["T"]
+    m1, m2 = ivc.Mlp(inp["mlp1"]).fold(), ivc.Mlp(inp["mlp2"]).fold()
+    r = ivc.Router(inp["router"])
+    ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_FLASH, T, 1024, m1, m2, r))
+    res = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(), inp["image_offsets"].cuda(),
+                             m1, m2, r, workspace=ws, routed=True)
+    torch.cuda.synchronize()
+    assert ivc.device_status(ws) == 0
+    padded = np.nonzero(inp["valid_len"].numpy() < 1024)[0].tolist()
+    rng = np.random.default_rng(12)
+    tiles = sorted(set(padded[:4] + rng.choice(T, 6, replace=False).tolist() + [T - 1]))
+    _flash_check(ivc, inp, res, tiles=tiles)
+    _routed_vs_dual(ivc, inp, m1, m2, r, res)

@@ -92,6 +92,8 @@ def lib() -> ctypes.CDLL:
                                          ctypes.POINTER(_CMlp), ctypes.POINTER(_CMlp),
                                          ctypes.POINTER(_CRouter), _vp, _vp, _vp, _vp, _vp, _vp,
                                          ctypes.c_size_t, _vp]
+        L.ivc_flash_compress_routed.restype = ctypes.c_int
+        L.ivc_flash_compress_routed.argtypes = L.ivc_flash_compress.argtypes
         L.ivc_device_status.restype = ctypes.c_int
         L.ivc_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int), _vp]
         _LIB = L
@@ -235,7 +237,10 @@ def vir_route(x: torch.Tensor, valid_len: Optional[torch.Tensor], image_offsets:
 def flash_compress(x: torch.Tensor, valid_len: Optional[torch.Tensor], image_offsets: torch.Tensor,
                    mlp1: Mlp, mlp2: Mlp, r: Router, out: Optional[torch.Tensor] = None,
                    workspace: Optional[torch.Tensor] = None, bufs: Optional[dict] = None,
-                   stream=None) -> dict:
+                   stream=None, routed: bool = False) -> dict:
+    """ivc_flash_compress (both paths for every tile, then compaction), or with
+    routed=True ivc_flash_compress_routed (router first, each tile through its
+    selected path only); same results."""
     T, _, _, C = x.shape
     dev = x.device
     H = mlp1.out_dim
@@ -249,12 +254,13 @@ def flash_compress(x: torch.Tensor, valid_len: Optional[torch.Tensor], image_off
     if workspace is None:
         workspace = new_workspace(workspace_size(OP_FLASH, T, C, mlp1, mlp2, r), dev)
     I = int(image_offsets.numel()) - 1
-    _check(lib().ivc_flash_compress(_ptr(x), _ptr(valid_len), T, C, _ptr(image_offsets), I,
-                                    ctypes.byref(mlp1.c), ctypes.byref(mlp2.c), ctypes.byref(r.c),
-                                    _ptr(out), _ptr(bufs["gate"]), _ptr(bufs["mask"]),
-                                    _ptr(bufs["offsets"]), _ptr(bufs["total"]), _ptr(workspace),
-                                    workspace.numel(), _stream(stream)),
-           "ivc_flash_compress")
+    fn = lib().ivc_flash_compress_routed if routed else lib().ivc_flash_compress
+    _check(fn(_ptr(x), _ptr(valid_len), T, C, _ptr(image_offsets), I,
+              ctypes.byref(mlp1.c), ctypes.byref(mlp2.c), ctypes.byref(r.c),
+              _ptr(out), _ptr(bufs["gate"]), _ptr(bufs["mask"]),
+              _ptr(bufs["offsets"]), _ptr(bufs["total"]), _ptr(workspace),
+              workspace.numel(), _stream(stream)),
+           "ivc_flash_compress_routed" if routed else "ivc_flash_compress")
     res = dict(bufs)
     res["out"] = out
     return res

@@ -154,9 +154,19 @@ void carve_route(Carver& cv, const ivc_router* r, int T, RouteBufs& b) {
     if (_rc != IVC_OK) return _rc; \
   } while (0)
 
-// pixel_shuffle + MLP with the statistics already in b.mean / b.rstd.
+// Tiles routed to one path (router-first flow), all on the device: the
+// listed tile ids, their count, and the first output row of each.
+struct Routed {
+  const int* list;
+  const int* count;
+  const int* base;
+};
+
+// pixel_shuffle + MLP with the statistics already in b.mean / b.rstd. With
+// rt, only the listed tiles are computed (rows in list order) and the last
+// Linear stores each tile's rows at its output offset in y.
 int ps_mlp(const void* x, int T, int C, bool half, int flags, const ivc_mlp* m, bf16* y,
-           const PsBufs& b, const Launch& L) {
+           const PsBufs& b, const Launch& L, const Routed* rt = nullptr) {
   static const char* const kTags[2][3] = {{"mlp2.fc1", "mlp2.fc2", "mlp2.fc3"},
                                           {"mlp1.fc1", "mlp1.fc2", "mlp1.fc3"}};
   const long long rows = static_cast<long long>(T) * (half ? 256 : 64);
@@ -192,6 +202,13 @@ int ps_mlp(const void* x, int T, int C, bool half, int flags, const ivc_mlp* m, 
   c.row_rstd = b.rstd;
   c.out = b.h1;
   c.ldo = m->dims[1];
+  const int item_rows = half ? 256 : 64;
+  if (rt) {
+    c.list = rt->list;
+    c.list_count = rt->count;
+    c.item_rows = item_rows;
+    c.stats_remap = 1;
+  }
   IVC_TRY(launch_gemm(c, L));
   const bf16* a = b.h1;
   for (int i = 1; i < m->n_linear; ++i) {
@@ -211,6 +228,11 @@ int ps_mlp(const void* x, int T, int C, bool half, int flags, const ivc_mlp* m, 
     d.remap = last ? remap : 0;
     d.out = last ? y : b.h2;
     d.ldo = m->dims[i + 1];
+    if (rt) {
+      d.list_count = rt->count;
+      d.item_rows = item_rows;
+      d.out_base = last ? rt->base : nullptr;
+    }
     IVC_TRY(launch_gemm(d, L));
     a = b.h2;
   }
@@ -274,11 +296,14 @@ int folded_layer(const void* x, const int32_t* valid_len, int T, const ivc_route
                            static_cast<const bf16*>(r->bv[l]), b.O, L);
 }
 
+// fused_default: use the persistent single-launch router when it applies and
+// IVC_ROUTER_FUSED does not say otherwise. It holds every SM for its whole
+// run, so it is the default only where nothing runs beside the router.
 int route_impl(const void* x, const int32_t* valid_len, int T, const int32_t* image_offsets,
                int I, const ivc_router* r, float* gate, uint8_t* mask, int32_t* offsets,
-               int32_t* total, const RouteBufs& b, const Launch& L) {
+               int32_t* total, const RouteBufs& b, const Launch& L, bool fused_default) {
   const int D = r->D;
-  if (r->pool_mode == IVC_POOL_FOLDED && router_fused_enabled()) {
+  if (router_fused_supported(r) && router_fused_wanted(fused_default)) {
     FusedRouterBufs f{b.Q, b.U2, b.cb, b.S, b.P2, b.z, b.O, b.q, b.h, b.u1, b.u2, b.bar};
     return launch_router_fused(r, x, valid_len, T, image_offsets, I, gate, mask, offsets, total,
                                f, L);
@@ -412,15 +437,48 @@ size_t route_ws(int T, const ivc_router* r) {
   return cv.off;
 }
 
+// Routed tile lists of the router-first flow: list_u, base_u, list_c,
+// base_c [T] and the two counts.
+struct ListBufs {
+  int* list_u;
+  int* base_u;
+  int* list_c;
+  int* base_c;
+  int* counts;
+};
+
+void carve_lists(Carver& cv, int T, ListBufs& l) {
+  l.list_u = cv.take<int>(T);
+  l.base_u = cv.take<int>(T);
+  l.list_c = cv.take<int>(T);
+  l.base_c = cv.take<int>(T);
+  l.counts = cv.take<int>(2);
+}
+
+// One layout for both flash flows (dual path and router-first), so that one
+// workspace size serves either entry point.
+struct FlashBufs {
+  PsBufs b1, b2;
+  bf16* Y256;
+  bf16* Y64;
+  RouteBufs br;
+  ListBufs lists;
+};
+
+void carve_flash(Carver& cv, int T, const ivc_mlp* m1, const ivc_mlp* m2, const ivc_router* r,
+                 FlashBufs& f) {
+  carve_ps(cv, m1, static_cast<long long>(T) * 256, true, f.b1);
+  carve_ps(cv, m2, static_cast<long long>(T) * 64, true, f.b2);
+  f.Y256 = cv.take<bf16>(static_cast<size_t>(T) * 256 * m1->dims[m1->n_linear]);
+  f.Y64 = cv.take<bf16>(static_cast<size_t>(T) * 64 * m2->dims[m2->n_linear]);
+  carve_route(cv, r, T, f.br);
+  carve_lists(cv, T, f.lists);
+}
+
 size_t flash_ws(int T, const ivc_mlp* m1, const ivc_mlp* m2, const ivc_router* r) {
   Carver cv(nullptr);
-  PsBufs b1, b2;
-  RouteBufs br;
-  carve_ps(cv, m1, static_cast<long long>(T) * 256, true, b1);
-  carve_ps(cv, m2, static_cast<long long>(T) * 64, true, b2);
-  cv.take<bf16>(static_cast<size_t>(T) * 256 * m1->dims[m1->n_linear]);
-  cv.take<bf16>(static_cast<size_t>(T) * 64 * m2->dims[m2->n_linear]);
-  carve_route(cv, r, T, br);
+  FlashBufs f;
+  carve_flash(cv, T, m1, m2, r, f);
   return cv.off;
 }
 
@@ -537,7 +595,8 @@ int ivc_vir_route(const void* x, const int32_t* valid_len, int T, int C,
   Carver cv(workspace);
   RouteBufs b;
   carve_route(cv, r, T, b);
-  return route_impl(x, valid_len, T, image_offsets, I, r, gate, mask, offsets, nullptr, b, L);
+  return route_impl(x, valid_len, T, image_offsets, I, r, gate, mask, offsets, nullptr, b, L,
+                    true);
 }
 
 int ivc_flash_compress(const void* x, const int32_t* valid_len, int T, int C,
@@ -562,13 +621,13 @@ int ivc_flash_compress(const void* x, const int32_t* valid_len, int T, int C,
   }
   Launch L{s, static_cast<int*>(workspace)};
   Carver cv(workspace);
-  PsBufs b1, b2;
-  RouteBufs br;
-  carve_ps(cv, mlp1, static_cast<long long>(T) * 256, true, b1);
-  carve_ps(cv, mlp2, static_cast<long long>(T) * 64, true, b2);
-  bf16* Y256 = cv.take<bf16>(static_cast<size_t>(T) * 256 * H);
-  bf16* Y64 = cv.take<bf16>(static_cast<size_t>(T) * 64 * H);
-  carve_route(cv, r, T, br);
+  FlashBufs f;
+  carve_flash(cv, T, mlp1, mlp2, r, f);
+  const PsBufs& b1 = f.b1;
+  const PsBufs& b2 = f.b2;
+  bf16* Y256 = f.Y256;
+  bf16* Y64 = f.Y64;
+  const RouteBufs& br = f.br;
   // The router (own buffers) runs on the side stream while the connector runs
   // on the caller's stream; they meet before compaction.
   SideStream* side = nullptr;
@@ -576,7 +635,8 @@ int ivc_flash_compress(const void* x, const int32_t* valid_len, int T, int C,
   Launch R{side->stream, L.status};
   IVC_TRY(cu_check(cudaEventRecord(side->fork, s)));
   IVC_TRY(cu_check(cudaStreamWaitEvent(side->stream, side->fork, 0)));
-  int rc = route_impl(x, valid_len, T, image_offsets, I, r, gate, mask, offsets, total, br, R);
+  int rc =
+      route_impl(x, valid_len, T, image_offsets, I, r, gate, mask, offsets, total, br, R, false);
   // join even on failure so that the caller's stream never runs ahead of work
   // already enqueued on the side stream
   const int rc_rec = cu_check(cudaEventRecord(side->join, side->stream));
@@ -589,6 +649,46 @@ int ivc_flash_compress(const void* x, const int32_t* valid_len, int T, int C,
   if (rc != IVC_OK) return rc;
   if (rc_wait != IVC_OK) return rc_wait;
   return launch_compact(Y256, Y64, mask, offsets, T, H, static_cast<bf16*>(out), L);
+}
+
+int ivc_flash_compress_routed(const void* x, const int32_t* valid_len, int T, int C,
+                              const int32_t* image_offsets, int I, const ivc_mlp* mlp1,
+                              const ivc_mlp* mlp2, const ivc_router* r, void* out, float* gate,
+                              uint8_t* mask, int32_t* offsets, int32_t* total, void* workspace,
+                              size_t ws_bytes, ivc_stream_t stream) {
+  if (T < 0 || C <= 0 || I < 0) return IVC_EINVAL;
+  IVC_TRY(ps_args_ok(x, T, C, mlp1, true));
+  IVC_TRY(ps_args_ok(x, T, C, mlp2, false));
+  const int H = mlp1->dims[mlp1->n_linear];
+  if (mlp2->dims[mlp2->n_linear] != H) return IVC_EUNSUPPORTED;
+  IVC_TRY(router_shape_ok(r, C));
+  if (!offsets || !total || (T > 0 && (!out || !gate || !mask))) return IVC_EINVAL;
+  if (T > 0 && r->quantile_scope == 0 && !image_offsets) return IVC_EINVAL;
+  if (!aligned16(out)) return IVC_EALIGN;
+  IVC_TRY(check_ws(workspace, ws_bytes, flash_ws(T, mlp1, mlp2, r)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    IVC_TRY(cu_check(cudaMemsetAsync(offsets, 0, sizeof(int32_t), s)));
+    return cu_check(cudaMemsetAsync(total, 0, sizeof(int32_t), s));
+  }
+  Launch L{s, static_cast<int*>(workspace)};
+  Carver cv(workspace);
+  FlashBufs f;
+  carve_flash(cv, T, mlp1, mlp2, r, f);
+  // Router first: it needs only x. Then each tile runs through the path it
+  // was routed to, and the last Linear of each MLP stores its rows at the
+  // tile's output offset, so no compaction pass remains.
+  IVC_TRY(launch_ps_stats(static_cast<const bf16*>(x), T, C, f.b1.mean, f.b1.rstd, f.b2.mean,
+                          f.b2.rstd, L));
+  IVC_TRY(route_impl(x, valid_len, T, image_offsets, I, r, gate, mask, offsets, total, f.br, L,
+                     true));
+  const ListBufs& lb = f.lists;
+  IVC_TRY(launch_route_lists(mask, offsets, T, lb.list_u, lb.base_u, lb.list_c, lb.base_c,
+                             lb.counts, L));
+  const Routed ru{lb.list_u, lb.counts, lb.base_u};
+  const Routed rc{lb.list_c, lb.counts + 1, lb.base_c};
+  IVC_TRY(ps_mlp(x, T, C, true, 0, mlp1, static_cast<bf16*>(out), f.b1, L, &ru));
+  return ps_mlp(x, T, C, false, 0, mlp2, static_cast<bf16*>(out), f.b2, L, &rc);
 }
 
 int ivc_device_status(void* workspace, int* bits, ivc_stream_t stream) {

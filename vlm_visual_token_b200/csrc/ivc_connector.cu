@@ -187,6 +187,10 @@ static int map_2d(CUtensorMap* m, const void* base, long long rows, long long co
   return encode(m, 2, base, dims, strides, box);
 }
 
+int map_rows_2d(CUtensorMap* m, const void* base, long long rows, long long cols, int box_rows) {
+  return map_2d(m, base, rows, cols, box_rows);
+}
+
 // Batched [batches][rows][inner] bf16 (row stride ld, batch stride bs elements),
 // box {box_inner, box_rows, 1}.
 static int map_3d(CUtensorMap* m, const void* base, long long batches, long long rows,
@@ -198,8 +202,9 @@ static int map_3d(CUtensorMap* m, const void* base, long long batches, long long
   return encode(m, 3, base, dims, strides, box);
 }
 
-// The [T,32,32,C] features seen as the pixel-shuffled [T*tokens, f*f*C] matrix.
-static int map_ps(CUtensorMap* m, const void* x, int T, int C, int f) {
+// The [T,32,32,C] features seen as the pixel-shuffled [T*tokens, f*f*C] matrix;
+// one box is 128 rows, or (one_tile, f = 4) the 64 rows of one tile.
+static int map_ps(CUtensorMap* m, const void* x, int T, int C, int f, bool one_tile = false) {
   const cuuint64_t Cu = static_cast<cuuint64_t>(C);
   const int g = 32 / f;  // output grid side
   cuuint64_t dims[5] = {Cu, static_cast<cuuint64_t>(f), static_cast<cuuint64_t>(g),
@@ -207,8 +212,8 @@ static int map_ps(CUtensorMap* m, const void* x, int T, int C, int f) {
   // strides (bytes) of dims 1..4: next column in the block, next output
   // column b, next row in the block, next output row (a) / tile.
   cuuint64_t strides[4] = {Cu * 2, Cu * f * 2, Cu * 32 * 2, Cu * 32 * f * 2};
-  cuuint32_t box[5] = {GEMM_BK, 1, static_cast<cuuint32_t>(g), 1,
-                       static_cast<cuuint32_t>(GEMM_BM / g)};
+  const int outer = one_tile && g * g < GEMM_BM ? g : GEMM_BM / g;
+  cuuint32_t box[5] = {GEMM_BK, 1, static_cast<cuuint32_t>(g), 1, static_cast<cuuint32_t>(outer)};
   return encode(m, 5, x, dims, strides, box);
 }
 
@@ -294,7 +299,7 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
   switch (c.a_mode) {
     case A_PLAIN: rc = map_2d(&maps.a, c.a, c.M, c.K, GEMM_BM); break;
     case A_PS_HALF: rc = map_ps(&maps.a, c.a, c.T, c.C, 2); break;
-    default: rc = map_ps(&maps.a, c.a, c.T, c.C, 4); break;
+    default: rc = map_ps(&maps.a, c.a, c.T, c.C, 4, c.list != nullptr); break;
   }
   if (rc) return rc;
   for (int g = 0; g < c.groups; ++g) {
@@ -333,6 +338,16 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
   a.fbias = c.fbias;
   a.row_mean = c.row_mean;
   a.row_rstd = c.row_rstd;
+  a.list = c.list;
+  a.list_count = c.list_count;
+  a.out_base = c.out_base;
+  a.item_rows = c.item_rows;
+  a.stats_remap = c.stats_remap;
+  if (c.list_count != nullptr && (c.item_rows <= 0 || (c.item_rows != 256 && c.item_rows != 64)))
+    return IVC_EINVAL;
+  if ((c.list != nullptr || c.stats_remap || c.out_base != nullptr) && c.list_count == nullptr)
+    return IVC_EINVAL;
+  if (c.stats_remap && c.list == nullptr) return IVC_EINVAL;
   switch (bn) {
     case 256: return cg == 2 ? run_gemm<256, 6, 2>(maps, a, c.tag, L)
                              : run_gemm<256, 4, 1>(maps, a, c.tag, L);

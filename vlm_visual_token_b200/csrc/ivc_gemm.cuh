@@ -84,6 +84,17 @@ struct GemmArgs {
   const float* fbias;            // EPI_LNFOLD
   const float* row_mean;         // EPI_LNFOLD
   const float* row_rstd;         // EPI_LNFOLD
+  // Routed rows (router-first flow). With list_count set, the row count is
+  // *list_count * item_rows (read on the device, at most M): the rows of the
+  // listed tiles in list order. The pixel_shuffle A modes then address tile
+  // list[row / item_rows]; stats_remap reads the LN statistics of that tile's
+  // row; out_base (if set) stores row r at out_base[r / item_rows] + r % item_rows
+  // (after the v1 remap inside the tile) instead of at r.
+  const int* list;
+  const int* list_count;
+  const int* out_base;
+  int item_rows;
+  int stats_remap;
 };
 
 template <int BN, int STAGES, int CG = 1>
@@ -149,9 +160,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const int rank = CG == 2 ? static_cast<int>(cluster_ctarank()) : 0;
   const int unit = blockIdx.x / CG;     // this CTA (pair) in the persistent grid
   const int n_units = gridDim.x / CG;
-  const int m_tiles = (args.M + TILE_M - 1) / TILE_M;
   const int n_tiles = (args.N + BN - 1) / BN;
-  const int n_total = m_tiles * n_tiles * args.groups;
   const int KT = args.K / GEMM_BK;
 
   if (warp == 0 && lane == 0) {
@@ -185,6 +194,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   // operands and outputs may belong to the previous kernel in the stream
   pdl_wait();
   pdl_trigger();
+  int M = args.M;
+  if (args.list_count != nullptr) {
+    const int c = *args.list_count;
+    const long long rows = static_cast<long long>(c < 0 ? 0 : c) * args.item_rows;
+    M = rows < M ? static_cast<int>(rows) : M;
+  }
+  const int m_tiles = (M + TILE_M - 1) / TILE_M;
+  const int n_total = m_tiles * n_tiles * args.groups;
+  const int n_listed = args.list_count != nullptr ? M / args.item_rows : 0;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -211,6 +229,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           uint8_t* b_dst = a_dst + L::A_BYTES;
           int ac[5];
           int a_rank = 2;
+          int ac4b = -1;  // routed factor 0.25: outer coordinate of the second 64-row box
           if (args.a_mode == A_PLAIN) {
             ac[0] = kk * GEMM_BK;
             ac[1] = my_m0;
@@ -220,6 +239,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             a_rank = 5;
             if (args.a_mode == A_PS_HALF) {
               ac[0] = c0; ac[1] = blk & 1; ac[2] = 0; ac[3] = blk >> 1; ac[4] = my_m0 >> 4;
+              if (args.list != nullptr)  // 128 rows = half of listed tile my_m0 / 256
+                ac[4] = args.list[my_m0 >> 8] * 16 + ((my_m0 >> 4) & 15);
             } else {
               int q, r;
               if (args.a_mode == A_PS_QUARTER) {
@@ -230,21 +251,36 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 r = 2 * ((blk >> 2) & 1) + (blk & 1);
               }
               ac[0] = c0; ac[1] = r; ac[2] = 0; ac[3] = q; ac[4] = my_m0 >> 3;
+              if (args.list != nullptr) {
+                // 128 rows = listed tiles j and j + 1 (64 rows each, one box
+                // apiece); past the last one, j again (rows >= M, not stored)
+                const int j = my_m0 >> 6;
+                ac[4] = args.list[j < n_listed ? j : (n_listed > 0 ? n_listed - 1 : 0)] * 8;
+                ac4b = args.list[j + 1 < n_listed ? j + 1 : (n_listed > 0 ? n_listed - 1 : 0)] * 8;
+              }
             }
           }
           if constexpr (CG == 2) {
             const uint32_t lb = pair_leader_addr(&full_bar[s]);
-            if (a_rank == 2)
+            if (a_rank == 2) {
               tma_load_2d_pair(a_dst, &maps.a, lb, ac[0], ac[1]);
-            else
+            } else {
               tma_load_5d_pair(a_dst, &maps.a, lb, ac[0], ac[1], ac[2], ac[3], ac[4]);
+              if (ac4b >= 0)
+                tma_load_5d_pair(a_dst + L::A_BYTES / 2, &maps.a, lb, ac[0], ac[1], ac[2], ac[3],
+                                 ac4b);
+            }
             tma_load_2d_pair(b_dst, &maps.b[tc.g], lb, kk * GEMM_BK, my_n0);
             continue;
           }
-          if (a_rank == 2)
+          if (a_rank == 2) {
             tma_load_2d(a_dst, &maps.a, &full_bar[s], ac[0], ac[1]);
-          else
+          } else {
             tma_load_5d(a_dst, &maps.a, &full_bar[s], ac[0], ac[1], ac[2], ac[3], ac[4]);
+            if (ac4b >= 0)
+              tma_load_5d(a_dst + L::A_BYTES / 2, &maps.a, &full_bar[s], ac[0], ac[1], ac[2], ac[3],
+                          ac4b);
+          }
           const CUtensorMap* bm = &maps.b[tc.g];
           if (args.b_mode == B_K2D) {
             tma_load_2d(b_dst, bm, &full_bar[s], kk * GEMM_BK, tc.n0);
@@ -336,9 +372,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       tc_fence_after();
       const int row = tc.m0 + GEMM_BM * rank + quad * 32 + lane;
       float mean = 0.f, rstd = 1.f;
-      if (args.epi_mode == EPI_LNFOLD && row < args.M) {
-        mean = args.row_mean[row];
-        rstd = args.row_rstd[row];
+      if (args.epi_mode == EPI_LNFOLD && row < M) {
+        const int sr = args.stats_remap
+                           ? args.list[row / args.item_rows] * args.item_rows + row % args.item_rows
+                           : row;
+        mean = args.row_mean[sr];
+        rstd = args.row_rstd[sr];
       }
       const float nms = -mean * rstd;
       long long out_row = row;
@@ -349,6 +388,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         const int t = row & 63;
         out_row = (row & ~63) | ((t & 7) << 3) | (t >> 3);
       }
+      if (args.out_base != nullptr && row < M)  // item_rows is 256 / 64, as the remaps
+        out_row = args.out_base[row / args.item_rows] + out_row % args.item_rows;
       const long long out_off =
           out_row * args.ldo + static_cast<long long>(tc.g) * args.group_col_stride + tc.n0;
       const uint32_t t_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
@@ -369,7 +410,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
               mbar_arrive(&tempty_bar[acc]);
           }
         }
-        if (row < args.M && tc.n0 + c < args.N && (args.m_valid == 0 || (row & 127) < args.m_valid)) {
+        if (row < M && tc.n0 + c < args.N && (args.m_valid == 0 || (row & 127) < args.m_valid)) {
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {

@@ -105,6 +105,13 @@ struct GemmCall {
   int out_f32;         // store fp32 (pooling K/V) instead of bf16
   int m_valid;         // >0: store only rows with (row % 128) < m_valid
   long long ldo;
+  // routed rows (router-first flow; GemmArgs in ivc_gemm.cuh): M is then the
+  // upper bound T * item_rows, the device count decides
+  const int* list;
+  const int* list_count;
+  const int* out_base;
+  int item_rows;
+  int stats_remap;
 };
 int launch_gemm(const GemmCall& c, const Launch& L);
 
@@ -144,9 +151,14 @@ struct FusedRouterBufs {
   float* u2;
   unsigned* bar;
 };
-// Folded pooling runs as one persistent cooperative kernel (grid barriers
-// between its phases) when IVC_ROUTER_FUSED=1; otherwise as separate kernels.
-bool router_fused_enabled();
+// Tensor map of a row-major [rows, cols] bf16 matrix, box 64 columns x
+// box_rows rows, 128-byte swizzle (ivc_connector.cu).
+int map_rows_2d(CUtensorMap* m, const void* base, long long rows, long long cols, int box_rows);
+// Folded pooling can run as one persistent cooperative kernel (grid barriers
+// between its phases) or as separate kernels. IVC_ROUTER_FUSED=1 / 0 forces
+// the choice; otherwise the caller's default_on decides.
+bool router_fused_wanted(bool default_on);
+bool router_fused_supported(const ivc_router* r);
 int launch_router_fused(const ivc_router* r, const void* x, const int32_t* valid_len, int T,
                         const int32_t* image_offsets, int I, float* gate, uint8_t* mask,
                         int32_t* offsets, int32_t* total, const FusedRouterBufs& b,
@@ -157,6 +169,11 @@ int launch_residual_ln(float* h, const float* u, const bf16* gamma, const bf16* 
 // gate[t] = softmax(Wout h[t] + bout), Wout [2, D].
 int launch_gate_head(const float* h, const bf16* Wout, const bf16* bout, int T, int D,
                      float* gate, const Launch& L);
+// From the routing mask and row offsets: the uncompressed tiles (list_u,
+// their first output rows base_u) and the compressed ones (list_c, base_c),
+// each in tile order; counts[0] = #uncompressed, counts[1] = #compressed.
+int launch_route_lists(const uint8_t* mask, const int32_t* offsets, int T, int* list_u,
+                       int* base_u, int* list_c, int* base_c, int* counts, const Launch& L);
 // Quantile + double threshold + row-count scan.
 int launch_route(const float* gate, int T, const int32_t* image_offsets, int I, double rel_q,
                  double abs_t, int scope, uint8_t* mask, int32_t* offsets, int32_t* total,

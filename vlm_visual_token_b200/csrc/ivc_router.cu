@@ -697,6 +697,70 @@ int launch_route(const float* gate, int T, const int32_t* image_offsets, int I, 
                   image_offsets, I, rel_q, abs_t, scope, mask, offsets, total, L.status);
 }
 
+// ---------------------------------------------------------------- routed lists
+// Single CTA (router-first flow). The compressed tiles, in tile order, are
+// list_c[0..n_c) with their first output rows base_c (= offsets[t]); the
+// others are list_u / base_u. n_u and n_c go to counts[0], counts[1].
+__global__ void __launch_bounds__(ROUTE_THREADS)
+    route_lists_kernel(const uint8_t* __restrict__ mask, const int32_t* __restrict__ offsets,
+                       int T, int* __restrict__ list_u, int* __restrict__ base_u,
+                       int* __restrict__ list_c, int* __restrict__ base_c,
+                       int* __restrict__ counts) {
+  __shared__ int s_warp[ROUTE_THREADS / 32];
+  __shared__ int s_carry;
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x == 0) s_carry = 0;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int base = 0; base < T; base += ROUTE_THREADS) {
+    const int i = base + threadIdx.x;
+    const int c = (i < T && mask[i]) ? 1 : 0;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int w = s_warp[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += v;
+      }
+      s_warp[lane] = w;
+    }
+    __syncthreads();
+    const int jc = (warp > 0 ? s_warp[warp - 1] : 0) + s_carry + incl - c;  // compressed before i
+    if (i < T) {
+      if (c) {
+        list_c[jc] = i;
+        base_c[jc] = offsets[i];
+      } else {
+        list_u[i - jc] = i;
+        base_u[i - jc] = offsets[i];
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == ROUTE_THREADS - 1) s_carry = jc + c;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    counts[0] = T - s_carry;
+    counts[1] = s_carry;
+  }
+}
+
+int launch_route_lists(const uint8_t* mask, const int32_t* offsets, int T, int* list_u,
+                       int* base_u, int* list_c, int* base_c, int* counts, const Launch& L) {
+  TraceScope ts("route.lists", L.stream);
+  return launch_k(route_lists_kernel, dim3(1), dim3(ROUTE_THREADS), 0, L.stream, 1, mask, offsets,
+                  T, list_u, base_u, list_c, base_c, counts);
+}
+
 // ---------------------------------------------------------------- compaction
 // Grid (T, 8): CTA (t, y) copies rows 32y..32y+31 of tile t when they exist
 // (64 rows for a compressed tile, 256 otherwise), 16 bytes per thread-step.

@@ -37,14 +37,18 @@ namespace {
 
 constexpr int RF_THREADS = 256;
 constexpr int RF_WARPS = RF_THREADS / 32;
-constexpr int RF_TOK = 1024;      // tokens per tile
-constexpr int RF_HD = 64;         // head width
-constexpr int RF_GEMV_COLS = 16;  // output columns per GEMV item (2 per warp)
-constexpr int RF_ROWS = 16;       // input rows staged per GEMV round
-constexpr int RF_MAXK = 2048;     // widest GEMV input
+constexpr int RF_TOK = 1024;    // tokens per tile
+constexpr int RF_HD = 64;       // head width
+constexpr int RF_MAXD = 1024;   // widest pooling width (scores staging)
+constexpr int RF_MAXK = 2048;   // widest projection input
+constexpr int GV_COLS = 8;      // output columns per projection item (one n8 MMA tile)
+constexpr int GV_ROWS = 16;     // input rows per projection round (one m16 MMA tile)
+constexpr int WS_BOX = 256;     // tokens per TMA box of the weighted-sum staging
+constexpr int WS_PPITCH = RF_TOK + 8;  // bf16 per staged P2 row
 
 struct RouterFusedArgs {
-  const bf16* x;  // [T, 1024, D]
+  CUtensorMap xmap;  // x as [T*1024, D], box 64 channels x WS_BOX tokens, 128-byte swizzle
+  const bf16* x;     // [T, 1024, D]
   const int32_t* valid_len;
   int T, D, G, heads;
   const bf16 *query, *Wq[4], *bq[4], *Wk[4], *bk[4], *Wv[4], *bv[4], *Wo[4], *bo[4];
@@ -79,15 +83,16 @@ __device__ __forceinline__ float gelu(float y) {
 
 // Grid-wide barrier over co-resident CTAs: one arrival counter that only
 // grows (barrier g completes when it reaches (g + 1) * gridDim.x), so no CTA
-// has to reset it; false after ~1 s without progress.
+// has to reset it. Arrival is a release reduction (this CTA's writes, ordered
+// by the __syncthreads before it, become visible with it), the wait an
+// acquire spin; false after ~1 s without progress.
 __device__ bool grid_sync(unsigned* bar, unsigned& gen) {
   __shared__ int s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
     const unsigned target = (gen + 1u) * gridDim.x;
-    __threadfence();
-    atomicAdd(bar, 1u);
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(bar), "r"(1u) : "memory");
     const long long t0 = clock64();
     while (true) {
       unsigned v;
@@ -97,9 +102,7 @@ __device__ bool grid_sync(unsigned* bar, unsigned& gen) {
         ok = 0;
         break;
       }
-      __nanosleep(20);
     }
-    __threadfence();
     s_ok = ok;
   }
   __syncthreads();
@@ -131,100 +134,123 @@ __device__ __forceinline__ void ldsm_x2_trans(uint32_t (&r)[2], const void* p) {
                : "=r"(r[0]), "=r"(r[1])
                : "r"(smem_u32(p)));
 }
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+// Orders this thread's later async-proxy (bulk copy / TMA) reads of global
+// memory after generic writes that other CTAs made before a grid barrier.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// Copies `rows` rows of `bytes` (multiple of 16) from src (row pitch
-// src_pitch bytes) into shared memory (row pitch dst_pitch bytes) with
-// 16-byte cp.async pieces, all in flight at once; caller commits/waits.
-__device__ __forceinline__ void async_rows(void* dst, int dst_pitch, const void* src,
-                                           long long src_pitch, int rows, int bytes) {
-  const int per_row = bytes >> 4;
-  const int n = rows * per_row;
-  for (int i = threadIdx.x; i < n; i += RF_THREADS) {
-    const int r = i / per_row, p = i - r * per_row;
-    cp_async16(static_cast<uint8_t*>(dst) + r * dst_pitch + p * 16,
-               static_cast<const uint8_t*>(src) + r * src_pitch + p * 16);
-  }
+// v = hi + lo with hi = bf16(v), lo = bf16(v - hi), two lanes packed per word.
+__device__ __forceinline__ void split_bf16x2(float2 v, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(v.x - __low2float(h), v.y - __high2float(h));
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
-// ------------------------------------------------------------------ GEMV phase
-// Y[m, n] = act(sum_k X(m)[k] W[n, k] + b[n]) for m < M. Items are blocks of
-// RF_GEMV_COLS columns (warp w owns columns 2w, 2w+1 of the item). The item's
-// weight rows (bf16) and up to RF_ROWS input rows (fp32, `row(m, c0)` = the
-// input row of output row m for the item's columns c0..) are staged with
-// cp.async in one go, then the dot products run from shared memory.
-// Shared memory: RF_ROWS*K*4 (x) + RF_GEMV_COLS*K*2 (w).
+// ------------------------------------------------------------------ projection phase
+// Y[m, n] = act(sum_k X(m)[k] W[n, k] + b[n]) for m < M (M = tiles, small).
+// Items are GV_COLS = 8 output columns (one n8 MMA tile). Per item the 8
+// weight rows (bf16, mbarrier 0) and up to 16 input rows (fp32, mbarrier 1;
+// `row(m, c0)` = the input row of output row m for columns c0..c0+7) are
+// brought into shared memory with bulk copies; warp w then multiplies the
+// k-range [w K/8, (w+1) K/8) with m16n8k16 MMAs, the fp32 inputs split into a
+// bf16 hi/lo pair (two MMAs per k-step, fp32 accumulate), and the 8 warps'
+// partial tiles are summed through shared memory. Shared memory:
+// x [16][K+8] f32 | w [8][K+8] bf16 | partials [8 warps][16][8] f32.
+__device__ __forceinline__ size_t gv_x_bytes(int K) {
+  return static_cast<size_t>(GV_ROWS) * (K + 8) * 4;
+}
+__device__ __forceinline__ size_t gv_w_bytes(int K) {
+  return static_cast<size_t>(GV_COLS) * (K + 8) * 2;
+}
+
+// Warp 0: the weight rows of item `item` into their slot, on mbarrier mb.
+__device__ __forceinline__ void gv_issue_w(const bf16* __restrict__ W, int K, int item,
+                                           uint8_t* sm, uint64_t* mb) {
+  const int lane = threadIdx.x & 31;
+  bf16* sw = reinterpret_cast<bf16*>(sm + gv_x_bytes(K));
+  if (lane == 0) mbar_arrive_expect_tx(mb, GV_COLS * K * 2);
+  __syncwarp();
+  if (lane < GV_COLS)
+    bulk_load(sw + lane * (K + 8), W + static_cast<size_t>(item * GV_COLS + lane) * K, K * 2, mb);
+}
+
 template <typename RowFn>
-__device__ void gemv_phase(int M, int K, int N, const bf16* __restrict__ W,
+__device__ bool gemv_phase(int M, int K, int N, const bf16* __restrict__ W,
                            const bf16* __restrict__ b, float* __restrict__ Y, int ldy, bool act,
-                           float* sx, RowFn row) {
+                           uint8_t* sm, uint64_t* mb, uint32_t* ph, bool w_prefetched, RowFn row) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_items = (N + RF_GEMV_COLS - 1) / RF_GEMV_COLS;
-  bf16* sw = reinterpret_cast<bf16*>(sx + RF_ROWS * K);
+  const int g = lane >> 2, t2 = (lane & 3) * 2;
+  const int pitch = K + 8;
+  float* sx = reinterpret_cast<float*>(sm);
+  const bf16* sw = reinterpret_cast<const bf16*>(sm + gv_x_bytes(K));
+  float* red = reinterpret_cast<float*>(sm + gv_x_bytes(K) + gv_w_bytes(K));
+  const int n_items = N / GV_COLS;
+  const int kw = K / RF_WARPS;
+  bool first = true;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-    const int c0 = item * RF_GEMV_COLS;
-    const int wrows = min(RF_GEMV_COLS, N - c0);
-    for (int m0 = 0; m0 < M; m0 += RF_ROWS) {
-      const int rows = min(RF_ROWS, M - m0);
-      __syncthreads();
-      if (m0 == 0) async_rows(sw, K * 2, W + static_cast<long long>(c0) * K, K * 2LL, wrows, K * 2);
-      for (int r = 0; r < rows; ++r) async_rows(sx + r * K, K * 4, row(m0 + r, c0), 0, 1, K * 4);
-      cp_async_commit();
-      cp_async_wait<0>();
-      __syncthreads();
-      const int n = c0 + 2 * warp;
-      float acc[RF_ROWS][2];
-#pragma unroll
-      for (int r = 0; r < RF_ROWS; ++r) acc[r][0] = acc[r][1] = 0.f;
-      const bf16* w0 = sw + min(2 * warp, wrows - 1) * K;
-      const bf16* w1 = sw + min(2 * warp + 1, wrows - 1) * K;
-      for (int k = lane * 4; k < K; k += 128) {
-        const uint2 a = *reinterpret_cast<const uint2*>(w0 + k);
-        const uint2 c = *reinterpret_cast<const uint2*>(w1 + k);
-        const float wa[4] = {__uint_as_float(a.x << 16), __uint_as_float(a.x & 0xffff0000u),
-                             __uint_as_float(a.y << 16), __uint_as_float(a.y & 0xffff0000u)};
-        const float wc[4] = {__uint_as_float(c.x << 16), __uint_as_float(c.x & 0xffff0000u),
-                             __uint_as_float(c.y << 16), __uint_as_float(c.y & 0xffff0000u)};
-#pragma unroll
-        for (int r = 0; r < RF_ROWS; ++r) {
-          if (r < rows) {
-            const float4 xv = *reinterpret_cast<const float4*>(sx + r * K + k);
-            acc[r][0] = fmaf(wa[0], xv.x, fmaf(wa[1], xv.y, fmaf(wa[2], xv.z, fmaf(wa[3], xv.w, acc[r][0]))));
-            acc[r][1] = fmaf(wc[0], xv.x, fmaf(wc[1], xv.y, fmaf(wc[2], xv.z, fmaf(wc[3], xv.w, acc[r][1]))));
-          }
+    const int c0 = item * GV_COLS;
+    if (!(first && w_prefetched)) {
+      __syncthreads();  // the previous item's reads of the weight slot are done
+      if (warp == 0) gv_issue_w(W, K, item, sm, &mb[0]);
+    }
+    first = false;
+    bool w_ready = false;
+    for (int m0 = 0; m0 < M; m0 += GV_ROWS) {
+      const int rows = min(GV_ROWS, M - m0);
+      __syncthreads();  // the previous round's reads of x and the partials are done
+      if (warp == 0) {
+        if (lane == 0) mbar_arrive_expect_tx(&mb[1], rows * K * 4);
+        __syncwarp();
+        if (lane < rows) {
+          fence_proxy_async_global();
+          bulk_load(sx + lane * pitch, row(m0 + lane, c0), K * 4, &mb[1]);
         }
       }
-#pragma unroll
-      for (int r = 0; r < RF_ROWS; ++r) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          acc[r][0] += __shfl_xor_sync(0xffffffffu, acc[r][0], o);
-          acc[r][1] += __shfl_xor_sync(0xffffffffu, acc[r][1], o);
-        }
+      if (!w_ready) {
+        if (!mbar_wait(&mb[0], ph[0])) return false;
+        ph[0] ^= 1;
+        w_ready = true;
       }
-      if (lane < 2 && n + lane < N) {
-        const float bias = b ? __bfloat162float(b[n + lane]) : 0.f;
+      if (!mbar_wait(&mb[1], ph[1])) return false;
+      ph[1] ^= 1;
+      // rows >= `rows` of the A tile hold stale values; they only reach
+      // output rows that are never stored
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const int kb = warp * kw;
+      for (int ks = 0; ks < kw; ks += 16) {
+        const int k = kb + ks + t2;
+        uint32_t ah[4], al[4], bw[2];
+        split_bf16x2(*reinterpret_cast<const float2*>(sx + g * pitch + k), ah[0], al[0]);
+        split_bf16x2(*reinterpret_cast<const float2*>(sx + (g + 8) * pitch + k), ah[1], al[1]);
+        split_bf16x2(*reinterpret_cast<const float2*>(sx + g * pitch + k + 8), ah[2], al[2]);
+        split_bf16x2(*reinterpret_cast<const float2*>(sx + (g + 8) * pitch + k + 8), ah[3], al[3]);
+        bw[0] = *reinterpret_cast<const uint32_t*>(sw + g * pitch + k);
+        bw[1] = *reinterpret_cast<const uint32_t*>(sw + g * pitch + k + 8);
+        mma_bf16_16816(acc, ah, bw);
+        mma_bf16_16816(acc, al, bw);
+      }
+      float* rw = red + warp * (GV_ROWS * GV_COLS);
+      rw[g * GV_COLS + t2] = acc[0];
+      rw[g * GV_COLS + t2 + 1] = acc[1];
+      rw[(g + 8) * GV_COLS + t2] = acc[2];
+      rw[(g + 8) * GV_COLS + t2 + 1] = acc[3];
+      __syncthreads();
+      if (threadIdx.x < GV_ROWS * GV_COLS) {
+        const int r = threadIdx.x / GV_COLS, c = threadIdx.x % GV_COLS;
+        if (r < rows) {
+          float v = 0.f;
 #pragma unroll
-        for (int r = 0; r < RF_ROWS; ++r) {
-          if (r < rows) {
-            float y = (lane == 0 ? acc[r][0] : acc[r][1]) + bias;
-            if (act) y = gelu(y);
-            Y[static_cast<long long>(m0 + r) * ldy + n + lane] = y;
-          }
+          for (int w = 0; w < RF_WARPS; ++w) v += red[w * GV_ROWS * GV_COLS + threadIdx.x];
+          if (b) v += __bfloat162float(b[c0 + c]);
+          if (act) v = gelu(v);
+          Y[static_cast<size_t>(m0 + r) * ldy + c0 + c] = v;
         }
       }
     }
   }
+  return true;
 }
 
 // dst = h + LN(u) * gamma + beta (inside = 0) or LN(h + u) * gamma + beta
@@ -320,31 +346,46 @@ __device__ void fold_phase(const RouterFusedArgs& a, int l, int Tq, const float*
 }
 
 // ------------------------------------------------------------------ scores phase
-// Items (tile, 64-token block). St[tile][j][t] = sum_c x[tile][t][c] U2[tu][j][c],
-// j < 32 (hi rows 0..15, lo rows 16..31); tu = tile, or 0 when the query is
-// shared. The item's 64 token rows and the tile's 32 U2 rows are staged in
-// one cp.async batch; warp w computes m16 tile (w & 3) x n8 tiles
-// 2(w >> 2), 2(w >> 2) + 1 with m16n8k16 bf16 MMAs over all channels.
-
-__device__ void scores_phase(const RouterFusedArgs& a, bool shared_query, bf16* sm) {
+// Items (tile, 64-token block), a contiguous range per CTA so that
+// consecutive items share the tile's U2 rows. St[tile][j][t] = sum_c
+// x[tile][t][c] U2[tu][j][c], j < 32 (hi rows 0..15, lo rows 16..31); tu =
+// tile, or 0 when the query is shared. The item's 64 token rows (and the
+// tile's 32 U2 rows when they change) arrive by bulk copies on mbarrier 1;
+// warp w computes m16 tile (w & 3) x n8 tiles 2(w >> 2), 2(w >> 2) + 1 with
+// m16n8k16 bf16 MMAs over all channels.
+__device__ bool scores_phase(const RouterFusedArgs& a, bool shared_query, uint8_t* sm,
+                             uint64_t* mb, uint32_t* ph) {
   const int D = a.D;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pitch = D + 8;
-  const int n_items = a.T * (RF_TOK / 64);
-  bf16* sx = sm;               // [64][pitch]
-  bf16* su = sm + 64 * pitch;  // [32][pitch]
+  const int per_tile = RF_TOK / 64;
+  const int n_items = a.T * per_tile;
+  const int i0 = static_cast<int>(static_cast<long long>(blockIdx.x) * n_items / gridDim.x);
+  const int i1 = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * n_items / gridDim.x);
+  bf16* sx = reinterpret_cast<bf16*>(sm);  // [64][pitch]
+  bf16* su = sx + 64 * pitch;              // [32][pitch]
   const int mt = warp & 3, nb0 = 2 * (warp >> 2);
   const int g = lane >> 2, t2 = (lane & 3) * 2;
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-    const int tile = item / (RF_TOK / 64), tb = item % (RF_TOK / 64);
+  int staged_u = -1;
+  for (int item = i0; item < i1; ++item) {
+    const int tile = item / per_tile, tb = item % per_tile;
+    const int tu = shared_query ? 0 : tile;
+    const bool need_u = tu != staged_u;
+    staged_u = tu;
     __syncthreads();
-    async_rows(sx, pitch * 2, a.x + (static_cast<long long>(tile) * RF_TOK + tb * 64) * D, D * 2LL,
-               64, D * 2);
-    async_rows(su, pitch * 2, a.U2 + static_cast<long long>(shared_query ? 0 : tile) * 32 * D,
-               D * 2LL, 32, D * 2);
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
+    if (warp == 0) {
+      if (lane == 0) mbar_arrive_expect_tx(&mb[1], (64 + (need_u ? 32 : 0)) * D * 2);
+      __syncwarp();
+      fence_proxy_async_global();
+      const bf16* xs = a.x + (static_cast<size_t>(tile) * RF_TOK + tb * 64) * D;
+      bulk_load(sx + lane * pitch, xs + static_cast<size_t>(lane) * D, D * 2, &mb[1]);
+      bulk_load(sx + (lane + 32) * pitch, xs + static_cast<size_t>(lane + 32) * D, D * 2, &mb[1]);
+      if (need_u)
+        bulk_load(su + lane * pitch, a.U2 + (static_cast<size_t>(tu) * 32 + lane) * D, D * 2,
+                  &mb[1]);
+    }
+    if (!mbar_wait(&mb[1], ph[1])) return false;
+    ph[1] ^= 1;
     float acc[2][4] = {};
     for (int ks = 0; ks < D / 16; ++ks) {
       uint32_t af[4];
@@ -356,16 +397,17 @@ __device__ void scores_phase(const RouterFusedArgs& a, bool shared_query, bf16* 
         mma_bf16_16816(acc[q], af, bfr);
       }
     }
-    float* st = a.S + static_cast<long long>(tile) * 32 * RF_TOK + tb * 64 + mt * 16;
+    float* st = a.S + static_cast<size_t>(tile) * 32 * RF_TOK + tb * 64 + mt * 16;
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       const int j = (nb0 + q) * 8 + t2;
-      st[static_cast<long long>(j) * RF_TOK + g] = acc[q][0];
-      st[static_cast<long long>(j + 1) * RF_TOK + g] = acc[q][1];
-      st[static_cast<long long>(j) * RF_TOK + g + 8] = acc[q][2];
-      st[static_cast<long long>(j + 1) * RF_TOK + g + 8] = acc[q][3];
+      st[static_cast<size_t>(j) * RF_TOK + g] = acc[q][0];
+      st[static_cast<size_t>(j + 1) * RF_TOK + g] = acc[q][1];
+      st[static_cast<size_t>(j) * RF_TOK + g + 8] = acc[q][2];
+      st[static_cast<size_t>(j + 1) * RF_TOK + g + 8] = acc[q][3];
     }
   }
+  return true;
 }
 
 // ------------------------------------------------------------------ softmax phase
@@ -449,39 +491,52 @@ __device__ void softmax_phase(const RouterFusedArgs& a, bool shared_cb, float* s
 }
 
 // ------------------------------------------------------------------ wsum phase
-// Items (tile, 64-channel block): z[tile][h][c] = sum_t (P_hi + P_lo)[h][t] x[tile][t][c].
-// P2[tile] (32 x 1024) and the tile's x columns (1024 tokens x 64 channels)
-// are staged in one cp.async batch; warp w computes channels 8w..8w+7 (one n8
+// Items (tile, 64-channel block), a contiguous range per CTA so that
+// consecutive items share the tile's P2 rows: z[tile][h][c] = sum_t
+// (P_hi + P_lo)[h][t] x[tile][t][c]. The tile's 1024 x 64 feature block comes
+// in 4 TMA boxes of 256 tokens x 128 bytes (128-byte swizzle: the 16-byte
+// chunk j of row r sits at chunk j ^ (r & 7)), P2[tile] (32 x 1024) by bulk
+// copies, both on mbarrier 1. Warp w computes channels 8w..8w+7 (one n8
 // tile) for both m16 tiles (hi rows, lo rows) over all 1024 tokens.
-constexpr int WS_PPITCH = RF_TOK + 8;  // bf16 per staged P2 row
-constexpr int WS_XPITCH = 64 + 8;      // bf16 per staged x row (64 channels)
-
-__device__ void wsum_phase(const RouterFusedArgs& a, bf16* sm) {
+__device__ bool wsum_phase(const RouterFusedArgs& a, uint8_t* sm, uint64_t* mb, uint32_t* ph) {
   const int D = a.D;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cblocks = D / 64;
   const int n_items = a.T * cblocks;
-  bf16* sp = sm;                     // [32][WS_PPITCH]
-  bf16* sx = sm + 32 * WS_PPITCH;    // [1024][WS_XPITCH]
+  const int i0 = static_cast<int>(static_cast<long long>(blockIdx.x) * n_items / gridDim.x);
+  const int i1 = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * n_items / gridDim.x);
+  uint8_t* sxb = sm;  // 4 boxes [256 tokens][128 B], 1024-byte aligned
+  bf16* sp = reinterpret_cast<bf16*>(sm + (RF_TOK / WS_BOX) * WS_BOX * 128);  // [32][WS_PPITCH]
   const int g = lane >> 2, t2 = (lane & 3) * 2;
   int staged_tile = -1;
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+  for (int item = i0; item < i1; ++item) {
     const int tile = item / cblocks, cbk = item % cblocks;
-    __syncthreads();
-    if (tile != staged_tile)
-      async_rows(sp, WS_PPITCH * 2, a.P2 + static_cast<long long>(tile) * 32 * RF_TOK,
-                 RF_TOK * 2LL, 32, RF_TOK * 2);
+    const bool need_p = tile != staged_tile;
     staged_tile = tile;
-    async_rows(sx, WS_XPITCH * 2, a.x + static_cast<long long>(tile) * RF_TOK * D + cbk * 64,
-               D * 2LL, RF_TOK, 128);
-    cp_async_commit();
-    cp_async_wait<0>();
     __syncthreads();
+    if (warp == 0) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&mb[1], RF_TOK * 128 + (need_p ? 32 * RF_TOK * 2 : 0));
+        for (int bx = 0; bx < RF_TOK / WS_BOX; ++bx)
+          tma_load_2d(sxb + bx * WS_BOX * 128, &a.xmap, &mb[1], cbk * 64,
+                      tile * RF_TOK + bx * WS_BOX);
+      }
+      __syncwarp();
+      if (need_p) {
+        fence_proxy_async_global();
+        bulk_load(sp + lane * WS_PPITCH, a.P2 + (static_cast<size_t>(tile) * 32 + lane) * RF_TOK,
+                  RF_TOK * 2, &mb[1]);
+      }
+    }
+    if (!mbar_wait(&mb[1], ph[1])) return false;
+    ph[1] ^= 1;
     float acc[2][4] = {};
     for (int ks = 0; ks < RF_TOK / 16; ++ks) {
-      uint32_t bfr[2];
       // B[k = token][n = channel] stored n-contiguous: transposed 8x8 loads
-      ldsm_x2_trans(bfr, sx + (ks * 16 + (lane & 15)) * WS_XPITCH + warp * 8);
+      const int r = ks * 16 + (lane & 15);
+      const int rr = r & (WS_BOX - 1);
+      uint32_t bfr[2];
+      ldsm_x2_trans(bfr, sxb + (r / WS_BOX) * WS_BOX * 128 + rr * 128 + ((warp ^ (rr & 7)) << 4));
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
         uint32_t af[4];
@@ -490,12 +545,13 @@ __device__ void wsum_phase(const RouterFusedArgs& a, bf16* sm) {
       }
     }
     // row g of m-tile 0 is the hi part of head g, row g of m-tile 1 its lo part
-    float* zt = a.z + static_cast<long long>(tile) * 16 * D + cbk * 64 + warp * 8 + t2;
-    *reinterpret_cast<float2*>(zt + static_cast<long long>(g) * D) =
+    float* zt = a.z + static_cast<size_t>(tile) * 16 * D + cbk * 64 + warp * 8 + t2;
+    *reinterpret_cast<float2*>(zt + static_cast<size_t>(g) * D) =
         make_float2(acc[0][0] + acc[1][0], acc[0][1] + acc[1][1]);
-    *reinterpret_cast<float2*>(zt + static_cast<long long>(g + 8) * D) =
+    *reinterpret_cast<float2*>(zt + static_cast<size_t>(g + 8) * D) =
         make_float2(acc[0][2] + acc[1][2], acc[0][3] + acc[1][3]);
   }
+  return true;
 }
 
 // ------------------------------------------------------------------ routing
@@ -604,70 +660,104 @@ __device__ void route_phase(const RouterFusedArgs& a, double* s_vals, double* s_
 // ------------------------------------------------------------------ the kernel
 __global__ void __launch_bounds__(RF_THREADS, 1)
     router_fused_kernel(const __grid_constant__ RouterFusedArgs a) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  float* sf = reinterpret_cast<float*>(smem);
-  bf16* sb = reinterpret_cast<bf16*>(smem);
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the swizzled TMA boxes (the launch adds the slack)
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  float* sf = reinterpret_cast<float*>(sm);
+  __shared__ __align__(8) uint64_t s_mb[2];  // 0: projection weights, 1: everything else
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(&s_mb[0], 1);
+    mbar_init(&s_mb[1], 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&a.xmap);
+  }
+  __syncthreads();
+  uint32_t ph[2] = {0u, 0u};
   unsigned gen = 0;
   bool ok = true;
+  bool w_pending = false;  // weight copies of the next projection phase in flight
   const int T = a.T, D = a.D, G = a.G;
   auto sync = [&]() {
     if (ok) ok = grid_sync(a.bar, gen);
     return ok;
   };
+  // The weights of the next projection phase do not depend on the previous
+  // phase: this CTA's first item's rows are requested before the barrier.
+  auto prefetch_w = [&](const bf16* W, int K, int N) {
+    __syncthreads();
+    w_pending = static_cast<int>(blockIdx.x) < N / GV_COLS;
+    if (w_pending && warp == 0) gv_issue_w(W, K, blockIdx.x, sm, &s_mb[0]);
+  };
+  auto project = [&](int M, int K, int N, const bf16* W, const bf16* b, float* Y, int ldy,
+                     bool act, auto row) {
+    const bool pre = w_pending;
+    w_pending = false;
+    if (ok) {
+      ok = gemv_phase(M, K, N, W, b, Y, ldy, act, sm, s_mb, ph, pre, row);
+    } else if (pre && mbar_wait(&s_mb[0], ph[0])) {
+      ph[0] ^= 1;  // drain the prefetched copies of a phase that does not run
+    }
+  };
   // layer 1's query is shared by all tiles: Q1 = Wq_1 query + bq_1 in row 0 of Q
   // (the bf16 query is widened into h first)
   if (blockIdx.x == 0)
     for (int k = threadIdx.x; k < D; k += RF_THREADS) a.h[k] = __bfloat162float(a.query[k]);
-  if (sync())
-    gemv_phase(1, D, D, a.Wq[0], a.bq[0], a.Q, D, false, sf, [&](int, int) { return a.h; });
-  for (int l = 0; l < 4; ++l) {
+  prefetch_w(a.Wq[0], D, D);
+  if (sync()) project(1, D, D, a.Wq[0], a.bq[0], a.Q, D, false, [&](int, int) { return a.h; });
+  for (int l = 0; l < 4 && ok; ++l) {
     if (!sync()) break;
     const bool shared_q = l == 0;
     fold_phase(a, l, shared_q ? 1 : T, a.Q, shared_q ? 0 : D, sf);
     if (!sync()) break;
-    scores_phase(a, shared_q, sb);
+    if (!scores_phase(a, shared_q, sm, s_mb, ph)) ok = false;
     if (!sync()) break;
     softmax_phase(a, shared_q, sf);
     if (!sync()) break;
-    wsum_phase(a, sb);
-    if (!sync()) break;
+    if (!wsum_phase(a, sm, s_mb, ph)) ok = false;
     // o = Wv_h z_h + bv: the input row of output row m for columns of head h is z[m][h]
-    gemv_phase(T, D, D, a.Wv[l], a.bv[l], a.O, D, false, sf, [&](int m, int c0) {
-      return a.z + (static_cast<long long>(m) * 16 + c0 / RF_HD) * D;
-    });
+    prefetch_w(a.Wv[l], D, D);
     if (!sync()) break;
-    gemv_phase(T, D, D, a.Wo[l], a.bo[l], a.q, D, false, sf,
-               [&](int m, int) { return a.O + static_cast<long long>(m) * D; });
+    project(T, D, D, a.Wv[l], a.bv[l], a.O, D, false, [&](int m, int c0) {
+      return a.z + (static_cast<size_t>(m) * 16 + c0 / RF_HD) * D;
+    });
+    prefetch_w(a.Wo[l], D, D);
+    if (!sync()) break;
+    project(T, D, D, a.Wo[l], a.bo[l], a.q, D, false,
+            [&](int m, int) { return a.O + static_cast<size_t>(m) * D; });
     if (l < 3) {
+      prefetch_w(a.Wq[l + 1], D, D);
       if (!sync()) break;
-      gemv_phase(T, D, D, a.Wq[l + 1], a.bq[l + 1], a.Q, D, false, sf,
-                 [&](int m, int) { return a.q + static_cast<long long>(m) * D; });
+      project(T, D, D, a.Wq[l + 1], a.bq[l + 1], a.Q, D, false,
+              [&](int m, int) { return a.q + static_cast<size_t>(m) * D; });
     }
   }
   // Gating: h_0 = pooled = q; block b: u1 = GELU(W1 h_b + b1), u2 = W2 u1 + b2,
-  // h_{b+1} = h_b + LN_b(u2) (rows spread over the CTAs, kept in h).
-  for (int b = 0; b < 4; ++b) {
-    if (!sync()) break;
+  // then the residual LayerNorm (rows spread over the CTAs, kept in h).
+  for (int b = 0; b < 4 && ok; ++b) {
     const float* hb = b == 0 ? a.q : a.h;
-    gemv_phase(T, D, G, a.gW1[b], a.gb1[b], a.u1, G, true, sf,
-               [&](int m, int) { return hb + static_cast<long long>(m) * D; });
+    prefetch_w(a.gW1[b], D, G);
     if (!sync()) break;
-    gemv_phase(T, G, D, a.gW2[b], a.gb2[b], a.u2, D, false, sf,
-               [&](int m, int) { return a.u1 + static_cast<long long>(m) * G; });
+    project(T, D, G, a.gW1[b], a.gb1[b], a.u1, G, true,
+            [&](int m, int) { return hb + static_cast<size_t>(m) * D; });
+    prefetch_w(a.gW2[b], G, D);
+    if (!sync()) break;
+    project(T, G, D, a.gW2[b], a.gb2[b], a.u2, D, false,
+            [&](int m, int) { return a.u1 + static_cast<size_t>(m) * G; });
     if (!sync()) break;
     for (int m = blockIdx.x; m < T; m += gridDim.x) {
-      residual_ln_row(hb + static_cast<long long>(m) * D, a.u2 + static_cast<long long>(m) * D,
+      residual_ln_row(hb + static_cast<size_t>(m) * D, a.u2 + static_cast<size_t>(m) * D,
                       a.gln_g[b], a.gln_b[b], sf, D, a.gate_inside);
       __syncthreads();
-      for (int i = threadIdx.x; i < D; i += RF_THREADS) a.h[static_cast<long long>(m) * D + i] = sf[i];
+      for (int i = threadIdx.x; i < D; i += RF_THREADS) a.h[static_cast<size_t>(m) * D + i] = sf[i];
       __syncthreads();
     }
   }
   // head: gate = softmax(Wout h_4 + bout), one warp per tile
   if (ok && sync()) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31;
     for (int t = blockIdx.x * RF_WARPS + warp; t < T; t += gridDim.x * RF_WARPS) {
-      const float* hr = a.h + static_cast<long long>(t) * D;
+      const float* hr = a.h + static_cast<size_t>(t) * D;
       float l0 = 0.f, l1 = 0.f;
       for (int i = lane; i < D; i += 32) {
         const float v = hr[i];
@@ -692,34 +782,43 @@ __global__ void __launch_bounds__(RF_THREADS, 1)
     }
   }
   if (ok && sync())
-    route_phase(a, reinterpret_cast<double*>(smem),
-                reinterpret_cast<double*>(smem) + IVC_MAX_QUANTILE_GROUP);
+    route_phase(a, reinterpret_cast<double*>(sm),
+                reinterpret_cast<double*>(sm) + IVC_MAX_QUANTILE_GROUP);
+  // a prefetch whose phase never ran (a barrier gave up): let its copies land
+  if (w_pending) (void)mbar_wait(&s_mb[0], ph[0]);
   if (!ok && threadIdx.x == 0) atomicOr(a.status, DEV_WAIT_TIMEOUT);
 }
 
 size_t router_fused_smem(int D, int G) {
   const size_t K = static_cast<size_t>(D > G ? D : G);
-  const size_t gemv = K * (RF_ROWS * sizeof(float) + RF_GEMV_COLS * sizeof(bf16));
+  const size_t gemv = GV_ROWS * (K + 8) * 4 + GV_COLS * (K + 8) * 2 +
+                      static_cast<size_t>(RF_WARPS) * GV_ROWS * GV_COLS * 4;
   const size_t route = 2 * static_cast<size_t>(IVC_MAX_QUANTILE_GROUP) * sizeof(double);
   const size_t scores = static_cast<size_t>(96) * (D + 8) * sizeof(bf16);
-  const size_t wsum = (static_cast<size_t>(32) * WS_PPITCH + static_cast<size_t>(RF_TOK) * WS_XPITCH) *
-                      sizeof(bf16);
+  const size_t wsum = static_cast<size_t>(RF_TOK) * 128 +
+                      static_cast<size_t>(32) * WS_PPITCH * sizeof(bf16);
+  const size_t fold = static_cast<size_t>(64) * RF_HD * sizeof(float);
   size_t m = gemv;
-  if (route > m) m = route;
-  if (scores > m) m = scores;
-  if (wsum > m) m = wsum;
-  return m;
+  for (size_t v : {route, scores, wsum, fold, static_cast<size_t>(D) * sizeof(float)})
+    if (v > m) m = v;
+  return m + 1024;  // alignment slack
 }
 
 }  // namespace
 
-bool router_fused_enabled() {
-  static int on = -1;
-  if (on < 0) {
+bool router_fused_wanted(bool default_on) {
+  static int env = -2;
+  if (env == -2) {
     const char* e = std::getenv("IVC_ROUTER_FUSED");
-    on = (e && e[0] == '1') ? 1 : 0;
+    env = e ? (e[0] == '1' ? 1 : 0) : -1;
   }
-  return on == 1;
+  return env < 0 ? default_on : env == 1;
+}
+
+bool router_fused_supported(const ivc_router* r) {
+  return r->pool_mode == IVC_POOL_FOLDED && r->D % 128 == 0 && r->D <= RF_MAXD &&
+         r->heads <= 16 && r->gate_hidden <= RF_MAXK && r->gate_hidden % 128 == 0 &&
+         router_fused_smem(r->D, r->gate_hidden) <= 227 * 1024;
 }
 
 int launch_router_fused(const ivc_router* r, const void* x, const int32_t* valid_len, int T,
@@ -727,9 +826,10 @@ int launch_router_fused(const ivc_router* r, const void* x, const int32_t* valid
                         int32_t* offsets, int32_t* total, const FusedRouterBufs& b,
                         const Launch& L) {
   if (T == 0) return IVC_OK;
-  if (r->D % 128 != 0 || r->heads > 16 || r->D > RF_MAXK || r->gate_hidden > RF_MAXK)
-    return IVC_EUNSUPPORTED;
+  if (!router_fused_supported(r)) return IVC_EUNSUPPORTED;
   RouterFusedArgs a{};
+  if (map_rows_2d(&a.xmap, x, static_cast<long long>(T) * RF_TOK, r->D, WS_BOX) != IVC_OK)
+    return IVC_ECUDA;
   a.x = static_cast<const bf16*>(x);
   a.valid_len = valid_len;
   a.T = T;
