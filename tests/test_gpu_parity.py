@@ -295,8 +295,9 @@ def test_flash_4b_batched_sampled(pool_mode):
 
 # ---------------------------------------------------------------- router-first flow
 def _routed_vs_dual(ivc, inp, m1, m2, r, routed_res):
-    """Rows of tiles routed alike in both flows are bit-identical: each output
-    row of a GEMM depends only on its own input row."""
+    """Rows of tiles routed alike in both flows agree. They are computed by
+    the same kernels; only the split-K slicing, chosen per launch from the
+    number of rows, can change the fp32 summation order."""
     dual = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(), inp["image_offsets"].cuda(),
                               m1, m2, r)
     torch.cuda.synchronize()
@@ -308,7 +309,8 @@ def _routed_vs_dual(ivc, inp, m1, m2, r, routed_res):
             continue
         a = dual["out"][od[t]:od[t + 1]]
         b = routed_res["out"][orr[t]:orr[t + 1]]
-        assert torch.equal(a, b), f"tile {t}: routed rows differ from the dual-path rows"
+        torch.testing.assert_close(b.float(), a.float(), rtol=2e-2, atol=2e-2,
+                                   msg=lambda m: f"tile {t}: routed vs dual-path rows: {m}")
         same += 1
     assert same > 0
 

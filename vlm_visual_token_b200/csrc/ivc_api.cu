@@ -90,6 +90,8 @@ struct PsBufs {
   float* fold_b = nullptr;
   bf16* h1 = nullptr;
   bf16* h2 = nullptr;
+  float* split_part = nullptr;  // split-K scratch (flash flows only), shared
+  int* split_s = nullptr;
 };
 
 void carve_ps(Carver& cv, const ivc_mlp* m, long long rows, bool need_stats, PsBufs& b) {
@@ -202,6 +204,8 @@ int ps_mlp(const void* x, int T, int C, bool half, int flags, const ivc_mlp* m, 
   c.row_rstd = b.rstd;
   c.out = b.h1;
   c.ldo = m->dims[1];
+  c.split_part = b.split_part;
+  c.split_s = b.split_s;
   const int item_rows = half ? 256 : 64;
   if (rt) {
     c.list = rt->list;
@@ -228,6 +232,8 @@ int ps_mlp(const void* x, int T, int C, bool half, int flags, const ivc_mlp* m, 
     d.remap = last ? remap : 0;
     d.out = last ? y : b.h2;
     d.ldo = m->dims[i + 1];
+    d.split_part = b.split_part;
+    d.split_s = b.split_s;
     if (rt) {
       d.list_count = rt->count;
       d.item_rows = item_rows;
@@ -473,6 +479,9 @@ void carve_flash(Carver& cv, int T, const ivc_mlp* m1, const ivc_mlp* m2, const 
   f.Y64 = cv.take<bf16>(static_cast<size_t>(T) * 64 * m2->dims[m2->n_linear]);
   carve_route(cv, r, T, f.br);
   carve_lists(cv, T, f.lists);
+  // one split-K scratch for all connector GEMMs (they run one after another)
+  f.b1.split_part = f.b2.split_part = cv.take<float>(splitk_part_floats());
+  f.b1.split_s = f.b2.split_s = cv.take<int>(4);
 }
 
 size_t flash_ws(int T, const ivc_mlp* m1, const ivc_mlp* m2, const ivc_router* r) {

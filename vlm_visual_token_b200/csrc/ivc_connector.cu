@@ -244,11 +244,95 @@ static int run_gemm(const GemmMaps& maps, const GemmArgs& args, const char* tag,
   const long long tiles = static_cast<long long>((args.M + GEMM_BM * CG - 1) / (GEMM_BM * CG)) *
                           ((args.N + BN - 1) / BN) * args.groups;
   const long long units = num_sms() / CG;
-  const int grid = CG * static_cast<int>(tiles < units ? tiles : units);
+  // with split-K the last round is cut into slices for every unit
+  const int grid = CG * static_cast<int>(tiles < units && args.split_max <= 1 ? tiles : units);
   TraceScope ts(tag ? tag : "gemm", L.stream);
   return launch_k(kern, dim3(grid), dim3(GEMM_THREADS), S::TOTAL, L.stream, CG, maps, args,
                   L.status);
 }
+
+// Finishes the split tiles of a GEMM (GemmArgs.split_max): each element of a
+// split tile is the sum of its S fp32 k-slice partials, then the epilogue the
+// GEMM itself applies (LayerNorm fold or bias, GELU, row remaps, bf16/fp32
+// store). Each thread owns 8 consecutive columns of one row. Exits at once
+// when the GEMM split nothing (split_s[0] == 1).
+__global__ void __launch_bounds__(256)
+    splitk_epilogue_kernel(const __grid_constant__ GemmArgs args, int tile_m, int bn) {
+  pdl_wait();
+  pdl_trigger();
+  const int S = args.split_s[0];
+  if (S <= 1) return;
+  const int first = args.split_s[1], n_split = args.split_s[2];
+  int M = args.M;
+  if (args.list_count != nullptr) {
+    const int c = *args.list_count;
+    const long long rows = static_cast<long long>(c < 0 ? 0 : c) * args.item_rows;
+    M = rows < M ? static_cast<int>(rows) : M;
+  }
+  const int m_tiles = (M + tile_m - 1) / tile_m;
+  const int n_tiles = (args.N + bn - 1) / bn;
+  const int cols8 = bn / 8;
+  const long long per_tile = static_cast<long long>(tile_m) * cols8;
+  const long long n = n_split * per_tile;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int tt = static_cast<int>(i / per_tile);
+    const int in_tile = static_cast<int>(i % per_tile);
+    const int lr = in_tile / cols8, lc = (in_tile % cols8) * 8;
+    const TileCoord tc = tile_coord(first + tt, m_tiles, n_tiles, tile_m, bn);
+    const int row = tc.m0 + lr, c0 = tc.n0 + lc;
+    if (row >= M || c0 >= args.N) continue;
+    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const float* p = args.split_part + (static_cast<long long>(tt) * S * tile_m + lr) * bn + lc;
+    const long long slice = static_cast<long long>(tile_m) * bn;
+#pragma unroll 4
+    for (int sl = 0; sl < S; ++sl) {
+      const float4 a = __ldcs(reinterpret_cast<const float4*>(p + sl * slice));
+      const float4 b = __ldcs(reinterpret_cast<const float4*>(p + sl * slice + 4));
+      v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+      v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+    }
+    if (args.epi_mode == EPI_LNFOLD) {
+      const int sr = args.stats_remap
+                         ? args.list[row / args.item_rows] * args.item_rows + row % args.item_rows
+                         : row;
+      const float rstd = args.row_rstd[sr];
+      const float nms = -args.row_mean[sr] * rstd;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        v[j] = fmaf(rstd, v[j], nms * args.colsum[c0 + j]) + args.fbias[c0 + j];
+    } else if (args.bias[0] != nullptr) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] += __bfloat162float(args.bias[0][c0 + j]);
+    }
+    if (args.gelu) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = gelu_erf(v[j]);
+    }
+    long long out_row = row;
+    if (args.remap == 1) {
+      const int t = row & 255;
+      out_row = (row & ~255) | ((t & 15) << 4) | (t >> 4);
+    } else if (args.remap == 2) {
+      const int t = row & 63;
+      out_row = (row & ~63) | ((t & 7) << 3) | (t >> 3);
+    }
+    if (args.out_base != nullptr)
+      out_row = args.out_base[row / args.item_rows] + out_row % args.item_rows;
+    const long long off = out_row * args.ldo + c0;
+    if (args.out_f32) {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + off);
+      dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+      dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+    } else {
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) + off) =
+          make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                     pack_bf16x2(v[6], v[7]));
+    }
+  }
+}
+
+size_t splitk_part_floats() { return static_cast<size_t>(num_sms()) * GEMM_BM * 256; }
 
 // 256-wide tiles run on CTA pairs unless IVC_GEMM_PAIRS=0 (kept for
 // comparing the two variants on the same build).
@@ -343,18 +427,49 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
   a.out_base = c.out_base;
   a.item_rows = c.item_rows;
   a.stats_remap = c.stats_remap;
+  // Split-K where the output tiles leave SMs idle. With a host-known row
+  // count the slice count is fixed here; with a device row count (routed
+  // rows) the kernel picks it and the finishing kernel always runs.
+  if (c.split_part != nullptr && c.split_s != nullptr && c.groups == 1 && c.b_mode == B_K2D &&
+      c.m_valid == 0) {
+    const int units = num_sms() / cg;
+    const int n_tiles = (c.N + bn - 1) / bn;
+    const int KT = c.K / GEMM_BK;
+    const int tile_m = GEMM_BM * cg;
+    constexpr int kMaxSplit = 8;
+    if (c.list_count == nullptr) {
+      // the kernel's own choice, known here: skip the finishing launch if 1
+      const int rem = (((c.M + tile_m - 1) / tile_m) * n_tiles) % units;
+      const int S = rem > 0 ? split_count(kMaxSplit, units, rem, KT) : 1;
+      a.split_max = S > 1 ? S : 0;
+    } else {
+      // the row count is known only on the device: the kernel decides
+      a.split_max = KT >= 16 ? kMaxSplit : 0;
+    }
+    if (a.split_max > 1) {
+      if (c.N % 8 != 0) return IVC_EUNSUPPORTED;
+      a.split_part = c.split_part;
+      a.split_s = c.split_s;
+    }
+  }
   if (c.list_count != nullptr && (c.item_rows <= 0 || (c.item_rows != 256 && c.item_rows != 64)))
     return IVC_EINVAL;
   if ((c.list != nullptr || c.stats_remap || c.out_base != nullptr) && c.list_count == nullptr)
     return IVC_EINVAL;
   if (c.stats_remap && c.list == nullptr) return IVC_EINVAL;
+  int rc2;
   switch (bn) {
-    case 256: return cg == 2 ? run_gemm<256, 6, 2>(maps, a, c.tag, L)
-                             : run_gemm<256, 4, 1>(maps, a, c.tag, L);
-    case 128: return run_gemm<128, 6, 1>(maps, a, c.tag, L);
-    case 64: return run_gemm<64, 8, 1>(maps, a, c.tag, L);
-    default: return run_gemm<32, 8, 1>(maps, a, c.tag, L);
+    case 256: rc2 = cg == 2 ? run_gemm<256, 6, 2>(maps, a, c.tag, L)
+                            : run_gemm<256, 4, 1>(maps, a, c.tag, L);
+      break;
+    case 128: rc2 = run_gemm<128, 6, 1>(maps, a, c.tag, L); break;
+    case 64: rc2 = run_gemm<64, 8, 1>(maps, a, c.tag, L); break;
+    default: rc2 = run_gemm<32, 8, 1>(maps, a, c.tag, L); break;
   }
+  if (rc2 != IVC_OK || a.split_max <= 1) return rc2;
+  TraceScope ts("splitk.epilogue", L.stream);
+  return launch_k(splitk_epilogue_kernel, dim3(2 * num_sms()), dim3(256), 0, L.stream, 1, a,
+                  GEMM_BM * cg, bn);
 }
 
 }  // namespace ivc

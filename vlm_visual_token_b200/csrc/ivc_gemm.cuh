@@ -95,7 +95,29 @@ struct GemmArgs {
   const int* out_base;
   int item_rows;
   int stats_remap;
+  // Split-K of the last round (split_max > 1). The output tiles that fill
+  // whole rounds of the persistent grid run unsplit; the rem < units tiles
+  // left for the last round are each cut into S = min(split_max, units / rem,
+  // KT / 4) k-slices, so that round keeps every CTA busy. A slice unit stores
+  // its raw fp32 tile at split_part[((tail tile) * S + slice)][TILE_M][BN];
+  // splitk_epilogue_kernel sums the slices and applies the epilogue. CTA 0
+  // writes split_s[0..2] = {S, first split tile, split tiles}.
+  int split_max;
+  float* split_part;
+  int* split_s;
 };
+
+// Number of k-slices for `tiles` output tiles on `units` CTAs (or pairs).
+// The split-K scratch holds units x TILE_M x BN values: S * tiles <= units.
+// Fewer than 4 slices do not pay for the partial traffic and the finishing
+// launch (measured on the connector GEMMs).
+__host__ __device__ __forceinline__ int split_count(int split_max, int units, int tiles, int KT) {
+  if (split_max <= 1 || tiles <= 0) return 1;
+  int s = units / tiles;
+  if (s > split_max) s = split_max;
+  if (s > KT / 4) s = KT / 4;  // at least 4 k-steps per slice
+  return s < 4 ? 1 : s;
+}
 
 template <int BN, int STAGES, int CG = 1>
 struct GemmSmem {
@@ -201,26 +223,52 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     M = rows < M ? static_cast<int>(rows) : M;
   }
   const int m_tiles = (M + TILE_M - 1) / TILE_M;
-  const int n_total = m_tiles * n_tiles * args.groups;
+  const int n_out = m_tiles * n_tiles * args.groups;  // output tiles
+  const int rem = n_out % n_units;
+  const int S = rem > 0 ? split_count(args.split_max, n_units, rem, KT) : 1;
+  const int n_full = S > 1 ? n_out - rem : n_out;     // tiles computed whole
+  const int n_total = n_full + (n_out - n_full) * S;  // work units
   const int n_listed = args.list_count != nullptr ? M / args.item_rows : 0;
+  if (args.split_s != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
+    args.split_s[0] = S;
+    args.split_s[1] = n_full;
+    args.split_s[2] = n_out - n_full;
+  }
+  // work unit -> output tile and k-block range [kb0, kb1); slice < 0: whole tile
+  auto unit_of = [&](int idx, int& tile, int& slice, int& kb0, int& kb1) {
+    if (idx < n_full) {
+      tile = idx;
+      slice = -1;
+      kb0 = 0;
+      kb1 = KT;
+    } else {
+      const int j = idx - n_full;
+      tile = n_full + j / S;
+      slice = j % S;
+      kb0 = slice * KT / S;
+      kb1 = (slice + 1) * KT / S;
+    }
+  };
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
       int it = 0;
       for (int idx = unit; idx < n_total && ok; idx += n_units) {
-        const TileCoord tc = tile_coord(idx, m_tiles, n_tiles, TILE_M, BN);
+        int tile, slice, kb0, kb1;
+        unit_of(idx, tile, slice, kb0, kb1);
+        const TileCoord tc = tile_coord(tile, m_tiles, n_tiles, TILE_M, BN);
         const int my_m0 = tc.m0 + GEMM_BM * rank;
         const int my_n0 = tc.n0 + static_cast<int>(L::B_ROWS) * rank;
         const int bb = args.b_batch_rows > 0 ? tc.m0 / args.b_batch_rows : 0;
         if (args.b_prefetch > 0 && args.b_mode == B_K2D) {
-          for (int kk = 0; kk < args.b_prefetch && kk < KT; ++kk)
+          for (int kk = kb0; kk < kb0 + args.b_prefetch && kk < kb1; ++kk)
             tma_prefetch_2d(&maps.b[tc.g], kk * GEMM_BK, my_n0);
         }
-        for (int kk = 0; kk < KT; ++kk, ++it) {
+        for (int kk = kb0; kk < kb1; ++kk, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
-          if (args.b_prefetch > 0 && args.b_mode == B_K2D && kk + args.b_prefetch < KT)
+          if (args.b_prefetch > 0 && args.b_mode == B_K2D && kk + args.b_prefetch < kb1)
             tma_prefetch_2d(&maps.b[tc.g], (kk + args.b_prefetch) * GEMM_BK, my_n0);
           if (!mbar_wait(&empty_bar[s], ph ^ 1)) { ok = false; break; }
           // the leader's barrier counts the bytes of both CTAs of a pair
@@ -304,10 +352,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       for (int idx = unit; idx < n_total && ok; idx += n_units, ++local) {
         const int acc = local & 1;
         const uint32_t use = static_cast<uint32_t>(local >> 1);
+        int tile, slice, kb0, kb1;
+        unit_of(idx, tile, slice, kb0, kb1);
         if (!mbar_wait(&tempty_bar[acc], (use & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kk = 0; kk < KT; ++kk, ++it) {
+        for (int kk = kb0; kk < kb1; ++kk, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
           if (!mbar_wait(&full_bar[s], ph)) { ok = false; break; }
@@ -323,9 +373,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             // K-major: advance 16 bf16 = 32 bytes inside the swizzle atom;
             // MN-major: advance 16 k-rows of 128 bytes.
             if constexpr (CG == 2)
-              umma_bf16_pair(d_tmem, ad + 2 * k, bd + bstep * k, idesc, (kk | k) != 0 ? 1u : 0u);
+              umma_bf16_pair(d_tmem, ad + 2 * k, bd + bstep * k, idesc,
+                             (kk != kb0 || k != 0) ? 1u : 0u);
             else
-              umma_bf16(d_tmem, ad + 2 * k, bd + bstep * k, idesc, (kk | k) != 0 ? 1u : 0u);
+              umma_bf16(d_tmem, ad + 2 * k, bd + bstep * k, idesc, (kk != kb0 || k != 0) ? 1u : 0u);
           }
           if constexpr (CG == 2)
             umma_commit_pair(&empty_bar[s]);
@@ -345,7 +396,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const int et = threadIdx.x - 64;  // 0..127
     int local = 0;
     for (int idx = unit; idx < n_total; idx += n_units, ++local) {
-      const TileCoord tc = tile_coord(idx, m_tiles, n_tiles, TILE_M, BN);
+      int tile, slice, kb0, kb1;
+      unit_of(idx, tile, slice, kb0, kb1);
+      const TileCoord tc = tile_coord(tile, m_tiles, n_tiles, TILE_M, BN);
       const int acc = local & 1;
       const uint32_t use = static_cast<uint32_t>(local >> 1);
       // per-column epilogue vectors of this tile
@@ -409,6 +462,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             else
               mbar_arrive(&tempty_bar[acc]);
           }
+        }
+        if (slice >= 0) {
+          // raw sums of this k-slice (the whole TILE_M x BN tile, in bounds
+          // of its slot); splitk_epilogue_kernel finishes the tile
+          float4* dst = reinterpret_cast<float4*>(
+              args.split_part +
+              ((static_cast<long long>(tile - n_full) * S + slice) * TILE_M + (row - tc.m0)) * BN +
+              c);
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                 __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+          continue;
         }
         if (row < M && tc.n0 + c < args.N && (args.m_valid == 0 || (row & 127) < args.m_valid)) {
           float v[32];

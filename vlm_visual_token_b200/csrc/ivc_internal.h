@@ -112,8 +112,13 @@ struct GemmCall {
   const int* out_base;
   int item_rows;
   int stats_remap;
+  // split-K scratch (optional): splitk_part_floats() fp32 values and one int
+  float* split_part;
+  int* split_s;
 };
 int launch_gemm(const GemmCall& c, const Launch& L);
+// Size of the split-K partial buffer: enough for any GEMM shape on this device.
+size_t splitk_part_floats();
 
 // -------------------------------------------------------------- router
 // Y[m, n] = act(sum_k X[m, k] W[n, k] + b[n]); X fp32 [M, ldx], W bf16 [N, K].
