@@ -191,6 +191,18 @@ int map_rows_2d(CUtensorMap* m, const void* base, long long rows, long long cols
   return map_2d(m, base, rows, cols, box_rows);
 }
 
+int map_bf16(CUtensorMap* m, int rank, const void* base, const unsigned long long* dims,
+             const unsigned long long* strides_bytes, const unsigned* box) {
+  cuuint64_t d[5], st[4];
+  cuuint32_t b[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    if (i + 1 < rank) st[i] = strides_bytes[i];
+  }
+  return encode(m, rank, base, d, st, b);
+}
+
 // Batched [batches][rows][inner] bf16 (row stride ld, batch stride bs elements),
 // box {box_inner, box_rows, 1}.
 static int map_3d(CUtensorMap* m, const void* base, long long batches, long long rows,

@@ -159,6 +159,10 @@ struct FusedRouterBufs {
 // Tensor map of a row-major [rows, cols] bf16 matrix, box 64 columns x
 // box_rows rows, 128-byte swizzle (ivc_connector.cu).
 int map_rows_2d(CUtensorMap* m, const void* base, long long rows, long long cols, int box_rows);
+// Tensor map of a bf16 tensor of `rank` dims (innermost first; strides in
+// bytes of dims 1..rank-1, in any order), box `box`, 128-byte swizzle.
+int map_bf16(CUtensorMap* m, int rank, const void* base, const unsigned long long* dims,
+             const unsigned long long* strides_bytes, const unsigned* box);
 // Folded pooling can run as one persistent cooperative kernel (grid barriers
 // between its phases) or as separate kernels. IVC_ROUTER_FUSED=1 / 0 forces
 // the choice; otherwise the caller's default_on decides.

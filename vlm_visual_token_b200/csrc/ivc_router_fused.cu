@@ -44,11 +44,16 @@ constexpr int RF_MAXK = 2048;   // widest projection input
 constexpr int GV_COLS = 8;      // output columns per projection item (one n8 MMA tile)
 constexpr int GV_ROWS = 16;     // input rows per projection round (one m16 MMA tile)
 constexpr int WS_BOX = 256;     // tokens per TMA box of the weighted-sum staging
-constexpr int WS_PPITCH = RF_TOK + 8;  // bf16 per staged P2 row
+constexpr int SC_TOK = 32;      // tokens per scores item
+constexpr int WS_HALF = RF_TOK / 2;  // tokens per weighted-sum item
 
 struct RouterFusedArgs {
-  CUtensorMap xmap;  // x as [T*1024, D], box 64 channels x WS_BOX tokens, 128-byte swizzle
-  const bf16* x;     // [T, 1024, D]
+  // 128-byte swizzled TMA views (one request per staged operand):
+  CUtensorMap xmap;   // x as [T*1024, D], box 64 channels x WS_BOX tokens
+  CUtensorMap xmap3;  // x as {64 ch, T*1024 tokens, D/64 chunks}, box {64, SC_TOK, D/64}
+  CUtensorMap u2map;  // U2 as {64, 32 rows, D/64 chunks, T}, box {64, 32, D/64, 1}
+  CUtensorMap p2map;  // P2 as {64 tokens, 32 rows, 16 chunks, T}, box {64, 32, 8, 1}
+  const bf16* x;      // [T, 1024, D]
   const int32_t* valid_len;
   int T, D, G, heads;
   const bf16 *query, *Wq[4], *bq[4], *Wk[4], *bk[4], *Wv[4], *bv[4], *Wo[4], *bo[4];
@@ -304,20 +309,42 @@ __device__ void residual_ln_row(const float* __restrict__ hrow, const float* __r
 // ------------------------------------------------------------------ fold phase
 // Items (c-block of 128, head): U2[t][h][c] hi, U2[t][16+h][c] lo of
 // u = Wk[h*64.., c] . Q[t, h*64..] / 8; cb[t][h] = bk . Q / 8 (c-block 0).
-__device__ void fold_phase(const RouterFusedArgs& a, int l, int Tq, const float* __restrict__ Q,
-                           long long ldq, float* s_q) {
+// The item's 64 x 128 block of Wk arrives by bulk copies on mbarrier 0 (the
+// first item's before the grid barrier, see fold_issue_w); Q rows are read
+// directly. Shared memory: Wk block [64][128] bf16 | Q block [64][64] f32.
+__device__ __forceinline__ void fold_issue_w(const bf16* __restrict__ Wk, int D, int item,
+                                             uint8_t* sm, uint64_t* mb) {
+  const int lane = threadIdx.x & 31;
+  const int cblocks = D / 128;
+  const int h = item / cblocks, cbk = item % cblocks;
+  bf16* sw = reinterpret_cast<bf16*>(sm);
+  if (lane == 0) mbar_arrive_expect_tx(mb, RF_HD * 128 * 2);
+  __syncwarp();
+  for (int d = lane; d < RF_HD; d += 32)
+    bulk_load(sw + d * 128, Wk + static_cast<size_t>(h * RF_HD + d) * D + cbk * 128, 256, mb);
+}
+
+__device__ bool fold_phase(const RouterFusedArgs& a, int l, int Tq, const float* __restrict__ Q,
+                           long long ldq, uint8_t* sm, uint64_t* mb, uint32_t* ph,
+                           bool w_prefetched) {
   const int D = a.D;
   const int cblocks = D / 128;
   const int n_items = cblocks * a.heads;
+  const bf16* sw = reinterpret_cast<const bf16*>(sm);
+  float* s_q = reinterpret_cast<float*>(sm + RF_HD * 128 * 2);
+  const int tid = threadIdx.x & 127;  // column within the block
+  const int half = threadIdx.x >> 7;  // two halves share the tiles
+  bool first = true;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     const int h = item / cblocks, cbk = item % cblocks;
-    const int tid = threadIdx.x & 127;   // column within the block
-    const int half = threadIdx.x >> 7;   // two halves share the tiles
     const int c = cbk * 128 + tid;
-    float w[RF_HD];
-#pragma unroll
-    for (int d = 0; d < RF_HD; ++d)
-      w[d] = __bfloat162float(a.Wk[l][static_cast<long long>(h * RF_HD + d) * D + c]);
+    if (!(first && w_prefetched)) {
+      __syncthreads();
+      if (threadIdx.x < 32) fold_issue_w(a.Wk[l], D, item, sm, &mb[0]);
+    }
+    first = false;
+    if (!mbar_wait(&mb[0], ph[0])) return false;
+    ph[0] ^= 1;
     for (int t0 = 0; t0 < Tq; t0 += 64) {
       const int nt = min(64, Tq - t0);
       __syncthreads();
@@ -326,13 +353,14 @@ __device__ void fold_phase(const RouterFusedArgs& a, int l, int Tq, const float*
       __syncthreads();
       for (int t = half; t < nt; t += 2) {
         float u = 0.f;
-#pragma unroll
-        for (int d = 0; d < RF_HD; ++d) u = fmaf(w[d], s_q[t * RF_HD + d], u);
+#pragma unroll 16
+        for (int d = 0; d < RF_HD; ++d)
+          u = fmaf(__bfloat162float(sw[d * 128 + tid]), s_q[t * RF_HD + d], u);
         const bf16 hi = __float2bfloat16_rn(u);
         const bf16 lo = __float2bfloat16_rn(u - __bfloat162float(hi));
-        bf16* base = a.U2 + static_cast<long long>(t0 + t) * 32 * D;
-        base[static_cast<long long>(h) * D + c] = hi;
-        base[static_cast<long long>(16 + h) * D + c] = lo;
+        bf16* base = a.U2 + static_cast<size_t>(t0 + t) * 32 * D;
+        base[static_cast<size_t>(h) * D + c] = hi;
+        base[static_cast<size_t>(16 + h) * D + c] = lo;
       }
       if (cbk == 0 && threadIdx.x < nt) {
         float acc = 0.f;
@@ -343,68 +371,118 @@ __device__ void fold_phase(const RouterFusedArgs& a, int l, int Tq, const float*
       }
     }
   }
+  return true;
 }
 
 // ------------------------------------------------------------------ scores phase
-// Items (tile, 64-token block), a contiguous range per CTA so that
+// Items (tile, SC_TOK-token block), a contiguous range per CTA so that
 // consecutive items share the tile's U2 rows. St[tile][j][t] = sum_c
 // x[tile][t][c] U2[tu][j][c], j < 32 (hi rows 0..15, lo rows 16..31); tu =
-// tile, or 0 when the query is shared. The item's 64 token rows (and the
-// tile's 32 U2 rows when they change) arrive by bulk copies on mbarrier 1;
-// warp w computes m16 tile (w & 3) x n8 tiles 2(w >> 2), 2(w >> 2) + 1 with
-// m16n8k16 bf16 MMAs over all channels.
+// tile, or 0 when the query is shared. Each operand arrives as one TMA
+// request in the 128-byte swizzled layout [D/64 chunks][rows][128 B] (the
+// 16-byte piece j of row r at j ^ (r & 7)): U2 on mbarrier 1 when the tile
+// changes, x double-buffered on mbarriers 2 and 3 (the CTA's first two x
+// items are requested before the grid barrier, x being an input). Warp w
+// computes m16 tile (w & 1) x n8 tile (w >> 1) with m16n8k16 bf16 MMAs.
+// Shared memory: U2 at 0, then x slots 0 and 1 (D/64 * 4 KB each); the x
+// slots start at or above FOLD_SMEM since they are filled while the fold
+// phase still uses that region.
+constexpr int FOLD_SMEM = RF_HD * 128 * 2 + 64 * RF_HD * 4;  // Wk block + Q block
+
+__device__ __forceinline__ uint8_t* scores_x_slot(uint8_t* sm, int D, int slot) {
+  const int slot_bytes = (D / 64) * SC_TOK * 128;
+  return sm + max(slot_bytes, FOLD_SMEM) + slot * slot_bytes;
+}
+
+__device__ __forceinline__ void scores_range(const RouterFusedArgs& a, int& i0, int& i1) {
+  const int n_items = a.T * (RF_TOK / SC_TOK);
+  i0 = static_cast<int>(static_cast<long long>(blockIdx.x) * n_items / gridDim.x);
+  i1 = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * n_items / gridDim.x);
+}
+
+// Lane 0: x of scores item `item` into slot `slot` (mbarrier 2 + slot).
+__device__ __forceinline__ void scores_issue_x(const RouterFusedArgs& a, int item, int slot,
+                                               uint8_t* sm, uint64_t* mb) {
+  const int slot_bytes = (a.D / 64) * SC_TOK * 128;
+  mbar_arrive_expect_tx(&mb[2 + slot], slot_bytes);
+  const int tile = item / (RF_TOK / SC_TOK), tb = item % (RF_TOK / SC_TOK);
+  tma_load_3d(scores_x_slot(sm, a.D, slot), &a.xmap3, &mb[2 + slot], 0,
+              tile * RF_TOK + tb * SC_TOK, 0);
+}
+
+// Before the grid barrier: this CTA's first two x items. Returns the slots
+// now in flight (bit s = slot s).
+__device__ __forceinline__ int scores_prefetch_x(const RouterFusedArgs& a, uint8_t* sm,
+                                                 uint64_t* mb) {
+  int i0, i1;
+  scores_range(a, i0, i1);
+  const int n = min(2, i1 - i0);
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int k = 0; k < n; ++k) scores_issue_x(a, i0 + k, k, sm, mb);
+  return (1 << n) - 1;
+}
+
 __device__ bool scores_phase(const RouterFusedArgs& a, bool shared_query, uint8_t* sm,
-                             uint64_t* mb, uint32_t* ph) {
+                             uint64_t* mb, uint32_t* ph, int& x_pending) {
   const int D = a.D;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pitch = D + 8;
-  const int per_tile = RF_TOK / 64;
-  const int n_items = a.T * per_tile;
-  const int i0 = static_cast<int>(static_cast<long long>(blockIdx.x) * n_items / gridDim.x);
-  const int i1 = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * n_items / gridDim.x);
-  bf16* sx = reinterpret_cast<bf16*>(sm);  // [64][pitch]
-  bf16* su = sx + 64 * pitch;              // [32][pitch]
-  const int mt = warp & 3, nb0 = 2 * (warp >> 2);
+  const int chunk_bytes = SC_TOK * 128;  // one 64-column chunk of 32 rows
+  const int slot_bytes = (D / 64) * chunk_bytes;
+  int i0, i1;
+  scores_range(a, i0, i1);
+  const uint8_t* su = sm;
+  const int mt = warp & 1, nt = warp >> 1;
   const int g = lane >> 2, t2 = (lane & 3) * 2;
+  const int ra = mt * 16 + (lane & 15), rb = nt * 8 + (lane & 7);
   int staged_u = -1;
-  for (int item = i0; item < i1; ++item) {
-    const int tile = item / per_tile, tb = item % per_tile;
+  for (int item = i0, k = 0; item < i1; ++item, ++k) {
+    const int slot = k & 1;
+    const int tile = item / (RF_TOK / SC_TOK), tb = item % (RF_TOK / SC_TOK);
     const int tu = shared_query ? 0 : tile;
-    const bool need_u = tu != staged_u;
-    staged_u = tu;
-    __syncthreads();
-    if (warp == 0) {
-      if (lane == 0) mbar_arrive_expect_tx(&mb[1], (64 + (need_u ? 32 : 0)) * D * 2);
-      __syncwarp();
-      fence_proxy_async_global();
-      const bf16* xs = a.x + (static_cast<size_t>(tile) * RF_TOK + tb * 64) * D;
-      bulk_load(sx + lane * pitch, xs + static_cast<size_t>(lane) * D, D * 2, &mb[1]);
-      bulk_load(sx + (lane + 32) * pitch, xs + static_cast<size_t>(lane + 32) * D, D * 2, &mb[1]);
-      if (need_u)
-        bulk_load(su + lane * pitch, a.U2 + (static_cast<size_t>(tu) * 32 + lane) * D, D * 2,
-                  &mb[1]);
-    }
-    if (!mbar_wait(&mb[1], ph[1])) return false;
-    ph[1] ^= 1;
-    float acc[2][4] = {};
-    for (int ks = 0; ks < D / 16; ++ks) {
-      uint32_t af[4];
-      ldsm_x4(af, sx + (mt * 16 + (lane & 15)) * pitch + ks * 16 + (lane >> 4) * 8);
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t bfr[2];
-        ldsm_x2(bfr, su + ((nb0 + q) * 8 + (lane & 7)) * pitch + ks * 16 + ((lane >> 3) & 1) * 8);
-        mma_bf16_16816(acc[q], af, bfr);
+    if (tu != staged_u) {
+      __syncthreads();  // every warp is done with the previous U2
+      if (threadIdx.x == 0) {
+        fence_proxy_async_global();  // U2 was written by the fold phase
+        mbar_arrive_expect_tx(&mb[1], slot_bytes);
+        tma_load_4d(sm, &a.u2map, &mb[1], 0, 0, 0, tu);
       }
+      if (!mbar_wait(&mb[1], ph[1])) return false;
+      ph[1] ^= 1;
+      staged_u = tu;
     }
-    float* st = a.S + static_cast<size_t>(tile) * 32 * RF_TOK + tb * 64 + mt * 16;
+    if (!mbar_wait(&mb[2 + slot], ph[2 + slot])) return false;
+    ph[2 + slot] ^= 1;
+    x_pending &= ~(1 << slot);
+    const uint8_t* sx = scores_x_slot(sm, D, slot);
+    // two independent accumulator chains (even / odd k-steps) for ILP
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc_b[4] = {0.f, 0.f, 0.f, 0.f};
+    auto step = [&](int ks, float (&d)[4]) {
+      const int c = ks >> 2;
+      const int ja = ((ks & 3) << 1) + (lane >> 4);
+      const int jb = ((ks & 3) << 1) + ((lane >> 3) & 1);
+      uint32_t af[4], bfr[2];
+      ldsm_x4(af, sx + c * chunk_bytes + ra * 128 + ((ja ^ (ra & 7)) << 4));
+      ldsm_x2(bfr, su + c * chunk_bytes + rb * 128 + ((jb ^ (rb & 7)) << 4));
+      mma_bf16_16816(d, af, bfr);
+    };
+#pragma unroll 2
+    for (int ks = 0; ks < D / 16; ks += 2) {  // D / 16 is even
+      step(ks, acc);
+      step(ks + 1, acc_b);
+    }
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int j = (nb0 + q) * 8 + t2;
-      st[static_cast<size_t>(j) * RF_TOK + g] = acc[q][0];
-      st[static_cast<size_t>(j + 1) * RF_TOK + g] = acc[q][1];
-      st[static_cast<size_t>(j) * RF_TOK + g + 8] = acc[q][2];
-      st[static_cast<size_t>(j + 1) * RF_TOK + g + 8] = acc[q][3];
+    for (int i = 0; i < 4; ++i) acc[i] += acc_b[i];
+    float* st = a.S + static_cast<size_t>(tile) * 32 * RF_TOK + tb * SC_TOK + mt * 16;
+    const int j = nt * 8 + t2;
+    st[static_cast<size_t>(j) * RF_TOK + g] = acc[0];
+    st[static_cast<size_t>(j + 1) * RF_TOK + g] = acc[1];
+    st[static_cast<size_t>(j) * RF_TOK + g + 8] = acc[2];
+    st[static_cast<size_t>(j + 1) * RF_TOK + g + 8] = acc[3];
+    if (item + 2 < i1) {
+      __syncthreads();  // every warp is done with this slot
+      if (threadIdx.x == 0) scores_issue_x(a, item + 2, slot, sm, mb);
+      x_pending |= 1 << slot;
     }
   }
   return true;
@@ -418,6 +496,13 @@ __device__ void softmax_phase(const RouterFusedArgs& a, bool shared_cb, float* s
   __shared__ float s_red[RF_WARPS];
   __shared__ float s_val;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  {  // the weighted sums of the next phase accumulate into a zeroed z
+    const size_t nz = static_cast<size_t>(a.T) * 16 * a.D / 4;
+    float4* z4 = reinterpret_cast<float4*>(a.z);
+    for (size_t i = static_cast<size_t>(blockIdx.x) * RF_THREADS + threadIdx.x; i < nz;
+         i += static_cast<size_t>(gridDim.x) * RF_THREADS)
+      z4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   const int n_items = a.T * 16;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     const int tile = item / 16, h = item % 16;
@@ -491,65 +576,118 @@ __device__ void softmax_phase(const RouterFusedArgs& a, bool shared_cb, float* s
 }
 
 // ------------------------------------------------------------------ wsum phase
-// Items (tile, 64-channel block), a contiguous range per CTA so that
-// consecutive items share the tile's P2 rows: z[tile][h][c] = sum_t
-// (P_hi + P_lo)[h][t] x[tile][t][c]. The tile's 1024 x 64 feature block comes
-// in 4 TMA boxes of 256 tokens x 128 bytes (128-byte swizzle: the 16-byte
-// chunk j of row r sits at chunk j ^ (r & 7)), P2[tile] (32 x 1024) by bulk
-// copies, both on mbarrier 1. Warp w computes channels 8w..8w+7 (one n8
-// tile) for both m16 tiles (hi rows, lo rows) over all 1024 tokens.
-__device__ bool wsum_phase(const RouterFusedArgs& a, uint8_t* sm, uint64_t* mb, uint32_t* ph) {
+// Items (tile, token half, 64-channel block), a contiguous range per CTA in
+// that order so that consecutive items share the half-tile's P2 rows:
+// z[tile][h][c] += sum_{t in half} (P_hi + P_lo)[h][t] x[tile][t][c]. The
+// half-tile's 512 x 64 feature block comes in 2 TMA boxes of 256 tokens x
+// 128 bytes, double-buffered on mbarriers 2 and 3 (the first two items
+// requested before the grid barrier); P2[tile][.][half] (32 x 512) in one
+// TMA request on mbarrier 1. Both are 128-byte swizzled (the 16-byte piece j
+// of row r at j ^ (r & 7)). Warp w computes channels 8w..8w+7 (one n8 tile)
+// for both m16 tiles (hi rows, lo rows). z was zeroed in the softmax phase;
+// each element receives exactly two additions (one per half), so the
+// result does not depend on their order.
+// Shared memory: P2 [8 chunks][32][128 B] | x slot 0 | x slot 1 (64 KB each).
+constexpr int WS_P_BYTES = (WS_HALF / 64) * 32 * 128;
+constexpr int WS_X_BYTES = WS_HALF * 128;
+
+__device__ __forceinline__ void red_add_f32x2(float* p, float a, float b) {
+  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(a), "f"(b) : "memory");
+}
+
+__device__ __forceinline__ void wsum_range(const RouterFusedArgs& a, int& i0, int& i1) {
+  const int n_items = a.T * 2 * (a.D / 64);
+  i0 = static_cast<int>(static_cast<long long>(blockIdx.x) * n_items / gridDim.x);
+  i1 = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * n_items / gridDim.x);
+}
+
+__device__ __forceinline__ void wsum_issue_x(const RouterFusedArgs& a, int item, int slot,
+                                             uint8_t* sm, uint64_t* mb) {
+  const int cblocks = a.D / 64;
+  const int th = item / cblocks, cbk = item % cblocks;
+  uint8_t* dst = sm + WS_P_BYTES + slot * WS_X_BYTES;
+  mbar_arrive_expect_tx(&mb[2 + slot], WS_X_BYTES);
+  for (int bx = 0; bx < WS_HALF / WS_BOX; ++bx)
+    tma_load_2d(dst + bx * WS_BOX * 128, &a.xmap, &mb[2 + slot], cbk * 64,
+                (th >> 1) * RF_TOK + (th & 1) * WS_HALF + bx * WS_BOX);
+}
+
+__device__ __forceinline__ int wsum_prefetch_x(const RouterFusedArgs& a, uint8_t* sm,
+                                               uint64_t* mb) {
+  int i0, i1;
+  wsum_range(a, i0, i1);
+  const int n = min(2, i1 - i0);
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int k = 0; k < n; ++k) wsum_issue_x(a, i0 + k, k, sm, mb);
+  return (1 << n) - 1;
+}
+
+__device__ bool wsum_phase(const RouterFusedArgs& a, uint8_t* sm, uint64_t* mb, uint32_t* ph,
+                           int& x_pending) {
   const int D = a.D;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cblocks = D / 64;
-  const int n_items = a.T * cblocks;
-  const int i0 = static_cast<int>(static_cast<long long>(blockIdx.x) * n_items / gridDim.x);
-  const int i1 = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * n_items / gridDim.x);
-  uint8_t* sxb = sm;  // 4 boxes [256 tokens][128 B], 1024-byte aligned
-  bf16* sp = reinterpret_cast<bf16*>(sm + (RF_TOK / WS_BOX) * WS_BOX * 128);  // [32][WS_PPITCH]
+  int i0, i1;
+  wsum_range(a, i0, i1);
+  const uint8_t* sp = sm;
   const int g = lane >> 2, t2 = (lane & 3) * 2;
-  int staged_tile = -1;
-  for (int item = i0; item < i1; ++item) {
-    const int tile = item / cblocks, cbk = item % cblocks;
-    const bool need_p = tile != staged_tile;
-    staged_tile = tile;
-    __syncthreads();
-    if (warp == 0) {
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&mb[1], RF_TOK * 128 + (need_p ? 32 * RF_TOK * 2 : 0));
-        for (int bx = 0; bx < RF_TOK / WS_BOX; ++bx)
-          tma_load_2d(sxb + bx * WS_BOX * 128, &a.xmap, &mb[1], cbk * 64,
-                      tile * RF_TOK + bx * WS_BOX);
+  int staged = -1;
+  for (int item = i0, k = 0; item < i1; ++item, ++k) {
+    const int slot = k & 1;
+    const int th = item / cblocks, cbk = item % cblocks;  // th = 2 tile + half
+    const int tile = th >> 1;
+    if (th != staged) {
+      __syncthreads();  // every warp is done with the previous P2
+      if (threadIdx.x == 0) {
+        fence_proxy_async_global();  // P2 was written by the softmax phase
+        mbar_arrive_expect_tx(&mb[1], WS_P_BYTES);
+        tma_load_4d(sm, &a.p2map, &mb[1], 0, 0, (th & 1) * (WS_HALF / 64), tile);
       }
-      __syncwarp();
-      if (need_p) {
-        fence_proxy_async_global();
-        bulk_load(sp + lane * WS_PPITCH, a.P2 + (static_cast<size_t>(tile) * 32 + lane) * RF_TOK,
-                  RF_TOK * 2, &mb[1]);
-      }
+      if (!mbar_wait(&mb[1], ph[1])) return false;
+      ph[1] ^= 1;
+      staged = th;
     }
-    if (!mbar_wait(&mb[1], ph[1])) return false;
-    ph[1] ^= 1;
-    float acc[2][4] = {};
-    for (int ks = 0; ks < RF_TOK / 16; ++ks) {
+    if (!mbar_wait(&mb[2 + slot], ph[2 + slot])) return false;
+    ph[2 + slot] ^= 1;
+    x_pending &= ~(1 << slot);
+    const uint8_t* sxb = sm + WS_P_BYTES + slot * WS_X_BYTES;
+    float acc[2][4] = {}, acc_b[2][4] = {};  // odd k-steps: a second chain for ILP
+    auto step = [&](int ks, float (&d)[2][4]) {
       // B[k = token][n = channel] stored n-contiguous: transposed 8x8 loads
       const int r = ks * 16 + (lane & 15);
       const int rr = r & (WS_BOX - 1);
       uint32_t bfr[2];
       ldsm_x2_trans(bfr, sxb + (r / WS_BOX) * WS_BOX * 128 + rr * 128 + ((warp ^ (rr & 7)) << 4));
+      const int c = ks >> 2;
+      const int ja = ((ks & 3) << 1) + (lane >> 4);
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
+        const int ra = mt * 16 + (lane & 15);
         uint32_t af[4];
-        ldsm_x4(af, sp + (mt * 16 + (lane & 15)) * WS_PPITCH + ks * 16 + (lane >> 4) * 8);
-        mma_bf16_16816(acc[mt], af, bfr);
+        ldsm_x4(af, sp + c * (32 * 128) + ra * 128 + ((ja ^ (ra & 7)) << 4));
+        mma_bf16_16816(d[mt], af, bfr);
       }
+    };
+#pragma unroll 2
+    for (int ks = 0; ks < WS_HALF / 16; ks += 2) {
+      step(ks, acc);
+      step(ks + 1, acc_b);
     }
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[mt][i] += acc_b[mt][i];
     // row g of m-tile 0 is the hi part of head g, row g of m-tile 1 its lo part
     float* zt = a.z + static_cast<size_t>(tile) * 16 * D + cbk * 64 + warp * 8 + t2;
-    *reinterpret_cast<float2*>(zt + static_cast<size_t>(g) * D) =
-        make_float2(acc[0][0] + acc[1][0], acc[0][1] + acc[1][1]);
-    *reinterpret_cast<float2*>(zt + static_cast<size_t>(g + 8) * D) =
-        make_float2(acc[0][2] + acc[1][2], acc[0][3] + acc[1][3]);
+    red_add_f32x2(zt + static_cast<size_t>(g) * D, acc[0][0] + acc[1][0], acc[0][1] + acc[1][1]);
+    red_add_f32x2(zt + static_cast<size_t>(g + 8) * D, acc[0][2] + acc[1][2],
+                  acc[0][3] + acc[1][3]);
+    if (item + 2 < i1) {
+      __syncthreads();  // every warp is done with this slot
+      if (threadIdx.x == 0) wsum_issue_x(a, item + 2, slot, sm, mb);
+      x_pending |= 1 << slot;
+    }
   }
   return true;
 }
@@ -664,19 +802,24 @@ __global__ void __launch_bounds__(RF_THREADS, 1)
   // 1024-byte alignment for the swizzled TMA boxes (the launch adds the slack)
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   float* sf = reinterpret_cast<float*>(sm);
-  __shared__ __align__(8) uint64_t s_mb[2];  // 0: projection weights, 1: everything else
+  // mbarriers: 0 weights (projections, fold), 1 other staged operands,
+  // 2 and 3 the two x slots of the scores and weighted-sum phases
+  __shared__ __align__(8) uint64_t s_mb[4];
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
-    mbar_init(&s_mb[0], 1);
-    mbar_init(&s_mb[1], 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&s_mb[i], 1);
     fence_mbar_init();
     tma_prefetch_desc(&a.xmap);
+    tma_prefetch_desc(&a.xmap3);
+    tma_prefetch_desc(&a.u2map);
+    tma_prefetch_desc(&a.p2map);
   }
   __syncthreads();
-  uint32_t ph[2] = {0u, 0u};
+  uint32_t ph[4] = {0u, 0u, 0u, 0u};
   unsigned gen = 0;
   bool ok = true;
   bool w_pending = false;  // weight copies of the next projection phase in flight
+  int x_pending = 0;       // x slots (bits) requested ahead of their phase
   const int T = a.T, D = a.D, G = a.G;
   auto sync = [&]() {
     if (ok) ok = grid_sync(a.bar, gen);
@@ -706,15 +849,26 @@ __global__ void __launch_bounds__(RF_THREADS, 1)
   prefetch_w(a.Wq[0], D, D);
   if (sync()) project(1, D, D, a.Wq[0], a.bq[0], a.Q, D, false, [&](int, int) { return a.h; });
   for (int l = 0; l < 4 && ok; ++l) {
+    // this CTA's first fold item: its Wk block is requested before the barrier
+    __syncthreads();
+    w_pending = static_cast<int>(blockIdx.x) < (D / 128) * a.heads;
+    if (w_pending && warp == 0) fold_issue_w(a.Wk[l], D, blockIdx.x, sm, &s_mb[0]);
     if (!sync()) break;
     const bool shared_q = l == 0;
-    fold_phase(a, l, shared_q ? 1 : T, a.Q, shared_q ? 0 : D, sf);
+    {
+      const bool pre = w_pending;
+      w_pending = false;
+      if (!fold_phase(a, l, shared_q ? 1 : T, a.Q, shared_q ? 0 : D, sm, s_mb, ph, pre)) ok = false;
+    }
+    // the scores phase's first x items (x is an input) before the barrier
+    x_pending = scores_prefetch_x(a, sm, s_mb);
     if (!sync()) break;
-    if (!scores_phase(a, shared_q, sm, s_mb, ph)) ok = false;
+    if (!scores_phase(a, shared_q, sm, s_mb, ph, x_pending)) ok = false;
+    x_pending = wsum_prefetch_x(a, sm, s_mb);  // the softmax phase uses no shared memory
     if (!sync()) break;
     softmax_phase(a, shared_q, sf);
     if (!sync()) break;
-    if (!wsum_phase(a, sm, s_mb, ph)) ok = false;
+    if (!wsum_phase(a, sm, s_mb, ph, x_pending)) ok = false;
     // o = Wv_h z_h + bv: the input row of output row m for columns of head h is z[m][h]
     prefetch_w(a.Wv[l], D, D);
     if (!sync()) break;
@@ -784,8 +938,10 @@ __global__ void __launch_bounds__(RF_THREADS, 1)
   if (ok && sync())
     route_phase(a, reinterpret_cast<double*>(sm),
                 reinterpret_cast<double*>(sm) + IVC_MAX_QUANTILE_GROUP);
-  // a prefetch whose phase never ran (a barrier gave up): let its copies land
+  // prefetches whose phase never ran (a barrier gave up): let their copies land
   if (w_pending) (void)mbar_wait(&s_mb[0], ph[0]);
+  for (int sl = 0; sl < 2; ++sl)
+    if (x_pending & (1 << sl)) (void)mbar_wait(&s_mb[2 + sl], ph[2 + sl]);
   if (!ok && threadIdx.x == 0) atomicOr(a.status, DEV_WAIT_TIMEOUT);
 }
 
@@ -794,10 +950,10 @@ size_t router_fused_smem(int D, int G) {
   const size_t gemv = GV_ROWS * (K + 8) * 4 + GV_COLS * (K + 8) * 2 +
                       static_cast<size_t>(RF_WARPS) * GV_ROWS * GV_COLS * 4;
   const size_t route = 2 * static_cast<size_t>(IVC_MAX_QUANTILE_GROUP) * sizeof(double);
-  const size_t scores = static_cast<size_t>(96) * (D + 8) * sizeof(bf16);
-  const size_t wsum = static_cast<size_t>(RF_TOK) * 128 +
-                      static_cast<size_t>(32) * WS_PPITCH * sizeof(bf16);
-  const size_t fold = static_cast<size_t>(64) * RF_HD * sizeof(float);
+  const size_t sc_slot = static_cast<size_t>(D / 64) * SC_TOK * 128;
+  const size_t scores = (sc_slot > FOLD_SMEM ? sc_slot : FOLD_SMEM) + 2 * sc_slot;  // U2, 2 x slots
+  const size_t wsum = static_cast<size_t>(WS_P_BYTES) + 2 * static_cast<size_t>(WS_X_BYTES);
+  const size_t fold = FOLD_SMEM;
   size_t m = gemv;
   for (size_t v : {route, scores, wsum, fold, static_cast<size_t>(D) * sizeof(float)})
     if (v > m) m = v;
@@ -830,6 +986,26 @@ int launch_router_fused(const ivc_router* r, const void* x, const int32_t* valid
   RouterFusedArgs a{};
   if (map_rows_2d(&a.xmap, x, static_cast<long long>(T) * RF_TOK, r->D, WS_BOX) != IVC_OK)
     return IVC_ECUDA;
+  {
+    const unsigned long long D2 = static_cast<unsigned long long>(r->D) * 2;  // row bytes
+    const unsigned long long chunks = static_cast<unsigned long long>(r->D) / 64;
+    // x: {64 ch, tokens, chunks}, rows of D2 bytes, chunks 128 bytes apart
+    const unsigned long long xd[3] = {64, static_cast<unsigned long long>(T) * RF_TOK, chunks};
+    const unsigned long long xs[2] = {D2, 128};
+    const unsigned xb[3] = {64, SC_TOK, static_cast<unsigned>(chunks)};
+    // U2: {64, 32 rows, chunks, T}
+    const unsigned long long ud[4] = {64, 32, chunks, static_cast<unsigned long long>(T)};
+    const unsigned long long us[3] = {D2, 128, 32 * D2};
+    const unsigned ub[4] = {64, 32, static_cast<unsigned>(chunks), 1};
+    // P2: {64 tokens, 32 rows, 16 chunks, T}, rows of 1024 tokens
+    const unsigned long long pd[4] = {64, 32, RF_TOK / 64, static_cast<unsigned long long>(T)};
+    const unsigned long long ps[3] = {RF_TOK * 2, 128, 32ull * RF_TOK * 2};
+    const unsigned pb[4] = {64, 32, WS_HALF / 64, 1};
+    if (map_bf16(&a.xmap3, 3, x, xd, xs, xb) != IVC_OK ||
+        map_bf16(&a.u2map, 4, b.U2, ud, us, ub) != IVC_OK ||
+        map_bf16(&a.p2map, 4, b.P2, pd, ps, pb) != IVC_OK)
+      return IVC_ECUDA;
+  }
   a.x = static_cast<const bf16*>(x);
   a.valid_len = valid_len;
   a.T = T;
