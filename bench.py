@@ -83,6 +83,8 @@ def algorithmic(w, T):
         "pool.wsum": (2.0 * T * 32 * 1024 * D, bf * (tok * D + T * 32 * 1024) + f32 * T * 32 * D),
         "pool.attention": (4.0 * tok * D, f32 * tok * 2 * D),          # per layer launch
         "ps_stats": (3.0 * tok * C, bf * tok * C + f32 * 2 * (r256 + r64)),
+        # compaction reads and writes the kept rows (all-256 upper bound here;
+        # the bench prices it with the step's actual mask)
         "compact": (0.0, bf * 2 * r256 * H),
         "route": (0.0, f32 * 2 * T),
     }
@@ -383,6 +385,18 @@ def run_ivc(args):
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                 "traffic": None, "kernel": dom, "peak_source": f"{src} hbm_gbs"}
+    # the HBM-bound kernels: algorithmic bytes per launch / traced launch time
+    hbm = {}
+    kept_rows = int(bufs["offsets"][-1].item())  # 256 (T - k) + 64 k of this image
+    for k in ("ps_stats", "compact"):
+        if k in trace and trace[k]["launches"] > 0:
+            us = 1e3 * trace[k]["ms"] / trace[k]["launches"]
+            b_launch = alg[k][1] / (trace[k]["launches"] / n_trace)
+            if k == "compact":
+                b_launch = 2.0 * 2 * kept_rows * w.H
+            gbs = b_launch / (us * 1e-6) / 1e9
+            hbm[k] = {"bytes_per_launch": b_launch, "us_per_launch": us, "achieved": gbs,
+                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"]}
     # whole-step roofline: algorithmic FLOPs at the dense bf16 peak vs bytes at HBM peak.
     # F_literal counts the method as the pages state it (K/V projections of all
     # tokens); F_folded is what the folded pooling actually has to compute.
@@ -464,7 +478,7 @@ def run_ivc(args):
                        "flow": ("router first, each tile through its selected path" if routed
                                 else "both paths for every tile, then compaction"),
                        "parallelism": f"replicas x{world}, one image per GPU, no collective"},
-            "roofline": roof, "step_roofline": step_roofline,
+            "roofline": roof, "step_roofline": step_roofline, "hbm_kernels": hbm,
             "kernels_ms_per_step": {k: round(v, 5) for k, v in per_step_ms.items()},
             "traced_ms_per_step": trace_total, "parts_graph_ms": parts,
             "clocks": clocks, "e2e": e2e, "gpu_launches": int(round(launches_per_step * args.steps)),

@@ -36,7 +36,9 @@ MHA layers with their own Q/K/V/out projections and biases, 16 heads, scale
 tokens are a suffix and are excluded from the softmax; gating residual wraps
 the listed block (h <- h + LN(block(h))), dropout is identity at inference;
 quantile by linear interpolation in fp64, per image; gate column 0 means
-"compress to 64"; compaction keeps images, tiles and tokens in order.
+"compress to 64"; compaction keeps images, tiles and tokens in order;
+sequence assembly: the k-th run of 256 placeholders is tile k, a compressed
+tile keeps its first 64, positions count the kept tokens per sequence.
 """
 from __future__ import annotations
 
@@ -263,6 +265,59 @@ def compact(Y256: np.ndarray, Y64: np.ndarray, mask: np.ndarray) -> np.ndarray:
     if not parts:
         return np.zeros((0, Y256.shape[-1]))
     return np.concatenate(parts, axis=0)
+
+
+# ----------------------------------------------------------------------------
+# Sequence assembly  ([VIR] section 4, compress_visual_tokens_in_sentence:
+# a compressed tile keeps 64 of its 256 <IMG_CONTEXT> positions and 192 are
+# deleted, the position indices following; [PS] "视觉 Token 如何注入": the
+# embedded prompt's <IMG_CONTEXT> positions take the visual rows in order)
+# ----------------------------------------------------------------------------
+def assemble_sequence(input_ids, seq_offsets, img_context_id: int, embed_table: np.ndarray,
+                      visual: np.ndarray, mask, offsets, keep: int = 64,
+                      full: int = 256) -> Dict[str, np.ndarray]:
+    """Splice the compacted visual rows into a batch of token sequences.
+
+    The j-th <IMG_CONTEXT> placeholder of the batch (sequence order) is
+    placeholder r = j % full of tile t = j // full. For a compressed tile
+    (mask[t] = 1) placeholders r >= keep are deleted; a kept placeholder takes
+    visual row offsets[t] + r; every other token takes its row of the
+    embedding table. Position ids count the kept tokens from 0 in each
+    sequence. Placeholders beyond full * T (a prompt with more than T tiles)
+    are treated as text tokens. Returns ids, embeds, positions, the new
+    sequence offsets and the number of placeholders seen."""
+    ids = np.asarray(input_ids)
+    T = len(mask)
+    out_ids: List[int] = []
+    rows: List[np.ndarray] = []
+    pos: List[int] = []
+    new_offs = [0]
+    j = 0
+    for b in range(len(seq_offsets) - 1):
+        start = len(out_ids)
+        for p in range(int(seq_offsets[b]), int(seq_offsets[b + 1])):
+            tok = int(ids[p])
+            if tok == img_context_id:
+                jj = j
+                j += 1
+                if jj < full * T:
+                    t, r = divmod(jj, full)
+                    if mask[t] and r >= keep:
+                        continue  # one of the deleted placeholders
+                    out_ids.append(tok)
+                    rows.append(visual[int(offsets[t]) + r])
+                    pos.append(len(out_ids) - 1 - start)
+                    continue
+            out_ids.append(tok)
+            rows.append(embed_table[tok])
+            pos.append(len(out_ids) - 1 - start)
+        new_offs.append(len(out_ids))
+    H = embed_table.shape[1]
+    return {"ids": np.array(out_ids, dtype=np.int64),
+            "embeds": np.array(rows).reshape(-1, H),
+            "positions": np.array(pos, dtype=np.int64),
+            "seq_offsets": np.array(new_offs, dtype=np.int64),
+            "placeholders": j}
 
 
 # ----------------------------------------------------------------------------

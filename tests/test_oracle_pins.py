@@ -431,3 +431,87 @@ def test_flash_compress_small_composes_steps():
     # gate override routes on the given vector
     res2 = O.flash_compress(x, lens, offs, mlp1, mlp2, r, gate_override=np.array([0.9, 0.95, 0.99, 0.2]))
     assert res2["mask"].tolist() == [0, 1, 1, 0]
+
+
+# ------------------------------------------------------------------ sequence assembly
+def test_assemble_worked_example_scaled_down():
+    """Hand-built example with 4 placeholders per tile, 1 kept when compressed
+    (the same rule as 256 / 64, scaled down): ids 5 [9 9 9 9] [9 9 9 9] 7 with
+    tile 0 compressed gives 5 9 9 9 9 9 7; tile 0's one row, then tile 1's
+    four rows, then the table row of 7."""
+    tab = np.arange(10 * 3, dtype=np.float64).reshape(10, 3)
+    vis = 100.0 + np.arange(5 * 3, dtype=np.float64).reshape(5, 3)
+    ids = np.array([5, 9, 9, 9, 9, 9, 9, 9, 9, 7])
+    res = O.assemble_sequence(ids, [0, 10], 9, tab, vis, mask=[1, 0], offsets=[0, 1, 5],
+                              keep=1, full=4)
+    np.testing.assert_array_equal(res["ids"], [5, 9, 9, 9, 9, 9, 7])
+    expect = np.stack([tab[5], vis[0], vis[1], vis[2], vis[3], vis[4], tab[7]])
+    np.testing.assert_array_equal(res["embeds"], expect)
+    np.testing.assert_array_equal(res["positions"], np.arange(7))
+    np.testing.assert_array_equal(res["seq_offsets"], [0, 7])
+    assert res["placeholders"] == 8
+
+
+def _prompt(tiles_per_seq, text=(3, 2), img_id=7, V=50, seed=0):
+    rng = np.random.default_rng(seed)
+    ids, offs = [], [0]
+    for n in tiles_per_seq:
+        seq = list(rng.integers(10, V, text[0])) + [img_id] * (256 * n) + list(rng.integers(10, V, text[1]))
+        ids += seq
+        offs.append(len(ids))
+    return np.array(ids), np.array(offs)
+
+
+def test_assemble_lengths_follow_the_page_counts():
+    """Every compressed tile removes 192 of its 256 placeholders; uncompressed
+    tiles keep all 256 (page numbers in tests/golden)."""
+    g = GOLD["compressed_tile"]["value"]
+    tiles = [3, 1, 2]
+    ids, offs = _prompt(tiles)
+    T = sum(tiles)
+    mask = np.array([1, 0, 1, 0, 0, 1])
+    vis_offs = O.compaction_offsets(mask)
+    H = 4
+    tab = RNG.standard_normal((50, H))
+    vis = RNG.standard_normal((int(vis_offs[-1]), H))
+    res = O.assemble_sequence(ids, offs, 7, tab, vis, mask, vis_offs)
+    k = int(mask.sum())
+    assert len(res["ids"]) == len(ids) - g["deleted"] * k
+    # per sequence: the tiles of sequence b are consecutive
+    t0 = 0
+    for b, n in enumerate(tiles):
+        kb = int(mask[t0:t0 + n].sum())
+        assert res["seq_offsets"][b + 1] - res["seq_offsets"][b] == (offs[b + 1] - offs[b]) - 192 * kb
+        seg = res["positions"][res["seq_offsets"][b]:res["seq_offsets"][b + 1]]
+        np.testing.assert_array_equal(seg, np.arange(len(seg)))
+        t0 += n
+    # the kept placeholders take every visual row exactly once, in order
+    sel = res["ids"] == 7
+    np.testing.assert_array_equal(res["embeds"][sel], vis)
+    assert sel.sum() == g["placeholders"] * (T - k) + g["kept"] * k
+    np.testing.assert_array_equal(res["embeds"][~sel], tab[res["ids"][~sel]])
+
+
+def test_assemble_no_compression_is_plain_injection():
+    """With no tile compressed the result is the plain injection of [PS]
+    "视觉 Token 如何注入": input_embeds[ids == IMG_CONTEXT] = visual rows."""
+    ids, offs = _prompt([2])
+    H = 3
+    tab = RNG.standard_normal((50, H))
+    vis = RNG.standard_normal((512, H))
+    res = O.assemble_sequence(ids, offs, 7, tab, vis, [0, 0], [0, 256, 512])
+    ref = tab[ids].copy()
+    ref[ids == 7] = vis
+    np.testing.assert_array_equal(res["ids"], ids)
+    np.testing.assert_array_equal(res["embeds"], ref)
+
+
+def test_assemble_extra_placeholders_stay_text():
+    ids, offs = _prompt([1])
+    ids = np.concatenate([ids, [7, 7]])
+    offs = np.array([0, len(ids)])
+    tab = RNG.standard_normal((50, 2))
+    vis = RNG.standard_normal((64, 2))
+    res = O.assemble_sequence(ids, offs, 7, tab, vis, [1], [0, 64])
+    assert res["placeholders"] == 258
+    np.testing.assert_array_equal(res["embeds"][-2:], tab[[7, 7]])

@@ -19,30 +19,22 @@
 namespace ivc {
 
 // ---------------------------------------------------------------- LN statistics
-// One CTA per 4x4 block of ViT tokens = one factor-0.25 row; its four 2x2
-// sub-blocks are four factor-0.5 rows. Warp w = 4q + r reduces token
-// (4a+q, 4b+r) over C channels (sums shifted by the token's first value to
-// keep the one-pass variance well conditioned); the token statistics are
-// then merged per row with the pairwise (Chan) update in fp64.
-__global__ void __launch_bounds__(512) ps_stats_kernel(const bf16* __restrict__ x, int C,
-                                                       float* __restrict__ mean_half,
-                                                       float* __restrict__ rstd_half,
-                                                       float* __restrict__ mean_quarter,
-                                                       float* __restrict__ rstd_quarter) {
-  __shared__ double s_mean[16], s_m2[16];
-  const int cell = blockIdx.x;  // tile * 64 + a * 8 + b
-  const int tile = cell >> 6, a = (cell >> 3) & 7, b = cell & 7;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q = warp >> 2, r = warp & 3;
-  pdl_wait();
-  pdl_trigger();
-  const bf16* tok = x + ((static_cast<long long>(tile) * 32 + 4 * a + q) * 32 + 4 * b + r) * C;
-  const float shift = __bfloat162float(tok[0]);
-  float s1 = 0.f, s2 = 0.f;
-  const uint4* v = reinterpret_cast<const uint4*>(tok);
-  for (int i = lane; i < C / 8; i += 32) {
-    const uint4 u = v[i];
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+// A 4x4 block of ViT tokens ("cell") is one factor-0.25 row; its four 2x2
+// sub-blocks are four factor-0.5 rows. Each CTA takes PS_CELLS adjacent
+// cells; warp w = 4q + r reduces token (4a+q, 4b+r) of each of them over C
+// channels (sums shifted by the token's first value to keep the one-pass
+// variance well conditioned), all of its loads in flight before their use.
+// The token statistics are then merged per row with the pairwise (Chan)
+// update in fp64.
+constexpr int PS_CELLS = 2;
+
+__device__ __forceinline__ void token_moments(const uint4* __restrict__ v, int pieces, int lane,
+                                              float shift, float& s1, float& s2,
+                                              const uint4 (&u)[4], int i0) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    if (i0 + k * 32 + lane >= pieces) continue;
+    const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const float lo = __uint_as_float(w[j] << 16) - shift;
@@ -51,43 +43,90 @@ __global__ void __launch_bounds__(512) ps_stats_kernel(const bf16* __restrict__ 
       s2 = fmaf(lo, lo, fmaf(hi, hi, s2));
     }
   }
+  (void)v;
+}
+
+__global__ void __launch_bounds__(512) ps_stats_kernel(const bf16* __restrict__ x, int C,
+                                                       float* __restrict__ mean_half,
+                                                       float* __restrict__ rstd_half,
+                                                       float* __restrict__ mean_quarter,
+                                                       float* __restrict__ rstd_quarter) {
+  __shared__ double s_mean[PS_CELLS][16], s_m2[PS_CELLS][16];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q = warp >> 2, r = warp & 3;
+  pdl_wait();
+  pdl_trigger();
+  const int pieces = C / 8;  // 16-byte pieces per token
+  const uint4* v[PS_CELLS];
+  float shift[PS_CELLS], s1[PS_CELLS], s2[PS_CELLS];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-    s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+  for (int e = 0; e < PS_CELLS; ++e) {
+    const int cell = blockIdx.x * PS_CELLS + e;  // tile * 64 + a * 8 + b
+    const int tile = cell >> 6, a = (cell >> 3) & 7, b = cell & 7;
+    const bf16* tok = x + ((static_cast<long long>(tile) * 32 + 4 * a + q) * 32 + 4 * b + r) * C;
+    v[e] = reinterpret_cast<const uint4*>(tok);
+    shift[e] = __bfloat162float(tok[0]);
+    s1[e] = s2[e] = 0.f;
   }
-  if (lane == 0) {
-    const double n = C;
-    s_mean[warp] = shift + s1 / n;
-    s_m2[warp] = fmax(static_cast<double>(s2) - static_cast<double>(s1) * s1 / n, 0.0);
+  for (int i0 = 0; i0 < pieces; i0 += 128) {
+    uint4 u[PS_CELLS][4];
+#pragma unroll
+    for (int e = 0; e < PS_CELLS; ++e)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int i = i0 + k * 32 + lane;
+        // plain loads: x stays in L2 for the GEMMs that follow
+        u[e][k] = i < pieces ? __ldg(v[e] + i) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+    for (int e = 0; e < PS_CELLS; ++e) token_moments(v[e], pieces, lane, shift[e], s1[e], s2[e], u[e], i0);
+  }
+#pragma unroll
+  for (int e = 0; e < PS_CELLS; ++e) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      s1[e] += __shfl_xor_sync(0xffffffffu, s1[e], o);
+      s2[e] += __shfl_xor_sync(0xffffffffu, s2[e], o);
+    }
+    if (lane == 0) {
+      const double n = C;
+      s_mean[e][warp] = shift[e] + s1[e] / n;
+      s_m2[e][warp] =
+          fmax(static_cast<double>(s2[e]) - static_cast<double>(s1[e]) * s1[e] / n, 0.0);
+    }
   }
   __syncthreads();
   const double eps = 1e-5;
-  if (threadIdx.x < 4 && mean_half != nullptr) {
-    const int sa = threadIdx.x >> 1, sb = threadIdx.x & 1;
+  if (threadIdx.x < 4 * PS_CELLS && mean_half != nullptr) {
+    const int e = threadIdx.x >> 2;
+    const int cell = blockIdx.x * PS_CELLS + e;
+    const int tile = cell >> 6, a = (cell >> 3) & 7, b = cell & 7;
+    const int sa = (threadIdx.x >> 1) & 1, sb = threadIdx.x & 1;
     const int w0 = 4 * (2 * sa) + 2 * sb;  // tokens (2sa+di, 2sb+dj)
     const int ids[4] = {w0, w0 + 1, w0 + 4, w0 + 5};
     double mu = 0.0;
-    for (int i = 0; i < 4; ++i) mu += s_mean[ids[i]];
+    for (int i = 0; i < 4; ++i) mu += s_mean[e][ids[i]];
     mu *= 0.25;
     double m2 = 0.0;
     for (int i = 0; i < 4; ++i) {
-      const double d = s_mean[ids[i]] - mu;
-      m2 += s_m2[ids[i]] + C * d * d;
+      const double d = s_mean[e][ids[i]] - mu;
+      m2 += s_m2[e][ids[i]] + C * d * d;
     }
     const double var = m2 / (4.0 * C);
     const long long row = static_cast<long long>(tile) * 256 + (2 * a + sa) * 16 + (2 * b + sb);
     mean_half[row] = static_cast<float>(mu);
     rstd_half[row] = static_cast<float>(1.0 / sqrt(var + eps));
   }
-  if (threadIdx.x == 32 && mean_quarter != nullptr) {
+  if (threadIdx.x >= 32 && threadIdx.x < 32 + PS_CELLS && mean_quarter != nullptr) {
+    const int e = threadIdx.x - 32;
+    const int cell = blockIdx.x * PS_CELLS + e;
     double mu = 0.0;
-    for (int i = 0; i < 16; ++i) mu += s_mean[i];
+    for (int i = 0; i < 16; ++i) mu += s_mean[e][i];
     mu *= 1.0 / 16.0;
     double m2 = 0.0;
     for (int i = 0; i < 16; ++i) {
-      const double d = s_mean[i] - mu;
-      m2 += s_m2[i] + C * d * d;
+      const double d = s_mean[e][i] - mu;
+      m2 += s_m2[e][i] + C * d * d;
     }
     const double var = m2 / (16.0 * C);
     mean_quarter[cell] = static_cast<float>(mu);
@@ -99,8 +138,9 @@ int launch_ps_stats(const bf16* x, int T, int C, float* mean_half, float* rstd_h
                     float* mean_quarter, float* rstd_quarter, const Launch& L) {
   if (T == 0) return IVC_OK;
   TraceScope ts("ps_stats", L.stream);
-  return launch_k(ps_stats_kernel, dim3(T * 64), dim3(512), 0, L.stream, 1, x, C, mean_half,
-                  rstd_half, mean_quarter, rstd_quarter);
+  // T * 64 cells, an even number
+  return launch_k(ps_stats_kernel, dim3(T * 64 / PS_CELLS), dim3(512), 0, L.stream, 1, x, C,
+                  mean_half, rstd_half, mean_quarter, rstd_quarter);
 }
 
 // ---------------------------------------------------------------- LN fold

@@ -762,15 +762,19 @@ int launch_route_lists(const uint8_t* mask, const int32_t* offsets, int T, int* 
 }
 
 // ---------------------------------------------------------------- compaction
-// Grid (T, 8): CTA (t, y) copies rows 32y..32y+31 of tile t when they exist
-// (64 rows for a compressed tile, 256 otherwise), 16 bytes per thread-step.
+// Grid (T, 32): CTA (t, y) copies rows 8y..8y+7 of tile t when they exist
+// (64 rows for a compressed tile, 256 otherwise): 8 rows x H bf16, each
+// thread first loading all of its 16-byte pieces (H / 128 of them per
+// thread-row pair, 8 for H = 2048), then storing them.
+constexpr int COMPACT_ROWS = 8;
+
 __global__ void __launch_bounds__(256) compact_kernel(const bf16* __restrict__ Y256,
                                                       const bf16* __restrict__ Y64,
                                                       const uint8_t* __restrict__ mask,
                                                       const int32_t* __restrict__ offsets, int H,
                                                       bf16* __restrict__ out) {
   const int t = blockIdx.x;
-  const int r0 = blockIdx.y * 32;
+  const int r0 = blockIdx.y * COMPACT_ROWS;
   pdl_wait();
   pdl_trigger();
   const bool comp = mask[t] != 0;
@@ -779,18 +783,30 @@ __global__ void __launch_bounds__(256) compact_kernel(const bf16* __restrict__ Y
   const bf16* src = comp ? Y64 + (static_cast<long long>(t) * 64 + r0) * H
                          : Y256 + (static_cast<long long>(t) * 256 + r0) * H;
   bf16* dst = out + (static_cast<long long>(offsets[t]) + r0) * H;
-  const int per_row = H / 8;
+  const int n = COMPACT_ROWS * H / 8;  // 16-byte pieces of the 8 rows (contiguous)
   const uint4* s4 = reinterpret_cast<const uint4*>(src);
   uint4* d4 = reinterpret_cast<uint4*>(dst);
-  for (int i = threadIdx.x; i < 32 * per_row; i += 256) d4[i] = s4[i];
+  for (int i0 = 0; i0 < n; i0 += 8 * 256) {
+    uint4 u[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i = i0 + k * 256 + threadIdx.x;
+      if (i < n) u[k] = __ldcs(s4 + i);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i = i0 + k * 256 + threadIdx.x;
+      if (i < n) __stcs(d4 + i, u[k]);
+    }
+  }
 }
 
 int launch_compact(const bf16* Y256, const bf16* Y64, const uint8_t* mask,
                    const int32_t* offsets, int T, int H, bf16* out, const Launch& L) {
   if (T == 0) return IVC_OK;
   TraceScope ts("compact", L.stream);
-  return launch_k(compact_kernel, dim3(T, 8), dim3(256), 0, L.stream, 1, Y256, Y64, mask, offsets,
-                  H, out);
+  return launch_k(compact_kernel, dim3(T, 256 / COMPACT_ROWS), dim3(256), 0, L.stream, 1, Y256,
+                  Y64, mask, offsets, H, out);
 }
 
 }  // namespace ivc
