@@ -503,7 +503,27 @@ def run_op(args):
     w, T = inp["workload"], inp["T"]
     x = inp["x"].cuda()
     vl, offs = inp["valid_len"].cuda(), inp["image_offsets"].cuda()
-    if args.op in ("flash_dual", "flash_routed"):
+    if args.op == "assemble":
+        # the image's rows into a prompt: 64 text tokens, 13 x 256 placeholders,
+        # 32 text tokens; a vocabulary of the Qwen3 size (151,936 x H table)
+        m1, m2 = ivc.Mlp(inp["mlp1"]).fold(), ivc.Mlp(inp["mlp2"]).fold()
+        r = ivc.Router(inp["router"])
+        fres = ivc.flash_compress(x, vl, offs, m1, m2, r)
+        V, img = 151936, 151667
+        g = torch.Generator(device="cuda").manual_seed(3)
+        table = (0.02 * torch.randn(V, w.H, device="cuda", generator=g)).to(torch.bfloat16)
+        text = torch.randint(0, img, (96,), device="cuda", generator=g, dtype=torch.int32)
+        ids = torch.cat([text[:64], torch.full((256 * T,), img, dtype=torch.int32, device="cuda"),
+                         text[64:]])
+        soffs = torch.tensor([0, ids.numel()], dtype=torch.int32, device="cuda")
+        ws_a = ivc.new_workspace(ivc.lib().ivc_assemble_workspace_size(ids.numel()))
+        aout = None
+
+        def fn():
+            nonlocal aout
+            aout = ivc.assemble_sequence(ids, soffs, img, table, fres["out"], fres["mask"],
+                                         fres["offsets"], workspace=ws_a, out=aout)
+    elif args.op in ("flash_dual", "flash_routed"):
         m1, m2 = ivc.Mlp(inp["mlp1"]).fold(), ivc.Mlp(inp["mlp2"]).fold()
         r = ivc.Router(inp["router"])
         fn = lambda: ivc.flash_compress(x, vl, offs, m1, m2, r, routed=args.op == "flash_routed")
@@ -529,6 +549,11 @@ def run_op(args):
     ms = a.elapsed_time(b) / args.steps
     line = {"op": args.op, "workload": WORKLOAD, "tiles": T, "ms_per_call": ms,
             "tiles_per_s": T / (ms / 1e3), "timing": "CUDA graph, back to back, no L2 flush"}
+    if args.op == "assemble":
+        n = int(aout["seq_offsets"][-1].item())
+        moved = 2.0 * n * w.H * 2  # each kept row read once and written once
+        line.update({"prompt_tokens": int(ids.numel()), "kept_tokens": n,
+                     "bytes_per_call": moved, "achieved_gbs": moved / (ms / 1e3) / 1e9})
     if args.trace:
         import ctypes
         L = ivc.lib()
@@ -561,7 +586,7 @@ def main(argv=None):
                     help="dual: ivc_flash_compress (both paths, then compaction); "
                          "routed: ivc_flash_compress_routed (router first)")
     ap.add_argument("--op", choices=["flash", "flash_dual", "flash_routed", "ps_half",
-                                     "ps_quarter", "route", "route_literal"],
+                                     "ps_quarter", "route", "route_literal", "assemble"],
                     default="flash", help="profiling aid: time one entry point alone "
                                           "(flash = the full benchmark)")
     ap.add_argument("--trace", action="store_true",

@@ -73,7 +73,9 @@ enum ivc_device_bits {
   IVC_DEV_BAD_VALID_LEN = 1,  /* valid_len[t] outside [1, 1024]; clamped */
   IVC_DEV_BAD_OFFSETS = 2,    /* image_offsets not 0 = o0 <= o1 <= ... = T */
   IVC_DEV_WAIT_TIMEOUT = 4,   /* a pipeline barrier wait ran out; outputs invalid */
-  IVC_DEV_GROUP_TOO_LARGE = 8 /* a quantile group above IVC_MAX_QUANTILE_GROUP */
+  IVC_DEV_GROUP_TOO_LARGE = 8, /* a quantile group above IVC_MAX_QUANTILE_GROUP */
+  IVC_DEV_BAD_PROMPT = 16      /* sequence assembly: placeholders != 256 T, a token id
+                                  outside [0, V) or seq_offsets not 0 <= ... = L */
 };
 
 #define IVC_MAX_QUANTILE_GROUP 8192
@@ -232,6 +234,38 @@ int ivc_flash_compress_routed(const void* x, const int32_t* valid_len, int T, in
                               const ivc_mlp* mlp2, const ivc_router* r, void* out, float* gate,
                               uint8_t* mask, int32_t* offsets, int32_t* total, void* workspace,
                               size_t ws_bytes, ivc_stream_t stream);
+
+/* Sequence assembly: the compacted visual rows spliced into the token
+ * sequences ([PS] "视觉 Token 如何注入 Qwen2.5 语言模型": the prompt's
+ * <IMG_CONTEXT> positions take the visual rows in order; [VIR] section 4 and
+ * [DP] "路由决策": a compressed tile keeps 64 of its 256 placeholders, the
+ * other 192 are deleted and the position indices follow).
+ *   input_ids       device int32 [L]: B sequences back to back.
+ *   seq_offsets     device int32 [B+1]: 0 = s_0 <= ... <= s_B = L.
+ *   img_context_id  the <IMG_CONTEXT> token id. The j-th placeholder of the
+ *                   batch is placeholder j % 256 of tile j / 256; a batch
+ *                   must hold exactly 256 T of them (else IVC_DEV_BAD_PROMPT,
+ *                   and placeholders beyond 256 T are treated as text).
+ *   embed_table     device bf16 [V, H]: the language model's token embeddings.
+ *   visual          device bf16 [offsets[T], H]: rows of ivc_flash_compress.
+ *   mask, offsets   device uint8 [T], int32 [T+1] of ivc_flash_compress.
+ *   out_ids         device int32 [L] capacity: the kept token ids.
+ *   out_embeds      device bf16 [L, H] capacity: row i = visual row of a kept
+ *                   placeholder, else embed_table[out_ids[i]] (a zero row and
+ *                   IVC_DEV_BAD_PROMPT for an id outside [0, V)).
+ *   out_positions   device int32 [L] capacity: position of row i within its
+ *                   sequence (0, 1, ...).
+ *   out_seq_offsets device int32 [B+1]: the shortened sequences; the total
+ *                   row count L - 192 k is out_seq_offsets[B].
+ *   workspace       >= ivc_assemble_workspace_size(L) bytes, status word first.
+ * H must be a multiple of 8; pointers to bf16 rows 16-byte aligned. */
+size_t ivc_assemble_workspace_size(int L);
+int ivc_assemble_sequence(const int32_t* input_ids, const int32_t* seq_offsets, int B, int L,
+                          int32_t img_context_id, const void* embed_table, int V, int H,
+                          const void* visual, const uint8_t* mask, const int32_t* offsets, int T,
+                          int32_t* out_ids, void* out_embeds, int32_t* out_positions,
+                          int32_t* out_seq_offsets, void* workspace, size_t ws_bytes,
+                          ivc_stream_t stream);
 
 /* Synchronise `stream`, copy the workspace's device status word to *bits and
  * clear it. Returns IVC_OK when no bit was set, IVC_EDEVICE otherwise. */

@@ -393,3 +393,88 @@ def test_flash_routed_4b_batched_sampled():
     tiles = sorted(set(padded[:4] + rng.choice(T, 6, replace=False).tolist() + [T - 1]))
     _flash_check(ivc, inp, res, tiles=tiles)
     _routed_vs_dual(ivc, inp, m1, m2, r, res)
+
+
+# ---------------------------------------------------------------- sequence assembly
+def _prompt_ids(tiles_per_seq, img_id, V, seed, text=(5, 3), extra_img=0):
+    rng = np.random.default_rng(seed)
+    ids, offs = [], [0]
+    for n in tiles_per_seq:
+        pre = [int(v) for v in rng.integers(0, V, text[0]) if v != img_id]
+        post = [int(v) for v in rng.integers(0, V, text[1]) if v != img_id]
+        ids += pre + [img_id] * (256 * n) + post
+        offs.append(len(ids))
+    ids += [img_id] * extra_img
+    offs[-1] = len(ids)
+    return np.array(ids, dtype=np.int32), np.array(offs, dtype=np.int32)
+
+
+def _assemble_check(ivc, ids, offs, img_id, table, visual, mask, v_offs, expect_status=0):
+    dev = "cuda"
+    res = ivc.assemble_sequence(torch.from_numpy(ids).to(dev), torch.from_numpy(offs).to(dev),
+                                img_id, table.to(dev), visual.to(dev),
+                                torch.from_numpy(mask.astype(np.uint8)).to(dev),
+                                torch.from_numpy(v_offs.astype(np.int32)).to(dev))
+    torch.cuda.synchronize()
+    assert ivc.device_status(res["workspace"]) == expect_status
+    ref = O.assemble_sequence(ids, offs, img_id, table.float().numpy(), visual.float().numpy(),
+                              mask, v_offs)
+    n = int(ref["seq_offsets"][-1])
+    np.testing.assert_array_equal(to_np(res["seq_offsets"]), ref["seq_offsets"])
+    np.testing.assert_array_equal(to_np(res["ids"])[:n], ref["ids"])
+    np.testing.assert_array_equal(to_np(res["positions"])[:n], ref["positions"])
+    # pure data movement: bit-exact rows
+    np.testing.assert_array_equal(res["embeds"][:n].float().cpu().numpy(), ref["embeds"])
+    return n
+
+
+@pytest.mark.parametrize("tiles", [(3, 1, 2), (1,), (0, 2, 0)])
+def test_assemble_sequence_small(tiles):
+    ivc = _ivc()
+    T = sum(tiles)
+    rng = np.random.default_rng(31 + T)
+    mask = (rng.random(T) < 0.5).astype(np.uint8)
+    v_offs = O.compaction_offsets(mask)
+    V, H, img = 600, 64, 599
+    g = torch.Generator().manual_seed(5)
+    table = torch.randn(V, H, generator=g).to(torch.bfloat16)
+    visual = torch.randn(max(int(v_offs[-1]), 1), H, generator=g).to(torch.bfloat16)
+    ids, offs = _prompt_ids(tiles, img, V, seed=T)
+    n = _assemble_check(ivc, ids, offs, img, table, visual, mask, v_offs)
+    assert n == len(ids) - 192 * int(mask.sum())
+
+
+def test_assemble_sequence_flags_a_bad_prompt():
+    """Two placeholders more than 256 T: flagged, and they stay text rows."""
+    ivc = _ivc()
+    mask = np.array([1, 0], dtype=np.uint8)
+    v_offs = O.compaction_offsets(mask)
+    V, H, img = 100, 32, 7
+    g = torch.Generator().manual_seed(6)
+    table = torch.randn(V, H, generator=g).to(torch.bfloat16)
+    visual = torch.randn(int(v_offs[-1]), H, generator=g).to(torch.bfloat16)
+    ids, offs = _prompt_ids((2,), img, V, seed=3, extra_img=2)
+    _assemble_check(ivc, ids, offs, img, table, visual, mask, v_offs, expect_status=16)
+
+
+def test_assemble_after_flash_compress():
+    """The 13-tile image through ivc_flash_compress, then into a two-turn
+    prompt; rows checked against the oracle's splice of the GPU's own rows."""
+    ivc = _ivc()
+    inp = W.make("flash_2b_13tiles")
+    m1, m2 = ivc.Mlp(inp["mlp1"]).fold(), ivc.Mlp(inp["mlp2"]).fold()
+    r = ivc.Router(inp["router"])
+    res = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(), inp["image_offsets"].cuda(),
+                             m1, m2, r)
+    torch.cuda.synchronize()
+    mask = to_np(res["mask"])
+    v_offs = to_np(res["offsets"])
+    total = int(v_offs[-1])
+    V, H, img = 4096, inp["H"], 4095
+    table = torch.randn(V, H, generator=torch.Generator().manual_seed(8)).to(torch.bfloat16)
+    ids, offs = _prompt_ids((13,), img, V, seed=13, text=(40, 12))
+    ids2, _ = _prompt_ids((0,), img, V, seed=14, text=(20, 0))
+    ids = np.concatenate([ids, ids2]).astype(np.int32)
+    offs = np.array([0, offs[1], len(ids)], dtype=np.int32)
+    n = _assemble_check(ivc, ids, offs, img, table, res["out"][:total].cpu(), mask, v_offs)
+    assert n == len(ids) - 192 * int(mask.sum())

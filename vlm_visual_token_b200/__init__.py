@@ -21,7 +21,7 @@ import torch
 
 POOL_FOLDED, POOL_LITERAL = 0, 1
 
-__all__ = ["Mlp", "Router", "POOL_FOLDED", "POOL_LITERAL", "ps_project", "vir_route", "flash_compress", "workspace_size",
+__all__ = ["Mlp", "Router", "POOL_FOLDED", "POOL_LITERAL", "ps_project", "vir_route", "flash_compress", "assemble_sequence", "workspace_size",
            "device_status", "IvcError", "lib", "LIB_PATH", "PS_V1", "PS_QUARTER_TWICE",
            "OP_PS_HALF", "OP_PS_QUARTER", "OP_VIR_ROUTE", "OP_FLASH"]
 
@@ -94,6 +94,13 @@ def lib() -> ctypes.CDLL:
                                          ctypes.c_size_t, _vp]
         L.ivc_flash_compress_routed.restype = ctypes.c_int
         L.ivc_flash_compress_routed.argtypes = L.ivc_flash_compress.argtypes
+        L.ivc_assemble_workspace_size.restype = ctypes.c_size_t
+        L.ivc_assemble_workspace_size.argtypes = [ctypes.c_int]
+        L.ivc_assemble_sequence.restype = ctypes.c_int
+        L.ivc_assemble_sequence.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int32,
+                                            _vp, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp,
+                                            ctypes.c_int, _vp, _vp, _vp, _vp, _vp,
+                                            ctypes.c_size_t, _vp]
         L.ivc_device_status.restype = ctypes.c_int
         L.ivc_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int), _vp]
         _LIB = L
@@ -263,6 +270,37 @@ def flash_compress(x: torch.Tensor, valid_len: Optional[torch.Tensor], image_off
            "ivc_flash_compress_routed" if routed else "ivc_flash_compress")
     res = dict(bufs)
     res["out"] = out
+    return res
+
+
+def assemble_sequence(input_ids: torch.Tensor, seq_offsets: torch.Tensor, img_context_id: int,
+                      embed_table: torch.Tensor, visual: torch.Tensor, mask: torch.Tensor,
+                      offsets: torch.Tensor, workspace: Optional[torch.Tensor] = None,
+                      out: Optional[dict] = None, stream=None) -> dict:
+    """ivc_assemble_sequence: the visual rows spliced into the token sequences
+    (compressed tiles keep 64 of their 256 placeholders). Returns device
+    tensors at full capacity L; the kept length is seq_offsets[-1]."""
+    L = int(input_ids.numel())
+    B = int(seq_offsets.numel()) - 1
+    V, H = embed_table.shape
+    T = int(mask.numel())
+    dev = input_ids.device
+    if out is None:
+        out = {"ids": torch.empty(max(L, 1), dtype=torch.int32, device=dev),
+               "embeds": torch.empty(max(L, 1), H, dtype=torch.bfloat16, device=dev),
+               "positions": torch.empty(max(L, 1), dtype=torch.int32, device=dev),
+               "seq_offsets": torch.empty(B + 1, dtype=torch.int32, device=dev)}
+    if workspace is None:
+        workspace = new_workspace(lib().ivc_assemble_workspace_size(L), dev)
+    _check(lib().ivc_assemble_sequence(_ptr(input_ids), _ptr(seq_offsets), B, L,
+                                       int(img_context_id), _ptr(embed_table), V, H, _ptr(visual),
+                                       _ptr(mask), _ptr(offsets), T, _ptr(out["ids"]),
+                                       _ptr(out["embeds"]), _ptr(out["positions"]),
+                                       _ptr(out["seq_offsets"]), _ptr(workspace),
+                                       workspace.numel(), _stream(stream)),
+           "ivc_assemble_sequence")
+    res = dict(out)
+    res["workspace"] = workspace
     return res
 
 

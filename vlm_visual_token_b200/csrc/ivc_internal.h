@@ -18,6 +18,7 @@ constexpr int DEV_BAD_VALID_LEN = IVC_DEV_BAD_VALID_LEN;
 constexpr int DEV_BAD_OFFSETS = IVC_DEV_BAD_OFFSETS;
 constexpr int DEV_WAIT_TIMEOUT = IVC_DEV_WAIT_TIMEOUT;
 constexpr int DEV_GROUP_TOO_LARGE = IVC_DEV_GROUP_TOO_LARGE;
+constexpr int DEV_BAD_PROMPT = IVC_DEV_BAD_PROMPT;
 
 struct Launch {
   cudaStream_t stream;
