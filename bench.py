@@ -62,6 +62,26 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def kernel_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture
+    (profiles/traffic.json), or None once the sources it was built from have
+    changed since the capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get("kernels", {}).get(kernel)
+    if e is None:
+        return None
+    for rel, digest in d.get("sources_sha256", {}).items():
+        fp = os.path.join(ROOT, rel)
+        if not os.path.exists(fp) or hashlib.sha256(open(fp, "rb").read()).hexdigest() != digest:
+            return None
+    return e["dram_bytes_read"] + e["dram_bytes_write"]
+
+
 def algorithmic(w, T):
     """Algorithmic FLOPs / bytes of each kernel role for T tiles of workload w.
 
@@ -378,13 +398,13 @@ def run_ivc(args):
         ach = fl / launches_dom / (per_launch_ms / 1e3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
         roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": ach / peak, "traffic": None,
+                "frac": ach / peak, "traffic": kernel_traffic(dom),
                 "kernel": dom, "peak_source": f"{src} bf16_tflops_sustained"}
     else:
         ach = by / launches_dom / (per_launch_ms / 1e3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
-                "traffic": None, "kernel": dom, "peak_source": f"{src} hbm_gbs"}
+                "traffic": kernel_traffic(dom), "kernel": dom, "peak_source": f"{src} hbm_gbs"}
     # the HBM-bound kernels: algorithmic bytes per launch / traced launch time
     hbm = {}
     kept_rows = int(bufs["offsets"][-1].item())  # 256 (T - k) + 64 k of this image
