@@ -282,7 +282,7 @@ int num_sms() {
 }
 
 template <int BN, int STAGES, int CG>
-static int run_gemm(const GemmMaps& maps, const GemmArgs& args, const char* tag,
+static int run_gemm(const GemmMaps& maps, const GemmArgs& args, const char* tag, int units_cap,
                     const Launch& L) {
   using S = GemmSmem<BN, STAGES, CG>;
   auto kern = gemm_sm100_kernel<BN, STAGES, CG>;
@@ -295,7 +295,7 @@ static int run_gemm(const GemmMaps& maps, const GemmArgs& args, const char* tag,
   }
   const long long tiles = static_cast<long long>((args.M + GEMM_BM * CG - 1) / (GEMM_BM * CG)) *
                           ((args.N + BN - 1) / BN) * args.groups;
-  const long long units = num_sms() / CG;
+  const long long units = units_cap;
   // with split-K the last round is cut into slices for every unit
   const int grid = CG * static_cast<int>(tiles < units && args.split_max <= 1 ? tiles : units);
   TraceScope ts(tag ? tag : "gemm", L.stream);
@@ -449,6 +449,16 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
                   GEMM_BK);
     if (rc) return rc;
   }
+  // persistent units (CTAs, or pairs): all SMs, or fewer when c.reserve_sms
+  // leaves room for concurrent work without adding a round of tiles
+  int units = num_sms() / cg;
+  if (c.reserve_sms > 0) {
+    const int tile_m = GEMM_BM * cg;
+    const long long tiles = static_cast<long long>((c.M + tile_m - 1) / tile_m) *
+                            ((c.N + bn - 1) / bn) * c.groups;
+    const int capped = (num_sms() - c.reserve_sms) / cg;
+    if (capped > 0 && (tiles + capped - 1) / capped == (tiles + units - 1) / units) units = capped;
+  }
   GemmArgs a{};
   a.M = c.M;
   a.N = c.N;
@@ -484,7 +494,6 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
   // rows) the kernel picks it and the finishing kernel always runs.
   if (c.split_part != nullptr && c.split_s != nullptr && c.groups == 1 && c.b_mode == B_K2D &&
       c.m_valid == 0) {
-    const int units = num_sms() / cg;
     const int n_tiles = (c.N + bn - 1) / bn;
     const int KT = c.K / GEMM_BK;
     const int tile_m = GEMM_BM * cg;
@@ -511,12 +520,12 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
   if (c.stats_remap && c.list == nullptr) return IVC_EINVAL;
   int rc2;
   switch (bn) {
-    case 256: rc2 = cg == 2 ? run_gemm<256, 6, 2>(maps, a, c.tag, L)
-                            : run_gemm<256, 4, 1>(maps, a, c.tag, L);
+    case 256: rc2 = cg == 2 ? run_gemm<256, 6, 2>(maps, a, c.tag, units, L)
+                            : run_gemm<256, 4, 1>(maps, a, c.tag, units, L);
       break;
-    case 128: rc2 = run_gemm<128, 6, 1>(maps, a, c.tag, L); break;
-    case 64: rc2 = run_gemm<64, 8, 1>(maps, a, c.tag, L); break;
-    default: rc2 = run_gemm<32, 8, 1>(maps, a, c.tag, L); break;
+    case 128: rc2 = run_gemm<128, 6, 1>(maps, a, c.tag, units, L); break;
+    case 64: rc2 = run_gemm<64, 8, 1>(maps, a, c.tag, units, L); break;
+    default: rc2 = run_gemm<32, 8, 1>(maps, a, c.tag, units, L); break;
   }
   if (rc2 != IVC_OK || a.split_max <= 1) return rc2;
   TraceScope ts("splitk.epilogue", L.stream);

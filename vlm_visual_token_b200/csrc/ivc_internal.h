@@ -116,6 +116,9 @@ struct GemmCall {
   // split-K scratch (optional): splitk_part_floats() fp32 values and one int
   float* split_part;
   int* split_s;
+  // SMs to leave to concurrent work (the router beside the connector) when
+  // that does not add a round of output tiles; 0 = use every SM
+  int reserve_sms;
 };
 int launch_gemm(const GemmCall& c, const Launch& L);
 // Size of the split-K partial buffer: enough for any GEMM shape on this device.
