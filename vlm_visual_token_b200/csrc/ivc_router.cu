@@ -34,100 +34,96 @@ __device__ __forceinline__ float gelu_f(float y) {
 }
 
 // ---------------------------------------------------------------- skinny GEMV
-// Y[m, n] = act(sum_k X[m, k] W[n, k] + b[n]) for few rows m (router vectors).
-// A CTA of GEMV_WARPS warps owns GEMV_CTA_COLS consecutive columns. One
-// thread brings the CTA's weight block (GEMV_CTA_COLS contiguous rows of W)
-// and up to GEMV_ROWS input rows into shared memory with bulk copies on one
-// mbarrier (the weight copy is issued before waiting for the previous
-// kernel), so the load latency is paid once. Warp w then keeps its
-// GEMV_COLS weight rows in registers (packed bf16, lane l holds
-// k = 128 j + 4 l .. +3) and reads each staged input row once for all of them.
-constexpr int GEMV_WARPS = 4;
-constexpr int GEMV_COLS = 4;
-constexpr int GEMV_CTA_COLS = GEMV_WARPS * GEMV_COLS;  // 16: one head of 64 spans 4 CTAs
+// Y[m, n] = act(sum_k X[m, k] W[n, k] + b[n]) for few rows m (router vectors),
+// on the tensor cores (m16n8k16). A CTA of 8 warps owns 8 consecutive columns
+// (one n8 tile). One thread brings their 8 weight rows (contiguous in W) into
+// shared memory with one bulk copy issued before waiting for the previous
+// kernel, and up to 16 input rows per round (one bulk copy per row) on the same
+// mbarrier. Warp w multiplies the k-range [w K/8, (w+1) K/8): fp32 inputs are
+// split into a bf16 pair hi + lo (two MMAs per k-step, fp32 accumulate, about
+// 16 significant bits of the input kept), bf16 inputs enter as they are. The
+// 8 partial m16n8 tiles are summed through shared memory.
+constexpr int GEMV_THREADS = 256;
+constexpr int GEMV_WARPS = GEMV_THREADS / 32;
+constexpr int GEMV_COLS = 8;   // output columns per CTA
+constexpr int GEMV_ROWS = 16;  // input rows per round
 
-template <int J>
-struct GemvRows {
-  static constexpr int value = J <= 8 ? 16 : 8;  // staged rows per round
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
+                                          const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// v = hi + lo, hi = bf16(v), lo = bf16(v - hi), two lanes per 32-bit word.
+__device__ __forceinline__ void split2(float2 v, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(v.x - __low2float(h), v.y - __high2float(h));
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+template <typename XT, bool PAIRED>
+struct GemvLayout {
+  // staged input rows (padded by 8 elements), the weight rows (unpadded, one
+  // copy), the warps' partial tiles; after a 16-byte mbarrier slot
+  __host__ __device__ static size_t x_bytes(int K) {
+    return (PAIRED ? 2 : 1) * static_cast<size_t>(GEMV_ROWS) * (K + 8) * sizeof(XT);
+  }
+  __host__ __device__ static size_t w_bytes(int K) { return static_cast<size_t>(GEMV_COLS) * K * 2; }
+  __host__ __device__ static size_t total(int K) {
+    return 16 + x_bytes(K) + w_bytes(K) + static_cast<size_t>(GEMV_WARPS) * GEMV_ROWS * GEMV_COLS * 4;
+  }
 };
-
-template <typename XT, int J, bool PAIRED>
-struct GemvSmem {
-  static constexpr int K = J * 128;
-  static constexpr int ROWS = GemvRows<J>::value;
-  static constexpr size_t W_BYTES = static_cast<size_t>(GEMV_CTA_COLS) * K * 2;
-  static constexpr size_t X_BYTES = static_cast<size_t>(ROWS) * K * sizeof(XT) * (PAIRED ? 2 : 1);
-  static constexpr size_t TOTAL = 16 + W_BYTES + X_BYTES;
-};
-
-template <typename XT>
-__device__ __forceinline__ float4 load4(const XT* p);
-template <>
-__device__ __forceinline__ float4 load4<float>(const float* p) {
-  return *reinterpret_cast<const float4*>(p);
-}
-template <>
-__device__ __forceinline__ float4 load4<bf16>(const bf16* p) {
-  const uint2 u = *reinterpret_cast<const uint2*>(p);
-  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
-                     __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
-}
-
-__device__ __forceinline__ float dot4(uint2 w, float4 x, float acc) {
-  acc = fmaf(__uint_as_float(w.x << 16), x.x, acc);
-  acc = fmaf(__uint_as_float(w.x & 0xffff0000u), x.y, acc);
-  acc = fmaf(__uint_as_float(w.y << 16), x.z, acc);
-  return fmaf(__uint_as_float(w.y & 0xffff0000u), x.w, acc);
-}
 
 // PAIRED: the input row m of the CTA's columns is Z[m*128 + h] + Z[m*128 + 16 + h]
 // with h = (first column) / 64 (the folded pooling's split weighted sums; ldx
 // is then the row length of Z).
-template <typename XT, int J, bool PAIRED = false>
-__global__ void __launch_bounds__(GEMV_WARPS * 32)
-    gemv_kernel(const XT* __restrict__ X, long long ldx, int M,
+template <typename XT, bool PAIRED>
+__global__ void __launch_bounds__(GEMV_THREADS)
+    gemv_kernel(const XT* __restrict__ X, long long ldx, int M, int K,
                 const bf16* __restrict__ W, const bf16* __restrict__ b, int N,
                 float* __restrict__ Y, long long ldy, int gelu, int* __restrict__ status) {
-  using S = GemvSmem<XT, J, PAIRED>;
-  constexpr int K = S::K;
-  constexpr int ROWS = S::ROWS;
+  using Lay = GemvLayout<XT, PAIRED>;
   extern __shared__ __align__(16) uint8_t smem[];
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
-  bf16* sw = reinterpret_cast<bf16*>(smem + 16);
-  XT* sx = reinterpret_cast<XT*>(smem + 16 + S::W_BYTES);
+  XT* sx = reinterpret_cast<XT*>(smem + 16);
+  const bf16* sw = reinterpret_cast<const bf16*>(smem + 16 + Lay::x_bytes(K));
+  float* red = reinterpret_cast<float*>(smem + 16 + Lay::x_bytes(K) + Lay::w_bytes(K));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cta_n0 = blockIdx.x * GEMV_CTA_COLS;
-  const int n0 = cta_n0 + warp * GEMV_COLS;
-  const int w_rows = min(GEMV_CTA_COLS, N - cta_n0);
-  const int h = PAIRED ? cta_n0 / 64 : 0;
-  const int rows0 = min(ROWS, M);
-  const uint32_t x_row_bytes = K * sizeof(XT);
+  const int g = lane >> 2, t2 = (lane & 3) * 2;
+  const int c0 = blockIdx.x * GEMV_COLS;
+  const int w_rows = min(GEMV_COLS, N - c0);
+  const int xp = K + 8;
+  const int h = PAIRED ? c0 / 64 : 0;
+  const uint32_t xrow = K * sizeof(XT);
+  const int rows0 = min(GEMV_ROWS, M);
   if (threadIdx.x == 0) {
     mbar_init(bar, 1);
     fence_mbar_init();
-    mbar_arrive_expect_tx(bar, w_rows * K * 2 + rows0 * x_row_bytes * (PAIRED ? 2 : 1));
-    bulk_load(sw, W + static_cast<long long>(cta_n0) * K, w_rows * K * 2, bar);
+    // the weights do not depend on the previous kernel: request them now,
+    // with the byte count of the first round of input rows as well
+    mbar_arrive_expect_tx(bar, w_rows * K * 2 + rows0 * xrow * (PAIRED ? 2 : 1));
+    bulk_load(const_cast<bf16*>(sw), W + static_cast<size_t>(c0) * K, w_rows * K * 2, bar);
   }
   __syncthreads();  // barrier initialised before anyone waits on it
-  float bias[GEMV_COLS];
-#pragma unroll
-  for (int c = 0; c < GEMV_COLS; ++c)
-    bias[c] = (n0 + c < N && b != nullptr) ? __bfloat162float(b[n0 + c]) : 0.f;
   pdl_wait();
   pdl_trigger();
   bool ok = true;
-  uint2 w[GEMV_COLS][J];
-  for (int m0 = 0, round = 0; m0 < M; m0 += ROWS, ++round) {
-    const int rows = min(ROWS, M - m0);
+  const int kw = K / GEMV_WARPS;
+  for (int m0 = 0, round = 0; m0 < M; m0 += GEMV_ROWS, ++round) {
+    const int rows = min(GEMV_ROWS, M - m0);
     if (threadIdx.x == 0) {
-      if (round > 0) mbar_arrive_expect_tx(bar, rows * x_row_bytes * (PAIRED ? 2 : 1));
+      if (round > 0) mbar_arrive_expect_tx(bar, rows * xrow * (PAIRED ? 2 : 1));
       for (int r = 0; r < rows; ++r) {
         if constexpr (PAIRED) {
           const XT* zr = X + (static_cast<long long>(m0 + r) * 128 + h) * ldx;
-          bulk_load(sx + r * K, zr, x_row_bytes, bar);
-          bulk_load(sx + (ROWS + r) * K, zr + 16 * ldx, x_row_bytes, bar);
+          bulk_load(sx + r * xp, zr, xrow, bar);
+          bulk_load(sx + (GEMV_ROWS + r) * xp, zr + 16 * ldx, xrow, bar);
         } else {
-          bulk_load(sx + r * K, X + static_cast<long long>(m0 + r) * ldx, x_row_bytes, bar);
+          bulk_load(sx + r * xp, X + static_cast<long long>(m0 + r) * ldx, xrow, bar);
         }
       }
     }
@@ -136,73 +132,83 @@ __global__ void __launch_bounds__(GEMV_WARPS * 32)
       if (threadIdx.x == 0) atomicOr(status, DEV_WAIT_TIMEOUT);
       break;
     }
-    if (round == 0) {
+    // rows >= `rows` of the A tile hold stale values; they only reach output
+    // rows that are never stored
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const int wr = g < w_rows ? g : 0;
+    for (int ks = warp * kw; ks < (warp + 1) * kw; ks += 16) {
+      const int k = ks + t2;
+      uint32_t bw[2];
+      bw[0] = *reinterpret_cast<const uint32_t*>(sw + static_cast<size_t>(wr) * K + k);
+      bw[1] = *reinterpret_cast<const uint32_t*>(sw + static_cast<size_t>(wr) * K + k + 8);
+      if constexpr (sizeof(XT) == 2) {
+        uint32_t a[4];
+        a[0] = *reinterpret_cast<const uint32_t*>(sx + g * xp + k);
+        a[1] = *reinterpret_cast<const uint32_t*>(sx + (g + 8) * xp + k);
+        a[2] = *reinterpret_cast<const uint32_t*>(sx + g * xp + k + 8);
+        a[3] = *reinterpret_cast<const uint32_t*>(sx + (g + 8) * xp + k + 8);
+        mma_16816(acc, a, bw);
+      } else {
+        const float* fx = reinterpret_cast<const float*>(sx);
+        float2 v[4] = {*reinterpret_cast<const float2*>(fx + g * xp + k),
+                       *reinterpret_cast<const float2*>(fx + (g + 8) * xp + k),
+                       *reinterpret_cast<const float2*>(fx + g * xp + k + 8),
+                       *reinterpret_cast<const float2*>(fx + (g + 8) * xp + k + 8)};
+        if constexpr (PAIRED) {
+          const float* fz = fx + GEMV_ROWS * xp;
+          const float2 z[4] = {*reinterpret_cast<const float2*>(fz + g * xp + k),
+                               *reinterpret_cast<const float2*>(fz + (g + 8) * xp + k),
+                               *reinterpret_cast<const float2*>(fz + g * xp + k + 8),
+                               *reinterpret_cast<const float2*>(fz + (g + 8) * xp + k + 8)};
 #pragma unroll
-      for (int c = 0; c < GEMV_COLS; ++c) {
-        const int wr = warp * GEMV_COLS + c < w_rows ? warp * GEMV_COLS + c : 0;
+          for (int i = 0; i < 4; ++i) v[i] = make_float2(v[i].x + z[i].x, v[i].y + z[i].y);
+        }
+        uint32_t ah[4], al[4];
 #pragma unroll
-        for (int j = 0; j < J; ++j)
-          w[c][j] = *reinterpret_cast<const uint2*>(sw + wr * K + j * 128 + lane * 4);
+        for (int i = 0; i < 4; ++i) split2(v[i], ah[i], al[i]);
+        mma_16816(acc, ah, bw);
+        mma_16816(acc, al, bw);
       }
     }
-    for (int r = 0; r < rows; ++r) {
-      float acc[GEMV_COLS] = {};
-#pragma unroll
-      for (int j = 0; j < J; ++j) {
-        float4 xv = load4<XT>(sx + r * K + j * 128 + lane * 4);
-        if constexpr (PAIRED) {
-          const float4 x2 = load4<XT>(sx + (ROWS + r) * K + j * 128 + lane * 4);
-          xv = make_float4(xv.x + x2.x, xv.y + x2.y, xv.z + x2.z, xv.w + x2.w);
-        }
-#pragma unroll
-        for (int c = 0; c < GEMV_COLS; ++c) acc[c] = dot4(w[c][j], xv, acc[c]);
-      }
-#pragma unroll
-      for (int c = 0; c < GEMV_COLS; ++c) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], o);
-      }
-      if (lane < GEMV_COLS) {
+    float* rw = red + warp * (GEMV_ROWS * GEMV_COLS);
+    rw[g * GEMV_COLS + t2] = acc[0];
+    rw[g * GEMV_COLS + t2 + 1] = acc[1];
+    rw[(g + 8) * GEMV_COLS + t2] = acc[2];
+    rw[(g + 8) * GEMV_COLS + t2 + 1] = acc[3];
+    __syncthreads();
+    if (threadIdx.x < GEMV_ROWS * GEMV_COLS) {
+      const int r = threadIdx.x / GEMV_COLS, c = threadIdx.x % GEMV_COLS;
+      if (r < rows && c < w_rows) {
         float y = 0.f;
 #pragma unroll
-        for (int c = 0; c < GEMV_COLS; ++c)
-          if (c == lane) y = acc[c] + bias[c];
+        for (int w = 0; w < GEMV_WARPS; ++w) y += red[w * GEMV_ROWS * GEMV_COLS + threadIdx.x];
+        if (b != nullptr) y += __bfloat162float(b[c0 + c]);
         if (gelu) y = gelu_f(y);
-        if (n0 + lane < N) Y[static_cast<long long>(m0 + r) * ldy + n0 + lane] = y;
+        Y[static_cast<long long>(m0 + r) * ldy + c0 + c] = y;
       }
     }
-    __syncthreads();  // staged rows consumed before the next round overwrites them
+    __syncthreads();  // staged rows and partials consumed before the next round
   }
-}
-
-template <typename XT, int J, bool PAIRED = false>
-static int run_gemv(const XT* X, long long ldx, int M, const bf16* W, const bf16* b, int N,
-                    float* Y, long long ldy, int gelu, const Launch& L) {
-  const int smem = static_cast<int>(GemvSmem<XT, J, PAIRED>::TOTAL);
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(gemv_kernel<XT, J, PAIRED>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return IVC_ECUDA;
-    attr = true;
-  }
-  TraceScope ts(PAIRED ? "pool.vproj" : (gelu ? "router.gemv_gelu" : "router.gemv"), L.stream);
-  return launch_k(gemv_kernel<XT, J, PAIRED>, dim3((N + GEMV_CTA_COLS - 1) / GEMV_CTA_COLS),
-                  dim3(GEMV_WARPS * 32), smem, L.stream, 1, X, ldx, M, W, b, N, Y, ldy, gelu,
-                  L.status);
 }
 
 template <typename XT, bool PAIRED = false>
 static int dispatch_gemv(const XT* X, long long ldx, int M, int K, const bf16* W, const bf16* b,
                          int N, float* Y, long long ldy, int gelu, const Launch& L) {
   if (M == 0 || N == 0) return IVC_OK;
-  switch (K) {
-    case 256: return run_gemv<XT, 2, PAIRED>(X, ldx, M, W, b, N, Y, ldy, gelu, L);
-    case 512: return run_gemv<XT, 4, PAIRED>(X, ldx, M, W, b, N, Y, ldy, gelu, L);
-    case 1024: return run_gemv<XT, 8, PAIRED>(X, ldx, M, W, b, N, Y, ldy, gelu, L);
-    case 2048: return run_gemv<XT, 16, PAIRED>(X, ldx, M, W, b, N, Y, ldy, gelu, L);
-    default: return IVC_EUNSUPPORTED;
+  if (K % (16 * GEMV_WARPS) != 0 || K > 2048 || N % GEMV_COLS != 0) return IVC_EUNSUPPORTED;
+  if (PAIRED && K > 1024) return IVC_EUNSUPPORTED;
+  const int smem = static_cast<int>(GemvLayout<XT, PAIRED>::total(K));
+  static bool attr = false;
+  if (!attr) {  // once, for the widest K this instantiation accepts
+    const int max_smem = static_cast<int>(GemvLayout<XT, PAIRED>::total(PAIRED ? 1024 : 2048));
+    if (cudaFuncSetAttribute(gemv_kernel<XT, PAIRED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             max_smem) != cudaSuccess)
+      return IVC_ECUDA;
+    attr = true;
   }
+  TraceScope ts(PAIRED ? "pool.vproj" : (gelu ? "router.gemv_gelu" : "router.gemv"), L.stream);
+  return launch_k(gemv_kernel<XT, PAIRED>, dim3(N / GEMV_COLS), dim3(GEMV_THREADS), smem,
+                  L.stream, 1, X, ldx, M, K, W, b, N, Y, ldy, gelu, L.status);
 }
 
 int launch_gemv(const float* X, long long ldx, int M, int K, const bf16* W, const bf16* b, int N,
