@@ -384,7 +384,21 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-size_t splitk_part_floats() { return static_cast<size_t>(num_sms()) * GEMM_BM * 256; }
+size_t splitk_part_floats() { return static_cast<size_t>(num_sms()) * GEMM_BM * 512; }
+
+// 512-wide pair tiles (see launch_gemm) with IVC_GEMM_WIDE=1. Off by
+// default: on the 13-tile image they cut mlp2.fc1 from ~145 to ~106 us, but
+// the split-K finishing launches they need (their partials re-read from
+// DRAM, ~13-20 us each) cost more than that in the whole step (0.514 against
+// 0.497 ms per call).
+static bool wide_tiles_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* e = std::getenv("IVC_GEMM_WIDE");
+    on = (e && e[0] == '1') ? 1 : 0;
+  }
+  return on == 1;
+}
 
 // 256-wide tiles run on CTA pairs unless IVC_GEMM_PAIRS=0 (kept for
 // comparing the two variants on the same build).
@@ -426,9 +440,18 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
   if (c.b_mode != B_K2D && (c.b_batch_rows <= 0 || c.b_batch_rows % GEMM_BM != 0))
     return IVC_EUNSUPPORTED;
   if (c.b_mode == B_MN3D && c.N % 64 != 0) return IVC_EUNSUPPORTED;
-  const int bn = pick_bn(c);
+  int bn = pick_bn(c);
   // CTA pairs (cta_group::2) for 256-wide tiles of plain K-major weights.
   const int cg = (bn == 256 && c.b_mode == B_K2D && pairs_enabled()) ? 2 : 1;
+  // 512-wide pair tiles where split-K can still fill the GPU: a host-known
+  // row count, split scratch, and at most half as many tiles as pair units
+  // (S >= 2). Per CTA and k-step they move 48 KB for 2x the MMA work of a
+  // 256-wide tile's 32 KB, and their weight box is one 32 KB request.
+  if (cg == 2 && c.N % 512 == 0 && c.list_count == nullptr && c.split_part != nullptr &&
+      c.groups == 1 && wide_tiles_enabled()) {
+    const long long tiles512 = static_cast<long long>((c.M + 255) / 256) * (c.N / 512);
+    if (2 * tiles512 <= num_sms() / 2 && c.K / GEMM_BK >= 16) bn = 512;
+  }
 
   GemmMaps maps;
   int rc;
@@ -498,10 +521,12 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
     const int KT = c.K / GEMM_BK;
     const int tile_m = GEMM_BM * cg;
     constexpr int kMaxSplit = 8;
+    const int split_min = bn > 256 ? 2 : 4;
+    a.split_min = split_min;
     if (c.list_count == nullptr) {
       // the kernel's own choice, known here: skip the finishing launch if 1
       const int rem = (((c.M + tile_m - 1) / tile_m) * n_tiles) % units;
-      const int S = rem > 0 ? split_count(kMaxSplit, units, rem, KT) : 1;
+      const int S = rem > 0 ? split_count(kMaxSplit, units, rem, KT, split_min) : 1;
       a.split_max = S > 1 ? S : 0;
     } else {
       // the row count is known only on the device: the kernel decides
@@ -520,6 +545,7 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
   if (c.stats_remap && c.list == nullptr) return IVC_EINVAL;
   int rc2;
   switch (bn) {
+    case 512: rc2 = run_gemm<512, 4, 2>(maps, a, c.tag, units, L); break;
     case 256: rc2 = cg == 2 ? run_gemm<256, 6, 2>(maps, a, c.tag, units, L)
                             : run_gemm<256, 4, 1>(maps, a, c.tag, units, L);
       break;
@@ -528,8 +554,12 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
     default: rc2 = run_gemm<32, 8, 1>(maps, a, c.tag, units, L); break;
   }
   if (rc2 != IVC_OK || a.split_max <= 1) return rc2;
+  // one thread per 8 output columns of a split tile (at most units tiles of
+  // TILE_M x bn), so that every partial load is in flight at once
+  const long long items = static_cast<long long>(units) * GEMM_BM * cg * (bn / 8);
+  const int blocks = static_cast<int>((items + 255) / 256);
   TraceScope ts("splitk.epilogue", L.stream);
-  return launch_k(splitk_epilogue_kernel, dim3(2 * num_sms()), dim3(256), 0, L.stream, 1, a,
+  return launch_k(splitk_epilogue_kernel, dim3(blocks), dim3(256), 0, L.stream, 1, a,
                   GEMM_BM * cg, bn);
 }
 

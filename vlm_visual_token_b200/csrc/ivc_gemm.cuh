@@ -103,20 +103,37 @@ struct GemmArgs {
   // splitk_epilogue_kernel sums the slices and applies the epilogue. CTA 0
   // writes split_s[0..2] = {S, first split tile, split tiles}.
   int split_max;
+  int split_min;
   float* split_part;
   int* split_s;
 };
 
 // Number of k-slices for `tiles` output tiles on `units` CTAs (or pairs).
 // The split-K scratch holds units x TILE_M x BN values: S * tiles <= units.
-// Fewer than 4 slices do not pay for the partial traffic and the finishing
-// launch (measured on the connector GEMMs).
-__host__ __device__ __forceinline__ int split_count(int split_max, int units, int tiles, int KT) {
+// Fewer than split_min slices do not pay for the partial traffic and the
+// finishing launch (measured on the connector GEMMs: 4 for 256-wide tiles,
+// 2 for the 512-wide ones, which exist to be split).
+__host__ __device__ __forceinline__ int split_count(int split_max, int units, int tiles, int KT,
+                                                    int split_min = 4) {
   if (split_max <= 1 || tiles <= 0) return 1;
   int s = units / tiles;
   if (s > split_max) s = split_max;
   if (s > KT / 4) s = KT / 4;  // at least 4 k-steps per slice
-  return s < 4 ? 1 : s;
+  return s < split_min ? 1 : s;
+}
+
+// Output column of TMEM column c. A 512-wide pair tile is two N = 256 pair
+// MMAs; CTA r of the pair holds weight rows [256 r, 256 r + 256) of the tile,
+// and MMA m reads rows [128 m, 128 m + 128) of both CTAs' blocks, so TMEM
+// column 256 m + 128 h + i is output column 128 m + 256 h + i.
+template <int BN>
+__host__ __device__ __forceinline__ int tmem_col_to_n(int c) {
+  if constexpr (BN > 256) {
+    const int m = c >> 8, h = (c >> 7) & 1, i = c & 127;
+    return 128 * m + 256 * h + i;
+  } else {
+    return c;
+  }
 }
 
 template <int BN, int STAGES, int CG = 1>
@@ -129,7 +146,10 @@ struct GemmSmem {
   static constexpr uint32_t BARS = (2 * STAGES + 4) * 8 + 16;
   static constexpr uint32_t COLS = 2 * BN * 4;
   static constexpr uint32_t TOTAL = 1024 + RING + BARS + COLS;
-  static constexpr uint32_t TMEM_COLS = 2 * BN;  // double-buffered accumulator
+  // double-buffered accumulator, except for 512-wide pair tiles, whose one
+  // accumulator fills the 512 columns of TMEM
+  static constexpr int ACC_BUFS = BN > 256 ? 1 : 2;
+  static constexpr uint32_t TMEM_COLS = ACC_BUFS * BN;
 };
 
 __device__ __forceinline__ float gelu_erf(float y) {
@@ -162,8 +182,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_sm100_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs args,
                       int* __restrict__ status) {
   using L = GemmSmem<BN, STAGES, CG>;
-  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
-  static_assert(CG == 1 || (CG == 2 && BN == 256), "CTA pairs use 256-wide tiles");
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 512, "BN");
+  static_assert(CG == 1 ? BN <= 256 : (BN == 256 || BN == 512),
+                "CTA pairs use 256- or 512-wide tiles, single CTAs up to 256");
   constexpr int TILE_M = GEMM_BM * CG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -225,7 +246,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const int m_tiles = (M + TILE_M - 1) / TILE_M;
   const int n_out = m_tiles * n_tiles * args.groups;  // output tiles
   const int rem = n_out % n_units;
-  const int S = rem > 0 ? split_count(args.split_max, n_units, rem, KT) : 1;
+  const int S = rem > 0 ? split_count(args.split_max, n_units, rem, KT, args.split_min) : 1;
   const int n_full = S > 1 ? n_out - rem : n_out;     // tiles computed whole
   const int n_total = n_full + (n_out - n_full) * S;  // work units
   const int n_listed = args.list_count != nullptr ? M / args.item_rows : 0;
@@ -346,12 +367,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       // ------------------------------------------------------------ MMA issuer
-      const uint32_t idesc = idesc_bf16_f32(TILE_M, BN) |
+      constexpr int MMA_N = BN > 256 ? 256 : BN;
+      const uint32_t idesc = idesc_bf16_f32(TILE_M, MMA_N) |
                              (args.b_mode == B_MN3D ? (1u << 16) : 0u);  // B MN-major
       int it = 0, local = 0;
       for (int idx = unit; idx < n_total && ok; idx += n_units, ++local) {
-        const int acc = local & 1;
-        const uint32_t use = static_cast<uint32_t>(local >> 1);
+        const int acc = local % L::ACC_BUFS;
+        const uint32_t use = static_cast<uint32_t>(local / L::ACC_BUFS);
         int tile, slice, kb0, kb1;
         unit_of(idx, tile, slice, kb0, kb1);
         if (!mbar_wait(&tempty_bar[acc], (use & 1) ^ 1)) { ok = false; break; }
@@ -372,11 +394,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           for (int k = 0; k < GEMM_BK / 16; ++k) {
             // K-major: advance 16 bf16 = 32 bytes inside the swizzle atom;
             // MN-major: advance 16 k-rows of 128 bytes.
-            if constexpr (CG == 2)
-              umma_bf16_pair(d_tmem, ad + 2 * k, bd + bstep * k, idesc,
-                             (kk != kb0 || k != 0) ? 1u : 0u);
-            else
-              umma_bf16(d_tmem, ad + 2 * k, bd + bstep * k, idesc, (kk != kb0 || k != 0) ? 1u : 0u);
+            const uint32_t accum = (kk != kb0 || k != 0) ? 1u : 0u;
+            if constexpr (CG == 2) {
+              umma_bf16_pair(d_tmem, ad + 2 * k, bd + bstep * k, idesc, accum);
+              if constexpr (BN > 256)  // rows 128..255 of each CTA's weight block (+16 KB)
+                umma_bf16_pair(d_tmem + 256, ad + 2 * k, bd + ((128 * 128) >> 4) + bstep * k,
+                               idesc, accum);
+            } else {
+              umma_bf16(d_tmem, ad + 2 * k, bd + bstep * k, idesc, accum);
+            }
           }
           if constexpr (CG == 2)
             umma_commit_pair(&empty_bar[s]);
@@ -399,12 +425,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       int tile, slice, kb0, kb1;
       unit_of(idx, tile, slice, kb0, kb1);
       const TileCoord tc = tile_coord(tile, m_tiles, n_tiles, TILE_M, BN);
-      const int acc = local & 1;
-      const uint32_t use = static_cast<uint32_t>(local >> 1);
-      // per-column epilogue vectors of this tile
+      const int acc = local % L::ACC_BUFS;
+      const uint32_t use = static_cast<uint32_t>(local / L::ACC_BUFS);
+      // per-column epilogue vectors of this tile, by TMEM column
       epi_bar_sync();
       for (int i = et; i < BN; i += 128) {
-        const int n = tc.n0 + i;
+        const int n = tc.n0 + tmem_col_to_n<BN>(i);
         float c0 = 0.f, c1 = 0.f;
         if (n < args.N) {
           if (args.epi_mode == EPI_LNFOLD) {
@@ -449,6 +475,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                               static_cast<uint32_t>(acc * BN);
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
+        const int cn = tmem_col_to_n<BN>(c);  // output column of this 32-column chunk
         uint32_t r[32];
         tmem_ld32(t_base + c, r);
         tmem_ld_wait();
@@ -469,14 +496,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           float4* dst = reinterpret_cast<float4*>(
               args.split_part +
               ((static_cast<long long>(tile - n_full) * S + slice) * TILE_M + (row - tc.m0)) * BN +
-              c);
+              cn);
 #pragma unroll
           for (int j = 0; j < 8; ++j)
             dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
                                  __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
           continue;
         }
-        if (row < M && tc.n0 + c < args.N && (args.m_valid == 0 || (row & 127) < args.m_valid)) {
+        if (row < M && tc.n0 + cn < args.N && (args.m_valid == 0 || (row & 127) < args.m_valid)) {
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
@@ -488,13 +515,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             v[i] = args.gelu ? gelu_erf(t) : t;
           }
           if (args.out_f32) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + out_off + c);
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.out) + out_off + cn);
 #pragma unroll
             for (int j = 0; j < 8; ++j)
               dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
           } else {
             uint4* dst =
-                reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) + out_off + c);
+                reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) + out_off + cn);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]),
