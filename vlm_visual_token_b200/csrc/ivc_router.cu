@@ -359,9 +359,11 @@ __global__ void __launch_bounds__(128) pool_fold_query_kernel(
           Q[(t0 + i / HEAD_DIM) * ldq + h * HEAD_DIM + i % HEAD_DIM] * 0.125f;
     __syncthreads();
     for (int t = 0; t < nt; ++t) {
-      float u = 0.f;
+      // four independent partial sums (ILP), then combined
+      float p[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int d = 0; d < HEAD_DIM; ++d) u = fmaf(w[d], s_q[t][d], u);
+      for (int d = 0; d < HEAD_DIM; ++d) p[d & 3] = fmaf(w[d], s_q[t][d], p[d & 3]);
+      const float u = (p[0] + p[1]) + (p[2] + p[3]);
       const bf16 hi = __float2bfloat16_rn(u);
       const bf16 lo = __float2bfloat16_rn(u - __bfloat162float(hi));
       bf16* base = U2 + static_cast<long long>(t0 + t) * 32 * D;
