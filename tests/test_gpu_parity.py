@@ -7,6 +7,7 @@ absolute, connector outputs within relative Frobenius 1e-2 and max-abs 3e-2
 (plus half a bf16 ulp where |y| >= 4, see tests/_parity.py).
 """
 import dataclasses
+import os
 
 import numpy as np
 import pytest
@@ -478,3 +479,41 @@ def test_assemble_after_flash_compress():
     offs = np.array([0, offs[1], len(ids)], dtype=np.int32)
     n = _assemble_check(ivc, ids, offs, img, table, res["out"][:total].cpu(), mask, v_offs)
     assert n == len(ids) - 192 * int(mask.sum())
+
+
+# ---------------------------------------------------------------- opt-in kernel variants
+_VARIANT_SNIPPET = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, {root!r})
+import oracle as O, workloads as W, vlm_visual_token_b200 as ivc
+inp = W.make("flash_2b_13tiles")
+m1, m2 = ivc.Mlp(inp["mlp1"]).fold(), ivc.Mlp(inp["mlp2"]).fold()
+r = ivc.Router(inp["router"])
+res = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(), inp["image_offsets"].cuda(),
+                         m1, m2, r)
+torch.cuda.synchronize()
+x64 = O.to64(inp["x"])
+mask = res["mask"].cpu().numpy(); offs = res["offsets"].cpu().numpy()
+for t in range(inp["T"]):
+    ref = (O.ps_project(x64[t:t + 1], 0.25, O.to64(inp["mlp2"])) if mask[t]
+           else O.ps_project(x64[t:t + 1], 0.5, O.to64(inp["mlp1"]))).reshape(-1, inp["H"])
+    got = res["out"][offs[t]:offs[t + 1]].float().cpu().double().numpy()
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rel <= 1e-2, (t, rel)
+print("variant ok")
+"""
+
+
+@pytest.mark.parametrize("env", [{"IVC_GEMM_WIDE": "1"}, {"IVC_GEMM_PAIRS": "0"},
+                                 {"IVC_ROUTER_FUSED": "1"}])
+def test_flash_kernel_variants(env):
+    """The opt-in kernel variants (512-wide pair tiles with split-K, single-CTA
+    256-wide tiles, the persistent router inside the dual flow), each in a fresh
+    process since the switches are read once."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, "-c", _VARIANT_SNIPPET.format(root=root)],
+                         env={**os.environ, **env}, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert "variant ok" in out.stdout
