@@ -208,6 +208,10 @@ int ps_mlp(const void* x, int T, int C, bool half, int flags, const ivc_mlp* m, 
   c.split_part = b.split_part;
   c.split_s = b.split_s;
   c.reserve_sms = reserve_sms;
+  // with weights folded ahead of time the first Linear reads only x and
+  // them; the statistics (ps_stats, which may still be running) are read in
+  // its epilogue alone. (A fold launched just above writes its weights.)
+  c.epi_dep_only = (rt == nullptr && m->fold_colsum != nullptr) ? 1 : 0;
   const int item_rows = half ? 256 : 64;
   if (rt) {
     c.list = rt->list;

@@ -543,6 +543,7 @@ int launch_gemm(const GemmCall& c, const Launch& L) {
   if ((c.list != nullptr || c.stats_remap || c.out_base != nullptr) && c.list_count == nullptr)
     return IVC_EINVAL;
   if (c.stats_remap && c.list == nullptr) return IVC_EINVAL;
+  a.epi_dep_only = (c.epi_dep_only && a.split_max <= 1 && c.list_count == nullptr) ? 1 : 0;
   int rc2;
   switch (bn) {
     case 512: rc2 = run_gemm<512, 4, 2>(maps, a, c.tag, units, L); break;

@@ -106,6 +106,10 @@ struct GemmArgs {
   int split_min;
   float* split_part;
   int* split_s;
+  // A and B are not written by the previous kernel in the stream (only the
+  // epilogue's inputs may be): only the epilogue warps wait for it, the
+  // mainloop starts as soon as the CTA is resident
+  int epi_dep_only;
 };
 
 // Number of k-slices for `tiles` output tiles on `units` CTAs (or pairs).
@@ -235,7 +239,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
   bool ok = true;
   // operands and outputs may belong to the previous kernel in the stream
-  pdl_wait();
+  if (!args.epi_dep_only || warp >= 2) pdl_wait();
   pdl_trigger();
   int M = args.M;
   if (args.list_count != nullptr) {

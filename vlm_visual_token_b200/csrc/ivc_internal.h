@@ -119,6 +119,8 @@ struct GemmCall {
   // SMs to leave to concurrent work (the router beside the connector) when
   // that does not add a round of output tiles; 0 = use every SM
   int reserve_sms;
+  // only the epilogue reads what the previous kernel wrote (GemmArgs)
+  int epi_dep_only;
 };
 int launch_gemm(const GemmCall& c, const Launch& L);
 // Size of the split-K partial buffer: enough for any GEMM shape on this device.
