@@ -484,12 +484,13 @@ def run_ivc(args):
                 "d2h_bytes_per_step": d2h_small + d2h_rows // e2e_steps, "steps": e2e_steps,
                 "timing": "wall clock, host sync per step (the row count read before the row copy)"}
 
-    # ---- the same, pipelined as a streaming user would: two buffer sets on
-    # two streams (each a CUDA graph of the call), so that one step's
-    # host-to-device copies overlap the other's compute and copies back. The
+    # ---- the same, pipelined as a streaming user would: three buffer sets
+    # on three streams (each a CUDA graph of the call), so that one step's
+    # host-to-device copies overlap the others' compute and copies back. The
     # whole row capacity is copied back, so no host sync is needed per step.
+    n_sets = 3
     sets = []
-    for _ in range(2):
+    for _ in range(n_sets):
         st = torch.cuda.Stream(device=dev)
         e = {"st": st, "x": torch.empty_like(x), "vl": torch.empty_like(vl),
              "offs": torch.empty_like(offs), "out": torch.empty_like(out),
@@ -515,7 +516,7 @@ def run_ivc(args):
     barrier()
     t0 = time.perf_counter()
     for i in range(e2e_steps):
-        e = sets[i % 2]
+        e = sets[i % n_sets]
         with torch.cuda.stream(e["st"]):
             e["x"].copy_(hx, non_blocking=True)
             e["vl"].copy_(hvl, non_blocking=True)
@@ -526,13 +527,13 @@ def run_ivc(args):
             e["hout"].copy_(e["out"], non_blocking=True)
     torch.cuda.synchronize()
     e2e_p = reduce_max(time.perf_counter() - t0, world, dev)
-    last = sets[(e2e_steps - 1) % 2]
+    last = sets[(e2e_steps - 1) % n_sets]
     if int(last["hsmall"]["total"][0]) != int(bufs["total"].item()):
         raise RuntimeError("pipelined end-to-end run returned a different row count")
     e2e = {"value": world * T * e2e_steps / e2e_p, "unit": UNIT, "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h_small + T * 256 * w.H * 2, "steps": e2e_steps,
-           "timing": "wall clock over all steps; two streams, inputs copied in and results "
-                     "(small outputs and the whole row capacity) copied out every step",
+           "timing": f"wall clock over all steps; {n_sets} streams, inputs copied in and "
+                     "results (small outputs and the whole row capacity) copied out every step",
            "synchronous": e2e_sync}
     for e in sets:
         del e["g"]
