@@ -22,8 +22,10 @@
 //   vproj    o_h = Wv_h z_h + bv_h
 //   oproj    q = Wo o + bo;  then Q of the next layer = Wq q + bq.
 // Gating: u1 = GELU(W1 h + b1), u2 = W2 u1 + b2, then the residual LayerNorm,
-// each a phase of its own. Selected with IVC_ROUTER_FUSED=1; the separate
-// kernels stay the default while they measure faster.
+// each a phase of its own. This kernel is the default wherever nothing runs
+// beside the router (ivc_vir_route, the router-first flow); beside the
+// connector, where it would have to wait for every SM, the separate kernels
+// are used. IVC_ROUTER_FUSED=1 / 0 forces the choice.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
