@@ -103,6 +103,10 @@ def algorithmic(w, T):
         "pool.scores": (4 * 2.0 * tok * D * 32, 4 * (bf * (tok * D + T * 32 * D) + f32 * tok * 32)),
         "pool.wsum": (4 * 2.0 * T * 32 * 1024 * D,
                       4 * (bf * (tok * D + T * 32 * 1024) + f32 * T * 32 * D)),
+        # the same two contractions in one pass over x per layer (single-pass
+        # form): x and u read once, the merged weighted sums written
+        "pool.attend": (4 * 2.0 * 2 * tok * D * 32,
+                        4 * (bf * (tok * D + T * 32 * D) + f32 * T * 16 * D)),
         "pool.attention": (4 * 4.0 * tok * D, 4 * f32 * tok * 2 * D),  # literal pooling
         "ps_stats": (3.0 * tok * C, bf * tok * C + f32 * 2 * (r256 + r64)),
         # compaction reads and writes the kept rows (all-256 upper bound here;
@@ -414,7 +418,7 @@ def run_ivc(args):
     # the HBM-bound kernels: algorithmic bytes per launch / traced launch time
     hbm = {}
     kept_rows = int(bufs["offsets"][-1].item())  # 256 (T - k) + 64 k of this image
-    for k in ("ps_stats", "compact"):
+    for k in ("ps_stats", "compact", "pool.attend"):
         if k in trace and trace[k]["launches"] > 0:
             us = 1e3 * trace[k]["ms"] / trace[k]["launches"]
             b_launch = alg[k][1] / (trace[k]["launches"] / n_trace)

@@ -249,6 +249,26 @@ def test_flash_compress_small(pool_mode):
     _flash_check(ivc, inp, res)
 
 
+def test_flash_compress_padding_extremes():
+    """The dual flow's router kernels on a tile with one valid token, one whose
+    second 128-token chunk holds a single valid token, and 4 heads of 64."""
+    ivc = _ivc()
+    inp = W.make(small_workload(C=256, H=128, tiles=(3, 2), var=0.6), affine="random")
+    vl = inp["valid_len"].clone()
+    vl[1] = 1
+    vl[3] = 129
+    inp["valid_len"] = vl
+    inp["x"] = W.features(inp["T"], 256, 1234 + 91, vl)
+    m1, m2 = ivc.Mlp(inp["mlp1"]), ivc.Mlp(inp["mlp2"])
+    r = ivc.Router(inp["router"])
+    ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_FLASH, inp["T"], 256, m1, m2, r))
+    res = ivc.flash_compress(inp["x"].cuda(), vl.cuda(), inp["image_offsets"].cuda(), m1, m2, r,
+                             workspace=ws)
+    torch.cuda.synchronize()
+    assert ivc.device_status(ws) == 0
+    _flash_check(ivc, inp, res)
+
+
 def test_flash_compress_empty():
     ivc = _ivc()
     inp = W.make(small_workload(C=256, H=128, tiles=(1,)))
@@ -493,6 +513,9 @@ res = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(), inp["image_of
                          m1, m2, r)
 torch.cuda.synchronize()
 x64 = O.to64(inp["x"])
+ref_gate = O.vir_gate(x64, inp["valid_len"].numpy(), O.to64(inp["router"]))
+gate_err = np.abs(res["gate"].cpu().double().numpy() - ref_gate).max()
+assert gate_err <= {gate_abs!r}, gate_err
 mask = res["mask"].cpu().numpy(); offs = res["offsets"].cpu().numpy()
 for t in range(inp["T"]):
     ref = (O.ps_project(x64[t:t + 1], 0.25, O.to64(inp["mlp2"])) if mask[t]
@@ -505,15 +528,16 @@ print("variant ok")
 
 
 @pytest.mark.parametrize("env", [{"IVC_GEMM_WIDE": "1"}, {"IVC_GEMM_PAIRS": "0"},
-                                 {"IVC_ROUTER_FUSED": "1"}])
+                                 {"IVC_ROUTER_FUSED": "1"}, {"IVC_POOL_ATTEND": "0"}])
 def test_flash_kernel_variants(env):
     """The opt-in kernel variants (512-wide pair tiles with split-K, single-CTA
-    256-wide tiles, the persistent router inside the dual flow), each in a fresh
+    256-wide tiles, the persistent router inside the dual flow, the pooling as
+    tensor-core scores / softmax / weighted-sum kernels), each in a fresh
     process since the switches are read once."""
     import subprocess
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    out = subprocess.run([sys.executable, "-c", _VARIANT_SNIPPET.format(root=root)],
+    out = subprocess.run([sys.executable, "-c", _VARIANT_SNIPPET.format(root=root, gate_abs=GATE_ABS)],
                          env={**os.environ, **env}, capture_output=True, text=True, timeout=600)
     assert out.returncode == 0, out.stderr[-2000:]
     assert "variant ok" in out.stdout

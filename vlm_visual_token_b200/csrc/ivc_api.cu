@@ -257,14 +257,22 @@ int gating_and_route(int T, const int32_t* image_offsets, int I, const ivc_route
                      const Launch& L);
 
 // One folded pooling layer (see ivc_router.cu): u/c from the layer's query,
-// scores = X u^T on the tensor cores, masked softmax, z = p X on the tensor
-// cores, o = Wv z + bv. Q is [T, D], or the shared query (ldq = 0, Tq = 1).
+// then either the single-pass attention (scores, running softmax and
+// weighted sums per 128-token chunk, chunks merged) or scores = X u^T on the
+// tensor cores, masked softmax, z = p X on the tensor cores; o = Wv z + bv.
+// Q is [T, D], or the shared query (ldq = 0, Tq = 1).
 int folded_layer(const void* x, const int32_t* valid_len, int T, const ivc_router* r, int l,
                  const float* Q, long long ldq, const RouteBufs& b, const Launch& L) {
   const int D = r->D;
   const int Tq = ldq == 0 ? 1 : T;
   IVC_TRY(launch_pool_fold_query(Q, ldq, Tq, static_cast<const bf16*>(r->Wk[l]),
                                  static_cast<const bf16*>(r->bk[l]), D, b.U2, b.cb, L));
+  if (pool_attend_wanted()) {
+    // chunk partials in Z, their statistics in S, merged sums in z
+    IVC_TRY(launch_pool_attend(x, b.U2, Tq, b.cb, valid_len, T, D, r->heads, b.Z, b.S, b.z, L));
+    return launch_pool_vproj_heads(b.z, T, D, static_cast<const bf16*>(r->Wv[l]),
+                                   static_cast<const bf16*>(r->bv[l]), b.O, L);
+  }
   GemmCall s{};
   s.tag = "pool.scores";
   s.a_mode = A_PLAIN;

@@ -146,6 +146,18 @@ int launch_pool_softmax(const float* S, const float* cb, int cb_stride, const in
                         int T, int heads, bf16* P2, const Launch& L);
 int launch_pool_vproj(const float* Z, int T, int D, const bf16* Wv, const bf16* bv, float* O,
                       const Launch& L);
+// The same scores, softmax and weighted sums in one pass over x (two
+// launches): per 128-token chunk unnormalised sums Zp [T*8*16, D] and their
+// running max / sum (stats: 2 * T*8*16 floats), merged into z [T*16, D];
+// then o = Wv z + bv reads z row (tile*16 + head).
+int launch_pool_attend(const void* x, const bf16* U2, int Tq, const float* cb,
+                       const int32_t* valid_len, int T, int D, int heads, float* Zp, float* stats,
+                       float* z, const Launch& L);
+int launch_pool_vproj_heads(const float* z, int T, int D, const bf16* Wv, const bf16* bv, float* O,
+                            const Launch& L);
+// Folded pooling through launch_pool_attend (default) or through the
+// tensor-core scores / softmax / weighted-sum kernels (IVC_POOL_ATTEND=0).
+bool pool_attend_wanted();
 // The whole folded router (pooling, gating, routing) as one cooperative
 // persistent kernel (ivc_router_fused.cu).
 struct FusedRouterBufs {

@@ -24,6 +24,8 @@
 // All router vectors between steps are fp32.
 #include <cuda_runtime.h>
 
+#include <cstdlib>
+
 #include "ivc_internal.h"
 #include "ivc_ptx.cuh"
 
@@ -65,12 +67,18 @@ __device__ __forceinline__ void split2(float2 v, uint32_t& hi, uint32_t& lo) {
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
-template <typename XT, bool PAIRED>
+// Where the input row of output row m comes from: row m of X (GV_PLAIN);
+// Z[m*128 + h] + Z[m*128 + 16 + h] (GV_PAIRED: the split weighted sums of the
+// tensor-core pooling form); z[m*16 + h] (GV_HEADROW: the combined weighted
+// sums of the single-pass form); h = (first column of the CTA) / 64.
+enum GemvRows { GV_PLAIN = 0, GV_PAIRED = 1, GV_HEADROW = 2 };
+
+template <typename XT, int ROWS>
 struct GemvLayout {
   // staged input rows (padded by 8 elements), the weight rows (unpadded, one
   // copy), the warps' partial tiles; after a 16-byte mbarrier slot
   __host__ __device__ static size_t x_bytes(int K) {
-    return (PAIRED ? 2 : 1) * static_cast<size_t>(GEMV_ROWS) * (K + 8) * sizeof(XT);
+    return (ROWS == GV_PAIRED ? 2 : 1) * static_cast<size_t>(GEMV_ROWS) * (K + 8) * sizeof(XT);
   }
   __host__ __device__ static size_t w_bytes(int K) { return static_cast<size_t>(GEMV_COLS) * K * 2; }
   __host__ __device__ static size_t total(int K) {
@@ -78,15 +86,14 @@ struct GemvLayout {
   }
 };
 
-// PAIRED: the input row m of the CTA's columns is Z[m*128 + h] + Z[m*128 + 16 + h]
-// with h = (first column) / 64 (the folded pooling's split weighted sums; ldx
-// is then the row length of Z).
-template <typename XT, bool PAIRED>
+// ROWS: see GemvRows (ldx is the row length of Z / z in the pooling modes).
+template <typename XT, int ROWS>
 __global__ void __launch_bounds__(GEMV_THREADS)
     gemv_kernel(const XT* __restrict__ X, long long ldx, int M, int K,
                 const bf16* __restrict__ W, const bf16* __restrict__ b, int N,
                 float* __restrict__ Y, long long ldy, int gelu, int* __restrict__ status) {
-  using Lay = GemvLayout<XT, PAIRED>;
+  using Lay = GemvLayout<XT, ROWS>;
+  constexpr bool PAIRED = ROWS == GV_PAIRED;
   extern __shared__ __align__(16) uint8_t smem[];
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
   XT* sx = reinterpret_cast<XT*>(smem + 16);
@@ -97,7 +104,7 @@ __global__ void __launch_bounds__(GEMV_THREADS)
   const int c0 = blockIdx.x * GEMV_COLS;
   const int w_rows = min(GEMV_COLS, N - c0);
   const int xp = K + 8;
-  const int h = PAIRED ? c0 / 64 : 0;
+  const int h = ROWS != GV_PLAIN ? c0 / 64 : 0;
   const uint32_t xrow = K * sizeof(XT);
   const int rows0 = min(GEMV_ROWS, M);
   if (threadIdx.x == 0) {
@@ -122,6 +129,8 @@ __global__ void __launch_bounds__(GEMV_THREADS)
           const XT* zr = X + (static_cast<long long>(m0 + r) * 128 + h) * ldx;
           bulk_load(sx + r * xp, zr, xrow, bar);
           bulk_load(sx + (GEMV_ROWS + r) * xp, zr + 16 * ldx, xrow, bar);
+        } else if constexpr (ROWS == GV_HEADROW) {
+          bulk_load(sx + r * xp, X + (static_cast<long long>(m0 + r) * 16 + h) * ldx, xrow, bar);
         } else {
           bulk_load(sx + r * xp, X + static_cast<long long>(m0 + r) * ldx, xrow, bar);
         }
@@ -191,23 +200,25 @@ __global__ void __launch_bounds__(GEMV_THREADS)
   }
 }
 
-template <typename XT, bool PAIRED = false>
+template <typename XT, int ROWS = GV_PLAIN>
 static int dispatch_gemv(const XT* X, long long ldx, int M, int K, const bf16* W, const bf16* b,
                          int N, float* Y, long long ldy, int gelu, const Launch& L) {
   if (M == 0 || N == 0) return IVC_OK;
   if (K % (16 * GEMV_WARPS) != 0 || K > 2048 || N % GEMV_COLS != 0) return IVC_EUNSUPPORTED;
+  constexpr bool PAIRED = ROWS == GV_PAIRED;
   if (PAIRED && K > 1024) return IVC_EUNSUPPORTED;
-  const int smem = static_cast<int>(GemvLayout<XT, PAIRED>::total(K));
+  const int smem = static_cast<int>(GemvLayout<XT, ROWS>::total(K));
   static bool attr = false;
   if (!attr) {  // once, for the widest K this instantiation accepts
-    const int max_smem = static_cast<int>(GemvLayout<XT, PAIRED>::total(PAIRED ? 1024 : 2048));
-    if (cudaFuncSetAttribute(gemv_kernel<XT, PAIRED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const int max_smem = static_cast<int>(GemvLayout<XT, ROWS>::total(PAIRED ? 1024 : 2048));
+    if (cudaFuncSetAttribute(gemv_kernel<XT, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              max_smem) != cudaSuccess)
       return IVC_ECUDA;
     attr = true;
   }
-  TraceScope ts(PAIRED ? "pool.vproj" : (gelu ? "router.gemv_gelu" : "router.gemv"), L.stream);
-  return launch_k(gemv_kernel<XT, PAIRED>, dim3(N / GEMV_COLS), dim3(GEMV_THREADS), smem,
+  TraceScope ts(ROWS != GV_PLAIN ? "pool.vproj" : (gelu ? "router.gemv_gelu" : "router.gemv"),
+                L.stream);
+  return launch_k(gemv_kernel<XT, ROWS>, dim3(N / GEMV_COLS), dim3(GEMV_THREADS), smem,
                   L.stream, 1, X, ldx, M, K, W, b, N, Y, ldy, gelu, L.status);
 }
 
@@ -223,7 +234,12 @@ int launch_gemv_bf16x(const bf16* x, int K, const bf16* W, const bf16* b, int N,
 
 int launch_pool_vproj(const float* Z, int T, int D, const bf16* Wv, const bf16* bv, float* O,
                       const Launch& L) {
-  return dispatch_gemv<float, true>(Z, D, T, D, Wv, bv, D, O, D, 0, L);
+  return dispatch_gemv<float, GV_PAIRED>(Z, D, T, D, Wv, bv, D, O, D, 0, L);
+}
+
+int launch_pool_vproj_heads(const float* z, int T, int D, const bf16* Wv, const bf16* bv, float* O,
+                            const Launch& L) {
+  return dispatch_gemv<float, GV_HEADROW>(z, D, T, D, Wv, bv, D, O, D, 0, L);
 }
 
 // ---------------------------------------------------------------- pooling attention
@@ -461,6 +477,371 @@ int launch_pool_softmax(const float* S, const float* cb, int cb_stride, const in
   TraceScope ts("pool.softmax", L.stream);
   return launch_k(pool_softmax_kernel, dim3(heads, T), dim3(ATT_THREADS), 0, L.stream, 1, S, cb,
                   cb_stride, valid_len, P2, L.status);
+}
+
+// ---------------------------------------------------------------- single-pass pooling attention
+// The same layer as scores + softmax + weighted sum above, with one read of
+// the features (the split-softmax, or flash-decoding, form of attention with
+// one query per head): CTA (tile, chunk of ATTN_CHUNK tokens) streams its
+// tokens ATTN_STEP at a time (one TMA box of {64 channels, 32 tokens, D/64
+// chunks}, 128-byte swizzle, double-buffered) and per step
+//   1. s[t][j] = x_t . U2[j] for the 32 split rows j (warp w multiplies its
+//      D/8 channels with m16n8k16 MMAs, the U2 fragments held in registers
+//      for the whole CTA; the 8 partial 32x32 tiles are summed in shared
+//      memory), s_h = s[t][h] + s[t][16 + h] + c_h, invalid tokens -inf;
+//   2. running max m_h and sum l_h (rescaled by exp(m_old - m_new)), the
+//      weights e = exp(s - m_h) split into a bf16 hi/lo pair;
+//   3. Zc[h][c] = Zc[h][c] * exp(m_old - m_new) + sum_t e_t x_t[c] with the
+//      hi and lo weights into the same fp32 accumulators (warp w owns
+//      channels [w D/8, (w+1) D/8), accumulators in registers).
+// The chunk's unnormalised Zc, m and l go to global memory; pool_combine_
+// kernel merges a tile's ATTN_NCH chunks:
+//   z_h = sum_c exp(m_c - M) Zc_h / sum_c exp(m_c - M) l_c,  M = max_c m_c.
+constexpr int ATTN_STEP = 32;                        // tokens per staged box
+constexpr int ATTN_CHUNK = 128;                      // tokens per CTA
+constexpr int ATTN_NCH = TILE_TOKENS / ATTN_CHUNK;   // chunks (partials) per tile
+constexpr int ATTN_RED_PITCH = 33;                   // floats per row of a partial score tile
+constexpr int ATTN_P_PITCH = 40;                     // bf16 per row of the weight tile (80 B)
+
+__device__ __forceinline__ void ldsm4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void ldsm4_trans(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+
+__host__ __device__ constexpr size_t attend_smem_bytes(int D) {
+  // alignment slack, two staging slots, 8 partial score tiles, hi/lo weights
+  return 1024 + 2 * static_cast<size_t>(D) * 64 + 8 * 32 * ATTN_RED_PITCH * 4 +
+         2 * 16 * ATTN_P_PITCH * 2;
+}
+
+// KS = D / 128: k16 steps of a warp's channel slice (D = 128 .. 1024).
+template <int KS>
+__global__ void __launch_bounds__(256, 1)
+    pool_attend_kernel(const __grid_constant__ CUtensorMap xmap, const bf16* __restrict__ U2,
+                       int u2_per_tile, const float* __restrict__ cb, int cb_stride,
+                       const int32_t* __restrict__ valid_len, int heads, float* __restrict__ Zp,
+                       float* __restrict__ mstat, float* __restrict__ lstat,
+                       int* __restrict__ status) {
+  constexpr int D = 128 * KS;
+  constexpr int SLOT = D * 64;  // D/64 chunks x 32 tokens x 128 B
+  constexpr int CHUNK_BYTES = ATTN_STEP * 128;
+  constexpr int NT = 2 * KS;    // n8 tiles of a warp's weighted-sum channels
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  float* red = reinterpret_cast<float*>(sm + 2 * SLOT);
+  bf16* sp = reinterpret_cast<bf16*>(red + 8 * 32 * ATTN_RED_PITCH);  // [hi, lo][16][pitch]
+  __shared__ float s_m[16], s_l[16], s_scale[16];
+  __shared__ __align__(8) uint64_t s_mb[2];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t2 = (lane & 3) * 2;
+  const int tile = blockIdx.x / ATTN_NCH, chunk = blockIdx.x % ATTN_NCH;
+  const int tok0 = chunk * ATTN_CHUNK;
+  // x and valid_len are inputs of the call and the previous kernel waited
+  // for its own predecessor before letting this one start: both are read
+  // before pdl_wait.
+  int n = TILE_TOKENS;
+  if (valid_len != nullptr) {
+    n = valid_len[tile];
+    if (n < 1 || n > TILE_TOKENS) {
+      if (threadIdx.x == 0 && chunk == 0) atomicOr(status, DEV_BAD_VALID_LEN);
+      n = n < 1 ? 1 : TILE_TOKENS;
+    }
+  }
+  const int nsteps = max(0, min(ATTN_CHUNK / ATTN_STEP, (n - tok0 + ATTN_STEP - 1) / ATTN_STEP));
+  if (threadIdx.x == 0) {
+    mbar_init(&s_mb[0], 1);
+    mbar_init(&s_mb[1], 1);
+    fence_mbar_init();
+    for (int st = 0; st < min(2, nsteps); ++st) {
+      mbar_arrive_expect_tx(&s_mb[st], SLOT);
+      tma_load_3d(sm + st * SLOT, &xmap, &s_mb[st], 0, tile * TILE_TOKENS + tok0 + st * ATTN_STEP,
+                  0);
+    }
+  }
+  if (threadIdx.x < 16) {
+    s_m[threadIdx.x] = -INFINITY;
+    s_l[threadIdx.x] = 0.f;
+  }
+  __syncthreads();
+  pdl_wait();
+  pdl_trigger();
+  const size_t row0 = (static_cast<size_t>(tile) * ATTN_NCH + chunk) * 16;
+  if (nsteps == 0) {  // every token of the chunk is padding
+    if (threadIdx.x < 16) {
+      mstat[row0 + threadIdx.x] = -INFINITY;
+      lstat[row0 + threadIdx.x] = 0.f;
+    }
+    return;
+  }
+  // B fragments of the scores (B[k = channel][n = split row] = U2[n][k]) for
+  // this warp's channels; rows of heads that do not exist are zero
+  const bf16* u = U2 + (u2_per_tile ? static_cast<size_t>(tile) * 32 * D : 0);
+  uint32_t ub[KS][4][2];
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    const int k = (warp * KS + ks) * 16 + t2;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const int r = nt * 8 + g;
+      const bool live = (r & 15) < heads;
+      const bf16* ur = u + static_cast<size_t>(r) * D + k;
+      ub[ks][nt][0] = live ? __ldg(reinterpret_cast<const unsigned*>(ur)) : 0u;
+      ub[ks][nt][1] = live ? __ldg(reinterpret_cast<const unsigned*>(ur + 8)) : 0u;
+    }
+  }
+  const int sh = threadIdx.x >> 4, stl = threadIdx.x & 15;  // softmax: head, token pair
+  const float c_h = sh < heads ? cb[static_cast<size_t>(tile) * cb_stride + sh] : 0.f;
+  float accz[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) accz[nt][i] = 0.f;
+  bool ok = true;
+  for (int st = 0; st < nsteps; ++st) {
+    const int slot = st & 1;
+    const uint8_t* sx = sm + slot * SLOT;
+    ok = mbar_wait(&s_mb[slot], (st >> 1) & 1) && ok;
+    // 1. partial scores of this warp's channels
+    float accs[2][4][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) accs[mt][nt][i] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const int kg = warp * KS + ks;
+      const int c = kg >> 2, ja = ((kg & 3) << 1) + (lane >> 4);
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const int ra = mt * 16 + (lane & 15);
+        uint32_t af[4];
+        ldsm4(af, sx + c * CHUNK_BYTES + ra * 128 + ((ja ^ (ra & 7)) << 4));
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) mma_16816(accs[mt][nt], af, ub[ks][nt]);
+      }
+    }
+    float* rw = red + warp * 32 * ATTN_RED_PITCH;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        const int r = mt * 16 + g, j = nt * 8 + t2;
+        rw[r * ATTN_RED_PITCH + j] = accs[mt][nt][0];
+        rw[r * ATTN_RED_PITCH + j + 1] = accs[mt][nt][1];
+        rw[(r + 8) * ATTN_RED_PITCH + j] = accs[mt][nt][2];
+        rw[(r + 8) * ATTN_RED_PITCH + j + 1] = accs[mt][nt][3];
+      }
+    ok = __syncthreads_and(ok) != 0;
+    if (!ok) break;
+    // 2. running softmax of head sh over tokens stl and stl + 16
+    {
+      const int tb = tok0 + st * ATTN_STEP;
+      float sv[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int t = stl + 16 * i;
+        float v = c_h;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          const float* rr = red + (w * 32 + t) * ATTN_RED_PITCH;
+          v += rr[sh] + rr[16 + sh];
+        }
+        sv[i] = (sh < heads && tb + t < n) ? v : -INFINITY;
+      }
+      float mx = fmaxf(sv[0], sv[1]);
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float m_old = s_m[sh];
+      const float m_new = fmaxf(m_old, mx);
+      float e[2] = {0.f, 0.f}, scale = 1.f;
+      if (m_new != -INFINITY) {
+        scale = expf(m_old - m_new);
+        e[0] = expf(sv[0] - m_new);
+        e[1] = expf(sv[1] - m_new);
+      }
+      float sum = e[0] + e[1];
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const bf16 hi = __float2bfloat16_rn(e[i]);
+        sp[sh * ATTN_P_PITCH + stl + 16 * i] = hi;
+        sp[(16 + sh) * ATTN_P_PITCH + stl + 16 * i] = __float2bfloat16_rn(e[i] - __bfloat162float(hi));
+      }
+      __syncwarp();  // every lane has read s_m[sh]
+      if (stl == 0) {
+        s_l[sh] = s_l[sh] * scale + sum;
+        s_m[sh] = m_new;
+        s_scale[sh] = scale;
+      }
+    }
+    __syncthreads();
+    // 3. rescale and accumulate this warp's channels of Zc
+    {
+      const float sc0 = s_scale[g], sc1 = s_scale[g + 8];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        accz[nt][0] *= sc0;
+        accz[nt][1] *= sc0;
+        accz[nt][2] *= sc1;
+        accz[nt][3] *= sc1;
+      }
+#pragma unroll
+      for (int kk = 0; kk < ATTN_STEP / 16; ++kk) {
+        uint32_t ah[4], al[4];
+        const int pr = lane & 15, pk = kk * 16 + 8 * (lane >> 4);
+        ldsm4(ah, sp + pr * ATTN_P_PITCH + pk);
+        ldsm4(al, sp + (16 + pr) * ATTN_P_PITCH + pk);
+        const int r = kk * 16 + (lane & 15);
+#pragma unroll
+        for (int nt = 0; nt < NT; nt += 2) {
+          const int cw = warp * (D / 8) + 8 * (nt + (lane >> 4));
+          const int c = cw >> 6, j = (cw & 63) >> 3;
+          uint32_t bf[4];
+          ldsm4_trans(bf, sx + c * CHUNK_BYTES + r * 128 + ((j ^ (r & 7)) << 4));
+          const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
+          mma_16816(accz[nt], ah, b0);
+          mma_16816(accz[nt], al, b0);
+          mma_16816(accz[nt + 1], ah, b1);
+          mma_16816(accz[nt + 1], al, b1);
+        }
+      }
+    }
+    __syncthreads();  // every warp is done with this slot and with the weights
+    if (threadIdx.x == 0 && st + 2 < nsteps) {
+      mbar_arrive_expect_tx(&s_mb[slot], SLOT);
+      tma_load_3d(sm + slot * SLOT, &xmap, &s_mb[slot], 0,
+                  tile * TILE_TOKENS + tok0 + (st + 2) * ATTN_STEP, 0);
+    }
+  }
+  if (!ok) {
+    if (threadIdx.x == 0) atomicOr(status, DEV_WAIT_TIMEOUT);
+    return;
+  }
+  float* zp = Zp + row0 * D;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int c = warp * (D / 8) + nt * 8 + t2;
+    *reinterpret_cast<float2*>(zp + static_cast<size_t>(g) * D + c) =
+        make_float2(accz[nt][0], accz[nt][1]);
+    *reinterpret_cast<float2*>(zp + static_cast<size_t>(g + 8) * D + c) =
+        make_float2(accz[nt][2], accz[nt][3]);
+  }
+  if (threadIdx.x < 16) {
+    mstat[row0 + threadIdx.x] = s_m[threadIdx.x];
+    lstat[row0 + threadIdx.x] = s_l[threadIdx.x];
+  }
+}
+
+// Grid (heads, T): z[tile][h] from the tile's ATTN_NCH chunk partials
+// (chunks without a valid token, l = 0, are skipped).
+__global__ void __launch_bounds__(256)
+    pool_combine_kernel(const float* __restrict__ Zp, const float* __restrict__ mstat,
+                        const float* __restrict__ lstat, int D, float* __restrict__ z) {
+  const int h = blockIdx.x, tile = blockIdx.y;
+  pdl_wait();
+  pdl_trigger();
+  const size_t r0 = static_cast<size_t>(tile) * ATTN_NCH * 16 + h;
+  float w[ATTN_NCH];
+  float M = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < ATTN_NCH; ++c) {
+    w[c] = lstat[r0 + 16 * c] > 0.f ? mstat[r0 + 16 * c] : -INFINITY;
+    M = fmaxf(M, w[c]);
+  }
+  float L = 0.f;
+#pragma unroll
+  for (int c = 0; c < ATTN_NCH; ++c) {
+    w[c] = w[c] == -INFINITY ? 0.f : expf(w[c] - M);
+    L += w[c] * lstat[r0 + 16 * c];
+  }
+  const float inv = 1.0f / L;
+  for (int c4 = threadIdx.x * 4; c4 < D; c4 += 1024) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < ATTN_NCH; ++c) {
+      if (w[c] == 0.f) continue;
+      const float4 v = __ldg(reinterpret_cast<const float4*>(Zp + (r0 + 16 * c) * D + c4));
+      acc.x = fmaf(w[c], v.x, acc.x);
+      acc.y = fmaf(w[c], v.y, acc.y);
+      acc.z = fmaf(w[c], v.z, acc.z);
+      acc.w = fmaf(w[c], v.w, acc.w);
+    }
+    *reinterpret_cast<float4*>(z + (static_cast<size_t>(tile) * 16 + h) * D + c4) =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  }
+}
+
+bool pool_attend_wanted() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("IVC_POOL_ATTEND");
+    v = (e && e[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+
+template <int KS>
+static int launch_attend_ks(const CUtensorMap& xmap, const bf16* U2, int u2_per_tile,
+                            const float* cb, int cb_stride, const int32_t* valid_len, int T,
+                            int heads, float* Zp, float* mstat, float* lstat, const Launch& L) {
+  const size_t smem = attend_smem_bytes(128 * KS);
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(pool_attend_kernel<KS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return IVC_ECUDA;
+    attr = true;
+  }
+  return launch_k(pool_attend_kernel<KS>, dim3(T * ATTN_NCH), dim3(256), smem, L.stream, 1, xmap,
+                  U2, u2_per_tile, cb, cb_stride, valid_len, heads, Zp, mstat, lstat, L.status);
+}
+
+int launch_pool_attend(const void* x, const bf16* U2, int Tq, const float* cb,
+                       const int32_t* valid_len, int T, int D, int heads, float* Zp, float* stats,
+                       float* z, const Launch& L) {
+  if (T == 0) return IVC_OK;
+  if (D % 128 != 0 || D > 1024 || heads < 1 || heads > 16 || heads * 64 != D)
+    return IVC_EUNSUPPORTED;
+  CUtensorMap xmap;
+  {
+    // x as {64 channels, T*1024 tokens, D/64 chunks}: rows of 2D bytes, chunks 128 B apart
+    const unsigned long long dims[3] = {64, static_cast<unsigned long long>(T) * TILE_TOKENS,
+                                        static_cast<unsigned long long>(D) / 64};
+    const unsigned long long strides[2] = {static_cast<unsigned long long>(D) * 2, 128};
+    const unsigned box[3] = {64, ATTN_STEP, static_cast<unsigned>(D / 64)};
+    if (map_bf16(&xmap, 3, x, dims, strides, box) != IVC_OK) return IVC_ECUDA;
+  }
+  float* mstat = stats;
+  float* lstat = stats + static_cast<size_t>(T) * ATTN_NCH * 16;
+  const int u2_per_tile = Tq == 1 ? 0 : 1;
+  const int cb_stride = Tq == 1 ? 0 : 16;
+  int rc;
+  {
+    TraceScope ts("pool.attend", L.stream);
+    switch (D / 128) {
+      case 1: rc = launch_attend_ks<1>(xmap, U2, u2_per_tile, cb, cb_stride, valid_len, T, heads, Zp, mstat, lstat, L); break;
+      case 2: rc = launch_attend_ks<2>(xmap, U2, u2_per_tile, cb, cb_stride, valid_len, T, heads, Zp, mstat, lstat, L); break;
+      case 3: rc = launch_attend_ks<3>(xmap, U2, u2_per_tile, cb, cb_stride, valid_len, T, heads, Zp, mstat, lstat, L); break;
+      case 4: rc = launch_attend_ks<4>(xmap, U2, u2_per_tile, cb, cb_stride, valid_len, T, heads, Zp, mstat, lstat, L); break;
+      case 5: rc = launch_attend_ks<5>(xmap, U2, u2_per_tile, cb, cb_stride, valid_len, T, heads, Zp, mstat, lstat, L); break;
+      case 6: rc = launch_attend_ks<6>(xmap, U2, u2_per_tile, cb, cb_stride, valid_len, T, heads, Zp, mstat, lstat, L); break;
+      case 7: rc = launch_attend_ks<7>(xmap, U2, u2_per_tile, cb, cb_stride, valid_len, T, heads, Zp, mstat, lstat, L); break;
+      default: rc = launch_attend_ks<8>(xmap, U2, u2_per_tile, cb, cb_stride, valid_len, T, heads, Zp, mstat, lstat, L); break;
+    }
+  }
+  if (rc != IVC_OK) return rc;
+  TraceScope ts("pool.combine", L.stream);
+  return launch_k(pool_combine_kernel, dim3(heads, T), dim3(256), 0, L.stream, 1, Zp, mstat, lstat,
+                  D, z);
 }
 
 // ---------------------------------------------------------------- residual + LayerNorm
