@@ -37,17 +37,18 @@ __device__ __forceinline__ float gelu_f(float y) {
 
 // ---------------------------------------------------------------- skinny GEMV
 // Y[m, n] = act(sum_k X[m, k] W[n, k] + b[n]) for few rows m (router vectors),
-// on the tensor cores (m16n8k16). A CTA of 8 warps owns 8 consecutive columns
-// (one n8 tile). One thread brings their 8 weight rows (contiguous in W) into
-// shared memory with one bulk copy issued before waiting for the previous
-// kernel, and up to 16 input rows per round (one bulk copy per row) on the same
-// mbarrier. Warp w multiplies the k-range [w K/8, (w+1) K/8): fp32 inputs are
+// on the tensor cores (m16n8k16). A CTA of 8 warps owns 16 consecutive columns
+// (two n8 tiles, so that each staged input row serves 16 columns). One thread
+// brings their 16 weight rows (contiguous in W) into shared memory with one
+// bulk copy issued before waiting for the previous kernel, and up to 16 input
+// rows per round (one bulk copy per row) on the same mbarrier. Warp w multiplies the k-range [w K/8, (w+1) K/8): fp32 inputs are
 // split into a bf16 pair hi + lo (two MMAs per k-step, fp32 accumulate, about
 // 16 significant bits of the input kept), bf16 inputs enter as they are. The
 // 8 partial m16n8 tiles are summed through shared memory.
 constexpr int GEMV_THREADS = 256;
 constexpr int GEMV_WARPS = GEMV_THREADS / 32;
-constexpr int GEMV_COLS = 8;   // output columns per CTA
+constexpr int GEMV_COLS = 16;  // output columns per CTA (two n8 tiles)
+constexpr int GEMV_NT = GEMV_COLS / 8;
 constexpr int GEMV_ROWS = 16;  // input rows per round
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
@@ -143,20 +144,26 @@ __global__ void __launch_bounds__(GEMV_THREADS)
     }
     // rows >= `rows` of the A tile hold stale values; they only reach output
     // rows that are never stored
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const int wr = g < w_rows ? g : 0;
+    float acc[GEMV_NT][4] = {};
+    int wr[GEMV_NT];  // weight row of this lane per n8 tile (rows past N read row 0)
+#pragma unroll
+    for (int j = 0; j < GEMV_NT; ++j) wr[j] = 8 * j + g < w_rows ? 8 * j + g : 0;
     for (int ks = warp * kw; ks < (warp + 1) * kw; ks += 16) {
       const int k = ks + t2;
-      uint32_t bw[2];
-      bw[0] = *reinterpret_cast<const uint32_t*>(sw + static_cast<size_t>(wr) * K + k);
-      bw[1] = *reinterpret_cast<const uint32_t*>(sw + static_cast<size_t>(wr) * K + k + 8);
+      uint32_t bw[GEMV_NT][2];
+#pragma unroll
+      for (int j = 0; j < GEMV_NT; ++j) {
+        bw[j][0] = *reinterpret_cast<const uint32_t*>(sw + static_cast<size_t>(wr[j]) * K + k);
+        bw[j][1] = *reinterpret_cast<const uint32_t*>(sw + static_cast<size_t>(wr[j]) * K + k + 8);
+      }
       if constexpr (sizeof(XT) == 2) {
         uint32_t a[4];
         a[0] = *reinterpret_cast<const uint32_t*>(sx + g * xp + k);
         a[1] = *reinterpret_cast<const uint32_t*>(sx + (g + 8) * xp + k);
         a[2] = *reinterpret_cast<const uint32_t*>(sx + g * xp + k + 8);
         a[3] = *reinterpret_cast<const uint32_t*>(sx + (g + 8) * xp + k + 8);
-        mma_16816(acc, a, bw);
+#pragma unroll
+        for (int j = 0; j < GEMV_NT; ++j) mma_16816(acc[j], a, bw[j]);
       } else {
         const float* fx = reinterpret_cast<const float*>(sx);
         float2 v[4] = {*reinterpret_cast<const float2*>(fx + g * xp + k),
@@ -175,22 +182,28 @@ __global__ void __launch_bounds__(GEMV_THREADS)
         uint32_t ah[4], al[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) split2(v[i], ah[i], al[i]);
-        mma_16816(acc, ah, bw);
-        mma_16816(acc, al, bw);
+#pragma unroll
+        for (int j = 0; j < GEMV_NT; ++j) {
+          mma_16816(acc[j], ah, bw[j]);
+          mma_16816(acc[j], al, bw[j]);
+        }
       }
     }
     float* rw = red + warp * (GEMV_ROWS * GEMV_COLS);
-    rw[g * GEMV_COLS + t2] = acc[0];
-    rw[g * GEMV_COLS + t2 + 1] = acc[1];
-    rw[(g + 8) * GEMV_COLS + t2] = acc[2];
-    rw[(g + 8) * GEMV_COLS + t2 + 1] = acc[3];
+#pragma unroll
+    for (int j = 0; j < GEMV_NT; ++j) {
+      rw[g * GEMV_COLS + 8 * j + t2] = acc[j][0];
+      rw[g * GEMV_COLS + 8 * j + t2 + 1] = acc[j][1];
+      rw[(g + 8) * GEMV_COLS + 8 * j + t2] = acc[j][2];
+      rw[(g + 8) * GEMV_COLS + 8 * j + t2 + 1] = acc[j][3];
+    }
     __syncthreads();
-    if (threadIdx.x < GEMV_ROWS * GEMV_COLS) {
-      const int r = threadIdx.x / GEMV_COLS, c = threadIdx.x % GEMV_COLS;
+    for (int o = threadIdx.x; o < GEMV_ROWS * GEMV_COLS; o += GEMV_THREADS) {
+      const int r = o / GEMV_COLS, c = o % GEMV_COLS;
       if (r < rows && c < w_rows) {
         float y = 0.f;
 #pragma unroll
-        for (int w = 0; w < GEMV_WARPS; ++w) y += red[w * GEMV_ROWS * GEMV_COLS + threadIdx.x];
+        for (int w = 0; w < GEMV_WARPS; ++w) y += red[w * GEMV_ROWS * GEMV_COLS + o];
         if (b != nullptr) y += __bfloat162float(b[c0 + c]);
         if (gelu) y = gelu_f(y);
         Y[static_cast<long long>(m0 + r) * ldy + c0 + c] = y;
@@ -204,7 +217,7 @@ template <typename XT, int ROWS = GV_PLAIN>
 static int dispatch_gemv(const XT* X, long long ldx, int M, int K, const bf16* W, const bf16* b,
                          int N, float* Y, long long ldy, int gelu, const Launch& L) {
   if (M == 0 || N == 0) return IVC_OK;
-  if (K % (16 * GEMV_WARPS) != 0 || K > 2048 || N % GEMV_COLS != 0) return IVC_EUNSUPPORTED;
+  if (K % (16 * GEMV_WARPS) != 0 || K > 2048 || N % 8 != 0) return IVC_EUNSUPPORTED;
   constexpr bool PAIRED = ROWS == GV_PAIRED;
   if (PAIRED && K > 1024) return IVC_EUNSUPPORTED;
   const int smem = static_cast<int>(GemvLayout<XT, ROWS>::total(K));
@@ -218,8 +231,9 @@ static int dispatch_gemv(const XT* X, long long ldx, int M, int K, const bf16* W
   }
   TraceScope ts(ROWS != GV_PLAIN ? "pool.vproj" : (gelu ? "router.gemv_gelu" : "router.gemv"),
                 L.stream);
-  return launch_k(gemv_kernel<XT, ROWS>, dim3(N / GEMV_COLS), dim3(GEMV_THREADS), smem,
-                  L.stream, 1, X, ldx, M, K, W, b, N, Y, ldy, gelu, L.status);
+  return launch_k(gemv_kernel<XT, ROWS>, dim3((N + GEMV_COLS - 1) / GEMV_COLS),
+                  dim3(GEMV_THREADS), smem, L.stream, 1, X, ldx, M, K, W, b, N, Y, ldy, gelu,
+                  L.status);
 }
 
 int launch_gemv(const float* X, long long ldx, int M, int K, const bf16* W, const bf16* b, int N,
