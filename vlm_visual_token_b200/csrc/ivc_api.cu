@@ -325,7 +325,7 @@ int route_impl(const void* x, const int32_t* valid_len, int T, const int32_t* im
                int32_t* total, const RouteBufs& b, const Launch& L, bool fused_default) {
   const int D = r->D;
   if (router_fused_supported(r) && router_fused_wanted(fused_default)) {
-    FusedRouterBufs f{b.Q, b.U2, b.cb, b.S, b.P2, b.z, b.O, b.q, b.h, b.u1, b.u2, b.bar};
+    FusedRouterBufs f{b.Q, b.U2, b.cb, b.S, b.Z, b.z, b.O, b.q, b.h, b.u1, b.u2, b.bar};
     return launch_router_fused(r, x, valid_len, T, image_offsets, I, gate, mask, offsets, total,
                                f, L);
   }

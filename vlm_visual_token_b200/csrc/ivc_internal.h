@@ -164,8 +164,8 @@ struct FusedRouterBufs {
   float* Q;
   bf16* U2;
   float* cb;
-  float* S;
-  bf16* P2;
+  float* stats;  // 2 * T*8*16 floats
+  float* Zp;     // [T*8*16, D]
   float* z;
   float* O;
   float* q;

@@ -16,9 +16,9 @@
 // guaranteed by the cooperative launch; every wait is bounded). Per pooling
 // layer (the folded form of the single-query attention, see ivc_router.cu):
 //   fold     u_h = Wk_h^T Q_h / 8, c_h = bk_h . Q_h / 8   (hi/lo bf16 split of u)
-//   scores   s[t, h] = x_t . u_h  for every token        (mma.sync, fp32 accumulate)
-//   softmax  p = softmax over the valid tokens, split hi/lo bf16
-//   wsum     z_h = sum_t p_t x_t                          (mma.sync, fp32 accumulate)
+//   attend   per 128-token chunk: s[t, h] = x_t . u_h + c_h, running softmax,
+//            Zc_h = sum_t exp(s - m) x_t  (mma.sync, fp32 accumulate; x read once)
+//   combine  z_h = softmax-weighted merge of the tile's 8 chunks
 //   vproj    o_h = Wv_h z_h + bv_h
 //   oproj    q = Wo o + bo;  then Q of the next layer = Wq q + bq.
 // Gating: u1 = GELU(W1 h + b1), u2 = W2 u1 + b2, then the residual LayerNorm,
@@ -45,16 +45,12 @@ constexpr int RF_MAXD = 1024;   // widest pooling width (scores staging)
 constexpr int RF_MAXK = 2048;   // widest projection input
 constexpr int GV_COLS = 8;      // output columns per projection item (one n8 MMA tile)
 constexpr int GV_ROWS = 16;     // input rows per projection round (one m16 MMA tile)
-constexpr int WS_BOX = 256;     // tokens per TMA box of the weighted-sum staging
-constexpr int SC_TOK = 32;      // tokens per scores item
-constexpr int WS_HALF = RF_TOK / 2;  // tokens per weighted-sum item
+constexpr int SC_TOK = 32;      // tokens per staged step of the attention phase
 
 struct RouterFusedArgs {
-  // 128-byte swizzled TMA views (one request per staged operand):
-  CUtensorMap xmap;   // x as [T*1024, D], box 64 channels x WS_BOX tokens
-  CUtensorMap xmap3;  // x as {64 ch, T*1024 tokens, D/64 chunks}, box {64, SC_TOK, D/64}
-  CUtensorMap u2map;  // U2 as {64, 32 rows, D/64 chunks, T}, box {64, 32, D/64, 1}
-  CUtensorMap p2map;  // P2 as {64 tokens, 32 rows, 16 chunks, T}, box {64, 32, 8, 1}
+  // x as {64 ch, T*1024 tokens, D/64 chunks}, box {64, SC_TOK, D/64}, 128-byte
+  // swizzle (one request per staged step)
+  CUtensorMap xmap3;
   const bf16* x;      // [T, 1024, D]
   const int32_t* valid_len;
   int T, D, G, heads;
@@ -67,9 +63,9 @@ struct RouterFusedArgs {
   float* Q;     // [T, D]
   bf16* U2;     // [T, 32, D]
   float* cb;    // [T, 16]
-  float* S;     // [T, 32, 1024] split scores, token-contiguous
-  bf16* P2;     // [T, 32, 1024] split softmax weights
-  float* z;     // [T, 16, D]
+  float* Zp;    // [T, 8 chunks, 16, D] unnormalised weighted sums per chunk
+  float* stats; // [2][T, 8 chunks, 16]: running max m, then sum l
+  float* z;     // [T, 16, D] merged weighted sums
   float* O;     // [T, D]
   float* q;     // [T, D]
   float* h;     // [T, D]
@@ -131,14 +127,9 @@ __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(smem_u32(p)));
 }
-__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
-               : "=r"(r[0]), "=r"(r[1])
-               : "r"(smem_u32(p)));
-}
-__device__ __forceinline__ void ldsm_x2_trans(uint32_t (&r)[2], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
-               : "=r"(r[0]), "=r"(r[1])
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(smem_u32(p)));
 }
 // Orders this thread's later async-proxy (bulk copy / TMA) reads of global
@@ -376,322 +367,362 @@ __device__ bool fold_phase(const RouterFusedArgs& a, int l, int Tq, const float*
   return true;
 }
 
-// ------------------------------------------------------------------ scores phase
-// Items (tile, SC_TOK-token block), a contiguous range per CTA so that
-// consecutive items share the tile's U2 rows. St[tile][j][t] = sum_c
-// x[tile][t][c] U2[tu][j][c], j < 32 (hi rows 0..15, lo rows 16..31); tu =
-// tile, or 0 when the query is shared. Each operand arrives as one TMA
-// request in the 128-byte swizzled layout [D/64 chunks][rows][128 B] (the
-// 16-byte piece j of row r at j ^ (r & 7)): U2 on mbarrier 1 when the tile
-// changes, x double-buffered on mbarriers 2 and 3 (the CTA's first two x
-// items are requested before the grid barrier, x being an input). Warp w
-// computes m16 tile (w & 1) x n8 tile (w >> 1) with m16n8k16 bf16 MMAs.
-// Shared memory: U2 at 0, then x slots 0 and 1 (D/64 * 4 KB each); the x
-// slots start at or above FOLD_SMEM since they are filled while the fold
-// phase still uses that region.
+// ------------------------------------------------------------------ attention phase
+// Scores, softmax and weighted sums of one pooling layer in one pass over x
+// (the split-softmax form of single-query attention). Items (tile, chunk of
+// AT_CHUNK tokens), a contiguous range per CTA; each item takes its tokens
+// SC_TOK at a time, one TMA request per step ({64 channels, 32 tokens, D/64
+// chunks}, 128-byte swizzle), double-buffered on mbarriers 2 and 3 across the
+// CTA's steps (the first two requested before the grid barrier, x being an
+// input). Per step:
+//   1. s[t][j] = x_t . U2[j] for the 32 split rows: warp w multiplies its D/8
+//      channels with m16n8k16 MMAs (its U2 fragments in registers for the
+//      item), the 8 partial 32x32 tiles are summed in shared memory;
+//      s_h = s[t][h] + s[t][16 + h] + c_h, tokens past valid_len -inf;
+//   2. running max m_h and sum l_h, weights e = exp(s - m_h) as a bf16 hi/lo
+//      pair;
+//   3. Zc[h][c] = Zc[h][c] exp(m_old - m_new) + sum_t e_t x_t[c] (warp w owns
+//      channels [w D/8, (w+1) D/8), hi and lo weights into the same fp32
+//      accumulators in registers).
+// Each item writes its unnormalised Zc to Zp[tile][chunk] and m, l to stats;
+// the combine phase merges a tile's chunks. U2 and c are read with plain loads:
+// they are written inside this kernel (the fold phase).
+// Shared memory: 8 partial score tiles | hi/lo weights | x slots 0 and 1
+// (D/64 * 4 KB each, above the fold phase's region since they are filled
+// before the barrier that ends it for every CTA).
+constexpr int AT_CHUNK = 128;                 // tokens per item
+constexpr int AT_NCH = RF_TOK / AT_CHUNK;     // items (partials) per tile
+constexpr int AT_RED_PITCH = 33;
+constexpr int AT_P_PITCH = 40;
+constexpr int AT_RED_BYTES = RF_WARPS * 32 * AT_RED_PITCH * 4;
+constexpr int AT_SLOT0 = ((AT_RED_BYTES + 2 * 16 * AT_P_PITCH * 2 + 1023) / 1024) * 1024;
 constexpr int FOLD_SMEM = RF_HD * 128 * 2 + 64 * RF_HD * 4;  // Wk block + Q block
+static_assert(AT_SLOT0 >= FOLD_SMEM, "x slots must not overlap the fold phase's staging");
 
-__device__ __forceinline__ uint8_t* scores_x_slot(uint8_t* sm, int D, int slot) {
-  const int slot_bytes = (D / 64) * SC_TOK * 128;
-  return sm + max(slot_bytes, FOLD_SMEM) + slot * slot_bytes;
-}
-
-__device__ __forceinline__ void scores_range(const RouterFusedArgs& a, int& i0, int& i1) {
-  const int n_items = a.T * (RF_TOK / SC_TOK);
+__device__ __forceinline__ void attend_range(const RouterFusedArgs& a, int& i0, int& i1) {
+  const int n_items = a.T * AT_NCH;
   i0 = static_cast<int>(static_cast<long long>(blockIdx.x) * n_items / gridDim.x);
   i1 = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * n_items / gridDim.x);
 }
 
-// Lane 0: x of scores item `item` into slot `slot` (mbarrier 2 + slot).
-__device__ __forceinline__ void scores_issue_x(const RouterFusedArgs& a, int item, int slot,
-                                               uint8_t* sm, uint64_t* mb) {
-  const int slot_bytes = (a.D / 64) * SC_TOK * 128;
+// Steps of an item holding at least one valid token (0: the chunk is padding).
+__device__ __forceinline__ int attend_steps(const RouterFusedArgs& a, int item) {
+  const int tile = item / AT_NCH, chunk = item % AT_NCH;
+  int n = RF_TOK;
+  if (a.valid_len) {
+    n = a.valid_len[tile];
+    n = n < 1 ? 1 : (n > RF_TOK ? RF_TOK : n);
+  }
+  return max(0, min(AT_CHUNK / SC_TOK, (n - chunk * AT_CHUNK + SC_TOK - 1) / SC_TOK));
+}
+
+// Cursor over this CTA's (item, step) sequence, past items without steps.
+struct StepCursor {
+  int item, st, end;
+  __device__ void settle(const RouterFusedArgs& a) {
+    while (item < end && st >= attend_steps(a, item)) {
+      ++item;
+      st = 0;
+    }
+  }
+  __device__ bool valid() const { return item < end; }
+  __device__ void next(const RouterFusedArgs& a) {
+    ++st;
+    settle(a);
+  }
+};
+
+__device__ __forceinline__ StepCursor attend_first(const RouterFusedArgs& a) {
+  StepCursor c;
+  attend_range(a, c.item, c.end);
+  c.st = 0;
+  c.settle(a);
+  return c;
+}
+
+// Lane 0: x of the cursor's step into slot `slot` (mbarrier 2 + slot).
+__device__ __forceinline__ void attend_issue_x(const RouterFusedArgs& a, const StepCursor& c,
+                                               int slot, uint8_t* sm, uint64_t* mb) {
+  const int slot_bytes = a.D * 64;
   mbar_arrive_expect_tx(&mb[2 + slot], slot_bytes);
-  const int tile = item / (RF_TOK / SC_TOK), tb = item % (RF_TOK / SC_TOK);
-  tma_load_3d(scores_x_slot(sm, a.D, slot), &a.xmap3, &mb[2 + slot], 0,
-              tile * RF_TOK + tb * SC_TOK, 0);
+  const int tile = c.item / AT_NCH, chunk = c.item % AT_NCH;
+  tma_load_3d(sm + AT_SLOT0 + slot * slot_bytes, &a.xmap3, &mb[2 + slot], 0,
+              tile * RF_TOK + chunk * AT_CHUNK + c.st * SC_TOK, 0);
 }
 
-// Before the grid barrier: this CTA's first two x items. Returns the slots
-// now in flight (bit s = slot s).
-__device__ __forceinline__ int scores_prefetch_x(const RouterFusedArgs& a, uint8_t* sm,
+// Before the grid barrier: this CTA's first two steps. Returns the slots now
+// in flight (bit s = slot s).
+__device__ __forceinline__ int attend_prefetch_x(const RouterFusedArgs& a, uint8_t* sm,
                                                  uint64_t* mb) {
-  int i0, i1;
-  scores_range(a, i0, i1);
-  const int n = min(2, i1 - i0);
   __syncthreads();
-  if (threadIdx.x == 0)
-    for (int k = 0; k < n; ++k) scores_issue_x(a, i0 + k, k, sm, mb);
-  return (1 << n) - 1;
+  StepCursor c = attend_first(a);
+  int pending = 0;
+  for (int s = 0; s < 2 && c.valid(); ++s, c.next(a)) {
+    if (threadIdx.x == 0) attend_issue_x(a, c, s, sm, mb);
+    pending |= 1 << s;
+  }
+  return pending;
 }
 
-__device__ bool scores_phase(const RouterFusedArgs& a, bool shared_query, uint8_t* sm,
-                             uint64_t* mb, uint32_t* ph, int& x_pending) {
-  const int D = a.D;
+// KS = D / 128 (the phase is instantiated per width; see attend_phase).
+template <int KS>
+__device__ __noinline__ bool attend_phase_ks(const RouterFusedArgs& a, bool shared_q, uint8_t* sm,
+                                uint64_t* mb, uint32_t* ph, int& x_pending, float* s_m,
+                                float* s_l, float* s_scale) {
+  constexpr int D = 128 * KS, NT = 2 * KS;
+  constexpr int slot_bytes = D * 64;
+  constexpr int CHUNK_BYTES = SC_TOK * 128;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chunk_bytes = SC_TOK * 128;  // one 64-column chunk of 32 rows
-  const int slot_bytes = (D / 64) * chunk_bytes;
-  int i0, i1;
-  scores_range(a, i0, i1);
-  const uint8_t* su = sm;
-  const int mt = warp & 1, nt = warp >> 1;
   const int g = lane >> 2, t2 = (lane & 3) * 2;
-  const int ra = mt * 16 + (lane & 15), rb = nt * 8 + (lane & 7);
-  int staged_u = -1;
-  for (int item = i0, k = 0; item < i1; ++item, ++k) {
-    const int slot = k & 1;
-    const int tile = item / (RF_TOK / SC_TOK), tb = item % (RF_TOK / SC_TOK);
-    const int tu = shared_query ? 0 : tile;
-    if (tu != staged_u) {
-      __syncthreads();  // every warp is done with the previous U2
-      if (threadIdx.x == 0) {
-        fence_proxy_async_global();  // U2 was written by the fold phase
-        mbar_arrive_expect_tx(&mb[1], slot_bytes);
-        tma_load_4d(sm, &a.u2map, &mb[1], 0, 0, 0, tu);
-      }
-      if (!mbar_wait(&mb[1], ph[1])) return false;
-      ph[1] ^= 1;
-      staged_u = tu;
-    }
-    if (!mbar_wait(&mb[2 + slot], ph[2 + slot])) return false;
-    ph[2 + slot] ^= 1;
-    x_pending &= ~(1 << slot);
-    const uint8_t* sx = scores_x_slot(sm, D, slot);
-    // two independent accumulator chains (even / odd k-steps) for ILP
-    float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc_b[4] = {0.f, 0.f, 0.f, 0.f};
-    auto step = [&](int ks, float (&d)[4]) {
-      const int c = ks >> 2;
-      const int ja = ((ks & 3) << 1) + (lane >> 4);
-      const int jb = ((ks & 3) << 1) + ((lane >> 3) & 1);
-      uint32_t af[4], bfr[2];
-      ldsm_x4(af, sx + c * chunk_bytes + ra * 128 + ((ja ^ (ra & 7)) << 4));
-      ldsm_x2(bfr, su + c * chunk_bytes + rb * 128 + ((jb ^ (rb & 7)) << 4));
-      mma_bf16_16816(d, af, bfr);
-    };
-#pragma unroll 2
-    for (int ks = 0; ks < D / 16; ks += 2) {  // D / 16 is even
-      step(ks, acc);
-      step(ks + 1, acc_b);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[i] += acc_b[i];
-    float* st = a.S + static_cast<size_t>(tile) * 32 * RF_TOK + tb * SC_TOK + mt * 16;
-    const int j = nt * 8 + t2;
-    st[static_cast<size_t>(j) * RF_TOK + g] = acc[0];
-    st[static_cast<size_t>(j + 1) * RF_TOK + g] = acc[1];
-    st[static_cast<size_t>(j) * RF_TOK + g + 8] = acc[2];
-    st[static_cast<size_t>(j + 1) * RF_TOK + g + 8] = acc[3];
-    if (item + 2 < i1) {
-      __syncthreads();  // every warp is done with this slot
-      if (threadIdx.x == 0) scores_issue_x(a, item + 2, slot, sm, mb);
-      x_pending |= 1 << slot;
-    }
-  }
-  return true;
-}
-
-// ------------------------------------------------------------------ softmax phase
-// Items (tile, head): p = softmax over the valid tokens of hi + lo + c, written
-// as a bf16 hi/lo pair into rows h and 16 + h of P2[tile] (zero rows for heads
-// that do not exist).
-__device__ void softmax_phase(const RouterFusedArgs& a, bool shared_cb, float* sf) {
-  __shared__ float s_red[RF_WARPS];
-  __shared__ float s_val;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  {  // the weighted sums of the next phase accumulate into a zeroed z
-    const size_t nz = static_cast<size_t>(a.T) * 16 * a.D / 4;
-    float4* z4 = reinterpret_cast<float4*>(a.z);
-    for (size_t i = static_cast<size_t>(blockIdx.x) * RF_THREADS + threadIdx.x; i < nz;
-         i += static_cast<size_t>(gridDim.x) * RF_THREADS)
-      z4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  const int n_items = a.T * 16;
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-    const int tile = item / 16, h = item % 16;
-    bf16* prow = a.P2 + (static_cast<long long>(tile) * 32 + h) * RF_TOK;
-    bf16* lrow = prow + 16 * RF_TOK;
-    if (h >= a.heads) {
-      for (int t = threadIdx.x; t < RF_TOK; t += RF_THREADS)
-        prow[t] = lrow[t] = __float2bfloat16_rn(0.f);
-      continue;
-    }
+  float* red = reinterpret_cast<float*>(sm);
+  bf16* sp = reinterpret_cast<bf16*>(sm + AT_RED_BYTES);  // [hi, lo][16][AT_P_PITCH]
+  const int sh = threadIdx.x >> 4, stl = threadIdx.x & 15;  // softmax: head, token pair
+  int i0, i1;
+  attend_range(a, i0, i1);
+  // the issue cursor runs two steps ahead of the consumed ones
+  StepCursor ic = attend_first(a);
+  for (int s = 0; s < 2 && ic.valid(); ++s) ic.next(a);
+  int k = 0;  // steps consumed: slot k & 1
+  for (int item = i0; item < i1; ++item) {
+    const int tile = item / AT_NCH, chunk = item % AT_NCH;
+    const size_t row0 = static_cast<size_t>(item) * 16;
     int n = RF_TOK;
     if (a.valid_len) {
       n = a.valid_len[tile];
       if (n < 1 || n > RF_TOK) {
-        if (threadIdx.x == 0 && h == 0) atomicOr(a.status, DEV_BAD_VALID_LEN);
+        if (threadIdx.x == 0 && chunk == 0) atomicOr(a.status, DEV_BAD_VALID_LEN);
         n = n < 1 ? 1 : RF_TOK;
       }
     }
-    const float c = a.cb[(shared_cb ? 0 : tile) * 16 + h];
-    const float* shi = a.S + (static_cast<long long>(tile) * 32 + h) * RF_TOK;
-    const float* slo = shi + 16 * RF_TOK;
-    float v[RF_TOK / RF_THREADS];
-    float mx = -INFINITY;
-#pragma unroll
-    for (int u = 0; u < RF_TOK / RF_THREADS; ++u) {
-      const int t = threadIdx.x + u * RF_THREADS;
-      v[u] = shi[t] + slo[t] + c;
-      if (t < n) mx = fmaxf(mx, v[u]);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    __syncthreads();
-    if (lane == 0) s_red[warp] = mx;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float m = s_red[0];
-      for (int i = 1; i < RF_WARPS; ++i) m = fmaxf(m, s_red[i]);
-      s_val = m;
-    }
-    __syncthreads();
-    mx = s_val;
-    float sum = 0.f;
-#pragma unroll
-    for (int u = 0; u < RF_TOK / RF_THREADS; ++u) {
-      const int t = threadIdx.x + u * RF_THREADS;
-      v[u] = t < n ? expf(v[u] - mx) : 0.f;
-      sum += v[u];
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    __syncthreads();
-    if (lane == 0) s_red[warp] = sum;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float t = 0.f;
-      for (int i = 0; i < RF_WARPS; ++i) t += s_red[i];
-      s_val = 1.0f / t;
-    }
-    __syncthreads();
-    const float inv = s_val;
-#pragma unroll
-    for (int u = 0; u < RF_TOK / RF_THREADS; ++u) {
-      const int t = threadIdx.x + u * RF_THREADS;
-      const float p = v[u] * inv;
-      const bf16 hi = __float2bfloat16_rn(p);
-      prow[t] = hi;
-      lrow[t] = __float2bfloat16_rn(p - __bfloat162float(hi));
-    }
-  }
-  (void)sf;
-}
-
-// ------------------------------------------------------------------ wsum phase
-// Items (tile, token half, 64-channel block), a contiguous range per CTA in
-// that order so that consecutive items share the half-tile's P2 rows:
-// z[tile][h][c] += sum_{t in half} (P_hi + P_lo)[h][t] x[tile][t][c]. The
-// half-tile's 512 x 64 feature block comes in 2 TMA boxes of 256 tokens x
-// 128 bytes, double-buffered on mbarriers 2 and 3 (the first two items
-// requested before the grid barrier); P2[tile][.][half] (32 x 512) in one
-// TMA request on mbarrier 1. Both are 128-byte swizzled (the 16-byte piece j
-// of row r at j ^ (r & 7)). Warp w computes channels 8w..8w+7 (one n8 tile)
-// for both m16 tiles (hi rows, lo rows). z was zeroed in the softmax phase;
-// each element receives exactly two additions (one per half), so the
-// result does not depend on their order.
-// Shared memory: P2 [8 chunks][32][128 B] | x slot 0 | x slot 1 (64 KB each).
-constexpr int WS_P_BYTES = (WS_HALF / 64) * 32 * 128;
-constexpr int WS_X_BYTES = WS_HALF * 128;
-
-__device__ __forceinline__ void red_add_f32x2(float* p, float a, float b) {
-  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(a), "f"(b) : "memory");
-}
-
-__device__ __forceinline__ void wsum_range(const RouterFusedArgs& a, int& i0, int& i1) {
-  const int n_items = a.T * 2 * (a.D / 64);
-  i0 = static_cast<int>(static_cast<long long>(blockIdx.x) * n_items / gridDim.x);
-  i1 = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * n_items / gridDim.x);
-}
-
-__device__ __forceinline__ void wsum_issue_x(const RouterFusedArgs& a, int item, int slot,
-                                             uint8_t* sm, uint64_t* mb) {
-  const int cblocks = a.D / 64;
-  const int th = item / cblocks, cbk = item % cblocks;
-  uint8_t* dst = sm + WS_P_BYTES + slot * WS_X_BYTES;
-  mbar_arrive_expect_tx(&mb[2 + slot], WS_X_BYTES);
-  for (int bx = 0; bx < WS_HALF / WS_BOX; ++bx)
-    tma_load_2d(dst + bx * WS_BOX * 128, &a.xmap, &mb[2 + slot], cbk * 64,
-                (th >> 1) * RF_TOK + (th & 1) * WS_HALF + bx * WS_BOX);
-}
-
-__device__ __forceinline__ int wsum_prefetch_x(const RouterFusedArgs& a, uint8_t* sm,
-                                               uint64_t* mb) {
-  int i0, i1;
-  wsum_range(a, i0, i1);
-  const int n = min(2, i1 - i0);
-  __syncthreads();
-  if (threadIdx.x == 0)
-    for (int k = 0; k < n; ++k) wsum_issue_x(a, i0 + k, k, sm, mb);
-  return (1 << n) - 1;
-}
-
-__device__ bool wsum_phase(const RouterFusedArgs& a, uint8_t* sm, uint64_t* mb, uint32_t* ph,
-                           int& x_pending) {
-  const int D = a.D;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cblocks = D / 64;
-  int i0, i1;
-  wsum_range(a, i0, i1);
-  const uint8_t* sp = sm;
-  const int g = lane >> 2, t2 = (lane & 3) * 2;
-  int staged = -1;
-  for (int item = i0, k = 0; item < i1; ++item, ++k) {
-    const int slot = k & 1;
-    const int th = item / cblocks, cbk = item % cblocks;  // th = 2 tile + half
-    const int tile = th >> 1;
-    if (th != staged) {
-      __syncthreads();  // every warp is done with the previous P2
-      if (threadIdx.x == 0) {
-        fence_proxy_async_global();  // P2 was written by the softmax phase
-        mbar_arrive_expect_tx(&mb[1], WS_P_BYTES);
-        tma_load_4d(sm, &a.p2map, &mb[1], 0, 0, (th & 1) * (WS_HALF / 64), tile);
+    const int ns = attend_steps(a, item);
+    if (ns == 0) {  // every token of the chunk is padding
+      if (threadIdx.x < 16) {
+        a.stats[row0 + threadIdx.x] = -INFINITY;
+        a.stats[static_cast<size_t>(a.T) * AT_NCH * 16 + row0 + threadIdx.x] = 0.f;
       }
-      if (!mbar_wait(&mb[1], ph[1])) return false;
-      ph[1] ^= 1;
-      staged = th;
+      continue;
     }
-    if (!mbar_wait(&mb[2 + slot], ph[2 + slot])) return false;
-    ph[2 + slot] ^= 1;
-    x_pending &= ~(1 << slot);
-    const uint8_t* sxb = sm + WS_P_BYTES + slot * WS_X_BYTES;
-    float acc[2][4] = {}, acc_b[2][4] = {};  // odd k-steps: a second chain for ILP
-    auto step = [&](int ks, float (&d)[2][4]) {
-      // B[k = token][n = channel] stored n-contiguous: transposed 8x8 loads
-      const int r = ks * 16 + (lane & 15);
-      const int rr = r & (WS_BOX - 1);
-      uint32_t bfr[2];
-      ldsm_x2_trans(bfr, sxb + (r / WS_BOX) * WS_BOX * 128 + rr * 128 + ((warp ^ (rr & 7)) << 4));
-      const int c = ks >> 2;
-      const int ja = ((ks & 3) << 1) + (lane >> 4);
+    // B fragments of the scores (B[k = channel][n = split row] = U2[n][k])
+    const bf16* u = a.U2 + (shared_q ? 0 : static_cast<size_t>(tile) * 32 * D);
+    uint32_t ub[KS][4][2];
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        const int ra = mt * 16 + (lane & 15);
-        uint32_t af[4];
-        ldsm_x4(af, sp + c * (32 * 128) + ra * 128 + ((ja ^ (ra & 7)) << 4));
-        mma_bf16_16816(d[mt], af, bfr);
+    for (int ks = 0; ks < KS; ++ks) {
+      const int kk = (warp * KS + ks) * 16 + t2;
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        const int r = nt * 8 + g;
+        const bool live = (r & 15) < a.heads;
+        const bf16* ur = u + static_cast<size_t>(r) * D + kk;
+        ub[ks][nt][0] = live ? *reinterpret_cast<const unsigned*>(ur) : 0u;
+        ub[ks][nt][1] = live ? *reinterpret_cast<const unsigned*>(ur + 8) : 0u;
       }
-    };
-#pragma unroll 2
-    for (int ks = 0; ks < WS_HALF / 16; ks += 2) {
-      step(ks, acc);
-      step(ks + 1, acc_b);
     }
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[mt][i] += acc_b[mt][i];
-    // row g of m-tile 0 is the hi part of head g, row g of m-tile 1 its lo part
-    float* zt = a.z + static_cast<size_t>(tile) * 16 * D + cbk * 64 + warp * 8 + t2;
-    red_add_f32x2(zt + static_cast<size_t>(g) * D, acc[0][0] + acc[1][0], acc[0][1] + acc[1][1]);
-    red_add_f32x2(zt + static_cast<size_t>(g + 8) * D, acc[0][2] + acc[1][2],
-                  acc[0][3] + acc[1][3]);
-    if (item + 2 < i1) {
-      __syncthreads();  // every warp is done with this slot
-      if (threadIdx.x == 0) wsum_issue_x(a, item + 2, slot, sm, mb);
-      x_pending |= 1 << slot;
+    const float c_h = sh < a.heads ? a.cb[(shared_q ? 0 : tile) * 16 + sh] : 0.f;
+    if (threadIdx.x < 16) {
+      s_m[threadIdx.x] = -INFINITY;
+      s_l[threadIdx.x] = 0.f;
     }
+    float accz[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) accz[nt][i] = 0.f;
+    for (int st = 0; st < ns; ++st, ++k) {
+      const int slot = k & 1;
+      const uint8_t* sx = sm + AT_SLOT0 + slot * slot_bytes;
+      if (!mbar_wait(&mb[2 + slot], ph[2 + slot])) return false;
+      ph[2 + slot] ^= 1;
+      x_pending &= ~(1 << slot);
+      // 1. partial scores of this warp's channels
+      float accs[2][4][4];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) accs[mt][nt][i] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const int kg = warp * KS + ks;
+        const int c = kg >> 2, ja = ((kg & 3) << 1) + (lane >> 4);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          const int ra = mt * 16 + (lane & 15);
+          uint32_t af[4];
+          ldsm_x4(af, sx + c * CHUNK_BYTES + ra * 128 + ((ja ^ (ra & 7)) << 4));
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt) {
+            const uint32_t bfr[2] = {ub[ks][nt][0], ub[ks][nt][1]};
+            mma_bf16_16816(accs[mt][nt], af, bfr);
+          }
+        }
+      }
+      float* rw = red + warp * 32 * AT_RED_PITCH;
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+          const int r = mt * 16 + g, j = nt * 8 + t2;
+          rw[r * AT_RED_PITCH + j] = accs[mt][nt][0];
+          rw[r * AT_RED_PITCH + j + 1] = accs[mt][nt][1];
+          rw[(r + 8) * AT_RED_PITCH + j] = accs[mt][nt][2];
+          rw[(r + 8) * AT_RED_PITCH + j + 1] = accs[mt][nt][3];
+        }
+      __syncthreads();
+      // 2. running softmax of head sh over tokens stl and stl + 16
+      {
+        const int tb = chunk * AT_CHUNK + st * SC_TOK;
+        float sv[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int t = stl + 16 * i;
+          float v = c_h;
+#pragma unroll
+          for (int w = 0; w < RF_WARPS; ++w) {
+            const float* rr = red + (w * 32 + t) * AT_RED_PITCH;
+            v += rr[sh] + rr[16 + sh];
+          }
+          sv[i] = (sh < a.heads && tb + t < n) ? v : -INFINITY;
+        }
+        float mx = fmaxf(sv[0], sv[1]);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float m_old = s_m[sh];
+        const float m_new = fmaxf(m_old, mx);
+        float e[2] = {0.f, 0.f}, scale = 1.f;
+        if (m_new != -INFINITY) {
+          scale = expf(m_old - m_new);
+          e[0] = expf(sv[0] - m_new);
+          e[1] = expf(sv[1] - m_new);
+        }
+        float sum = e[0] + e[1];
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const bf16 hi = __float2bfloat16_rn(e[i]);
+          sp[sh * AT_P_PITCH + stl + 16 * i] = hi;
+          sp[(16 + sh) * AT_P_PITCH + stl + 16 * i] =
+              __float2bfloat16_rn(e[i] - __bfloat162float(hi));
+        }
+        __syncwarp();  // every lane has read s_m[sh]
+        if (stl == 0) {
+          s_l[sh] = s_l[sh] * scale + sum;
+          s_m[sh] = m_new;
+          s_scale[sh] = scale;
+        }
+      }
+      __syncthreads();
+      // 3. rescale and accumulate this warp's channels of Zc
+      {
+        const float sc0 = s_scale[g], sc1 = s_scale[g + 8];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          accz[nt][0] *= sc0;
+          accz[nt][1] *= sc0;
+          accz[nt][2] *= sc1;
+          accz[nt][3] *= sc1;
+        }
+#pragma unroll
+        for (int kk = 0; kk < SC_TOK / 16; ++kk) {
+          uint32_t ah[4], al[4];
+          const int pr = lane & 15, pk = kk * 16 + 8 * (lane >> 4);
+          ldsm_x4(ah, sp + pr * AT_P_PITCH + pk);
+          ldsm_x4(al, sp + (16 + pr) * AT_P_PITCH + pk);
+          const int r = kk * 16 + (lane & 15);
+#pragma unroll
+          for (int nt = 0; nt < NT; nt += 2) {
+            const int cw = warp * (D / 8) + 8 * (nt + (lane >> 4));
+            const int c = cw >> 6, j = (cw & 63) >> 3;
+            uint32_t bf[4];
+            ldsm_x4_trans(bf, sx + c * CHUNK_BYTES + r * 128 + ((j ^ (r & 7)) << 4));
+            const uint32_t b0[2] = {bf[0], bf[1]}, b1[2] = {bf[2], bf[3]};
+            mma_bf16_16816(accz[nt], ah, b0);
+            mma_bf16_16816(accz[nt], al, b0);
+            mma_bf16_16816(accz[nt + 1], ah, b1);
+            mma_bf16_16816(accz[nt + 1], al, b1);
+          }
+        }
+      }
+      __syncthreads();  // every warp is done with this slot and with the weights
+      if (ic.valid()) {
+        if (threadIdx.x == 0) attend_issue_x(a, ic, slot, sm, mb);
+        x_pending |= 1 << slot;
+        ic.next(a);
+      }
+    }
+    float* zp = a.Zp + row0 * D;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int c = warp * (D / 8) + nt * 8 + t2;
+      *reinterpret_cast<float2*>(zp + static_cast<size_t>(g) * D + c) =
+          make_float2(accz[nt][0], accz[nt][1]);
+      *reinterpret_cast<float2*>(zp + static_cast<size_t>(g + 8) * D + c) =
+          make_float2(accz[nt][2], accz[nt][3]);
+    }
+    if (threadIdx.x < 16) {  // s_m / s_l were last written before the final barrier
+      a.stats[row0 + threadIdx.x] = s_m[threadIdx.x];
+      a.stats[static_cast<size_t>(a.T) * AT_NCH * 16 + row0 + threadIdx.x] = s_l[threadIdx.x];
+    }
+    __syncthreads();  // stats read before the next item resets them
   }
   return true;
+}
+
+__device__ bool attend_phase(const RouterFusedArgs& a, bool shared_q, uint8_t* sm, uint64_t* mb,
+                             uint32_t* ph, int& x_pending) {
+  __shared__ float s_m[16], s_l[16], s_scale[16];
+  switch (a.D / 128) {
+    case 1: return attend_phase_ks<1>(a, shared_q, sm, mb, ph, x_pending, s_m, s_l, s_scale);
+    case 2: return attend_phase_ks<2>(a, shared_q, sm, mb, ph, x_pending, s_m, s_l, s_scale);
+    case 3: return attend_phase_ks<3>(a, shared_q, sm, mb, ph, x_pending, s_m, s_l, s_scale);
+    case 4: return attend_phase_ks<4>(a, shared_q, sm, mb, ph, x_pending, s_m, s_l, s_scale);
+    case 5: return attend_phase_ks<5>(a, shared_q, sm, mb, ph, x_pending, s_m, s_l, s_scale);
+    case 6: return attend_phase_ks<6>(a, shared_q, sm, mb, ph, x_pending, s_m, s_l, s_scale);
+    case 7: return attend_phase_ks<7>(a, shared_q, sm, mb, ph, x_pending, s_m, s_l, s_scale);
+    default: return attend_phase_ks<8>(a, shared_q, sm, mb, ph, x_pending, s_m, s_l, s_scale);
+  }
+}
+
+// ------------------------------------------------------------------ combine phase
+// Items (tile, head): z[tile][h] = sum_c exp(m_c - M) Zc / sum_c exp(m_c - M) l_c
+// over the tile's AT_NCH chunks (chunks without a valid token, l = 0, skipped).
+__device__ void combine_phase(const RouterFusedArgs& a) {
+  const int D = a.D;
+  const size_t lofs = static_cast<size_t>(a.T) * AT_NCH * 16;
+  const int n_items = a.T * a.heads;
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const int tile = item / a.heads, h = item % a.heads;
+    const size_t r0 = static_cast<size_t>(tile) * AT_NCH * 16 + h;
+    float w[AT_NCH];
+    float M = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < AT_NCH; ++c) {
+      w[c] = a.stats[lofs + r0 + 16 * c] > 0.f ? a.stats[r0 + 16 * c] : -INFINITY;
+      M = fmaxf(M, w[c]);
+    }
+    float L = 0.f;
+#pragma unroll
+    for (int c = 0; c < AT_NCH; ++c) {
+      w[c] = w[c] == -INFINITY ? 0.f : expf(w[c] - M);
+      L += w[c] * a.stats[lofs + r0 + 16 * c];
+    }
+    const float inv = 1.0f / L;
+    for (int c4 = threadIdx.x * 4; c4 < D; c4 += RF_THREADS * 4) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < AT_NCH; ++c) {
+        if (w[c] == 0.f) continue;
+        const float4 v = *reinterpret_cast<const float4*>(a.Zp + (r0 + 16 * c) * D + c4);
+        acc.x = fmaf(w[c], v.x, acc.x);
+        acc.y = fmaf(w[c], v.y, acc.y);
+        acc.z = fmaf(w[c], v.z, acc.z);
+        acc.w = fmaf(w[c], v.w, acc.w);
+      }
+      *reinterpret_cast<float4*>(a.z + (static_cast<size_t>(tile) * 16 + h) * D + c4) =
+          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    }
+  }
 }
 
 // ------------------------------------------------------------------ routing
@@ -804,17 +835,14 @@ __global__ void __launch_bounds__(RF_THREADS, 1)
   // 1024-byte alignment for the swizzled TMA boxes (the launch adds the slack)
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   float* sf = reinterpret_cast<float*>(sm);
-  // mbarriers: 0 weights (projections, fold), 1 other staged operands,
-  // 2 and 3 the two x slots of the scores and weighted-sum phases
+  // mbarriers: 0 weights (projections, fold), 1 the projections' input rows,
+  // 2 and 3 the two x slots of the attention phase
   __shared__ __align__(8) uint64_t s_mb[4];
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int i = 0; i < 4; ++i) mbar_init(&s_mb[i], 1);
     fence_mbar_init();
-    tma_prefetch_desc(&a.xmap);
     tma_prefetch_desc(&a.xmap3);
-    tma_prefetch_desc(&a.u2map);
-    tma_prefetch_desc(&a.p2map);
   }
   __syncthreads();
   uint32_t ph[4] = {0u, 0u, 0u, 0u};
@@ -862,15 +890,12 @@ __global__ void __launch_bounds__(RF_THREADS, 1)
       w_pending = false;
       if (!fold_phase(a, l, shared_q ? 1 : T, a.Q, shared_q ? 0 : D, sm, s_mb, ph, pre)) ok = false;
     }
-    // the scores phase's first x items (x is an input) before the barrier
-    x_pending = scores_prefetch_x(a, sm, s_mb);
+    // the attention phase's first x steps (x is an input) before the barrier
+    x_pending = attend_prefetch_x(a, sm, s_mb);
     if (!sync()) break;
-    if (!scores_phase(a, shared_q, sm, s_mb, ph, x_pending)) ok = false;
-    x_pending = wsum_prefetch_x(a, sm, s_mb);  // the softmax phase uses no shared memory
+    if (!attend_phase(a, shared_q, sm, s_mb, ph, x_pending)) ok = false;
     if (!sync()) break;
-    softmax_phase(a, shared_q, sf);
-    if (!sync()) break;
-    if (!wsum_phase(a, sm, s_mb, ph, x_pending)) ok = false;
+    combine_phase(a);
     // o = Wv_h z_h + bv: the input row of output row m for columns of head h is z[m][h]
     prefetch_w(a.Wv[l], D, D);
     if (!sync()) break;
@@ -952,12 +977,10 @@ size_t router_fused_smem(int D, int G) {
   const size_t gemv = GV_ROWS * (K + 8) * 4 + GV_COLS * (K + 8) * 2 +
                       static_cast<size_t>(RF_WARPS) * GV_ROWS * GV_COLS * 4;
   const size_t route = 2 * static_cast<size_t>(IVC_MAX_QUANTILE_GROUP) * sizeof(double);
-  const size_t sc_slot = static_cast<size_t>(D / 64) * SC_TOK * 128;
-  const size_t scores = (sc_slot > FOLD_SMEM ? sc_slot : FOLD_SMEM) + 2 * sc_slot;  // U2, 2 x slots
-  const size_t wsum = static_cast<size_t>(WS_P_BYTES) + 2 * static_cast<size_t>(WS_X_BYTES);
+  const size_t attend = AT_SLOT0 + 2 * static_cast<size_t>(D) * 64;  // partials, weights, 2 x slots
   const size_t fold = FOLD_SMEM;
   size_t m = gemv;
-  for (size_t v : {route, scores, wsum, fold, static_cast<size_t>(D) * sizeof(float)})
+  for (size_t v : {route, attend, fold, static_cast<size_t>(D) * sizeof(float)})
     if (v > m) m = v;
   return m + 1024;  // alignment slack
 }
@@ -986,8 +1009,6 @@ int launch_router_fused(const ivc_router* r, const void* x, const int32_t* valid
   if (T == 0) return IVC_OK;
   if (!router_fused_supported(r)) return IVC_EUNSUPPORTED;
   RouterFusedArgs a{};
-  if (map_rows_2d(&a.xmap, x, static_cast<long long>(T) * RF_TOK, r->D, WS_BOX) != IVC_OK)
-    return IVC_ECUDA;
   {
     const unsigned long long D2 = static_cast<unsigned long long>(r->D) * 2;  // row bytes
     const unsigned long long chunks = static_cast<unsigned long long>(r->D) / 64;
@@ -995,18 +1016,7 @@ int launch_router_fused(const ivc_router* r, const void* x, const int32_t* valid
     const unsigned long long xd[3] = {64, static_cast<unsigned long long>(T) * RF_TOK, chunks};
     const unsigned long long xs[2] = {D2, 128};
     const unsigned xb[3] = {64, SC_TOK, static_cast<unsigned>(chunks)};
-    // U2: {64, 32 rows, chunks, T}
-    const unsigned long long ud[4] = {64, 32, chunks, static_cast<unsigned long long>(T)};
-    const unsigned long long us[3] = {D2, 128, 32 * D2};
-    const unsigned ub[4] = {64, 32, static_cast<unsigned>(chunks), 1};
-    // P2: {64 tokens, 32 rows, 16 chunks, T}, rows of 1024 tokens
-    const unsigned long long pd[4] = {64, 32, RF_TOK / 64, static_cast<unsigned long long>(T)};
-    const unsigned long long ps[3] = {RF_TOK * 2, 128, 32ull * RF_TOK * 2};
-    const unsigned pb[4] = {64, 32, WS_HALF / 64, 1};
-    if (map_bf16(&a.xmap3, 3, x, xd, xs, xb) != IVC_OK ||
-        map_bf16(&a.u2map, 4, b.U2, ud, us, ub) != IVC_OK ||
-        map_bf16(&a.p2map, 4, b.P2, pd, ps, pb) != IVC_OK)
-      return IVC_ECUDA;
+    if (map_bf16(&a.xmap3, 3, x, xd, xs, xb) != IVC_OK) return IVC_ECUDA;
   }
   a.x = static_cast<const bf16*>(x);
   a.valid_len = valid_len;
@@ -1042,8 +1052,8 @@ int launch_router_fused(const ivc_router* r, const void* x, const int32_t* valid
   a.Q = b.Q;
   a.U2 = b.U2;
   a.cb = b.cb;
-  a.S = b.S;
-  a.P2 = b.P2;
+  a.Zp = b.Zp;
+  a.stats = b.stats;
   a.z = b.z;
   a.O = b.O;
   a.q = b.q;
