@@ -25,6 +25,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdlib>
+#include <type_traits>
 
 #include "ivc_internal.h"
 #include "ivc_ptx.cuh"
@@ -41,10 +42,11 @@ __device__ __forceinline__ float gelu_f(float y) {
 // (two n8 tiles, so that each staged input row serves 16 columns). One thread
 // brings their 16 weight rows (contiguous in W) into shared memory with one
 // bulk copy issued before waiting for the previous kernel, and up to 16 input
-// rows per round (one bulk copy per row) on the same mbarrier. Warp w multiplies the k-range [w K/8, (w+1) K/8): fp32 inputs are
-// split into a bf16 pair hi + lo (two MMAs per k-step, fp32 accumulate, about
-// 16 significant bits of the input kept), bf16 inputs enter as they are. The
-// 8 partial m16n8 tiles are summed through shared memory.
+// rows per round (one bulk copy per row) on the same mbarrier. Warp w
+// multiplies the k-range [w K/8, (w+1) K/8): fp32 inputs are split into a bf16
+// pair hi + lo (two MMAs per k-step, fp32 accumulate, about 16 significant
+// bits of the input kept), bf16 inputs enter as they are. The 8 warps' partial
+// tiles are summed through shared memory.
 constexpr int GEMV_THREADS = 256;
 constexpr int GEMV_WARPS = GEMV_THREADS / 32;
 constexpr int GEMV_COLS = 16;  // output columns per CTA (two n8 tiles)
@@ -501,8 +503,9 @@ int launch_pool_softmax(const float* S, const float* cb, int cb_stride, const in
 // chunks}, 128-byte swizzle, double-buffered) and per step
 //   1. s[t][j] = x_t . U2[j] for the 32 split rows j (warp w multiplies its
 //      D/8 channels with m16n8k16 MMAs, the U2 fragments held in registers
-//      for the whole CTA; the 8 partial 32x32 tiles are summed in shared
-//      memory), s_h = s[t][h] + s[t][16 + h] + c_h, invalid tokens -inf;
+//      for the whole CTA; the 8 partial 32x32 tiles, stored column by
+//      column, are summed in shared memory), s_h = s[t][h] + s[t][16 + h] +
+//      c_h, invalid tokens -inf;
 //   2. running max m_h and sum l_h (rescaled by exp(m_old - m_new)), the
 //      weights e = exp(s - m_h) split into a bf16 hi/lo pair;
 //   3. Zc[h][c] = Zc[h][c] * exp(m_old - m_new) + sum_t e_t x_t[c] with the
@@ -514,7 +517,7 @@ int launch_pool_softmax(const float* S, const float* cb, int cb_stride, const in
 constexpr int ATTN_STEP = 32;                        // tokens per staged box
 constexpr int ATTN_CHUNK = 128;                      // tokens per CTA
 constexpr int ATTN_NCH = TILE_TOKENS / ATTN_CHUNK;   // chunks (partials) per tile
-constexpr int ATTN_RED_PITCH = 33;                   // floats per row of a partial score tile
+constexpr int ATTN_RED_PITCH = 36;                   // floats per column of a partial score tile
 constexpr int ATTN_P_PITCH = 40;                     // bf16 per row of the weight tile (80 B)
 
 __device__ __forceinline__ void ldsm4(uint32_t (&r)[4], const void* p) {
@@ -648,28 +651,30 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt) {
         const int r = mt * 16 + g, j = nt * 8 + t2;
-        rw[r * ATTN_RED_PITCH + j] = accs[mt][nt][0];
-        rw[r * ATTN_RED_PITCH + j + 1] = accs[mt][nt][1];
-        rw[(r + 8) * ATTN_RED_PITCH + j] = accs[mt][nt][2];
-        rw[(r + 8) * ATTN_RED_PITCH + j + 1] = accs[mt][nt][3];
+        rw[j * ATTN_RED_PITCH + r] = accs[mt][nt][0];
+        rw[(j + 1) * ATTN_RED_PITCH + r] = accs[mt][nt][1];
+        rw[j * ATTN_RED_PITCH + r + 8] = accs[mt][nt][2];
+        rw[(j + 1) * ATTN_RED_PITCH + r + 8] = accs[mt][nt][3];
       }
     ok = __syncthreads_and(ok) != 0;
     if (!ok) break;
-    // 2. running softmax of head sh over tokens stl and stl + 16
+    // 2. running softmax of head sh over tokens 2 stl and 2 stl + 1
     {
       const int tb = tok0 + st * ATTN_STEP;
-      float sv[2];
+      // column sh of the hi part and 16 + sh of the lo part, token-contiguous
+      float sv[2] = {c_h, c_h};
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int t = stl + 16 * i;
-        float v = c_h;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          const float* rr = red + (w * 32 + t) * ATTN_RED_PITCH;
-          v += rr[sh] + rr[16 + sh];
-        }
-        sv[i] = (sh < heads && tb + t < n) ? v : -INFINITY;
+      for (int w = 0; w < 8; ++w) {
+        const float* rc = red + w * 32 * ATTN_RED_PITCH;
+        const float2 hi = *reinterpret_cast<const float2*>(rc + sh * ATTN_RED_PITCH + 2 * stl);
+        const float2 lo =
+            *reinterpret_cast<const float2*>(rc + (16 + sh) * ATTN_RED_PITCH + 2 * stl);
+        sv[0] += hi.x + lo.x;
+        sv[1] += hi.y + lo.y;
       }
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+        if (!(sh < heads && tb + 2 * stl + i < n)) sv[i] = -INFINITY;
       float mx = fmaxf(sv[0], sv[1]);
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -687,8 +692,9 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         const bf16 hi = __float2bfloat16_rn(e[i]);
-        sp[sh * ATTN_P_PITCH + stl + 16 * i] = hi;
-        sp[(16 + sh) * ATTN_P_PITCH + stl + 16 * i] = __float2bfloat16_rn(e[i] - __bfloat162float(hi));
+        sp[sh * ATTN_P_PITCH + 2 * stl + i] = hi;
+        sp[(16 + sh) * ATTN_P_PITCH + 2 * stl + i] =
+            __float2bfloat16_rn(e[i] - __bfloat162float(hi));
       }
       __syncwarp();  // every lane has read s_m[sh]
       if (stl == 0) {
@@ -841,15 +847,20 @@ int launch_pool_attend(const void* x, const bf16* U2, int Tq, const float* cb,
   int rc;
   {
     TraceScope ts("pool.attend", L.stream);
+    // one instantiation per width (the warps' register tiles are sized by it)
+    auto run = [&](auto ks) {
+      return launch_attend_ks<decltype(ks)::value>(xmap, U2, u2_per_tile, cb, cb_stride,
+                                                   valid_len, T, heads, Zp, mstat, lstat, L);
+    };
     switch (D / 128) {
-      case 1: rc = launch_attend_ks<1>(xmap, U2, u2_per_tile, cb, cb_stride, valid_len, T, heads, Zp, mstat, lstat, L); break;
-      case 2: rc = launch_attend_ks<2>(xmap, U2, u2_per_tile, cb, cb_stride, valid_len, T, heads, Zp, mstat, lstat, L); break;
-      case 3: rc = launch_attend_ks<3>(xmap, U2, u2_per_tile, cb, cb_stride, valid_len, T, heads, Zp, mstat, lstat, L); break;
-      case 4: rc = launch_attend_ks<4>(xmap, U2, u2_per_tile, cb, cb_stride, valid_len, T, heads, Zp, mstat, lstat, L); break;
-      case 5: rc = launch_attend_ks<5>(xmap, U2, u2_per_tile, cb, cb_stride, valid_len, T, heads, Zp, mstat, lstat, L); break;
-      case 6: rc = launch_attend_ks<6>(xmap, U2, u2_per_tile, cb, cb_stride, valid_len, T, heads, Zp, mstat, lstat, L); break;
-      case 7: rc = launch_attend_ks<7>(xmap, U2, u2_per_tile, cb, cb_stride, valid_len, T, heads, Zp, mstat, lstat, L); break;
-      default: rc = launch_attend_ks<8>(xmap, U2, u2_per_tile, cb, cb_stride, valid_len, T, heads, Zp, mstat, lstat, L); break;
+      case 1: rc = run(std::integral_constant<int, 1>{}); break;
+      case 2: rc = run(std::integral_constant<int, 2>{}); break;
+      case 3: rc = run(std::integral_constant<int, 3>{}); break;
+      case 4: rc = run(std::integral_constant<int, 4>{}); break;
+      case 5: rc = run(std::integral_constant<int, 5>{}); break;
+      case 6: rc = run(std::integral_constant<int, 6>{}); break;
+      case 7: rc = run(std::integral_constant<int, 7>{}); break;
+      default: rc = run(std::integral_constant<int, 8>{}); break;
     }
   }
   if (rc != IVC_OK) return rc;

@@ -377,7 +377,8 @@ __device__ bool fold_phase(const RouterFusedArgs& a, int l, int Tq, const float*
 // input). Per step:
 //   1. s[t][j] = x_t . U2[j] for the 32 split rows: warp w multiplies its D/8
 //      channels with m16n8k16 MMAs (its U2 fragments in registers for the
-//      item), the 8 partial 32x32 tiles are summed in shared memory;
+//      item), the 8 partial 32x32 tiles, stored column by column, are summed
+//      in shared memory;
 //      s_h = s[t][h] + s[t][16 + h] + c_h, tokens past valid_len -inf;
 //   2. running max m_h and sum l_h, weights e = exp(s - m_h) as a bf16 hi/lo
 //      pair;
@@ -392,7 +393,7 @@ __device__ bool fold_phase(const RouterFusedArgs& a, int l, int Tq, const float*
 // before the barrier that ends it for every CTA).
 constexpr int AT_CHUNK = 128;                 // tokens per item
 constexpr int AT_NCH = RF_TOK / AT_CHUNK;     // items (partials) per tile
-constexpr int AT_RED_PITCH = 33;
+constexpr int AT_RED_PITCH = 36;  // floats per column of a partial score tile
 constexpr int AT_P_PITCH = 40;
 constexpr int AT_RED_BYTES = RF_WARPS * 32 * AT_RED_PITCH * 4;
 constexpr int AT_SLOT0 = ((AT_RED_BYTES + 2 * 16 * AT_P_PITCH * 2 + 1023) / 1024) * 1024;
@@ -563,27 +564,29 @@ __device__ __noinline__ bool attend_phase_ks(const RouterFusedArgs& a, bool shar
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) {
           const int r = mt * 16 + g, j = nt * 8 + t2;
-          rw[r * AT_RED_PITCH + j] = accs[mt][nt][0];
-          rw[r * AT_RED_PITCH + j + 1] = accs[mt][nt][1];
-          rw[(r + 8) * AT_RED_PITCH + j] = accs[mt][nt][2];
-          rw[(r + 8) * AT_RED_PITCH + j + 1] = accs[mt][nt][3];
+          rw[j * AT_RED_PITCH + r] = accs[mt][nt][0];
+          rw[(j + 1) * AT_RED_PITCH + r] = accs[mt][nt][1];
+          rw[j * AT_RED_PITCH + r + 8] = accs[mt][nt][2];
+          rw[(j + 1) * AT_RED_PITCH + r + 8] = accs[mt][nt][3];
         }
       __syncthreads();
-      // 2. running softmax of head sh over tokens stl and stl + 16
+      // 2. running softmax of head sh over tokens 2 stl and 2 stl + 1
       {
         const int tb = chunk * AT_CHUNK + st * SC_TOK;
-        float sv[2];
+        // column sh of the hi part and 16 + sh of the lo part, token-contiguous
+        float sv[2] = {c_h, c_h};
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int t = stl + 16 * i;
-          float v = c_h;
-#pragma unroll
-          for (int w = 0; w < RF_WARPS; ++w) {
-            const float* rr = red + (w * 32 + t) * AT_RED_PITCH;
-            v += rr[sh] + rr[16 + sh];
-          }
-          sv[i] = (sh < a.heads && tb + t < n) ? v : -INFINITY;
+        for (int w = 0; w < RF_WARPS; ++w) {
+          const float* rc = red + w * 32 * AT_RED_PITCH;
+          const float2 hi = *reinterpret_cast<const float2*>(rc + sh * AT_RED_PITCH + 2 * stl);
+          const float2 lo =
+              *reinterpret_cast<const float2*>(rc + (16 + sh) * AT_RED_PITCH + 2 * stl);
+          sv[0] += hi.x + lo.x;
+          sv[1] += hi.y + lo.y;
         }
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+          if (!(sh < a.heads && tb + 2 * stl + i < n)) sv[i] = -INFINITY;
         float mx = fmaxf(sv[0], sv[1]);
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -601,8 +604,8 @@ __device__ __noinline__ bool attend_phase_ks(const RouterFusedArgs& a, bool shar
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
           const bf16 hi = __float2bfloat16_rn(e[i]);
-          sp[sh * AT_P_PITCH + stl + 16 * i] = hi;
-          sp[(16 + sh) * AT_P_PITCH + stl + 16 * i] =
+          sp[sh * AT_P_PITCH + 2 * stl + i] = hi;
+          sp[(16 + sh) * AT_P_PITCH + 2 * stl + i] =
               __float2bfloat16_rn(e[i] - __bfloat162float(hi));
         }
         __syncwarp();  // every lane has read s_m[sh]
