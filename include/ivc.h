@@ -136,8 +136,12 @@ typedef struct ivc_router {
  *   grouped tensor-core GEMM, fp32 K/V), then per head softmax(Q.K/8) V.
  * FOLDED: with one query per tile the projections are reassociated exactly:
  *   scores = X (Wk_h^T Q_h / 8) + bk_h.Q_h / 8 and o_h = Wv_h (sum_t p_t x_t) + bv_h,
- *   two thin tensor-core GEMMs over the raw features per layer (~60x fewer
- *   FLOPs, no K/V tensor). */
+ *   evaluated in one pass over the raw features per layer (scores, running
+ *   softmax and weighted sums per 128-token chunk, the chunks then merged;
+ *   ~60x fewer FLOPs, no K/V tensor). The environment variable
+ *   IVC_POOL_ATTEND=0 selects the earlier form of the separate kernels
+ *   (scores and weighted sums as two tensor-core GEMMs with a softmax kernel
+ *   between them). */
 enum ivc_pool_mode { IVC_POOL_FOLDED = 0, IVC_POOL_LITERAL = 1 };
 
 enum ivc_op {
