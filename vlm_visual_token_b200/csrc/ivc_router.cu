@@ -500,7 +500,8 @@ int launch_pool_softmax(const float* S, const float* cb, int cb_stride, const in
 // the features (the split-softmax, or flash-decoding, form of attention with
 // one query per head): CTA (tile, chunk of ATTN_CHUNK tokens) streams its
 // tokens ATTN_STEP at a time (one TMA box of {64 channels, 32 tokens, D/64
-// chunks}, 128-byte swizzle, double-buffered) and per step
+// chunks}, 128-byte swizzle, double-buffered; a slot is refilled after the
+// next step's scores are summed, two CTA barriers per step) and per step
 //   1. s[t][j] = x_t . U2[j] for the 32 split rows j (warp w multiplies its
 //      D/8 channels with m16n8k16 MMAs, the U2 fragments held in registers
 //      for the whole CTA; the 8 partial 32x32 tiles, stored column by
@@ -658,6 +659,13 @@ __global__ void __launch_bounds__(256, 1)
       }
     ok = __syncthreads_and(ok) != 0;
     if (!ok) break;
+    // every warp has finished the previous step's weighted sums: its slot takes
+    // the step after this one
+    if (threadIdx.x == 0 && st >= 1 && st + 1 < nsteps) {
+      mbar_arrive_expect_tx(&s_mb[slot ^ 1], SLOT);
+      tma_load_3d(sm + (slot ^ 1) * SLOT, &xmap, &s_mb[slot ^ 1], 0,
+                  tile * TILE_TOKENS + tok0 + (st + 1) * ATTN_STEP, 0);
+    }
     // 2. running softmax of head sh over tokens 2 stl and 2 stl + 1
     {
       const int tb = tok0 + st * ATTN_STEP;
@@ -735,12 +743,8 @@ __global__ void __launch_bounds__(256, 1)
         }
       }
     }
-    __syncthreads();  // every warp is done with this slot and with the weights
-    if (threadIdx.x == 0 && st + 2 < nsteps) {
-      mbar_arrive_expect_tx(&s_mb[slot], SLOT);
-      tma_load_3d(sm + slot * SLOT, &xmap, &s_mb[slot], 0,
-                  tile * TILE_TOKENS + tok0 + (st + 2) * ATTN_STEP, 0);
-    }
+    // no barrier here: the weights and s_scale are rewritten only after the
+    // next step's first barrier, and the score partials were read before the last
   }
   if (!ok) {
     if (threadIdx.x == 0) atomicOr(status, DEV_WAIT_TIMEOUT);

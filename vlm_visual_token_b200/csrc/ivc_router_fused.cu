@@ -374,7 +374,8 @@ __device__ bool fold_phase(const RouterFusedArgs& a, int l, int Tq, const float*
 // SC_TOK at a time, one TMA request per step ({64 channels, 32 tokens, D/64
 // chunks}, 128-byte swizzle), double-buffered on mbarriers 2 and 3 across the
 // CTA's steps (the first two requested before the grid barrier, x being an
-// input). Per step:
+// input; later ones once the scores of the step before them are summed, when
+// every warp is done with the slot). Two CTA barriers per step. Per step:
 //   1. s[t][j] = x_t . U2[j] for the 32 split rows: warp w multiplies its D/8
 //      channels with m16n8k16 MMAs (its U2 fragments in registers for the
 //      item), the 8 partial 32x32 tiles, stored column by column, are summed
@@ -570,6 +571,13 @@ __device__ __noinline__ bool attend_phase_ks(const RouterFusedArgs& a, bool shar
           rw[(j + 1) * AT_RED_PITCH + r + 8] = accs[mt][nt][3];
         }
       __syncthreads();
+      // every warp has finished the previous step's weighted sums: its slot
+      // takes the step after this one
+      if (k >= 1 && ic.valid()) {
+        if (threadIdx.x == 0) attend_issue_x(a, ic, slot ^ 1, sm, mb);
+        x_pending |= 1 << (slot ^ 1);
+        ic.next(a);
+      }
       // 2. running softmax of head sh over tokens 2 stl and 2 stl + 1
       {
         const int tb = chunk * AT_CHUNK + st * SC_TOK;
@@ -647,12 +655,8 @@ __device__ __noinline__ bool attend_phase_ks(const RouterFusedArgs& a, bool shar
           }
         }
       }
-      __syncthreads();  // every warp is done with this slot and with the weights
-      if (ic.valid()) {
-        if (threadIdx.x == 0) attend_issue_x(a, ic, slot, sm, mb);
-        x_pending |= 1 << slot;
-        ic.next(a);
-      }
+      // no barrier here: the weights and s_scale are rewritten only after the
+      // next step's first barrier, and the score partials were read before the last
     }
     float* zp = a.Zp + row0 * D;
 #pragma unroll
