@@ -257,8 +257,6 @@ def run_reference(args):
 
 # ----------------------------------------------------------------- GPU leg
 def run_ivc(args):
-    import ctypes
-
     import torch
 
     rank, world, local = dist_env()
@@ -374,21 +372,16 @@ def run_ivc(args):
     del ws_r, ws_1, ws_2, y256, y64
 
     # ---- traced pass: per-kernel device time of the same steps (eager launches)
-    L = ivc.lib()
-    L.ivc_trace_enable.argtypes = [ctypes.c_int]
-    L.ivc_trace_report.argtypes = [ctypes.c_char_p, ctypes.c_size_t]
     n_trace = min(args.steps, 50)
-    L.ivc_trace_reset()
-    L.ivc_trace_enable(1)
+    ivc.trace_reset()
+    ivc.trace_enable(True)
     for _ in range(n_trace):
         flush.zero_()
         step()
     torch.cuda.synchronize()
-    L.ivc_trace_enable(0)
-    buf = ctypes.create_string_buffer(1 << 16)
-    L.ivc_trace_report(buf, len(buf))
-    trace = json.loads(buf.value.decode())
-    L.ivc_trace_reset()
+    ivc.trace_enable(False)
+    trace = ivc.trace_report()
+    ivc.trace_reset()
     launches_per_step = sum(v["launches"] for v in trace.values()) / n_trace
     per_step_ms = {k: v["ms"] / n_trace for k, v in trace.items()}
     trace_total = sum(per_step_ms.values())
@@ -640,19 +633,14 @@ def run_op(args):
         line.update({"prompt_tokens": int(ids.numel()), "kept_tokens": n,
                      "bytes_per_call": moved, "achieved_gbs": moved / (ms / 1e3) / 1e9})
     if args.trace:
-        import ctypes
-        L = ivc.lib()
-        L.ivc_trace_enable.argtypes = [ctypes.c_int]
-        L.ivc_trace_report.argtypes = [ctypes.c_char_p, ctypes.c_size_t]
-        L.ivc_trace_reset()
-        L.ivc_trace_enable(1)
+        ivc.trace_reset()
+        ivc.trace_enable(True)
         for _ in range(args.steps):
             fn()
         torch.cuda.synchronize()
-        L.ivc_trace_enable(0)
-        buf = ctypes.create_string_buffer(1 << 16)
-        L.ivc_trace_report(buf, len(buf))
-        tr = json.loads(buf.value.decode())
+        ivc.trace_enable(False)
+        tr = ivc.trace_report()
+        ivc.trace_reset()
         line["traced_us_per_launch"] = {k: round(1e3 * v["ms"] / v["launches"], 2)
                                         for k, v in tr.items()}
         line["traced_launches_per_call"] = {k: v["launches"] // args.steps for k, v in tr.items()}

@@ -29,6 +29,17 @@ def test_library_exports_every_declared_symbol():
     assert L.ivc_version() >= 100
 
 
+def test_trace_without_records_needs_no_gpu():
+    """The tracing calls only touch CUDA for recorded launches: with none, the
+    report is an empty object and a too-small buffer is refused."""
+    import vlm_visual_token_b200 as ivc
+    ivc.trace_enable(False)
+    ivc.trace_reset()
+    assert ivc.trace_report() == {}
+    with pytest.raises(ivc.IvcError):
+        ivc.trace_report(max_bytes=1)
+
+
 def test_status_strings():
     import vlm_visual_token_b200 as ivc
     L = ivc.lib()

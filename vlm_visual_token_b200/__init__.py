@@ -14,6 +14,7 @@ is no fallback implementation.
 from __future__ import annotations
 
 import ctypes
+import json
 import os
 from typing import Optional, Sequence
 
@@ -103,6 +104,12 @@ def lib() -> ctypes.CDLL:
                                             ctypes.c_size_t, _vp]
         L.ivc_device_status.restype = ctypes.c_int
         L.ivc_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int), _vp]
+        L.ivc_trace_enable.restype = ctypes.c_int
+        L.ivc_trace_enable.argtypes = [ctypes.c_int]
+        L.ivc_trace_reset.restype = ctypes.c_int
+        L.ivc_trace_reset.argtypes = []
+        L.ivc_trace_report.restype = ctypes.c_int
+        L.ivc_trace_report.argtypes = [ctypes.c_char_p, ctypes.c_size_t]
         _LIB = L
     return _LIB
 
@@ -311,3 +318,21 @@ def device_status(workspace: torch.Tensor, stream=None) -> int:
     if rc not in (0, -5):
         raise IvcError(rc, "ivc_device_status")
     return bits.value
+
+
+def trace_enable(on: bool = True) -> None:
+    """Start (or stop) recording the device time of each of the library's launches."""
+    _check(lib().ivc_trace_enable(1 if on else 0), "ivc_trace_enable")
+
+
+def trace_reset() -> None:
+    """Forget the recorded launches."""
+    _check(lib().ivc_trace_reset(), "ivc_trace_reset")
+
+
+def trace_report(max_bytes: int = 1 << 16) -> dict:
+    """{role: {"launches": n, "ms": total device ms}} of the launches recorded
+    since the last reset (waits for them to finish)."""
+    buf = ctypes.create_string_buffer(max_bytes)
+    _check(lib().ivc_trace_report(buf, len(buf)), "ivc_trace_report")
+    return json.loads(buf.value.decode())
