@@ -113,10 +113,12 @@ struct RouteBufs {
   float* KV = nullptr;   // literal pooling: K/V of the 4 layers
   bf16* U2 = nullptr;    // folded pooling: split u of one layer [T][32][D]
   float* cb = nullptr;   //   c [T][16]
-  float* S = nullptr;    //   split scores [T*1024][32]
-  bf16* P2 = nullptr;    //   split softmax weights [T*128][1024] (multi-kernel form)
-  float* Z = nullptr;    //   split weighted sums [T*128][D] (multi-kernel form)
-  float* z = nullptr;    //   fused router: weighted sums [T][16][D]
+  float* S = nullptr;    //   single-pass attention: chunk max / sum [2][T*8*16];
+                         //   tensor-core form: split scores [T*1024][32]
+  bf16* P2 = nullptr;    //   tensor-core form: split softmax weights [T*128][1024]
+  float* Z = nullptr;    //   single-pass attention: chunk sums [T][8][16][D];
+                         //   tensor-core form: split weighted sums [T*128][D]
+  float* z = nullptr;    //   merged weighted sums [T][16][D]
   float* h = nullptr;    //   fused router: gating state [T][D]
   unsigned* bar = nullptr;  // fused router: grid barrier words
   float* Q1;
@@ -135,8 +137,6 @@ void carve_route(Carver& cv, const ivc_router* r, int T, RouteBufs& b) {
     b.U2 = cv.take<bf16>(static_cast<size_t>(T) * 32 * D);
     b.cb = cv.take<float>(static_cast<size_t>(T) * 16);
     b.S = cv.take<float>(static_cast<size_t>(T) * 1024 * 32);
-    // P2 in the multi-kernel form [T*128][1024]; the persistent kernel uses
-    // its first T*32*1024 entries as [T][32][1024]
     b.P2 = cv.take<bf16>(static_cast<size_t>(T) * 128 * 1024);
     b.Z = cv.take<float>(static_cast<size_t>(T) * 128 * D);
     b.z = cv.take<float>(static_cast<size_t>(T) * 16 * D);

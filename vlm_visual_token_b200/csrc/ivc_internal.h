@@ -138,8 +138,9 @@ int launch_pool_attention(const float* Q, long long ldq, const float* KV, long l
                           int koff, int voff, const int32_t* valid_len, int T, int D, int heads,
                           float* O, const Launch& L);
 // Folded pooling (up to 16 heads of 64): u/c of one layer from Q [Tq, D] (Tq = 1:
-// the same query for every tile), scores' softmax into the split P2 operand,
-// and o = Wv z + bv from the split weighted sums Z [T*128, D].
+// the same query for every tile); in the tensor-core form the scores' softmax
+// into the split P2 operand and o = Wv z + bv from the split weighted sums
+// Z [T*128, D].
 int launch_pool_fold_query(const float* Q, long long ldq, int Tq, const bf16* Wk, const bf16* bk,
                            int D, bf16* U2, float* cb, const Launch& L);
 int launch_pool_softmax(const float* S, const float* cb, int cb_stride, const int32_t* valid_len,
