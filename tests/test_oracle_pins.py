@@ -293,6 +293,72 @@ def test_pooling_matches_torch_multihead_attention_chain():
 
 
 # ------------------------------------------------------------------ gating
+def _pool_chunked(X, valid_len, r, rescale=True, merge=True, chunk=128, step=32):
+    """Single-query pooling in the single-pass form (fp64): per layer and head
+    the key projection folded into the query (u, c), per chunk of `chunk` tokens
+    a running max m and sum l over steps of `step` tokens with the weighted sum
+    kept relative to m, chunks without a valid token skipped, chunks merged
+    with weights exp(m_c - M); the value projection applied to the merged sum."""
+    T, N, D = X.shape
+    H = int(r["heads"])
+    dh = D // H
+    q = np.broadcast_to(r["query"], (T, D)).copy()
+    for l in range(len(r["Wq"])):
+        Q = q @ r["Wq"][l].T + r["bq"][l]
+        o = np.zeros((T, D))
+        for t in range(T):
+            n = int(valid_len[t])
+            for h in range(H):
+                sl = slice(h * dh, (h + 1) * dh)
+                u = r["Wk"][l][sl].T @ Q[t, sl] / math.sqrt(dh)
+                c = r["bk"][l][sl] @ Q[t, sl] / math.sqrt(dh)
+                parts = []
+                for c0 in range(0, N, chunk):
+                    m, lsum, z = -math.inf, 0.0, np.zeros(D)
+                    for s0 in range(c0, min(c0 + chunk, n), step):
+                        xs = X[t, s0:min(s0 + step, n)]
+                        sc = xs @ u + c
+                        m_new = max(m, float(sc.max()))
+                        f = math.exp(m - m_new) if rescale else 1.0
+                        e = np.exp(sc - m_new)
+                        lsum, z, m = lsum * f + e.sum(), z * f + e @ xs, m_new
+                    if lsum > 0:
+                        parts.append((m, lsum, z))
+                M = max(pm for pm, _, _ in parts)
+                w = [math.exp(pm - M) if merge else 1.0 for pm, _, _ in parts]
+                zt = sum(wi * pz for wi, (_, _, pz) in zip(w, parts)) / \
+                    sum(wi * pl for wi, (_, pl, _) in zip(w, parts))
+                o[t, sl] = r["Wv"][l][sl] @ zt + r["bv"][l][sl]
+        q = o @ r["Wo"][l].T + r["bo"][l]
+    return q
+
+
+def test_pooling_single_pass_form_equals_definition():
+    """The reassociation the pooling kernels compute (folded key projection,
+    running softmax per 128-token chunk, chunks merged) equals the oracle's
+    attention to rounding, including a one-token tile and a tile whose second
+    chunk holds a single valid token; dropping the running rescale or the
+    max-relative merge weights breaks it."""
+    rng = np.random.default_rng(11)
+    T, N, D, H = 3, 1024, 128, 2
+
+    def mat(o, i):
+        return rng.normal(size=(o, i)) / math.sqrt(i)
+
+    r = {"heads": H, "query": rng.normal(size=D)}
+    for k in ("Wq", "Wk", "Wv", "Wo"):
+        r[k] = [mat(D, D) for _ in range(4)]
+    for k in ("bq", "bk", "bv", "bo"):
+        r[k] = [0.1 * rng.normal(size=D) for _ in range(4)]
+    # growing scale along the tokens: the running max changes from chunk to chunk
+    X = rng.normal(size=(T, N, D)) * np.linspace(1.0, 4.0, N)[None, :, None]
+    vl = np.array([1, 129, 1024])
+    ref = O.cross_attention_pooling(X, vl, r)
+    np.testing.assert_allclose(_pool_chunked(X, vl, r), ref, rtol=1e-9, atol=1e-12)
+    assert not np.allclose(_pool_chunked(X, vl, r, rescale=False), ref, rtol=1e-3)
+    assert not np.allclose(_pool_chunked(X, vl, r, merge=False), ref, rtol=1e-3)
+
+
 def test_gating_rows_sum_to_one_and_sigmoid_identity():
     r = _router()
     h = RNG.standard_normal((7, 32))
