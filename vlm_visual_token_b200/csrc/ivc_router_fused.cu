@@ -113,6 +113,13 @@ __device__ bool grid_sync(unsigned* bar, unsigned& gen) {
   return s_ok != 0;
 }
 
+// Bounded wait whose give-up is decided for the whole CTA: every thread waits,
+// then one barrier combines the results, so no thread returns while others go
+// on to a later CTA barrier.
+__device__ __forceinline__ bool cta_wait(uint64_t* bar, uint32_t parity) {
+  return __syncthreads_and(mbar_wait(bar, parity) ? 1 : 0) != 0;
+}
+
 // ------------------------------------------------------------------ mma.sync
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
                                                const uint32_t (&b)[2]) {
@@ -207,11 +214,11 @@ __device__ bool gemv_phase(int M, int K, int N, const bf16* __restrict__ W,
         }
       }
       if (!w_ready) {
-        if (!mbar_wait(&mb[0], ph[0])) return false;
+        if (!cta_wait(&mb[0], ph[0])) return false;
         ph[0] ^= 1;
         w_ready = true;
       }
-      if (!mbar_wait(&mb[1], ph[1])) return false;
+      if (!cta_wait(&mb[1], ph[1])) return false;
       ph[1] ^= 1;
       // rows >= `rows` of the A tile hold stale values; they only reach
       // output rows that are never stored
@@ -336,7 +343,7 @@ __device__ bool fold_phase(const RouterFusedArgs& a, int l, int Tq, const float*
       if (threadIdx.x < 32) fold_issue_w(a.Wk[l], D, item, sm, &mb[0]);
     }
     first = false;
-    if (!mbar_wait(&mb[0], ph[0])) return false;
+    if (!cta_wait(&mb[0], ph[0])) return false;
     ph[0] ^= 1;
     for (int t0 = 0; t0 < Tq; t0 += 64) {
       const int nt = min(64, Tq - t0);
@@ -532,9 +539,8 @@ __device__ __noinline__ bool attend_phase_ks(const RouterFusedArgs& a, bool shar
     for (int st = 0; st < ns; ++st, ++k) {
       const int slot = k & 1;
       const uint8_t* sx = sm + AT_SLOT0 + slot * slot_bytes;
-      if (!mbar_wait(&mb[2 + slot], ph[2 + slot])) return false;
-      ph[2 + slot] ^= 1;
-      x_pending &= ~(1 << slot);
+      // the give-up is decided for the whole CTA at the barrier after the scores
+      const bool got = mbar_wait(&mb[2 + slot], ph[2 + slot]);
       // 1. partial scores of this warp's channels
       float accs[2][4][4];
 #pragma unroll
@@ -570,7 +576,10 @@ __device__ __noinline__ bool attend_phase_ks(const RouterFusedArgs& a, bool shar
           rw[j * AT_RED_PITCH + r + 8] = accs[mt][nt][2];
           rw[(j + 1) * AT_RED_PITCH + r + 8] = accs[mt][nt][3];
         }
-      __syncthreads();
+      // a copy that never landed leaves its bit set (drained at exit)
+      if (__syncthreads_and(got ? 1 : 0) == 0) return false;
+      ph[2 + slot] ^= 1;
+      x_pending &= ~(1 << slot);
       // every warp has finished the previous step's weighted sums: its slot
       // takes the step after this one
       if (k >= 1 && ic.valid()) {
