@@ -219,8 +219,14 @@ def gating(pooled: np.ndarray, r: dict, residual: str = "outside") -> np.ndarray
 def quantile_linear(values: np.ndarray, q: float) -> float:
     """Linear-interpolation quantile: sort ascending, pos = q (n - 1),
     lo = floor(pos), hi = ceil(pos), result = v[lo] + (pos - lo) (v[hi] - v[lo]).
-    Evaluated in fp64 with each operation rounded separately."""
+    Evaluated in fp64 with each operation rounded separately.
+
+    The threshold of [VIR] section 4 is torch.quantile's, which is NaN as soon
+    as one input is NaN (NaN inputs are not skipped); every comparison with a
+    NaN threshold is false, so no tile of that group is compressed."""
     v = np.sort(np.asarray(values, dtype=np.float64))
+    if np.isnan(v).any():
+        return float("nan")
     n = v.shape[0]
     pos = float(q) * float(n - 1)
     lo = int(math.floor(pos))

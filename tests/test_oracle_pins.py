@@ -427,6 +427,24 @@ def test_quantile_matches_numpy_and_torch(n):
         np.testing.assert_allclose(got, torch.quantile(torch.from_numpy(v), q).item(), rtol=1e-15, atol=1e-16)
 
 
+def test_quantile_nan_propagates_like_torch():
+    """A NaN gate makes torch.quantile NaN (the pages' threshold); the oracle
+    follows, and then no tile of the group passes the strict > test."""
+    rng = np.random.default_rng(5)
+    for n in (1, 2, 5, 13):
+        v = rng.random(n)
+        v[rng.integers(n)] = np.nan
+        ref = torch.quantile(torch.from_numpy(v), 0.1).item()
+        assert math.isnan(ref)
+        assert math.isnan(O.quantile_linear(v, 0.1))
+        mask = O.route(np.concatenate([v, [0.9, 0.8, 0.3]]), np.array([0, n, n + 3]))
+        assert mask[:n].sum() == 0               # the image holding the NaN
+        assert mask[n:].tolist() == [1, 1, 0]     # the other image is untouched
+    # batch scope: one NaN anywhere disables compression for the batch
+    g = np.array([0.9, 0.8, np.nan, 0.7])
+    assert O.route(g, np.array([0, 4]), scope="batch").sum() == 0
+
+
 def test_quantile_brute_cases():
     assert O.quantile_linear([0.7], 0.1) == 0.7
     v = np.array([5., 1., 4., 2., 3., 9., 8., 7., 6., 0., 10.])  # n = 11, pos = 1.0 exactly
