@@ -1,24 +1,32 @@
 """Throughput of the InternVL visual-token compression hot path on B200.
 
-One step = one ivc_flash_compress over one image of 12 tiles + thumbnail
-(T = 13 tiles of [32, 32, 1024] bf16, InternVL3.5-2B-Flash dims): pixel_shuffle
-0.5 -> mlp1 and 0.25 -> mlp2 for every tile, the ViR router (CrossAttentionPooling,
-Gating, quantile + absolute threshold) and compaction to 64/256 rows per tile.
+Default workload (``flash_2b_13tiles``): one step = one ivc_flash_compress over
+one image of 12 tiles + thumbnail (T = 13 tiles of [32, 32, 1024] bf16,
+InternVL3.5-2B-Flash dims): pixel_shuffle 0.5 -> mlp1 and 0.25 -> mlp2 for
+every tile, the ViR router (CrossAttentionPooling, Gating, quantile + absolute
+threshold) and compaction to 64/256 rows per tile.
+
+``--workload`` selects another configuration (``workloads.WORKLOADS``): the
+batched 4B-Flash flow (``flash_4b_batched``, one step = one
+ivc_flash_compress over 16 images), or a connector alone (``single_tile_2b``,
+``connector_14b_832tiles``, ``connector_38b_416tiles``: one step = one
+ivc_ps_project at factor 0.5 over the whole batch).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ivc|reference]
+                    [--workload NAME]
 
 Prints one JSON line (rank 0). Metric: tiles per second (whole job). Inputs
 are resident in HBM; L2 is flushed (512 MiB write) between timed steps, each
 step timed with CUDA events on the launching stream; max over ranks. With
-N > 1 every rank processes its own image (weights replicated, no data-path
+N > 1 every rank processes its own batch (weights replicated, no data-path
 collective): weak scaling. ``--impl reference`` times the fp64 CPU oracle on
 a bounded per-step sample of the same workload (rank 0 only).
 """
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -32,8 +40,11 @@ if ROOT not in sys.path:
 
 METRIC = "ViT tiles/sec through ps+MLP connector & ViR router; % of bf16 tensor/HBM peak"
 UNIT = "tiles/s"
-WORKLOAD = "flash_2b_13tiles"
+DEFAULT_WORKLOAD = "flash_2b_13tiles"
+WORKLOAD_NAMES = ("single_tile_2b", "flash_2b_13tiles", "flash_4b_batched",
+                  "connector_14b_832tiles", "connector_38b_416tiles")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GEMM_ROLES = ("mlp1.fc1", "mlp1.fc2", "mlp2.fc1", "mlp2.fc2", "mlp2.fc3")
 
 
 # ----------------------------------------------------------------- helpers (CPU-testable)
@@ -62,16 +73,18 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_traffic(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu capture
-    (profiles/traffic.json), or None once the sources it was built from have
-    changed since the capture."""
+def kernel_traffic(kernel, workload=DEFAULT_WORKLOAD):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    capture (profiles/traffic.json), or None once the sources it was built
+    from have changed since the capture."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
+    if d.get("workload", DEFAULT_WORKLOAD) != workload:
+        return None
     e = d.get("kernels", {}).get(kernel)
     if e is None:
         return None
@@ -117,17 +130,36 @@ def algorithmic(w, T):
     return f
 
 
-def image_gen(rank: int):
+def router_bytes(w, T):
+    """Algorithmic bytes of the whole folded router for T tiles: the features
+    once, every pooling and gating weight and bias once, the gates written."""
+    D, G = w.D, w.gate_hidden
+    pool_w = 4 * (4 * D * D + 4 * D) + D          # Wq/Wk/Wv/Wo + biases x 4 layers, query
+    gate_w = 4 * (2 * D * G + G + 3 * D) + 2 * D + 2  # W1/W2, b1/b2, LN gamma/beta x 4, head
+    return 2.0 * T * 1024 * w.C + 2.0 * (pool_w + gate_w) + 4.0 * 2 * T
+
+
+def connector_roles(w):
+    return GEMM_ROLES if w.path == "flash" else GEMM_ROLES[:2]
+
+
+def image_gen(rank: int, workload: str = DEFAULT_WORKLOAD):
     import workloads as W
-    return W.make(WORKLOAD, seed_offset=1000 * rank)
+    return W.make(workload, seed_offset=1000 * rank)
 
 
 class ClockSampler:
-    """nvidia-smi clocks/throttle reasons sampled every 100 ms while running."""
+    """nvidia-smi clocks/throttle reasons, sampled every 50 ms while running.
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Each sample carries its timestamp, so the summary separates the samples
+    taken inside the timed region from those of the whole loaded window
+    (the untimed preheat and warm-up steps right before it, and the timed
+    steps)."""
+
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, gpu_index: int):
         self.idx = gpu_index
@@ -140,7 +172,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -154,22 +186,47 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
+    @staticmethod
+    def parse(lines):
+        """Rows of (epoch seconds, sm MHz, max MHz, power W or None, reasons)."""
+        out = []
+        for line in lines:
+            p = [v.strip() for v in line.split(",")]
+            if len(p) < 10 or not p[2].replace(".", "").isdigit():
+                continue
+            try:
+                ts = datetime.datetime.strptime(p[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            pw = float(p[4]) if p[4].replace(".", "").isdigit() else None
+            reasons = {ClockSampler.REASONS[i] for i in range(4) if p[6 + i].lower() == "active"}
+            out.append((ts, float(p[2]), float(p[3]), pw, reasons))
+        return out
+
+    @staticmethod
+    def summarise(rows, t0, t1):
+        """Clock summary of the samples in [t0, t1] (the loaded window) and
+        the count of those inside the timed region's own bounds, if given."""
+        win = [r for r in rows if t0 - 0.05 <= r[0] <= t1 + 0.05]
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [r[1] for r in win]
+        pw = [r[3] for r in win if r[3] is not None]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": win[0][2],
+                "sm_mhz_min": min(sm), "reasons": sorted(set().union(*[r[4] for r in win])),
+                "samples": len(win), "power_w_max": max(pw) if pw else None}
+
+    def summary(self, t0, t1, timed=None):
         rows = []
         if self.path and os.path.exists(self.path):
-            for line in open(self.path):
-                p = [v.strip() for v in line.split(",")]
-                if len(p) >= 9 and p[1].replace(".", "").isdigit():
-                    rows.append(p)
+            with open(self.path) as f:
+                rows = self.parse(f)
             os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        sm = [float(r[1]) for r in rows]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
-                "reasons": reasons, "samples": len(rows),
-                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+        s = self.summarise(rows, t0, t1)
+        s["window"] = "preheat + warm-up + timed steps (GPU loaded throughout)"
+        if timed is not None:
+            s["samples_in_timed"] = sum(1 for r in rows if timed[0] <= r[0] <= timed[1])
+        return s
 
 
 def thread_count() -> int:
@@ -184,19 +241,32 @@ def thread_count() -> int:
 
 
 # ----------------------------------------------------------------- oracle (CPU) legs
+def _oracle_params(inp):
+    import oracle as O
+    if "_m1_64" not in inp:
+        inp["_m1_64"] = O.to64(inp["mlp1"])
+        if "mlp2" in inp:
+            inp["_m2_64"] = O.to64(inp["mlp2"])
+            inp["_r_64"] = O.to64(inp["router"])
+
+
 def oracle_sample(inp, tile: int, frac: float):
     """The oracle's whole path for `frac` of one tile: mlp1 on the first
-    256*frac shuffled rows, mlp2 on the first 64*frac, pooling over the first
-    1024*frac tokens (fewer K/V rows), gating, routing of the one-tile group
-    and the compaction offsets. Returns the tiles processed (= frac)."""
+    256*frac shuffled rows and, on the flash workloads, mlp2 on the first
+    64*frac, pooling over the first 1024*frac tokens, gating, routing of the
+    one-tile group and the compaction offsets. Returns the tiles processed
+    (= frac)."""
     import numpy as np
 
     import oracle as O
+    _oracle_params(inp)
     x = O.to64(inp["x"][tile:tile + 1])
     n256, n64, ntok = max(1, round(256 * frac)), max(1, round(64 * frac)), max(1, round(1024 * frac))
     P = O.pixel_shuffle(x, 0.5)[0, :n256]
     m1 = inp["_m1_64"]
     O.mlp(P, m1["ln_g"], m1["ln_b"], m1["W"], m1["b"])
+    if "mlp2" not in inp:
+        return frac
     Q = O.pixel_shuffle_quarter(x)[0, :n64]
     m2 = inp["_m2_64"]
     O.mlp(Q, m2["ln_g"], m2["ln_b"], m2["W"], m2["b"])
@@ -208,26 +278,55 @@ def oracle_sample(inp, tile: int, frac: float):
     return frac
 
 
+def cpu_sample_plan(inp):
+    """What the CPU baseline runs: whole images (routing couples the tiles of
+    an image) up to at least 8 tiles on the flash workloads, the whole image
+    when it has at most 16 tiles; 8 seeded tiles of a connector workload."""
+    import numpy as np
+    T = inp["T"]
+    w = inp["workload"]
+    if w.path == "flash":
+        offs = inp["image_offsets"].numpy()
+        if T <= 16:
+            return "images", len(offs) - 1
+        n = 1
+        while n < len(offs) - 1 and offs[n] < 8:
+            n += 1
+        return "images", n
+    k = min(8, T)
+    rng = np.random.default_rng(2024)
+    return "tiles", sorted(rng.choice(T, k, replace=False).tolist())
+
+
 def cpu_baseline(inp):
-    """The oracle, as it stands, over the whole 13-tile image once."""
+    """The oracle, as it stands, on the sample cpu_sample_plan picks; the
+    value is tiles processed per second of host time."""
     import oracle as O
+    _oracle_params(inp)
+    kind, what = cpu_sample_plan(inp)
     t0 = time.perf_counter()
-    O.flash_compress(O.to64(inp["x"]), inp["valid_len"].numpy(), inp["image_offsets"].numpy(),
-                     inp["_m1_64"], inp["_m2_64"], inp["_r_64"])
+    if kind == "images":
+        offs = inp["image_offsets"].numpy()
+        n_t = int(offs[what])
+        O.flash_compress(O.to64(inp["x"][:n_t]), inp["valid_len"].numpy()[:n_t], offs[:what + 1],
+                         inp["_m1_64"], inp["_m2_64"], inp["_r_64"])
+        desc = (f"the first {what} image(s), {n_t} tiles, whole path (fp64)" if n_t < inp["T"]
+                else f"one full batch of {n_t} tiles, whole path (fp64)")
+    else:
+        n_t = len(what)
+        O.ps_project(O.to64(inp["x"][what]), 0.5, inp["_m1_64"])
+        desc = f"{n_t} seeded tiles of {inp['T']} (ps 0.5 + mlp1, fp64), rate scales linearly in T"
     dt = time.perf_counter() - t0
-    return {"value": inp["T"] / dt, "unit": UNIT, "cores": thread_count(), "kind": "oracle",
-            "sample": f"one full image of {inp['T']} tiles (whole path, fp64), {dt:.1f} s"}
+    return {"value": n_t / dt, "unit": UNIT, "cores": thread_count(), "kind": "oracle",
+            "sample": f"{desc}, {dt:.1f} s"}
 
 
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
-    import oracle as O
-    inp = image_gen(0)
-    inp["_m1_64"], inp["_m2_64"], inp["_r_64"] = (O.to64(inp["mlp1"]), O.to64(inp["mlp2"]),
-                                                   O.to64(inp["router"]))
-    T = inp["T"]
+    inp = image_gen(0, args.workload)
+    w, T = inp["workload"], inp["T"]
     t0 = time.perf_counter()
     oracle_sample(inp, 0, 1.0)
     t_tile = time.perf_counter() - t0
@@ -243,26 +342,72 @@ def run_reference(args):
         units += oracle_sample(inp, i % T, frac)
         dt += time.perf_counter() - t0
     value = units / dt
+    path = "whole path" if w.path == "flash" else "ps 0.5 + mlp1"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": WORKLOAD, "tiles": T, "C": 1024, "H": 2048},
+            "data": "synthetic", "config": {"workload": w.name, "tiles": T, "C": w.C, "H": w.H},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": thread_count(), "kind": "oracle",
                              "sample": f"per step {frac:g} of one tile (rows/tokens subsampled), "
-                                       f"whole path in fp64"},
+                                       f"{path} in fp64"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
 # ----------------------------------------------------------------- GPU leg
+class Problem:
+    """Device-resident inputs, outputs and the one call a step makes."""
+
+    def __init__(self, ivc, inp, dev, routed):
+        import torch
+        self.ivc, self.inp, self.dev, self.routed = ivc, inp, dev, routed
+        w, T = inp["workload"], inp["T"]
+        self.w, self.T = w, T
+        self.flash = w.path == "flash"
+        self.x = inp["x"].to(dev)
+        self.m1 = ivc.Mlp(inp["mlp1"], dev).fold()
+        if self.flash:
+            self.vl = inp["valid_len"].to(dev)
+            self.offs = inp["image_offsets"].to(dev)
+            self.m2 = ivc.Mlp(inp["mlp2"], dev).fold()
+            self.r = ivc.Router(inp["router"], device=dev)
+            self.ws = ivc.new_workspace(
+                ivc.workspace_size(ivc.OP_FLASH, T, w.C, self.m1, self.m2, self.r), dev)
+            self.bufs = {"gate": torch.empty(T, 2, dtype=torch.float32, device=dev),
+                         "mask": torch.empty(T, dtype=torch.uint8, device=dev),
+                         "offsets": torch.empty(T + 1, dtype=torch.int32, device=dev),
+                         "total": torch.empty(1, dtype=torch.int32, device=dev)}
+        else:
+            self.ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_PS_HALF, T, w.C, self.m1), dev)
+            self.bufs = {}
+        self.out = torch.empty(T * 256, w.H, dtype=torch.bfloat16, device=dev)
+
+    def call(self, x=None, vl=None, offs=None, out=None, ws=None, bufs=None):
+        x = self.x if x is None else x
+        out = self.out if out is None else out
+        ws = self.ws if ws is None else ws
+        if self.flash:
+            self.ivc.flash_compress(x, self.vl if vl is None else vl,
+                                    self.offs if offs is None else offs, self.m1, self.m2, self.r,
+                                    out=out, workspace=ws, bufs=self.bufs if bufs is None else bufs,
+                                    routed=self.routed)
+        else:
+            self.ivc.ps_project(x, 0.5, self.m1, out=out, workspace=ws)
+
+    def inputs(self):
+        """The per-step inputs a user copies in (name -> device tensor)."""
+        d = {"x": self.x}
+        if self.flash:
+            d.update({"vl": self.vl, "offs": self.offs})
+        return d
+
+
 def run_ivc(args):
     import torch
 
     rank, world, local = dist_env()
     if world > 1:
-        import datetime
-
         import torch.distributed as dist
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
@@ -277,32 +422,18 @@ def run_ivc(args):
             import torch.distributed as dist
             dist.barrier()
 
-    inp = image_gen(rank)
-    w, T = inp["workload"], inp["T"]
-    x = inp["x"].to(dev)
-    vl = inp["valid_len"].to(dev)
-    offs = inp["image_offsets"].to(dev)
-    m1 = ivc.Mlp(inp["mlp1"], dev).fold()
-    m2 = ivc.Mlp(inp["mlp2"], dev).fold()
-    r = ivc.Router(inp["router"], device=dev)
-    ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_FLASH, T, w.C, m1, m2, r), dev)
-    bufs = {"gate": torch.empty(T, 2, dtype=torch.float32, device=dev),
-            "mask": torch.empty(T, dtype=torch.uint8, device=dev),
-            "offsets": torch.empty(T + 1, dtype=torch.int32, device=dev),
-            "total": torch.empty(1, dtype=torch.int32, device=dev)}
-    out = torch.empty(T * 256, w.H, dtype=torch.bfloat16, device=dev)
+    inp = image_gen(rank, args.workload)
+    routed = args.flow == "routed"
+    P = Problem(ivc, inp, dev, routed)
+    w, T = P.w, P.T
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-
-    routed = args.flow == "routed"
-
-    def step():
-        ivc.flash_compress(x, vl, offs, m1, m2, r, out=out, workspace=ws, bufs=bufs, routed=routed)
+    step = P.call
 
     for _ in range(3):
         step()
     torch.cuda.synchronize()
-    assert ivc.device_status(ws) == 0
+    assert ivc.device_status(P.ws) == 0
     graph = None
     try:
         g = torch.cuda.CUDAGraph()
@@ -313,15 +444,26 @@ def run_ivc(args):
         graph = None
     run = graph.replay if graph is not None else step
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        run()
-    torch.cuda.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
     with ClockSampler(local) as clk:
+        t_load0 = time.time()
+        # untimed preheat (at least a second of the same loaded loop) so that
+        # the clock sampler sees the GPU under this load right up to the
+        # timed steps, however short those are
+        t_end = time.perf_counter() + 1.0
+        while time.perf_counter() < t_end:
+            for _ in range(8):
+                flush.zero_()
+                run()
+            torch.cuda.synchronize()
+        for _ in range(args.warmup):
+            flush.zero_()
+            run()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        t_timed0 = time.time()
         t_wall = time.perf_counter()
         for a, b in evs:
             flush.zero_()
@@ -330,17 +472,17 @@ def run_ivc(args):
             b.record(stream)
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
+        t_timed1 = time.time()
+        time.sleep(0.1)  # let the sampler write its last row
     barrier()
     torch.cuda.synchronize()
     step_ms = [a.elapsed_time(b) for a, b in evs]
     total_ms = reduce_max(sum(step_ms), world, dev)
     value = world * T * args.steps / (total_ms / 1e3)
-    clocks = clk.summary()
-    if ivc.device_status(ws) != 0:
+    clocks = clk.summary(t_load0, t_timed1, (t_timed0, t_timed1))
+    if ivc.device_status(P.ws) != 0:
         raise RuntimeError("device status word set during the timed steps")
 
-    # ---- the two halves of the step alone (CUDA graphs, L2 flushed): the
-    # router (ivc_vir_route) and the connector (both ivc_ps_project calls)
     def graph_ms(fn, reps=50):
         g = torch.cuda.CUDAGraph()
         fn()
@@ -359,17 +501,23 @@ def run_ivc(args):
         del g
         return tot / reps
 
-    ws_r = ivc.new_workspace(ivc.workspace_size(ivc.OP_VIR_ROUTE, T, w.C, r=r), dev)
-    y256 = torch.empty(T * 256, w.H, dtype=torch.bfloat16, device=dev)
-    y64 = torch.empty(T * 64, w.H, dtype=torch.bfloat16, device=dev)
-    ws_1 = ivc.new_workspace(ivc.workspace_size(ivc.OP_PS_HALF, T, w.C, m1), dev)
-    ws_2 = ivc.new_workspace(ivc.workspace_size(ivc.OP_PS_QUARTER, T, w.C, m2), dev)
-    parts = {
-        "router_ms": graph_ms(lambda: ivc.vir_route(x, vl, offs, r, workspace=ws_r)),
-        "connector_ms": graph_ms(lambda: (ivc.ps_project(x, 0.5, m1, out=y256, workspace=ws_1),
-                                          ivc.ps_project(x, 0.25, m2, out=y64, workspace=ws_2))),
-    }
-    del ws_r, ws_1, ws_2, y256, y64
+    peaks, src = load_peaks()
+    parts = {}
+    if P.flash:
+        # ---- the two halves of the step alone (CUDA graphs, L2 flushed): the
+        # router (ivc_vir_route) and the connector (both ivc_ps_project calls)
+        ws_r = ivc.new_workspace(ivc.workspace_size(ivc.OP_VIR_ROUTE, T, w.C, r=P.r), dev)
+        y256 = torch.empty(T * 256, w.H, dtype=torch.bfloat16, device=dev)
+        y64 = torch.empty(T * 64, w.H, dtype=torch.bfloat16, device=dev)
+        ws_1 = ivc.new_workspace(ivc.workspace_size(ivc.OP_PS_HALF, T, w.C, P.m1), dev)
+        ws_2 = ivc.new_workspace(ivc.workspace_size(ivc.OP_PS_QUARTER, T, w.C, P.m2), dev)
+        parts = {
+            "router_ms": graph_ms(lambda: ivc.vir_route(P.x, P.vl, P.offs, P.r, workspace=ws_r)),
+            "connector_ms": graph_ms(lambda: (ivc.ps_project(P.x, 0.5, P.m1, out=y256, workspace=ws_1),
+                                              ivc.ps_project(P.x, 0.25, P.m2, out=y64,
+                                                             workspace=ws_2))),
+        }
+        del ws_r, ws_1, ws_2, y256, y64
 
     # ---- traced pass: per-kernel device time of the same steps (eager launches)
     n_trace = min(args.steps, 50)
@@ -386,31 +534,31 @@ def run_ivc(args):
     per_step_ms = {k: v["ms"] / n_trace for k, v in trace.items()}
     trace_total = sum(per_step_ms.values())
     alg = algorithmic(w, T)
-    # dominant kernel: the connector contraction with the largest traced
-    # time. (Inside the step the router's launches wait for SMs the GEMMs
-    # hold, so their traced times include that wait; by device time in the
-    # ncu launch list the connector GEMMs dominate.) The HBM-bound kernels
-    # are reported on their own below.
-    gemm_roles = ("mlp1.fc1", "mlp1.fc2", "mlp2.fc1", "mlp2.fc2", "mlp2.fc3")
-    dom = max((k for k in per_step_ms if k in gemm_roles), key=per_step_ms.get)
-    peaks, src = load_peaks()
-    fl, by = alg.get(dom, (0.0, 0.0))
-    per_launch_ms = trace[dom]["ms"] / trace[dom]["launches"]
-    launches_dom = trace[dom]["launches"] / n_trace
-    if fl / max(by, 1) > peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9):
-        ach = fl / launches_dom / (per_launch_ms / 1e3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": ach / peak, "traffic": kernel_traffic(dom),
-                "kernel": dom, "peak_source": f"{src} bf16_tflops_sustained"}
-    else:
-        ach = by / launches_dom / (per_launch_ms / 1e3) / 1e9
-        peak = peaks["hbm_gbs"]
-        roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
-                "traffic": kernel_traffic(dom), "kernel": dom, "peak_source": f"{src} hbm_gbs"}
+    burst = peaks["bf16_tflops"]
+    sustained = peaks.get("bf16_tflops_sustained", burst)
+    # every connector Linear against the dense bf16 peak: the burst figure,
+    # since each runs for well under a second inside a short step
+    gemm = {}
+    for k in connector_roles(w):
+        if k in trace and trace[k]["launches"] > 0:
+            us = 1e3 * trace[k]["ms"] / trace[k]["launches"]
+            fl = alg[k][0] / (trace[k]["launches"] / n_trace)
+            tf = fl / (us * 1e-6) / 1e12
+            gemm[k] = {"gflop_per_launch": fl / 1e9, "us_per_launch": us, "tflops": tf,
+                       "frac": tf / burst, "frac_vs_sustained": tf / sustained}
+    # dominant kernel: the connector contraction with the largest traced time.
+    # (Inside the step the router's launches wait for SMs the GEMMs hold, so
+    # their traced times include that wait; by device time in the ncu launch
+    # list the connector GEMMs dominate.) The HBM-bound kernels are reported
+    # on their own below.
+    dom = max(gemm, key=lambda k: per_step_ms[k])
+    roof = {"bound": "tensor", "achieved": gemm[dom]["tflops"], "peak": burst, "unit": "TFLOP/s",
+            "frac": gemm[dom]["frac"], "traffic": kernel_traffic(dom, w.name), "kernel": dom,
+            "peak_source": f"{src} bf16_tflops (burst)",
+            "frac_vs_sustained": gemm[dom]["frac_vs_sustained"]}
     # the HBM-bound kernels: algorithmic bytes per launch / traced launch time
     hbm = {}
-    kept_rows = int(bufs["offsets"][-1].item())  # 256 (T - k) + 64 k of this image
+    kept_rows = int(P.bufs["offsets"][-1].item()) if P.flash else T * 256
     for k in ("ps_stats", "compact", "pool.attend"):
         if k in trace and trace[k]["launches"] > 0:
             us = 1e3 * trace[k]["ms"] / trace[k]["launches"]
@@ -420,19 +568,32 @@ def run_ivc(args):
             gbs = b_launch / (us * 1e-6) / 1e9
             hbm[k] = {"bytes_per_launch": b_launch, "us_per_launch": us, "achieved": gbs,
                       "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"]}
+    router_roof = None
+    if P.flash and not routed:
+        rb = router_bytes(w, T)
+        gbs = rb / (parts["router_ms"] * 1e-3) / 1e9
+        router_roof = {"bound": "hbm", "bytes": rb, "us": parts["router_ms"] * 1e3,
+                       "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                       "frac": gbs / peaks["hbm_gbs"],
+                       "note": "ivc_vir_route alone (CUDA graph, L2 flushed); bytes = x once + "
+                               "pooling and gating weights once"}
     # whole-step roofline: algorithmic FLOPs at the dense bf16 peak vs bytes at HBM peak.
-    # F_literal counts the method as the pages state it (K/V projections of all
-    # tokens); F_folded is what the folded pooling actually has to compute.
-    conn = sum(alg[k][0] for k in ("mlp1.fc1", "mlp1.fc2", "mlp2.fc1", "mlp2.fc2", "mlp2.fc3"))
-    gate_f = 2.0 * T * (8 * w.D * w.gate_hidden + 2 * w.D)
-    F = conn + alg["pool.kv"][0] + alg["pool.attention"][0] + gate_f + 2.0 * T * 8 * w.D * w.D
-    F_folded = (conn + alg["pool.scores"][0] + alg["pool.wsum"][0] + gate_f +
-                2.0 * T * 16 * w.D * w.D)
-    B_alg = 2 * (T * 1024 * w.C) + 2 * (4 * w.C * w.H + w.H * w.H + 16 * w.C * w.mlp2_mid +
-                                        w.mlp2_mid * w.H + w.H * w.H + 16 * w.D * w.D +
-                                        8 * w.D * w.gate_hidden) + 2 * T * 256 * w.H
-    t_roof = max(F / (peaks["bf16_tflops"] * 1e12), B_alg / (peaks["hbm_gbs"] * 1e9))
-    t_roof_f = max(F_folded / (peaks["bf16_tflops"] * 1e12), B_alg / (peaks["hbm_gbs"] * 1e9))
+    conn = sum(alg[k][0] for k in connector_roles(w))
+    if P.flash:
+        # F_literal counts the method as the pages state it (K/V projections
+        # of all tokens); F_folded is what the folded pooling has to compute.
+        gate_f = 2.0 * T * (8 * w.D * w.gate_hidden + 2 * w.D)
+        F = conn + alg["pool.kv"][0] + alg["pool.attention"][0] + gate_f + 2.0 * T * 8 * w.D * w.D
+        F_folded = (conn + alg["pool.scores"][0] + alg["pool.wsum"][0] + gate_f +
+                    2.0 * T * 16 * w.D * w.D)
+        B_alg = 2 * (T * 1024 * w.C) + 2 * (4 * w.C * w.H + w.H * w.H + 16 * w.C * w.mlp2_mid +
+                                            w.mlp2_mid * w.H + w.H * w.H + 16 * w.D * w.D +
+                                            8 * w.D * w.gate_hidden) + 2 * T * 256 * w.H
+    else:
+        F = F_folded = conn
+        B_alg = 2 * (T * 1024 * w.C) + 2 * (4 * w.C * w.H + w.H * w.H) + 2 * T * 256 * w.H
+    t_roof = max(F / (burst * 1e12), B_alg / (peaks["hbm_gbs"] * 1e9))
+    t_roof_f = max(F_folded / (burst * 1e12), B_alg / (peaks["hbm_gbs"] * 1e9))
     meas = total_ms / args.steps / 1e3
     step_roofline = {"flops_literal": F, "flops_folded": F_folded, "bytes": B_alg,
                      "roofline_us_literal": t_roof * 1e6, "roofline_us_folded": t_roof_f * 1e6,
@@ -441,102 +602,20 @@ def run_ivc(args):
                      "peak_source": f"{src} bf16_tflops (burst), hbm_gbs"}
     if routed:
         # router-first: only the selected path of each tile is computed
-        k = int(bufs["mask"].sum().item())
+        k = int(P.bufs["mask"].sum().item())
         m1f = (alg["mlp1.fc1"][0] + alg["mlp1.fc2"][0]) * (T - k) / T
         m2f = (alg["mlp2.fc1"][0] + alg["mlp2.fc2"][0] + alg["mlp2.fc3"][0]) * k / T
         F_routed = F_folded - conn + m1f + m2f
         B_routed = B_alg - 2 * T * 256 * w.H + 2 * (256 * (T - k) + 64 * k) * w.H
-        t_roof_r = max(F_routed / (peaks["bf16_tflops"] * 1e12), B_routed / (peaks["hbm_gbs"] * 1e9))
+        t_roof_r = max(F_routed / (burst * 1e12), B_routed / (peaks["hbm_gbs"] * 1e9))
         step_roofline.update({"compressed_tiles": k, "flops_routed": F_routed,
                               "bytes_routed": B_routed, "roofline_us_routed": t_roof_r * 1e6,
                               "frac_vs_routed": t_roof_r / meas})
 
-    # ---- end to end through the public API with host buffers
-    e2e_steps = min(args.steps, 100)
-    hx = inp["x"].pin_memory()
-    hvl = inp["valid_len"].pin_memory()
-    hoffs = inp["image_offsets"].pin_memory()
-    hout = torch.empty(T * 256, w.H, dtype=torch.bfloat16).pin_memory()
-    hsmall = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in bufs.items()}
-    h2d = hx.numel() * 2 + hvl.numel() * 4 + hoffs.numel() * 4
-    d2h_small = sum(v.numel() * v.element_size() for v in bufs.values())
-    d2h_rows = 0
-    torch.cuda.synchronize()
-    barrier()
-    t0 = time.perf_counter()
-    for _ in range(e2e_steps):
-        x.copy_(hx, non_blocking=True)
-        vl.copy_(hvl, non_blocking=True)
-        offs.copy_(hoffs, non_blocking=True)
-        run()
-        for k in bufs:
-            hsmall[k].copy_(bufs[k], non_blocking=True)
-        torch.cuda.current_stream().synchronize()
-        rows = int(hsmall["total"][0])
-        hout[:rows].copy_(out[:rows], non_blocking=True)
-        torch.cuda.current_stream().synchronize()
-        d2h_rows += rows * w.H * 2
-    e2e_s = reduce_max(time.perf_counter() - t0, world, dev)
-    e2e_sync = {"value": world * T * e2e_steps / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h_small + d2h_rows // e2e_steps, "steps": e2e_steps,
-                "timing": "wall clock, host sync per step (the row count read before the row copy)"}
+    e2e = run_e2e(args, P, run, world, dev, barrier)
 
-    # ---- the same, pipelined as a streaming user would: three buffer sets
-    # on three streams (each a CUDA graph of the call), so that one step's
-    # host-to-device copies overlap the others' compute and copies back. The
-    # whole row capacity is copied back, so no host sync is needed per step.
-    n_sets = 3
-    sets = []
-    for _ in range(n_sets):
-        st = torch.cuda.Stream(device=dev)
-        e = {"st": st, "x": torch.empty_like(x), "vl": torch.empty_like(vl),
-             "offs": torch.empty_like(offs), "out": torch.empty_like(out),
-             "bufs": {k: torch.empty_like(v) for k, v in bufs.items()},
-             "ws": ivc.new_workspace(ws.numel(), dev),
-             "hout": torch.empty(T * 256, w.H, dtype=torch.bfloat16).pin_memory(),
-             "hsmall": {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in bufs.items()}}
-        st.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(st):
-            e["x"].copy_(x)
-            e["vl"].copy_(vl)
-            e["offs"].copy_(offs)
-            for _ in range(2):
-                ivc.flash_compress(e["x"], e["vl"], e["offs"], m1, m2, r, out=e["out"],
-                                   workspace=e["ws"], bufs=e["bufs"], routed=routed)
-        st.synchronize()
-        e["g"] = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(e["g"], stream=st):
-            ivc.flash_compress(e["x"], e["vl"], e["offs"], m1, m2, r, out=e["out"],
-                               workspace=e["ws"], bufs=e["bufs"], routed=routed)
-        sets.append(e)
-    torch.cuda.synchronize()
-    barrier()
-    t0 = time.perf_counter()
-    for i in range(e2e_steps):
-        e = sets[i % n_sets]
-        with torch.cuda.stream(e["st"]):
-            e["x"].copy_(hx, non_blocking=True)
-            e["vl"].copy_(hvl, non_blocking=True)
-            e["offs"].copy_(hoffs, non_blocking=True)
-            e["g"].replay()
-            for k in bufs:
-                e["hsmall"][k].copy_(e["bufs"][k], non_blocking=True)
-            e["hout"].copy_(e["out"], non_blocking=True)
-    torch.cuda.synchronize()
-    e2e_p = reduce_max(time.perf_counter() - t0, world, dev)
-    last = sets[(e2e_steps - 1) % n_sets]
-    if int(last["hsmall"]["total"][0]) != int(bufs["total"].item()):
-        raise RuntimeError("pipelined end-to-end run returned a different row count")
-    e2e = {"value": world * T * e2e_steps / e2e_p, "unit": UNIT, "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h_small + T * 256 * w.H * 2, "steps": e2e_steps,
-           "timing": f"wall clock over all steps; {n_sets} streams, inputs copied in and "
-                     "results (small outputs and the whole row capacity) copied out every step",
-           "synchronous": e2e_sync}
-    for e in sets:
-        del e["g"]
-    sets = None
-
-    fn_name = "ivc_flash_compress_routed" if routed else "ivc_flash_compress"
+    fn_name = ("ivc_flash_compress_routed" if routed else "ivc_flash_compress") if P.flash \
+        else "ivc_ps_project (factor 0.5)"
     launch_desc = (f"CUDA graph of one {fn_name}" if graph is not None else f"eager {fn_name}")
     run = None
     graph = None
@@ -546,28 +625,127 @@ def run_ivc(args):
         dist.destroy_process_group()
     if rank != 0:
         return 0
+    config = {"workload": w.name, "tiles_per_step": T, "C": w.C, "H": w.H}
+    if P.flash:
+        config.update({"mlp2_mid": w.mlp2_mid, "pool_heads": w.D // 64,
+                       "gate_hidden": w.gate_hidden, "images": int(inp["image_offsets"].numel() - 1),
+                       "flow": ("router first, each tile through its selected path" if routed
+                                else "both paths for every tile, then compaction")})
+    else:
+        config["flow"] = "pixel_shuffle 0.5 + mlp1 (LayerNorm, Linear, GELU, Linear)"
+    config.update({"l2": "flushed between steps (512 MiB write, outside the timed events)",
+                   "launch": launch_desc,
+                   "parallelism": f"replicas x{world}, one batch per GPU, no collective"})
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "tiles_per_step": T, "C": w.C, "H": w.H,
-                       "mlp2_mid": w.mlp2_mid, "pool_heads": 16, "gate_hidden": w.gate_hidden,
-                       "l2": "flushed between steps (512 MiB write, outside the timed events)",
-                       "launch": launch_desc,
-                       "flow": ("router first, each tile through its selected path" if routed
-                                else "both paths for every tile, then compaction"),
-                       "parallelism": f"replicas x{world}, one image per GPU, no collective"},
-            "roofline": roof, "step_roofline": step_roofline, "hbm_kernels": hbm,
-            "kernels_ms_per_step": {k: round(v, 5) for k, v in per_step_ms.items()},
-            "traced_ms_per_step": trace_total, "parts_graph_ms": parts,
-            "clocks": clocks, "e2e": e2e, "gpu_launches": int(round(launches_per_step * args.steps)),
-            "wall_s_timed": t_wall}
+            "config": config, "roofline": roof, "gemm": gemm, "step_roofline": step_roofline,
+            "hbm_kernels": hbm, "kernels_ms_per_step": {k: round(v, 5) for k, v in per_step_ms.items()},
+            "traced_ms_per_step": trace_total, "clocks": clocks, "e2e": e2e,
+            "gpu_launches": int(round(launches_per_step * args.steps)), "wall_s_timed": t_wall}
+    if parts:
+        line["parts_graph_ms"] = parts
+    if router_roof:
+        line["router_roofline"] = router_roof
     if world == 1 and not args.no_cpu_baseline:
-        import oracle as O
-        inp["_m1_64"], inp["_m2_64"], inp["_r_64"] = (O.to64(inp["mlp1"]), O.to64(inp["mlp2"]),
-                                                       O.to64(inp["router"]))
         line["cpu_baseline"] = cpu_baseline(inp)
     print(json.dumps(line), flush=True)
     return 0
+
+
+def run_e2e(args, P, run, world, dev, barrier):
+    """The same metric end to end through the public API with host buffers:
+    every step copies its inputs in from pinned host memory and its results
+    out. First with a host sync per step, then pipelined over buffer sets on
+    their own streams, as a streaming user would run it."""
+    import torch
+    w, T, ivc = P.w, P.T, P.ivc
+    host_in = {k: v.cpu().pin_memory() for k, v in P.inputs().items()}
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    out_bytes = T * 256 * w.H * 2
+    small_bytes = sum(v.numel() * v.element_size() for v in P.bufs.values())
+    big = h2d + out_bytes > (1 << 30)
+    e2e_steps = min(args.steps, 10 if big else 100)
+    n_sets = 2 if big else 3
+    hout = torch.empty(T * 256, w.H, dtype=torch.bfloat16).pin_memory()
+    hsmall = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in P.bufs.items()}
+    d2h_rows = 0
+    dev_in = P.inputs()
+    torch.cuda.synchronize()
+    barrier()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        for k, v in dev_in.items():
+            v.copy_(host_in[k], non_blocking=True)
+        run()
+        if P.flash:
+            for k in P.bufs:
+                hsmall[k].copy_(P.bufs[k], non_blocking=True)
+            torch.cuda.current_stream().synchronize()
+            rows = int(hsmall["total"][0])
+        else:
+            rows = T * 256
+        hout[:rows].copy_(P.out[:rows], non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        d2h_rows += rows * w.H * 2
+    e2e_s = reduce_max(time.perf_counter() - t0, world, dev)
+    e2e_sync = {"value": world * T * e2e_steps / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": small_bytes + d2h_rows // e2e_steps, "steps": e2e_steps,
+                "timing": "wall clock, host sync per step" +
+                          (" (the row count read before the row copy)" if P.flash else "")}
+    del hout
+
+    sets = []
+    for i in range(n_sets):
+        st = torch.cuda.Stream(device=dev)
+        e = {"st": st, "in": {k: torch.empty_like(v) for k, v in dev_in.items()},
+             "out": torch.empty_like(P.out),
+             "bufs": {k: torch.empty_like(v) for k, v in P.bufs.items()},
+             "ws": ivc.new_workspace(P.ws.numel(), dev),
+             "hout": torch.empty(T * 256, w.H, dtype=torch.bfloat16).pin_memory(),
+             "hsmall": {k: torch.empty(v.shape, dtype=v.dtype).pin_memory()
+                        for k, v in P.bufs.items()}}
+        st.wait_stream(torch.cuda.current_stream())
+
+        def call(e=e):
+            P.call(x=e["in"]["x"], vl=e["in"].get("vl"), offs=e["in"].get("offs"), out=e["out"],
+                   ws=e["ws"], bufs=e["bufs"])
+        with torch.cuda.stream(st):
+            for k, v in dev_in.items():
+                e["in"][k].copy_(v)
+            for _ in range(2):
+                call()
+        st.synchronize()
+        e["g"] = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(e["g"], stream=st):
+            call()
+        sets.append(e)
+    torch.cuda.synchronize()
+    barrier()
+    t0 = time.perf_counter()
+    for i in range(e2e_steps):
+        e = sets[i % n_sets]
+        with torch.cuda.stream(e["st"]):
+            for k, v in e["in"].items():
+                v.copy_(host_in[k], non_blocking=True)
+            e["g"].replay()
+            for k in P.bufs:
+                e["hsmall"][k].copy_(e["bufs"][k], non_blocking=True)
+            e["hout"].copy_(e["out"], non_blocking=True)
+    torch.cuda.synchronize()
+    e2e_p = reduce_max(time.perf_counter() - t0, world, dev)
+    if P.flash:
+        last = sets[(e2e_steps - 1) % n_sets]
+        if int(last["hsmall"]["total"][0]) != int(P.bufs["total"].item()):
+            raise RuntimeError("pipelined end-to-end run returned a different row count")
+    e2e = {"value": world * T * e2e_steps / e2e_p, "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": small_bytes + out_bytes, "steps": e2e_steps,
+           "timing": f"wall clock over all steps; {n_sets} streams, inputs copied in and "
+                     "results (small outputs and the whole row capacity) copied out every step",
+           "synchronous": e2e_sync}
+    for e in sets:
+        del e["g"]
+    return e2e
 
 
 def run_op(args):
@@ -577,8 +755,10 @@ def run_op(args):
 
     import vlm_visual_token_b200 as ivc
     torch.cuda.set_device(0)
-    inp = image_gen(0)
+    inp = image_gen(0, args.workload)
     w, T = inp["workload"], inp["T"]
+    if w.path != "flash" and args.op not in ("ps_half",):
+        raise SystemExit(f"--op {args.op} needs a flash workload; {w.name} has mlp1 only")
     x = inp["x"].cuda()
     vl, offs = inp["valid_len"].cuda(), inp["image_offsets"].cuda()
     if args.op == "assemble":
@@ -625,7 +805,7 @@ def run_op(args):
     b.record()
     b.synchronize()
     ms = a.elapsed_time(b) / args.steps
-    line = {"op": args.op, "workload": WORKLOAD, "tiles": T, "ms_per_call": ms,
+    line = {"op": args.op, "workload": w.name, "tiles": T, "ms_per_call": ms,
             "tiles_per_s": T / (ms / 1e3), "timing": "CUDA graph, back to back, no L2 flush"}
     if args.op == "assemble":
         n = int(aout["seq_offsets"][-1].item())
@@ -655,6 +835,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ivc", "reference"], default="ivc")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=WORKLOAD_NAMES, default=DEFAULT_WORKLOAD,
+                    help="configuration to run (default: the 13-tile 2B-Flash image)")
     ap.add_argument("--flow", choices=["dual", "routed"], default="dual",
                     help="dual: ivc_flash_compress (both paths, then compaction); "
                          "routed: ivc_flash_compress_routed (router first)")
@@ -671,6 +853,8 @@ def main(argv=None):
         return run_reference(args)
     if args.op != "flash":
         return run_op(args)
+    if args.flow == "routed" and args.workload not in WORKLOAD_NAMES[1:3]:
+        ap.error("--flow routed needs a flash workload")
     return run_ivc(args)
 
 

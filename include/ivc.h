@@ -199,6 +199,7 @@ int ivc_ps_project(const void* x, int T, int C, float scale, int flags, const iv
  *   mask           device uint8 [T]: 1 = compressed (64 rows), 0 = 256 rows.
  *   offsets        device int32 [T+1]: exclusive scan of the row counts;
  *                  offsets[T] = total rows = 256 (T - k) + 64 k.
+ * rel_q outside [0, 1] (or NaN) is IVC_EINVAL.
  * Unsupported: D != C, D % 256 != 0, heads * 64 != D, gate_hidden % 256 != 0.
  * With folded pooling, D <= 1024 and at most 16 heads, the router runs as one
  * cooperative persistent kernel that holds every SM until it ends (the
@@ -207,6 +208,29 @@ int ivc_vir_route(const void* x, const int32_t* valid_len, int T, int C,
                   const int32_t* image_offsets, int I, const ivc_router* r, float* gate,
                   uint8_t* mask, int32_t* offsets, void* workspace, size_t ws_bytes,
                   ivc_stream_t stream);
+
+/* Routing alone ([VIR] section 4; [DP] "路由决策：相对 + 绝对双阈值判定"): the
+ * double threshold and the row-count scan that end ivc_vir_route, applied to
+ * a gate vector the caller supplies (for instance gates computed by another
+ * implementation of the router). Tile t is compressed iff
+ * gate[t,0] > quantile(gate[.,0] over its group, rel_q) and gate[t,0] >= abs_t,
+ * the quantile by linear interpolation in fp64, each operation rounded on its
+ * own. As with torch.quantile, a NaN gate makes its group's quantile NaN, so
+ * no tile of that group is compressed.
+ *   gate           device fp32 [T, 2]; only column 0 is read.
+ *   image_offsets  device int32 [I+1] as in ivc_vir_route (scope 0); may be
+ *                  NULL for scope 1 (one group: the whole batch).
+ *   rel_q          in [0, 1], else IVC_EINVAL; abs_t any value.
+ *   mask, offsets  as in ivc_vir_route; total: device int32 [1] or NULL.
+ *   workspace      >= IVC_ROUTE_WORKSPACE_BYTES (the device status word),
+ *                  256-byte aligned. Bad image offsets set IVC_DEV_BAD_OFFSETS
+ *                  (nothing compressed); a group above IVC_MAX_QUANTILE_GROUP
+ *                  tiles sets IVC_DEV_GROUP_TOO_LARGE (that group uncompressed).
+ * One CTA; T == 0 writes offsets[0] = 0 (and *total = 0). */
+#define IVC_ROUTE_WORKSPACE_BYTES 256u
+int ivc_route(const float* gate, int T, const int32_t* image_offsets, int I, double rel_q,
+              double abs_t, int scope, uint8_t* mask, int32_t* offsets, int32_t* total,
+              void* workspace, size_t ws_bytes, ivc_stream_t stream);
 
 /* The Flash dual path ([DP] "双路压缩管线全流程拆解"; [VIR] section 5):
  * ivc_ps_project at 0.5 with mlp1 and at 0.25 with mlp2, ivc_vir_route, then
@@ -289,7 +313,10 @@ int ivc_device_status(void* workspace, int* bits, ivc_stream_t stream);
  *   ivc_workspace_size of the same op) return IVC_EWORKSPACE and enqueue
  *   nothing: e.g. up to 15 tiles of mlp1 4096->2048->2048 fit.
  *   The first call on a device looks up the array's device address (with that
- *   device current); make that first call before any stream capture.
+ *   device current); make that first call before any stream capture. The
+ *   address is looked up again when the device's current context changes
+ *   (e.g. after cudaDeviceReset); the first call after such a change must
+ *   also come before any capture.
  *   All calls share the one array and it keeps the last call's contents:
  *   calls whose GPU work can overlap (other streams, other host threads on
  *   the same device) race on it. The device status word inside the array is

@@ -139,3 +139,36 @@ def test_flash_entry_points_reject_bad_arguments(name):
     assert call(out=ctypes.c_void_p((1 << 26) + 4)) == -6
     assert call(nbytes=64) == -3
     assert call(xx=ctypes.c_void_p((1 << 24) + 2)) == -6
+
+
+def test_route_rejects_bad_arguments_without_touching_the_gpu():
+    """ivc_route (the double threshold on a given gate vector) checks its
+    arguments on the host; rel_q outside [0, 1] would index past the sorted
+    gates, so it is refused, for ivc_vir_route too."""
+    import vlm_visual_token_b200 as ivc
+    L = ivc.lib()
+    g = ctypes.c_void_p(1 << 24)
+    o = ctypes.c_void_p(1 << 25)
+    m = ctypes.c_void_p(1 << 26)
+    ws = ctypes.c_void_p(1 << 20)
+
+    def call(T=4, offs=o, I=1, rel_q=0.1, scope=0, mask=m, offsets=o, ws=ws, nbytes=256):
+        return L.ivc_route(g, T, offs, I, rel_q, 0.5, scope, mask, offsets, None, ws, nbytes, None)
+
+    assert call(rel_q=1.5) == -1
+    assert call(rel_q=-0.1) == -1
+    assert call(rel_q=float("nan")) == -1
+    assert call(scope=2) == -1
+    assert call(T=-1) == -1
+    assert call(offsets=None) == -1
+    assert call(mask=None) == -1
+    assert call(offs=None) == -1                 # per-image scope needs the offsets
+    assert call(nbytes=128) == -3                # the status word needs 256 bytes
+    assert call(ws=ctypes.c_void_p((1 << 20) + 64)) == -6
+    r = ivc._CRouter()
+    r.D, r.heads, r.gate_hidden = 1024, 16, 1024
+    r.rel_q = 2.0
+    x = ctypes.c_void_p(1 << 24)
+    y = ctypes.c_void_p(1 << 26)
+    assert L.ivc_vir_route(x, None, 1, 1024, x, 1, ctypes.byref(r), y, y, y, ws, 1 << 40,
+                           None) == -1

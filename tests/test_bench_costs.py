@@ -53,3 +53,46 @@ def test_single_pass_attention_counts_both_contractions_and_one_read_of_x():
     # four layers, each reading x once (the tensor-core form reads it twice)
     assert 4 * x_per_layer < alg["pool.attend"][1] < 4 * x_per_layer * 1.1
     assert alg["pool.scores"][1] + alg["pool.wsum"][1] > 8 * x_per_layer
+
+
+def test_router_bytes_are_features_and_weights_once():
+    w = W.WORKLOADS["flash_2b_13tiles"]
+    x = T * 1024 * C * 2
+    pool_w = 2 * 4 * 4 * D * D        # Wq, Wk, Wv, Wo of 4 layers, bf16
+    gate_w = 2 * 4 * 2 * D * 1024     # W1 and W2 of 4 gating blocks, bf16
+    b = bench.router_bytes(w, T)
+    assert x + pool_w + gate_w < b < (x + pool_w + gate_w) * 1.01
+    assert abs(b - 77.7e6) < 0.2e6    # 27.3 MB of features + 33.5 + 16.8 MB of weights
+
+
+def test_clock_summary_separates_the_timed_window():
+    lines = [
+        "2026/12/03 10:00:00.000, 0, 1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "2026/12/03 10:00:00.500, 0, 1950, 1965, 900.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "2026/12/03 10:00:01.000, 0, 1965, 1965, 650.5, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+    ]
+    rows = bench.ClockSampler.parse(lines)
+    assert len(rows) == 3
+    t0, t1 = rows[0][0], rows[2][0]
+    s = bench.ClockSampler.summarise(rows, t0, t1)
+    assert s["samples"] == 3 and s["sm_mhz"] == 1965 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"] and s["power_w_max"] == 900.0
+    assert bench.ClockSampler.summarise(rows, t1 + 10, t1 + 20)["reasons"] == ["unsampled"]
+
+
+def test_cpu_sample_plans():
+    """Whole images (routing couples an image's tiles) on the flash
+    workloads, 8 seeded tiles of the large connector batches."""
+    import torch
+    w2 = W.WORKLOADS["flash_2b_13tiles"]
+    inp = {"workload": w2, "T": 13, "image_offsets": torch.tensor([0, 13], dtype=torch.int32)}
+    assert bench.cpu_sample_plan(inp) == ("images", 1)
+    w3 = W.WORKLOADS["flash_4b_batched"]
+    offs = torch.tensor([0, 3, 5, 12, 20, 31, 40, 41, 50, 60, 70, 80, 90, 97, 100, 105, 110],
+                        dtype=torch.int32)
+    kind, n = bench.cpu_sample_plan({"workload": w3, "T": 110, "image_offsets": offs})
+    assert kind == "images" and offs[n] >= 8 and offs[n - 1] < 8
+    w4 = W.WORKLOADS["connector_14b_832tiles"]
+    kind, tiles = bench.cpu_sample_plan({"workload": w4, "T": 832})
+    assert kind == "tiles" and len(tiles) == 8 and len(set(tiles)) == 8 and max(tiles) < 832

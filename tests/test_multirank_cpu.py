@@ -24,7 +24,7 @@ def _worker(rank, world, port, q):
     r, w, lr = bench.dist_env()
     got = bench.reduce_max(float(10 * (rank + 1)), w)
     import workloads as W
-    wl = W.WORKLOADS[bench.WORKLOAD]
+    wl = W.WORKLOADS[bench.DEFAULT_WORKLOAD]
     offs, valid = W.layout(wl, seed=777 + wl.seed_base + 1000 * rank)
     x = W.features(1, 8, 1234 + wl.seed_base + 1000 * rank)
     q.put((r, w, got, int(offs[-1]), float(x.float().sum())))

@@ -6,6 +6,7 @@ functions keep the C names without the ``ivc_`` prefix:
 
     ps_project(x, scale, mlp, flags=0)           -> y [T*tokens, H] bf16
     vir_route(x, valid_len, image_offsets, r)    -> gate, mask, offsets
+    route(gate, image_offsets)                   -> mask, offsets, total
     flash_compress(x, valid_len, image_offsets, mlp1, mlp2, r) -> dict
 
 Importing this module fails loudly when the shared library is missing; there
@@ -22,7 +23,8 @@ import torch
 
 POOL_FOLDED, POOL_LITERAL = 0, 1
 
-__all__ = ["Mlp", "Router", "POOL_FOLDED", "POOL_LITERAL", "ps_project", "vir_route", "flash_compress", "assemble_sequence", "workspace_size",
+__all__ = ["Mlp", "Router", "POOL_FOLDED", "POOL_LITERAL", "ps_project", "vir_route", "route",
+           "flash_compress", "assemble_sequence", "workspace_size",
            "device_status", "IvcError", "lib", "LIB_PATH", "PS_V1", "PS_QUARTER_TWICE",
            "OP_PS_HALF", "OP_PS_QUARTER", "OP_VIR_ROUTE", "OP_FLASH"]
 
@@ -88,6 +90,10 @@ def lib() -> ctypes.CDLL:
         L.ivc_vir_route.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, _vp, ctypes.c_int,
                                     ctypes.POINTER(_CRouter), _vp, _vp, _vp, _vp, ctypes.c_size_t,
                                     _vp]
+        L.ivc_route.restype = ctypes.c_int
+        L.ivc_route.argtypes = [_vp, ctypes.c_int, _vp, ctypes.c_int, ctypes.c_double,
+                                ctypes.c_double, ctypes.c_int, _vp, _vp, _vp, _vp, ctypes.c_size_t,
+                                _vp]
         L.ivc_flash_compress.restype = ctypes.c_int
         L.ivc_flash_compress.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, _vp, ctypes.c_int,
                                          ctypes.POINTER(_CMlp), ctypes.POINTER(_CMlp),
@@ -246,6 +252,29 @@ def vir_route(x: torch.Tensor, valid_len: Optional[torch.Tensor], image_offsets:
                                _ptr(workspace), workspace.numel(), _stream(stream)),
            "ivc_vir_route")
     return gate, mask, offsets
+
+
+ROUTE_WORKSPACE_BYTES = 256
+
+
+def route(gate: torch.Tensor, image_offsets: Optional[torch.Tensor], rel_q: float = 0.1,
+          abs_t: float = 0.5, scope: int = 0, workspace: Optional[torch.Tensor] = None,
+          stream=None):
+    """ivc_route: the double threshold and row offsets for a given fp32 gate
+    [T, 2]. Returns mask [T] uint8, offsets [T+1] int32, total [1] int32."""
+    T = int(gate.shape[0])
+    dev = gate.device
+    mask = torch.empty(T, dtype=torch.uint8, device=dev)
+    offsets = torch.empty(T + 1, dtype=torch.int32, device=dev)
+    total = torch.empty(1, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = new_workspace(ROUTE_WORKSPACE_BYTES, dev)
+    I = int(image_offsets.numel()) - 1 if image_offsets is not None else 0
+    _check(lib().ivc_route(_ptr(gate), T, _ptr(image_offsets), I, float(rel_q), float(abs_t),
+                           int(scope), _ptr(mask), _ptr(offsets), _ptr(total), _ptr(workspace),
+                           workspace.numel(), _stream(stream)),
+           "ivc_route")
+    return mask, offsets, total
 
 
 def flash_compress(x: torch.Tensor, valid_len: Optional[torch.Tensor], image_offsets: torch.Tensor,

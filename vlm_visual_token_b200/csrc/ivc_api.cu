@@ -65,6 +65,7 @@ int router_shape_ok(const ivc_router* r, int C) {
   }
   if (!d_ok || !g_ok) return IVC_EUNSUPPORTED;
   if (r->quantile_scope != 0 && r->quantile_scope != 1) return IVC_EINVAL;
+  if (!(r->rel_q >= 0.0 && r->rel_q <= 1.0)) return IVC_EINVAL;  // also NaN
   if (r->pool_mode != IVC_POOL_FOLDED && r->pool_mode != IVC_POOL_LITERAL) return IVC_EINVAL;
   if (r->gate_residual != 0 && r->gate_residual != 1) return IVC_EINVAL;
   if (r->pool_mode == IVC_POOL_FOLDED && (r->heads > 16 || r->D % 128 != 0))
@@ -644,6 +645,23 @@ int ivc_vir_route(const void* x, const int32_t* valid_len, int T, int C,
   carve_route(cv, r, T, b);
   return route_impl(x, valid_len, T, image_offsets, I, r, gate, mask, offsets, nullptr, b, L,
                     true);
+}
+
+int ivc_route(const float* gate, int T, const int32_t* image_offsets, int I, double rel_q,
+              double abs_t, int scope, uint8_t* mask, int32_t* offsets, int32_t* total,
+              void* workspace, size_t ws_bytes, ivc_stream_t stream) {
+  if (T < 0 || I < 0 || (scope != 0 && scope != 1)) return IVC_EINVAL;
+  if (!(rel_q >= 0.0 && rel_q <= 1.0)) return IVC_EINVAL;
+  if (!offsets || (T > 0 && (!gate || !mask))) return IVC_EINVAL;
+  if (T > 0 && scope == 0 && !image_offsets) return IVC_EINVAL;
+  IVC_TRY(check_ws(workspace, ws_bytes, IVC_ROUTE_WORKSPACE_BYTES));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    IVC_TRY(cu_check(cudaMemsetAsync(offsets, 0, sizeof(int32_t), s)));
+    return total ? cu_check(cudaMemsetAsync(total, 0, sizeof(int32_t), s)) : IVC_OK;
+  }
+  Launch L{s, static_cast<int*>(workspace)};
+  return launch_route(gate, T, image_offsets, I, rel_q, abs_t, scope, mask, offsets, total, L);
 }
 
 int ivc_flash_compress(const void* x, const int32_t* valid_len, int T, int C,

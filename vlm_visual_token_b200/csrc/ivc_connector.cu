@@ -13,6 +13,7 @@
 #include <cstdlib>
 #include <mutex>
 
+#include "ivc_device_once.h"
 #include "ivc_gemm.cuh"
 #include "ivc_internal.h"
 
@@ -269,16 +270,34 @@ static int map_ps(CUtensorMap* m, const void* x, int T, int C, int f, bool one_t
   return encode(m, 5, x, dims, strides, box);
 }
 
+static DeviceTable& device_table() {
+  static DeviceTable t;
+  return t;
+}
+
 int num_sms() {
-  static int n = 0;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    int dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+  static const char key = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  int n = device_table().get(&key, dev);
+  if (n > 0) return n;
+  int q = 0;
+  if (cudaDeviceGetAttribute(&q, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || q <= 0)
+    q = 148;
+  device_table().raise(&key, dev, q, [] { return 0; });
+  return q;
+}
+
+int smem_optin(const void* kern, size_t bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return IVC_ECUDA;
+  const int rc = device_table().raise(kern, dev, static_cast<int>(bytes), [&] {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(bytes)) == cudaSuccess
+               ? 0
+               : 1;
   });
-  return n;
+  return rc == 0 ? IVC_OK : IVC_ECUDA;
 }
 
 template <int BN, int STAGES, int CG>
@@ -286,13 +305,7 @@ static int run_gemm(const GemmMaps& maps, const GemmArgs& args, const char* tag,
                     const Launch& L) {
   using S = GemmSmem<BN, STAGES, CG>;
   auto kern = gemm_sm100_kernel<BN, STAGES, CG>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL) !=
-        cudaSuccess)
-      return IVC_ECUDA;
-    attr_set = true;
-  }
+  if (smem_optin(reinterpret_cast<const void*>(kern), S::TOTAL) != IVC_OK) return IVC_ECUDA;
   const long long tiles = static_cast<long long>((args.M + GEMM_BM * CG - 1) / (GEMM_BM * CG)) *
                           ((args.N + BN - 1) / BN) * args.groups;
   const long long units = units_cap;

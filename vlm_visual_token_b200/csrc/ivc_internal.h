@@ -210,6 +210,12 @@ int launch_route(const float* gate, int T, const int32_t* image_offsets, int I, 
 int launch_compact(const bf16* Y256, const bf16* Y64, const uint8_t* mask,
                    const int32_t* offsets, int T, int H, bf16* out, const Launch& L);
 
+// SMs of the current device (queried once per device).
 int num_sms();
+
+// Raises `kern`'s dynamic shared-memory limit to at least `bytes` on the
+// current device, once per (kernel, device) for the largest size asked so far
+// (ivc_device_once.h). IVC_OK, or IVC_ECUDA when the attribute call fails.
+int smem_optin(const void* kern, size_t bytes);
 
 }  // namespace ivc

@@ -14,6 +14,7 @@
 // array, not its device address: the address is obtained once per device,
 // with that device current, through cudaGetSymbolAddress and then passed to
 // the kernels like any workspace pointer.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -26,17 +27,41 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// The driver's current context (nullptr if it cannot be queried).
+CUcontext current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  CUcontext c = nullptr;
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
 // Device address of g_noalloc_scratch on `dev` (the current device), looked
-// up on the first call for that device. Returns nullptr on failure.
+// up on the first call for that device and again whenever the device's
+// current context has changed since (after cudaDeviceReset the array lives in
+// a new context, at an address that may differ). Returns nullptr on failure.
 void* scratch_address(int dev) {
   static std::mutex mu;
   static void* addr[kMaxDevices] = {};
+  static CUcontext ctx_of[kMaxDevices] = {};
   if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  const CUcontext ctx = current_context();
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+  if (addr[dev] == nullptr || ctx == nullptr || ctx != ctx_of[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
     addr[dev] = p;
+    ctx_of[dev] = ctx;
   }
   return addr[dev];
 }

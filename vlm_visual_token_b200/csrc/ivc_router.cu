@@ -223,14 +223,10 @@ static int dispatch_gemv(const XT* X, long long ldx, int M, int K, const bf16* W
   constexpr bool PAIRED = ROWS == GV_PAIRED;
   if (PAIRED && K > 1024) return IVC_EUNSUPPORTED;
   const int smem = static_cast<int>(GemvLayout<XT, ROWS>::total(K));
-  static bool attr = false;
-  if (!attr) {  // once, for the widest K this instantiation accepts
-    const int max_smem = static_cast<int>(GemvLayout<XT, ROWS>::total(PAIRED ? 1024 : 2048));
-    if (cudaFuncSetAttribute(gemv_kernel<XT, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             max_smem) != cudaSuccess)
-      return IVC_ECUDA;
-    attr = true;
-  }
+  // once per device, for the widest K this instantiation accepts
+  if (smem_optin(reinterpret_cast<const void*>(gemv_kernel<XT, ROWS>),
+                 GemvLayout<XT, ROWS>::total(PAIRED ? 1024 : 2048)) != IVC_OK)
+    return IVC_ECUDA;
   TraceScope ts(ROWS != GV_PLAIN ? "pool.vproj" : (gelu ? "router.gemv_gelu" : "router.gemv"),
                 L.stream);
   return launch_k(gemv_kernel<XT, ROWS>, dim3((N + GEMV_COLS - 1) / GEMV_COLS),
@@ -818,13 +814,8 @@ static int launch_attend_ks(const CUtensorMap& xmap, const bf16* U2, int u2_per_
                             const float* cb, int cb_stride, const int32_t* valid_len, int T,
                             int heads, float* Zp, float* mstat, float* lstat, const Launch& L) {
   const size_t smem = attend_smem_bytes(128 * KS);
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(pool_attend_kernel<KS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return IVC_ECUDA;
-    attr = true;
-  }
+  if (smem_optin(reinterpret_cast<const void*>(pool_attend_kernel<KS>), smem) != IVC_OK)
+    return IVC_ECUDA;
   return launch_k(pool_attend_kernel<KS>, dim3(T * ATTN_NCH), dim3(256), smem, L.stream, 1, xmap,
                   U2, u2_per_tile, cb, cb_stride, valid_len, heads, Zp, mstat, lstat, L.status);
 }
@@ -1028,20 +1019,30 @@ __global__ void __launch_bounds__(ROUTE_THREADS)
       __syncthreads();
       continue;
     }
-    for (int i = threadIdx.x; i < n; i += ROUTE_THREADS)
-      s_vals[i] = static_cast<double>(gate[2 * (s + i)]);
-    __syncthreads();
+    int my_nan = 0;
     for (int i = threadIdx.x; i < n; i += ROUTE_THREADS) {
-      const double v = s_vals[i];
-      int rank = 0;
-      for (int j = 0; j < n; ++j) {
-        const double u = s_vals[j];
-        rank += (u < v) || (u == v && j < i);
+      const double v = static_cast<double>(gate[2 * (s + i)]);
+      s_vals[i] = v;
+      my_nan |= isnan(v) ? 1 : 0;
+    }
+    // a NaN gate makes the group's quantile NaN (as torch.quantile does), so
+    // no tile of the group passes the strict > test; the rank sort, whose
+    // ranks assume a total order, is skipped
+    const int any_nan = __syncthreads_or(my_nan);
+    if (!any_nan) {
+      for (int i = threadIdx.x; i < n; i += ROUTE_THREADS) {
+        const double v = s_vals[i];
+        int rank = 0;
+        for (int j = 0; j < n; ++j) {
+          const double u = s_vals[j];
+          rank += (u < v) || (u == v && j < i);
+        }
+        s_sorted[rank] = v;
       }
-      s_sorted[rank] = v;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && any_nan) s_qv = __longlong_as_double(0x7ff8000000000000LL);
+    if (threadIdx.x == 0 && !any_nan) {
       const double pos = __dmul_rn(rel_q, static_cast<double>(n - 1));
       const double flo = floor(pos);
       const int lo = static_cast<int>(flo);
@@ -1103,13 +1104,7 @@ int launch_route(const float* gate, int T, const int32_t* image_offsets, int I, 
                  double abs_t, int scope, uint8_t* mask, int32_t* offsets, int32_t* total,
                  const Launch& L) {
   const size_t smem = 2 * IVC_MAX_QUANTILE_GROUP * sizeof(double);
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return IVC_ECUDA;
-    attr = true;
-  }
+  if (smem_optin(reinterpret_cast<const void*>(route_kernel), smem) != IVC_OK) return IVC_ECUDA;
   TraceScope ts("route", L.stream);
   return launch_k(route_kernel, dim3(1), dim3(ROUTE_THREADS), smem, L.stream, 1, gate, T,
                   image_offsets, I, rel_q, abs_t, scope, mask, offsets, total, L.status);

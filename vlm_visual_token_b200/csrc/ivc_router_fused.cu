@@ -181,10 +181,15 @@ __device__ __forceinline__ void gv_issue_w(const bf16* __restrict__ W, int K, in
     bulk_load(sw + lane * (K + 8), W + static_cast<size_t>(item * GV_COLS + lane) * K, K * 2, mb);
 }
 
+// `pend` tracks the bulk copies this CTA has in flight on mbarriers 0 and 1
+// (bits 0 and 1): bit 0 set on entry means the first item's weight rows were
+// requested before the grid barrier. A bit is set when copies are issued and
+// cleared only when their wait succeeds, so after a give-up (false) the
+// kernel's exit still waits for every copy that may land in shared memory.
 template <typename RowFn>
 __device__ bool gemv_phase(int M, int K, int N, const bf16* __restrict__ W,
                            const bf16* __restrict__ b, float* __restrict__ Y, int ldy, bool act,
-                           uint8_t* sm, uint64_t* mb, uint32_t* ph, bool w_prefetched, RowFn row) {
+                           uint8_t* sm, uint64_t* mb, uint32_t* ph, int& pend, RowFn row) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t2 = (lane & 3) * 2;
   const int pitch = K + 8;
@@ -193,14 +198,13 @@ __device__ bool gemv_phase(int M, int K, int N, const bf16* __restrict__ W,
   float* red = reinterpret_cast<float*>(sm + gv_x_bytes(K) + gv_w_bytes(K));
   const int n_items = N / GV_COLS;
   const int kw = K / RF_WARPS;
-  bool first = true;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     const int c0 = item * GV_COLS;
-    if (!(first && w_prefetched)) {
+    if (!(pend & 1)) {
       __syncthreads();  // the previous item's reads of the weight slot are done
       if (warp == 0) gv_issue_w(W, K, item, sm, &mb[0]);
+      pend |= 1;
     }
-    first = false;
     bool w_ready = false;
     for (int m0 = 0; m0 < M; m0 += GV_ROWS) {
       const int rows = min(GV_ROWS, M - m0);
@@ -213,13 +217,16 @@ __device__ bool gemv_phase(int M, int K, int N, const bf16* __restrict__ W,
           bulk_load(sx + lane * pitch, row(m0 + lane, c0), K * 4, &mb[1]);
         }
       }
+      pend |= 2;
       if (!w_ready) {
         if (!cta_wait(&mb[0], ph[0])) return false;
         ph[0] ^= 1;
+        pend &= ~1;
         w_ready = true;
       }
       if (!cta_wait(&mb[1], ph[1])) return false;
       ph[1] ^= 1;
+      pend &= ~2;
       // rows >= `rows` of the A tile hold stale values; they only reach
       // output rows that are never stored
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -324,9 +331,9 @@ __device__ __forceinline__ void fold_issue_w(const bf16* __restrict__ Wk, int D,
     bulk_load(sw + d * 128, Wk + static_cast<size_t>(h * RF_HD + d) * D + cbk * 128, 256, mb);
 }
 
+// `pend`: as in gemv_phase (bit 0, the Wk block copies on mbarrier 0).
 __device__ bool fold_phase(const RouterFusedArgs& a, int l, int Tq, const float* __restrict__ Q,
-                           long long ldq, uint8_t* sm, uint64_t* mb, uint32_t* ph,
-                           bool w_prefetched) {
+                           long long ldq, uint8_t* sm, uint64_t* mb, uint32_t* ph, int& pend) {
   const int D = a.D;
   const int cblocks = D / 128;
   const int n_items = cblocks * a.heads;
@@ -334,17 +341,17 @@ __device__ bool fold_phase(const RouterFusedArgs& a, int l, int Tq, const float*
   float* s_q = reinterpret_cast<float*>(sm + RF_HD * 128 * 2);
   const int tid = threadIdx.x & 127;  // column within the block
   const int half = threadIdx.x >> 7;  // two halves share the tiles
-  bool first = true;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     const int h = item / cblocks, cbk = item % cblocks;
     const int c = cbk * 128 + tid;
-    if (!(first && w_prefetched)) {
+    if (!(pend & 1)) {
       __syncthreads();
       if (threadIdx.x < 32) fold_issue_w(a.Wk[l], D, item, sm, &mb[0]);
+      pend |= 1;
     }
-    first = false;
     if (!cta_wait(&mb[0], ph[0])) return false;
     ph[0] ^= 1;
+    pend &= ~1;
     for (int t0 = 0; t0 < Tq; t0 += 64) {
       const int nt = min(64, Tq - t0);
       __syncthreads();
@@ -776,19 +783,30 @@ __device__ void route_phase(const RouterFusedArgs& a, double* s_vals, double* s_
       __syncthreads();
       continue;
     }
-    for (int i = threadIdx.x; i < n; i += RF_THREADS) s_vals[i] = static_cast<double>(a.gate[2 * (s + i)]);
-    __syncthreads();
+    int my_nan = 0;
     for (int i = threadIdx.x; i < n; i += RF_THREADS) {
-      const double v = s_vals[i];
-      int rank = 0;
-      for (int j = 0; j < n; ++j) {
-        const double u = s_vals[j];
-        rank += (u < v) || (u == v && j < i);
+      const double v = static_cast<double>(a.gate[2 * (s + i)]);
+      s_vals[i] = v;
+      my_nan |= isnan(v) ? 1 : 0;
+    }
+    // a NaN gate makes the group's quantile NaN (as torch.quantile does), so
+    // no tile of the group passes the strict > test; the rank sort, whose
+    // ranks assume a total order, is skipped
+    const int any_nan = __syncthreads_or(my_nan);
+    if (!any_nan) {
+      for (int i = threadIdx.x; i < n; i += RF_THREADS) {
+        const double v = s_vals[i];
+        int rank = 0;
+        for (int j = 0; j < n; ++j) {
+          const double u = s_vals[j];
+          rank += (u < v) || (u == v && j < i);
+        }
+        s_sorted[rank] = v;
       }
-      s_sorted[rank] = v;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && any_nan) s_qv = __longlong_as_double(0x7ff8000000000000LL);
+    if (threadIdx.x == 0 && !any_nan) {
       const double pos = __dmul_rn(a.rel_q, static_cast<double>(n - 1));
       const double flo = floor(pos);
       const int lo = static_cast<int>(flo);
@@ -864,7 +882,9 @@ __global__ void __launch_bounds__(RF_THREADS, 1)
   uint32_t ph[4] = {0u, 0u, 0u, 0u};
   unsigned gen = 0;
   bool ok = true;
-  bool w_pending = false;  // weight copies of the next projection phase in flight
+  // bulk copies in flight on mbarriers 0 (weights) and 1 (projection input
+  // rows), bits 0 and 1: set when issued, cleared when their wait succeeds
+  int mb_pending = 0;
   int x_pending = 0;       // x slots (bits) requested ahead of their phase
   const int T = a.T, D = a.D, G = a.G;
   auto sync = [&]() {
@@ -875,18 +895,16 @@ __global__ void __launch_bounds__(RF_THREADS, 1)
   // phase: this CTA's first item's rows are requested before the barrier.
   auto prefetch_w = [&](const bf16* W, int K, int N) {
     __syncthreads();
-    w_pending = static_cast<int>(blockIdx.x) < N / GV_COLS;
-    if (w_pending && warp == 0) gv_issue_w(W, K, blockIdx.x, sm, &s_mb[0]);
+    if (static_cast<int>(blockIdx.x) < N / GV_COLS) {
+      if (warp == 0) gv_issue_w(W, K, blockIdx.x, sm, &s_mb[0]);
+      mb_pending |= 1;
+    }
   };
+  // a phase that does not run (an earlier wait gave up) leaves its
+  // prefetched copies to the drain at the end of the kernel
   auto project = [&](int M, int K, int N, const bf16* W, const bf16* b, float* Y, int ldy,
                      bool act, auto row) {
-    const bool pre = w_pending;
-    w_pending = false;
-    if (ok) {
-      ok = gemv_phase(M, K, N, W, b, Y, ldy, act, sm, s_mb, ph, pre, row);
-    } else if (pre && mbar_wait(&s_mb[0], ph[0])) {
-      ph[0] ^= 1;  // drain the prefetched copies of a phase that does not run
-    }
+    if (ok) ok = gemv_phase(M, K, N, W, b, Y, ldy, act, sm, s_mb, ph, mb_pending, row);
   };
   // layer 1's query is shared by all tiles: Q1 = Wq_1 query + bq_1 in row 0 of Q
   // (the bf16 query is widened into h first)
@@ -897,15 +915,14 @@ __global__ void __launch_bounds__(RF_THREADS, 1)
   for (int l = 0; l < 4 && ok; ++l) {
     // this CTA's first fold item: its Wk block is requested before the barrier
     __syncthreads();
-    w_pending = static_cast<int>(blockIdx.x) < (D / 128) * a.heads;
-    if (w_pending && warp == 0) fold_issue_w(a.Wk[l], D, blockIdx.x, sm, &s_mb[0]);
+    if (static_cast<int>(blockIdx.x) < (D / 128) * a.heads) {
+      if (warp == 0) fold_issue_w(a.Wk[l], D, blockIdx.x, sm, &s_mb[0]);
+      mb_pending |= 1;
+    }
     if (!sync()) break;
     const bool shared_q = l == 0;
-    {
-      const bool pre = w_pending;
-      w_pending = false;
-      if (!fold_phase(a, l, shared_q ? 1 : T, a.Q, shared_q ? 0 : D, sm, s_mb, ph, pre)) ok = false;
-    }
+    if (!fold_phase(a, l, shared_q ? 1 : T, a.Q, shared_q ? 0 : D, sm, s_mb, ph, mb_pending))
+      ok = false;
     // the attention phase's first x steps (x is an input) before the barrier
     x_pending = attend_prefetch_x(a, sm, s_mb);
     if (!sync()) break;
@@ -981,8 +998,10 @@ __global__ void __launch_bounds__(RF_THREADS, 1)
   if (ok && sync())
     route_phase(a, reinterpret_cast<double*>(sm),
                 reinterpret_cast<double*>(sm) + IVC_MAX_QUANTILE_GROUP);
-  // prefetches whose phase never ran (a barrier gave up): let their copies land
-  if (w_pending) (void)mbar_wait(&s_mb[0], ph[0]);
+  // copies whose wait never succeeded (a prefetch whose phase never ran, or a
+  // phase that gave up with copies in flight): let them land before exit
+  if (mb_pending & 1) (void)mbar_wait(&s_mb[0], ph[0]);
+  if (mb_pending & 2) (void)mbar_wait(&s_mb[1], ph[1]);
   for (int sl = 0; sl < 2; ++sl)
     if (x_pending & (1 << sl)) (void)mbar_wait(&s_mb[2 + sl], ph[2 + sl]);
   if (!ok && threadIdx.x == 0) atomicOr(a.status, DEV_WAIT_TIMEOUT);
@@ -1084,8 +1103,7 @@ int launch_router_fused(const ivc_router* r, const void* x, const int32_t* valid
   a.status = L.status;
   const size_t smem = router_fused_smem(r->D, r->gate_hidden);
   if (smem > 227 * 1024) return IVC_EUNSUPPORTED;
-  if (cudaFuncSetAttribute(router_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
+  if (smem_optin(reinterpret_cast<const void*>(router_fused_kernel), smem) != IVC_OK)
     return IVC_ECUDA;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, router_fused_kernel, RF_THREADS,
