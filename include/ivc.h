@@ -299,6 +299,19 @@ int ivc_assemble_sequence(const int32_t* input_ids, const int32_t* seq_offsets, 
  * clear it. Returns IVC_OK when no bit was set, IVC_EDEVICE otherwise. */
 int ivc_device_status(void* workspace, int* bits, ivc_stream_t stream);
 
+/* Failure detection (diagnostics). Every wait inside the kernels is bounded
+ * (about one second of clock cycles): a wait that runs out sets
+ * IVC_DEV_WAIT_TIMEOUT in the status word, the kernel skips its remaining
+ * work, lets the copies it issued land, and returns; no trap is used and the
+ * context stays usable. To exercise that path, `cycles` > 0 makes the
+ * persistent router (ivc_vir_route's single-kernel form) give up its
+ * software grid barriers from the one before the gating head on after that
+ * many clock cycles; no bulk copy is in flight at those barriers. With a
+ * limit of a few cycles the call's outputs are invalid and the status bit is
+ * set. 0 restores the default bound; negative values are IVC_EINVAL.
+ * Process-wide, read at each launch. */
+int ivc_set_router_wait_limit(long long cycles);
+
 /* ivc_ps_project for callers that cannot allocate device memory.
  * No counterpart on the pages: this is a deployment variant of the call above.
  * Callers such as an inference-engine plugin whose device memory is planned

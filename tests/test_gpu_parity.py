@@ -548,3 +548,41 @@ def test_flash_kernel_variants(env):
                          env={**os.environ, **env}, capture_output=True, text=True, timeout=600)
     assert out.returncode == 0, out.stderr[-2000:]
     assert "variant ok" in out.stdout
+
+
+# ---------------------------------------------------------------- multi-Linear launch
+@pytest.mark.parametrize("flags,scale", [(0, 0.5), (1, 0.5), (0, 0.25), (1, 0.25), (2, 0.25)])
+def test_ps_project_single_launch_small(flags, scale):
+    """Shapes the single persistent launch of all Linears takes (widths
+    multiples of 128): 5 tiles, so the factor-0.25 rows (320) end inside a
+    256-row block, every pixel_shuffle flag."""
+    ivc = _ivc()
+    inp = W.make(small_workload(C=128, H=256, mid=384, tiles=(5,)), affine="random")
+    key = "mlp1" if scale == 0.5 else "mlp2"
+    y = ivc.ps_project(inp["x"].cuda(), scale, ivc.Mlp(inp[key]).fold(), flags=flags)
+    torch.cuda.synchronize()
+    x64 = O.to64(inp["x"])
+    if flags == 2:
+        ref = O.ps_project(x64, 0.25, O.to64(inp[key]), quarter_order="twice")
+    else:
+        ref = O.ps_project(x64, scale, O.to64(inp[key]), ps_version="v1" if flags else "v2")
+        if flags == 1 and scale == 0.25:
+            ref = ref.reshape(5, 8, 8, -1).transpose(0, 2, 1, 3).reshape(5, 64, -1)
+    assert_connector_close(y, ref.reshape(-1, ref.shape[-1]), f"{key} flags={flags}")
+
+
+@pytest.mark.parametrize("tiles", [(3, 1, 4), (1,), (9, 8)])
+def test_flash_single_launch_small(tiles):
+    """Both MLPs in one persistent launch beside the router: 1, 8 and 17
+    tiles (1..5 row blocks of 256 for mlp1, ragged ones for mlp2)."""
+    ivc = _ivc()
+    inp = W.make(small_workload(C=256, H=256, mid=384, tiles=tiles, var=0.3), affine="random")
+    m1, m2 = ivc.Mlp(inp["mlp1"]), ivc.Mlp(inp["mlp2"]).fold()
+    r = ivc.Router(inp["router"])
+    ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_FLASH, inp["T"], 256, m1, m2, r))
+    for _ in range(2):  # the row-block counters start from zero on every call
+        res = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(),
+                                 inp["image_offsets"].cuda(), m1, m2, r, workspace=ws)
+        torch.cuda.synchronize()
+        assert ivc.device_status(ws) == 0
+        _flash_check(ivc, inp, res)

@@ -108,6 +108,8 @@ def lib() -> ctypes.CDLL:
                                             _vp, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp,
                                             ctypes.c_int, _vp, _vp, _vp, _vp, _vp,
                                             ctypes.c_size_t, _vp]
+        L.ivc_set_router_wait_limit.restype = ctypes.c_int
+        L.ivc_set_router_wait_limit.argtypes = [ctypes.c_longlong]
         L.ivc_device_status.restype = ctypes.c_int
         L.ivc_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int), _vp]
         L.ivc_trace_enable.restype = ctypes.c_int

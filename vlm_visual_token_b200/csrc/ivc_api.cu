@@ -8,6 +8,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "ivc_gemm.cuh"
 #include "ivc_internal.h"
@@ -94,6 +95,7 @@ struct PsBufs {
   bf16* h2 = nullptr;
   float* split_part = nullptr;  // split-K scratch (flash flows only), shared
   int* split_s = nullptr;
+  int* done = nullptr;          // row-block counters of the multi-Linear launch
 };
 
 void carve_ps(Carver& cv, const ivc_mlp* m, long long rows, bool need_stats, PsBufs& b) {
@@ -108,6 +110,8 @@ void carve_ps(Carver& cv, const ivc_mlp* m, long long rows, bool need_stats, PsB
   }
   b.h1 = cv.take<bf16>(rows * m->dims[1]);
   if (m->n_linear == 3) b.h2 = cv.take<bf16>(rows * m->dims[2]);
+  // one counter per 256-row block and Linear
+  b.done = cv.take<int>(static_cast<size_t>((rows + 255) / 256) * m->n_linear);
 }
 
 struct RouteBufs {
@@ -250,6 +254,82 @@ int ps_mlp(const void* x, int T, int C, bool half, int flags, const ivc_mlp* m, 
     IVC_TRY(launch_gemm(d, L));
     a = b.h2;
   }
+  return IVC_OK;
+}
+
+// The connector's Linears run as one persistent launch (ivc_gemm_graph.cuh)
+// with IVC_GEMM_GRAPH=1; otherwise one launch per Linear.
+bool gemm_graph_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("IVC_GEMM_GRAPH");
+    v = (e && e[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
+// The Linears of one pixel_shuffle + MLP as graph problems (appended to
+// `probs`; the first reads x through the pixel_shuffle view with the
+// LayerNorm fold, each later one the previous one's output). The weights
+// must be folded already (W0, cs, fb).
+void mlp_problems(const void* x, int T, int C, bool half, int flags, const ivc_mlp* m,
+                  const bf16* W0, const float* cs, const float* fb, bf16* y, const PsBufs& b,
+                  std::vector<GraphProblemCall>& probs) {
+  const int rows = T * (half ? 256 : 64);
+  const int remap = (flags & IVC_PS_V1) ? (half ? 1 : 2) : 0;
+  GraphProblemCall c{};
+  c.a_mode = half ? A_PS_HALF : ((flags & IVC_PS_QUARTER_TWICE) ? A_PS_QUARTER_TWICE : A_PS_QUARTER);
+  c.a = x;
+  c.T = T;
+  c.C = C;
+  c.M = rows;
+  c.N = m->dims[1];
+  c.K = m->dims[0];
+  c.B = W0;
+  c.epi_mode = EPI_LNFOLD;
+  c.gelu = 1;
+  c.colsum = cs;
+  c.fbias = fb;
+  c.row_mean = b.mean;
+  c.row_rstd = b.rstd;
+  c.out = b.h1;
+  c.ldo = m->dims[1];
+  c.dep = -1;
+  probs.push_back(c);
+  for (int i = 1; i < m->n_linear; ++i) {
+    const bool last = i + 1 == m->n_linear;
+    GraphProblemCall d{};
+    d.a_mode = A_PLAIN;
+    d.a = i == 1 ? b.h1 : b.h2;
+    d.M = rows;
+    d.N = m->dims[i + 1];
+    d.K = m->dims[i];
+    d.B = m->W[i];
+    d.bias = static_cast<const bf16*>(m->b[i]);
+    d.epi_mode = EPI_BIAS;
+    d.gelu = last ? 0 : 1;
+    d.remap = last ? remap : 0;
+    d.out = last ? static_cast<void*>(y) : static_cast<void*>(b.h2);
+    d.ldo = m->dims[i + 1];
+    d.dep = i - 1;  // the previous Linear of this MLP, as an index into this MLP's list
+    probs.push_back(d);
+  }
+}
+
+// LayerNorm-folded weights of the first Linear: the caller's (ivc_mlp_fold)
+// or folded now into the workspace.
+int folded_weights(const ivc_mlp* m, const PsBufs& b, const Launch& L, const bf16** W0,
+                   const float** cs, const float** fb) {
+  *W0 = static_cast<const bf16*>(m->fold_W0);
+  *cs = m->fold_colsum;
+  *fb = m->fold_bias;
+  if (*cs) return IVC_OK;
+  IVC_TRY(launch_fold(static_cast<const bf16*>(m->W[0]), static_cast<const bf16*>(m->b[0]),
+                      static_cast<const bf16*>(m->ln_gamma), static_cast<const bf16*>(m->ln_beta),
+                      m->dims[1], m->dims[0], b.fold_W0, b.fold_cs, b.fold_b, L));
+  *W0 = b.fold_W0;
+  *cs = b.fold_cs;
+  *fb = b.fold_b;
   return IVC_OK;
 }
 
@@ -508,6 +588,7 @@ struct FlashBufs {
   bf16* Y64;
   RouteBufs br;
   ListBufs lists;
+  int* done;
 };
 
 void carve_flash(Carver& cv, int T, const ivc_mlp* m1, const ivc_mlp* m2, const ivc_router* r,
@@ -521,6 +602,9 @@ void carve_flash(Carver& cv, int T, const ivc_mlp* m1, const ivc_mlp* m2, const 
   // one split-K scratch for all connector GEMMs (they run one after another)
   f.b1.split_part = f.b2.split_part = cv.take<float>(splitk_part_floats());
   f.b1.split_s = f.b2.split_s = cv.take<int>(4);
+  // row-block counters of both MLPs' Linears in one launch
+  f.done = cv.take<int>(static_cast<size_t>(T) * m1->n_linear +
+                        static_cast<size_t>((T * 64 + 255) / 256) * m2->n_linear);
 }
 
 size_t flash_ws(int T, const ivc_mlp* m1, const ivc_mlp* m2, const ivc_router* r) {
@@ -621,6 +705,26 @@ int ivc_ps_project(const void* x, int T, int C, float scale, int flags, const iv
   PsBufs b;
   const long long rows = static_cast<long long>(T) * (half ? 256 : 64);
   carve_ps(cv, m, rows, true, b);
+  std::vector<GraphProblemCall> probs;
+  if (gemm_graph_enabled())
+    mlp_problems(x, T, C, half, flags, m, nullptr, nullptr, nullptr, static_cast<bf16*>(y), b,
+                 probs);
+  if (!probs.empty() && graph_supported(probs.data(), static_cast<int>(probs.size()))) {
+    // fold (if needed), counters, statistics, then every Linear in one
+    // launch that overlaps the statistics kernel's tail
+    const bf16* W0;
+    const float *cs, *fb;
+    IVC_TRY(folded_weights(m, b, L, &W0, &cs, &fb));
+    probs[0].B = W0;
+    probs[0].colsum = cs;
+    probs[0].fbias = fb;
+    const int n_ctr = graph_counters(probs.data(), static_cast<int>(probs.size()));
+    IVC_TRY(cu_check(cudaMemsetAsync(b.done, 0, sizeof(int) * n_ctr, L.stream)));
+    IVC_TRY(launch_ps_stats(static_cast<const bf16*>(x), T, C, half ? b.mean : nullptr,
+                            half ? b.rstd : nullptr, half ? nullptr : b.mean,
+                            half ? nullptr : b.rstd, L));
+    return launch_gemm_graph(probs.data(), static_cast<int>(probs.size()), b.done, 0, L);
+  }
   IVC_TRY(launch_ps_stats(static_cast<const bf16*>(x), T, C, half ? b.mean : nullptr,
                           half ? b.rstd : nullptr, half ? nullptr : b.mean,
                           half ? nullptr : b.rstd, L));
@@ -706,15 +810,59 @@ int ivc_flash_compress(const void* x, const int32_t* valid_len, int T, int C,
   // already enqueued on the side stream
   const int rc_rec = cu_check(cudaEventRecord(side->join, side->stream));
   if (rc == IVC_OK) rc = rc_rec;
-  if (rc == IVC_OK)
-    rc = launch_ps_stats(static_cast<const bf16*>(x), T, C, b1.mean, b1.rstd, b2.mean, b2.rstd, L);
   const int reserve = dual_reserve_sms();
-  if (dual_mlp2_first()) {
-    if (rc == IVC_OK) rc = ps_mlp(x, T, C, false, 0, mlp2, Y64, b2, L, nullptr, reserve);
-    if (rc == IVC_OK) rc = ps_mlp(x, T, C, true, 0, mlp1, Y256, b1, L, nullptr, reserve);
-  } else {
-    if (rc == IVC_OK) rc = ps_mlp(x, T, C, true, 0, mlp1, Y256, b1, L, nullptr, reserve);
-    if (rc == IVC_OK) rc = ps_mlp(x, T, C, false, 0, mlp2, Y64, b2, L, nullptr, reserve);
+  // both MLPs' Linears in one persistent launch, in the priority order
+  // mlp2.fc1, mlp1.fc1, mlp2.fc2, mlp1.fc2, mlp2.fc3 (the long first Linear
+  // of mlp2 first; each later Linear right after its input's)
+  std::vector<GraphProblemCall> p1, p2, probs;
+  std::vector<int> pos1, pos2;
+  if (gemm_graph_enabled()) {
+    mlp_problems(x, T, C, true, 0, mlp1, nullptr, nullptr, nullptr, Y256, b1, p1);
+    mlp_problems(x, T, C, false, 0, mlp2, nullptr, nullptr, nullptr, Y64, b2, p2);
+    pos1.resize(p1.size());
+    pos2.resize(p2.size());
+    for (size_t i = 0; i < p1.size() || i < p2.size(); ++i) {
+      if (i < p2.size()) {
+        pos2[i] = static_cast<int>(probs.size());
+        probs.push_back(p2[i]);
+        if (p2[i].dep >= 0) probs.back().dep = pos2[p2[i].dep];
+      }
+      if (i < p1.size()) {
+        pos1[i] = static_cast<int>(probs.size());
+        probs.push_back(p1[i]);
+        if (p1[i].dep >= 0) probs.back().dep = pos1[p1[i].dep];
+      }
+    }
+  }
+  if (rc == IVC_OK && !probs.empty() &&
+      graph_supported(probs.data(), static_cast<int>(probs.size()))) {
+    const bf16 *W01, *W02;
+    const float *cs1, *fb1, *cs2, *fb2;
+    rc = folded_weights(mlp1, b1, L, &W01, &cs1, &fb1);
+    if (rc == IVC_OK) rc = folded_weights(mlp2, b2, L, &W02, &cs2, &fb2);
+    probs[pos1[0]].B = W01;
+    probs[pos1[0]].colsum = cs1;
+    probs[pos1[0]].fbias = fb1;
+    probs[pos2[0]].B = W02;
+    probs[pos2[0]].colsum = cs2;
+    probs[pos2[0]].fbias = fb2;
+    const int n_ctr = graph_counters(probs.data(), static_cast<int>(probs.size()));
+    if (rc == IVC_OK) rc = cu_check(cudaMemsetAsync(f.done, 0, sizeof(int) * n_ctr, s));
+    if (rc == IVC_OK)
+      rc = launch_ps_stats(static_cast<const bf16*>(x), T, C, b1.mean, b1.rstd, b2.mean, b2.rstd,
+                           L);
+    if (rc == IVC_OK)
+      rc = launch_gemm_graph(probs.data(), static_cast<int>(probs.size()), f.done, reserve, L);
+  } else if (rc == IVC_OK) {
+    // one launch per Linear (IVC_GEMM_GRAPH=0)
+    rc = launch_ps_stats(static_cast<const bf16*>(x), T, C, b1.mean, b1.rstd, b2.mean, b2.rstd, L);
+    const bool mlp2_first = dual_mlp2_first();
+    for (int k = 0; k < 2 && rc == IVC_OK; ++k) {
+      if ((k == 0) == mlp2_first)
+        rc = ps_mlp(x, T, C, false, 0, mlp2, Y64, b2, L, nullptr, reserve);
+      else
+        rc = ps_mlp(x, T, C, true, 0, mlp1, Y256, b1, L, nullptr, reserve);
+    }
   }
   const int rc_wait = rc_rec == IVC_OK ? cu_check(cudaStreamWaitEvent(s, side->join, 0)) : rc_rec;
   if (rc != IVC_OK) return rc;
@@ -760,6 +908,12 @@ int ivc_flash_compress_routed(const void* x, const int32_t* valid_len, int T, in
   const Routed rc{lb.list_c, lb.counts + 1, lb.base_c};
   IVC_TRY(ps_mlp(x, T, C, true, 0, mlp1, static_cast<bf16*>(out), f.b1, L, &ru));
   return ps_mlp(x, T, C, false, 0, mlp2, static_cast<bf16*>(out), f.b2, L, &rc);
+}
+
+int ivc_set_router_wait_limit(long long cycles) {
+  if (cycles < 0) return IVC_EINVAL;
+  set_router_late_wait_cycles(cycles);
+  return IVC_OK;
 }
 
 int ivc_device_status(void* workspace, int* bits, ivc_stream_t stream) {

@@ -1,0 +1,144 @@
+// ivc_graph.cu — host side of the multi-Linear persistent launch
+// (ivc_gemm_graph.cuh): tensor maps, problem table, list schedule, launch.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <vector>
+
+#include "ivc_gemm_graph.cuh"
+#include "ivc_graph_schedule.h"
+#include "ivc_internal.h"
+
+namespace ivc {
+
+// Two-k-block views (box: 128 rows x 2 chunks of 64 channels, the chunk
+// outermost; see ivc_gemm_graph.cuh).
+// Row-major [rows, cols] bf16: {64, rows, cols / 64}.
+static int map_rows_2k(CUtensorMap* m, const void* base, long long rows, long long cols) {
+  const unsigned long long d[3] = {64, static_cast<unsigned long long>(rows),
+                                   static_cast<unsigned long long>(cols / 64)};
+  const unsigned long long st[2] = {static_cast<unsigned long long>(cols) * 2, 128};
+  const unsigned box[3] = {64, static_cast<unsigned>(GEMM_BM), GG_KPER};
+  return map_bf16(m, 3, base, d, st, box);
+}
+
+// The [T,32,32,C] features at factor 1/f: one view per pixel_shuffle block
+// (qb, rb), maps[qb * f + rb] = {64, b: g, tile * g + a, C / 64} over the
+// pixels (f a + qb, f b + rb), g = 32 / f.
+static int map_ps_2k(CUtensorMap* maps, const void* x, int T, int C, int f) {
+  const int g = 32 / f;
+  const unsigned long long Cu = static_cast<unsigned long long>(C);
+  for (int qb = 0; qb < f; ++qb)
+    for (int rb = 0; rb < f; ++rb) {
+      const char* base = static_cast<const char*>(x) + (static_cast<size_t>(qb) * 32 + rb) * C * 2;
+      const unsigned long long d[4] = {64, static_cast<unsigned long long>(g),
+                                       static_cast<unsigned long long>(T) * g, Cu / 64};
+      const unsigned long long st[3] = {Cu * f * 2, Cu * 32 * f * 2, 128};
+      const unsigned box[4] = {64, static_cast<unsigned>(g), static_cast<unsigned>(GEMM_BM / g),
+                               GG_KPER};
+      const int rc = map_bf16(&maps[qb * f + rb], 4, base, d, st, box);
+      if (rc) return rc;
+    }
+  return IVC_OK;
+}
+
+bool graph_supported(const GraphProblemCall* probs, int n) {
+  if (n <= 0 || n > GG_MAX_PROBLEMS) return false;
+  int amaps = 0;
+  for (int i = 0; i < n; ++i) {
+    const GraphProblemCall& c = probs[i];
+    if (c.M <= 0 || c.N <= 0 || c.N % 32 != 0 || c.K % (GEMM_BK * GG_KPER) != 0) return false;
+    if (c.dep >= i || (c.dep >= 0 && probs[c.dep].M != c.M)) return false;
+    if (c.a_mode != A_PLAIN && (c.C % (GEMM_BK * GG_KPER) != 0)) return false;
+    amaps += c.a_mode == A_PLAIN ? 1 : (c.a_mode == A_PS_HALF ? 4 : 16);
+  }
+  return amaps <= GG_MAX_AMAPS;
+}
+
+int graph_counters(const GraphProblemCall* probs, int n) {
+  int c = 0;
+  for (int i = 0; i < n; ++i) c += (probs[i].M + GG_TILE_M - 1) / GG_TILE_M;
+  return c;
+}
+
+int launch_gemm_graph(const GraphProblemCall* probs, int n, int* done, int reserve_sms,
+                      const Launch& L) {
+  if (done == nullptr) return IVC_EINVAL;
+  if (!graph_supported(probs, n)) return IVC_EUNSUPPORTED;
+  GraphArgs g{};
+  g.n_problems = n;
+  g.done = done;
+  std::vector<SchedProblem> sp(n);
+  int amap = 0, ctr = 0;
+  GraphMaps m{};
+  for (int i = 0; i < n; ++i) {
+    const GraphProblemCall& c = probs[i];
+    GraphProblem& P = g.p[i];
+    P.M = c.M;
+    P.N = c.N;
+    P.K = c.K;
+    P.a_mode = c.a_mode;
+    P.a_map = amap;
+    P.c_blocks = c.C / GEMM_BK;
+    P.m_tiles = (c.M + GG_TILE_M - 1) / GG_TILE_M;
+    P.n_tiles = (c.N + GG_BN - 1) / GG_BN;
+    P.epi_mode = c.epi_mode;
+    P.gelu = c.gelu;
+    P.remap = c.remap;
+    P.dep = c.dep;
+    P.done_base = ctr;
+    P.bias = c.bias;
+    P.colsum = c.colsum;
+    P.fbias = c.fbias;
+    P.row_mean = c.row_mean;
+    P.row_rstd = c.row_rstd;
+    P.out = c.out;
+    P.ldo = c.ldo;
+    ctr += P.m_tiles;
+    int rc;
+    if (c.a_mode == A_PLAIN) {
+      rc = map_rows_2k(&m.a[amap], c.a, c.M, c.K);
+      P.a_views = 1;
+    } else {
+      const int f = c.a_mode == A_PS_HALF ? 2 : 4;
+      rc = map_ps_2k(&m.a[amap], c.a, c.T, c.C, f);
+      P.a_views = f * f;
+    }
+    if (rc) return rc;
+    amap += P.a_views;
+    rc = map_rows_2k(&m.b[i], c.B, c.N, c.K);
+    if (rc) return rc;
+    sp[i] = {P.m_tiles, P.n_tiles, c.K / GEMM_BK, c.dep};
+  }
+  for (int i = 0; i < n; ++i)
+    if (g.p[i].dep >= 0) g.p[i].dep_target = 2 * g.p[g.p[i].dep].n_tiles;
+  g.n_amaps = amap;
+  const std::vector<int> ub = schedule_unit_begin(sp);
+  for (int i = 0; i <= n; ++i) g.unit_begin[i] = ub[i];
+  const int units = ub[n];
+  int pairs = (num_sms() - (reserve_sms > 0 ? reserve_sms : 0)) / 2;
+  if (pairs > GG_MAX_PAIRS) pairs = GG_MAX_PAIRS;
+  if (pairs > units) pairs = units;
+  if (pairs < 1) pairs = 1;
+  g.n_pairs = pairs;
+  g.scheduled = 0;
+  if (units <= GG_MAX_SCHED) {
+    std::vector<std::vector<int>> lists;
+    if (!list_schedule(sp, pairs, 4, lists)) return IVC_EINVAL;
+    int off = 0;
+    for (int q = 0; q < pairs; ++q) {
+      g.sched_off[q] = static_cast<unsigned short>(off);
+      for (int u : lists[q]) g.sched[off++] = static_cast<unsigned short>(u);
+    }
+    g.sched_off[pairs] = static_cast<unsigned short>(off);
+    g.scheduled = 1;
+  }
+  using S = GraphSmem;
+  if (smem_optin(reinterpret_cast<const void*>(gemm_graph_kernel), S::TOTAL) != IVC_OK)
+    return IVC_ECUDA;
+  TraceScope ts("connector.graph", L.stream);
+  return launch_k(gemm_graph_kernel, dim3(2 * pairs), dim3(GEMM_THREADS), S::TOTAL, L.stream, 2, m,
+                  g, L.status);
+}
+
+}  // namespace ivc

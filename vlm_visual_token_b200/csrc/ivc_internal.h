@@ -123,6 +123,36 @@ struct GemmCall {
   int epi_dep_only;
 };
 int launch_gemm(const GemmCall& c, const Launch& L);
+
+// Several connector Linears in one persistent launch (ivc_gemm_graph.cuh).
+// Problems are given in priority order; `dep` names an earlier problem whose
+// output rows (256-row block m) tile row block m reads (its A operand), or -1.
+// Every problem uses 256 x 256 tiles on CTA pairs, K-major weights and a bf16
+// output; `done` holds graph_counters() ints that must be zero at launch.
+struct GraphProblemCall {
+  int a_mode;          // AMode
+  const void* a;       // A base (features for the pixel_shuffle modes)
+  int T, C;            // pixel_shuffle modes
+  int M, N, K;
+  const void* B;       // nn.Linear weight [N, K]
+  const bf16* bias;    // EPI_BIAS (may be null)
+  int epi_mode, gelu, remap;
+  const float* colsum;
+  const float* fbias;
+  const float* row_mean;
+  const float* row_rstd;
+  void* out;
+  long long ldo;
+  int dep;
+};
+int launch_gemm_graph(const GraphProblemCall* probs, int n, int* done, int reserve_sms,
+                      const Launch& L);
+// Row-block counters launch_gemm_graph needs for these problems.
+int graph_counters(const GraphProblemCall* probs, int n);
+// Whether launch_gemm_graph takes these problems: K a multiple of 128 (two
+// k-blocks per stage), C a multiple of 128 for the pixel_shuffle views, N a
+// multiple of 32, dependencies on earlier problems with the same rows.
+bool graph_supported(const GraphProblemCall* probs, int n);
 // Size of the split-K partial buffer: enough for any GEMM shape on this device.
 size_t splitk_part_floats();
 
@@ -178,6 +208,7 @@ struct FusedRouterBufs {
 // Tensor map of a row-major [rows, cols] bf16 matrix, box 64 columns x
 // box_rows rows, 128-byte swizzle (ivc_connector.cu).
 int map_rows_2d(CUtensorMap* m, const void* base, long long rows, long long cols, int box_rows);
+
 // Tensor map of a bf16 tensor of `rank` dims (innermost first; strides in
 // bytes of dims 1..rank-1, in any order), box `box`, 128-byte swizzle.
 int map_bf16(CUtensorMap* m, int rank, const void* base, const unsigned long long* dims,
@@ -186,6 +217,10 @@ int map_bf16(CUtensorMap* m, int rank, const void* base, const unsigned long lon
 // between its phases) or as separate kernels. IVC_ROUTER_FUSED=1 / 0 forces
 // the choice; otherwise the caller's default_on decides.
 bool router_fused_wanted(bool default_on);
+// The test limit of the persistent router's grid barriers after the gating
+// (ivc_set_router_wait_limit): 0 = the default bound.
+long long router_late_wait_cycles();
+void set_router_late_wait_cycles(long long cycles);
 bool router_fused_supported(const ivc_router* r);
 int launch_router_fused(const ivc_router* r, const void* x, const int32_t* valid_len, int T,
                         const int32_t* image_offsets, int I, float* gate, uint8_t* mask,

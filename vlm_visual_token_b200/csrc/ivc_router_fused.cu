@@ -29,6 +29,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdlib>
 
 #include "ivc_internal.h"
@@ -78,6 +79,10 @@ struct RouterFusedArgs {
   int32_t* offsets;
   int32_t* total;
   int* status;
+  // > 0: the grid barriers from the one before the gating head on give up
+  // after this many clock cycles (failure-detection tests; no bulk copy is
+  // in flight at those barriers). 0: every barrier uses IVC_WAIT_CYCLES.
+  long long late_wait_cycles;
 };
 
 __device__ __forceinline__ float gelu(float y) {
@@ -89,7 +94,7 @@ __device__ __forceinline__ float gelu(float y) {
 // has to reset it. Arrival is a release reduction (this CTA's writes, ordered
 // by the __syncthreads before it, become visible with it), the wait an
 // acquire spin; false after ~1 s without progress.
-__device__ bool grid_sync(unsigned* bar, unsigned& gen) {
+__device__ bool grid_sync(unsigned* bar, unsigned& gen, long long limit) {
   __shared__ int s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -101,7 +106,7 @@ __device__ bool grid_sync(unsigned* bar, unsigned& gen) {
       unsigned v;
       asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
       if (static_cast<int>(v - target) >= 0) break;
-      if (clock64() - t0 > IVC_WAIT_CYCLES) {
+      if (clock64() - t0 > limit) {
         ok = 0;
         break;
       }
@@ -887,8 +892,9 @@ __global__ void __launch_bounds__(RF_THREADS, 1)
   int mb_pending = 0;
   int x_pending = 0;       // x slots (bits) requested ahead of their phase
   const int T = a.T, D = a.D, G = a.G;
+  long long wait_limit = IVC_WAIT_CYCLES;
   auto sync = [&]() {
-    if (ok) ok = grid_sync(a.bar, gen);
+    if (ok) ok = grid_sync(a.bar, gen, wait_limit);
     return ok;
   };
   // The weights of the next projection phase do not depend on the previous
@@ -967,7 +973,10 @@ __global__ void __launch_bounds__(RF_THREADS, 1)
       __syncthreads();
     }
   }
-  // head: gate = softmax(Wout h_4 + bout), one warp per tile
+  // head: gate = softmax(Wout h_4 + bout), one warp per tile. From here on no
+  // bulk copy is in flight (the last projection's waits succeeded, the
+  // attention slots were consumed), so a short test limit may apply.
+  if (a.late_wait_cycles > 0) wait_limit = a.late_wait_cycles;
   if (ok && sync()) {
     const int lane = threadIdx.x & 31;
     for (int t = blockIdx.x * RF_WARPS + warp; t < T; t += gridDim.x * RF_WARPS) {
@@ -1021,6 +1030,16 @@ size_t router_fused_smem(int D, int G) {
 }
 
 }  // namespace
+
+// Test limit of the persistent router's late grid barriers (ivc.h,
+// ivc_set_router_wait_limit); read at every launch.
+static std::atomic<long long> g_late_wait_cycles{0};
+
+long long router_late_wait_cycles() { return g_late_wait_cycles.load(std::memory_order_relaxed); }
+
+void set_router_late_wait_cycles(long long cycles) {
+  g_late_wait_cycles.store(cycles > 0 ? cycles : 0, std::memory_order_relaxed);
+}
 
 bool router_fused_wanted(bool default_on) {
   static int env = -2;
@@ -1101,6 +1120,7 @@ int launch_router_fused(const ivc_router* r, const void* x, const int32_t* valid
   a.offsets = offsets;
   a.total = total;
   a.status = L.status;
+  a.late_wait_cycles = router_late_wait_cycles();
   const size_t smem = router_fused_smem(r->D, r->gate_hidden);
   if (smem > 227 * 1024) return IVC_EUNSUPPORTED;
   if (smem_optin(reinterpret_cast<const void*>(router_fused_kernel), smem) != IVC_OK)
