@@ -546,6 +546,15 @@ def run_ivc(args):
             tf = fl / (us * 1e-6) / 1e12
             gemm[k] = {"gflop_per_launch": fl / 1e9, "us_per_launch": us, "tflops": tf,
                        "frac": tf / burst, "frac_vs_sustained": tf / sustained}
+    # all connector Linears in one persistent launch: priced as their sum
+    if "connector.graph" in trace and trace["connector.graph"]["launches"] > 0:
+        k = "connector.graph"
+        us = 1e3 * trace[k]["ms"] / trace[k]["launches"]
+        fl = sum(alg[r][0] for r in connector_roles(w)) / (trace[k]["launches"] / n_trace)
+        tf = fl / (us * 1e-6) / 1e12
+        gemm[k] = {"gflop_per_launch": fl / 1e9, "us_per_launch": us, "tflops": tf,
+                   "frac": tf / burst, "frac_vs_sustained": tf / sustained,
+                   "linears": list(connector_roles(w))}
     # dominant kernel: the connector contraction with the largest traced time.
     # (Inside the step the router's launches wait for SMs the GEMMs hold, so
     # their traced times include that wait; by device time in the ncu launch

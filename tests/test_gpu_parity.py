@@ -192,6 +192,51 @@ def test_vir_route_gating_residual_inside(pool_mode):
     assert np.abs(ref - outside).max() > 10 * GATE_ABS  # the variant really differs
 
 
+_GATING_SNIPPET = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, {root!r})
+import oracle as O, workloads as W, vlm_visual_token_b200 as ivc
+G, inside = {G!r}, {inside!r}
+w = W.Workload("gw", "flash", C=256, H=128, tiles_per_image=(3, 18), n_images=2, mlp2_mid=256,
+               D=256, gate_hidden=G, seed_base=93)
+inp = W.make(w, affine="random")
+r = ivc.Router(inp["router"], pool_mode=1, gate_residual=inside)
+ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_VIR_ROUTE, inp["T"], 256, r=r))
+gate, mask, offsets = ivc.vir_route(inp["x"].cuda(), None, inp["image_offsets"].cuda(), r,
+                                    workspace=ws)
+torch.cuda.synchronize()
+assert ivc.device_status(ws) == 0
+ref = O.vir_gate(O.to64(inp["x"]), inp["valid_len"].numpy(), O.to64(inp["router"]),
+                 residual="inside" if inside else "outside")
+g = gate.cpu().double().numpy()
+assert np.abs(g - ref).max() <= {gate_abs!r}, np.abs(g - ref).max()
+ref_mask = O.route(g[:, 0], inp["image_offsets"].numpy())
+np.testing.assert_array_equal(mask.cpu().numpy(), ref_mask)
+np.testing.assert_array_equal(offsets.cpu().numpy(), O.compaction_offsets(ref_mask))
+print("gating ok")
+"""
+
+
+@pytest.mark.parametrize("fused", ["0", "1"])
+@pytest.mark.parametrize("G,inside", [(512, 0), (2048, 0), (256, 1)])
+def test_vir_route_gating_widths(G, inside, fused):
+    """The Gating of the separate-kernel router (here through literal
+    pooling), as 13 launches or as one cooperative kernel (IVC_GATING_FUSED=1:
+    items of 64 or 16 columns, CTAs without an item in one of the two
+    projections, 21 rows in two rounds), for a gating width unlike the
+    pooling width and for the LN(h + u) reading; in a fresh process since the
+    switch is read once."""
+    _ivc()
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = _GATING_SNIPPET.format(root=root, G=G, inside=inside, gate_abs=GATE_ABS)
+    out = subprocess.run([sys.executable, "-c", code], env={**os.environ, "IVC_GATING_FUSED": fused},
+                         capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert "gating ok" in out.stdout
+
+
 def test_bad_valid_len_sets_status_bit():
     ivc = _ivc()
     inp = W.make(small_workload(C=256, H=128, tiles=(2,)))
@@ -535,7 +580,8 @@ print("variant ok")
 
 
 @pytest.mark.parametrize("env", [{"IVC_GEMM_WIDE": "1"}, {"IVC_GEMM_PAIRS": "0"},
-                                 {"IVC_ROUTER_FUSED": "1"}, {"IVC_POOL_ATTEND": "0"}])
+                                 {"IVC_ROUTER_FUSED": "1"}, {"IVC_POOL_ATTEND": "0"},
+                                 {"IVC_GATING_FUSED": "1"}, {"IVC_POOL_TAIL": "1"}])
 def test_flash_kernel_variants(env):
     """The opt-in kernel variants (512-wide pair tiles with split-K, single-CTA
     256-wide tiles, the persistent router inside the dual flow, the pooling as

@@ -124,7 +124,7 @@ struct RouteBufs {
   float* Z = nullptr;    //   single-pass attention: chunk sums [T][8][16][D];
                          //   tensor-core form: split weighted sums [T*128][D]
   float* z = nullptr;    //   merged weighted sums [T][16][D]
-  float* h = nullptr;    //   fused router: gating state [T][D]
+  float* h = nullptr;    //   gating state [T][D] (persistent router, fused Gating)
   unsigned* bar = nullptr;  // fused router: grid barrier words
   float* Q1;
   float* Q;
@@ -145,9 +145,9 @@ void carve_route(Carver& cv, const ivc_router* r, int T, RouteBufs& b) {
     b.P2 = cv.take<bf16>(static_cast<size_t>(T) * 128 * 1024);
     b.Z = cv.take<float>(static_cast<size_t>(T) * 128 * D);
     b.z = cv.take<float>(static_cast<size_t>(T) * 16 * D);
-    b.h = cv.take<float>(static_cast<size_t>(T) * D);
-    b.bar = cv.take<unsigned>(2);
   }
+  b.h = cv.take<float>(static_cast<size_t>(T) * D);
+  b.bar = cv.take<unsigned>(2);
   b.Q1 = cv.take<float>(D);
   b.Q = cv.take<float>(static_cast<size_t>(T) * D);
   b.O = cv.take<float>(static_cast<size_t>(T) * D);
@@ -398,6 +398,20 @@ int folded_layer(const void* x, const int32_t* valid_len, int T, const ivc_route
                            static_cast<const bf16*>(r->bv[l]), b.O, L);
 }
 
+// The tail of each folded pooling layer as one cooperative launch
+// (ivc_router_coop.cu) with IVC_POOL_TAIL=1. Off by default: on the 16 CTAs
+// it can have beside the connector its merge of the chunk partials and its
+// projections are bandwidth-starved (73 us per call; dual flow 0.557 against
+// 0.399 ms with the separate kernels).
+bool pool_tail_wanted() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("IVC_POOL_TAIL");
+    v = (e && e[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
 // fused_default: use the persistent single-launch router when it applies and
 // IVC_ROUTER_FUSED does not say otherwise. It holds every SM for its whole
 // run, so it is the default only where nothing runs beside the router.
@@ -409,6 +423,25 @@ int route_impl(const void* x, const int32_t* valid_len, int T, const int32_t* im
     FusedRouterBufs f{b.Q, b.U2, b.cb, b.S, b.Z, b.z, b.O, b.q, b.h, b.u1, b.u2, b.bar};
     return launch_router_fused(r, x, valid_len, T, image_offsets, I, gate, mask, offsets, total,
                                f, L);
+  }
+  if (r->pool_mode == IVC_POOL_FOLDED && pool_tail_wanted() && pool_attend_wanted() &&
+      pool_tail_supported(D, r->heads)) {
+    // per layer: the single-pass attention, then its tail (merge, value,
+    // output and next query projections, next key fold) in one cooperative
+    // launch; layer 1's query is shared by every tile
+    IVC_TRY(launch_gemv_bf16x(static_cast<const bf16*>(r->query), D,
+                              static_cast<const bf16*>(r->Wq[0]),
+                              static_cast<const bf16*>(r->bq[0]), D, b.Q1, L));
+    IVC_TRY(launch_pool_fold_query(b.Q1, 0, 1, static_cast<const bf16*>(r->Wk[0]),
+                                   static_cast<const bf16*>(r->bk[0]), D, b.U2, b.cb, L));
+    float* mstat = b.S;
+    float* lstat = b.S + static_cast<size_t>(T) * 8 * 16;
+    for (int l = 0; l < 4; ++l) {
+      IVC_TRY(launch_pool_attend(x, b.U2, l == 0 ? 1 : T, b.cb, valid_len, T, D, r->heads, b.Z,
+                                 b.S, b.z, L, false));
+      IVC_TRY(launch_pool_tail(r, l, b.Z, mstat, lstat, T, b.O, b.q, b.Q, b.U2, b.cb, b.bar, L));
+    }
+    return gating_and_route(T, image_offsets, I, r, gate, mask, offsets, total, b, L);
   }
   if (r->pool_mode == IVC_POOL_FOLDED) {
     IVC_TRY(launch_gemv_bf16x(static_cast<const bf16*>(r->query), D,
@@ -469,12 +502,32 @@ int route_impl(const void* x, const int32_t* valid_len, int T, const int32_t* im
   return gating_and_route(T, image_offsets, I, r, gate, mask, offsets, total, b, L);
 }
 
+// The Gating as one cooperative kernel (ivc_router_coop.cu) with
+// IVC_GATING_FUSED=1. Off by default: beside the connector (16 CTAs on the
+// SMs it leaves free) it measured 66 us per call against its 13 separate
+// launches, which overlap through programmatic dependent launch (dual flow
+// 0.399 vs 0.379 ms per call on the 13-tile image).
+bool gating_fused_wanted() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("IVC_GATING_FUSED");
+    v = (e && e[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
 // Gating on the pooled vectors (in b.q), the 2-way head, then routing.
 int gating_and_route(int T, const int32_t* image_offsets, int I, const ivc_router* r, float* gate,
                      uint8_t* mask, int32_t* offsets, int32_t* total, const RouteBufs& b,
                      const Launch& L) {
   const int D = r->D;
   const int G = r->gate_hidden;
+  if (gating_fused_wanted() && gating_fused_supported(D, G)) {
+    // the whole Gating MLP and its softmax head in one cooperative launch
+    IVC_TRY(launch_gating_fused(b.q, T, D, G, r, b.h, b.u1, b.u2, gate, b.bar, L));
+    return launch_route(gate, T, image_offsets, I, r->rel_q, r->abs_t, r->quantile_scope, mask,
+                        offsets, total, L);
+  }
   for (int k = 0; k < 4; ++k) {
     IVC_TRY(launch_gemv(b.q, D, T, D, static_cast<const bf16*>(r->gW1[k]),
                         static_cast<const bf16*>(r->gb1[k]), G, b.u1, G, 1, L));

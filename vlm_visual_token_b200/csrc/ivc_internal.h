@@ -181,9 +181,19 @@ int launch_pool_vproj(const float* Z, int T, int D, const bf16* Wv, const bf16* 
 // launches): per 128-token chunk unnormalised sums Zp [T*8*16, D] and their
 // running max / sum (stats: 2 * T*8*16 floats), merged into z [T*16, D];
 // then o = Wv z + bv reads z row (tile*16 + head).
+// combine = false: the chunk partials are left for launch_pool_tail to merge.
 int launch_pool_attend(const void* x, const bf16* U2, int Tq, const float* cb,
                        const int32_t* valid_len, int T, int D, int heads, float* Zp, float* stats,
-                       float* z, const Launch& L);
+                       float* z, const Launch& L, bool combine = true);
+// The tail of folded pooling layer l as one cooperative launch of D/64 CTAs
+// (ivc_router_coop.cu): merge of the chunk partials (Zp, stats as left by
+// launch_pool_attend with combine = false), O = Wv z + bv, q = Wo O + bo, and
+// unless l is the last layer Q = Wq' q + bq' and the next layer's folded key
+// projection U2, cb. bar: one zeroed counter word.
+bool pool_tail_supported(int D, int heads);
+int launch_pool_tail(const ivc_router* r, int l, const float* Zp, const float* mstat,
+                     const float* lstat, int T, float* O, float* q, float* Q, bf16* U2, float* cb,
+                     unsigned* bar, const Launch& L);
 int launch_pool_vproj_heads(const float* z, int T, int D, const bf16* Wv, const bf16* bv, float* O,
                             const Launch& L);
 // Folded pooling through launch_pool_attend (default) or through the
@@ -229,6 +239,13 @@ int launch_router_fused(const ivc_router* r, const void* x, const int32_t* valid
 // h[t] += LN(u[t]) * gamma + beta over D (inside = 1: h[t] = LN(h[t] + u[t]) ...).
 int launch_residual_ln(float* h, const float* u, const bf16* gamma, const bf16* beta, int T,
                        int D, int inside, const Launch& L);
+// The whole Gating (4 residual blocks and the softmax head) as one
+// cooperative launch of up to 16 CTAs (ivc_gating.cu): pooled [T, D] in,
+// gate [T, 2] out; h [T, D], u1 [T, G], u2 [T, D] scratch, bar one zeroed
+// counter word.
+bool gating_fused_supported(int D, int G);
+int launch_gating_fused(const float* pooled, int T, int D, int G, const ivc_router* r, float* h,
+                        float* u1, float* u2, float* gate, unsigned* bar, const Launch& L);
 // gate[t] = softmax(Wout h[t] + bout), Wout [2, D].
 int launch_gate_head(const float* h, const bf16* Wout, const bf16* bout, int T, int D,
                      float* gate, const Launch& L);

@@ -822,7 +822,7 @@ static int launch_attend_ks(const CUtensorMap& xmap, const bf16* U2, int u2_per_
 
 int launch_pool_attend(const void* x, const bf16* U2, int Tq, const float* cb,
                        const int32_t* valid_len, int T, int D, int heads, float* Zp, float* stats,
-                       float* z, const Launch& L) {
+                       float* z, const Launch& L, bool combine) {
   if (T == 0) return IVC_OK;
   if (D % 128 != 0 || D > 1024 || heads < 1 || heads > 16 || heads * 64 != D)
     return IVC_EUNSUPPORTED;
@@ -858,7 +858,7 @@ int launch_pool_attend(const void* x, const bf16* U2, int Tq, const float* cb,
       default: rc = run(std::integral_constant<int, 8>{}); break;
     }
   }
-  if (rc != IVC_OK) return rc;
+  if (rc != IVC_OK || !combine) return rc;
   TraceScope ts("pool.combine", L.stream);
   return launch_k(pool_combine_kernel, dim3(heads, T), dim3(256), 0, L.stream, 1, Zp, mstat, lstat,
                   D, z);
