@@ -258,12 +258,13 @@ int ps_mlp(const void* x, int T, int C, bool half, int flags, const ivc_mlp* m, 
 }
 
 // The connector's Linears run as one persistent launch (ivc_gemm_graph.cuh)
-// with IVC_GEMM_GRAPH=1; otherwise one launch per Linear.
+// where the shapes allow it, unless IVC_GEMM_GRAPH=0 selects one launch per
+// Linear.
 bool gemm_graph_enabled() {
   static int v = -1;
   if (v < 0) {
     const char* e = std::getenv("IVC_GEMM_GRAPH");
-    v = (e && e[0] == '1') ? 1 : 0;
+    v = (e && e[0] == '0') ? 0 : 1;
   }
   return v == 1;
 }
