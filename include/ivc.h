@@ -201,9 +201,10 @@ int ivc_ps_project(const void* x, int T, int C, float scale, int flags, const iv
  *                  offsets[T] = total rows = 256 (T - k) + 64 k.
  * rel_q outside [0, 1] (or NaN) is IVC_EINVAL.
  * Unsupported: D != C, D % 256 != 0, heads * 64 != D, gate_hidden % 256 != 0.
- * With folded pooling, D <= 1024 and at most 16 heads, the router runs as one
- * cooperative persistent kernel that holds every SM until it ends (the
- * environment variable IVC_ROUTER_FUSED=0 selects separate kernels instead). */
+ * The router runs as a chain of kernels overlapped by programmatic dependent
+ * launch. With folded pooling, D <= 1024 and at most 16 heads, the
+ * environment variable IVC_ROUTER_FUSED=1 selects instead one cooperative
+ * persistent kernel that holds every SM until it ends. */
 int ivc_vir_route(const void* x, const int32_t* valid_len, int T, int C,
                   const int32_t* image_offsets, int I, const ivc_router* r, float* gate,
                   uint8_t* mask, int32_t* offsets, void* workspace, size_t ws_bytes,
@@ -304,7 +305,7 @@ int ivc_device_status(void* workspace, int* bits, ivc_stream_t stream);
  * IVC_DEV_WAIT_TIMEOUT in the status word, the kernel skips its remaining
  * work, lets the copies it issued land, and returns; no trap is used and the
  * context stays usable. To exercise that path, `cycles` > 0 makes the
- * persistent router (ivc_vir_route's single-kernel form) give up its
+ * persistent router (ivc_vir_route's single-kernel form, IVC_ROUTER_FUSED=1) give up its
  * software grid barriers from the one before the gating head on after that
  * many clock cycles; no bulk copy is in flight at those barriers. With a
  * limit of a few cycles the call's outputs are invalid and the status bit is

@@ -414,8 +414,10 @@ bool pool_tail_wanted() {
 }
 
 // fused_default: use the persistent single-launch router when it applies and
-// IVC_ROUTER_FUSED does not say otherwise. It holds every SM for its whole
-// run, so it is the default only where nothing runs beside the router.
+// IVC_ROUTER_FUSED does not say otherwise. The separate kernels, overlapped
+// through programmatic dependent launch, now measure faster even alone
+// (0.191 against 0.224 ms per ivc_vir_route on the 13-tile image), so every
+// caller passes false; IVC_ROUTER_FUSED=1 selects the persistent kernel.
 int route_impl(const void* x, const int32_t* valid_len, int T, const int32_t* image_offsets,
                int I, const ivc_router* r, float* gate, uint8_t* mask, int32_t* offsets,
                int32_t* total, const RouteBufs& b, const Launch& L, bool fused_default) {
@@ -544,15 +546,16 @@ int gating_and_route(int T, const int32_t* image_offsets, int I, const ivc_route
 }
 
 // Connector GEMMs beside the router in ivc_flash_compress: SMs they leave to
-// the router's small kernels when that costs no round of tiles
-// (IVC_DUAL_RESERVE, default 20: measured 0.555 -> 0.538 ms per call on the
-// 13-tile image; 36 and mlp2-first measured no better), and whether mlp2 runs
-// before mlp1 (IVC_DUAL_MLP2_FIRST).
+// the router's small kernels (IVC_DUAL_RESERVE, default 36). With the
+// connector's Linears in one persistent launch the router is the longer of
+// the two: 0.382 / 0.377 / 0.367 / 0.352 / 0.353 ms per call on the 13-tile
+// image for 12 / 20 / 28 / 36 / 44 SMs. IVC_DUAL_MLP2_FIRST=1 puts mlp2
+// before mlp1 when the Linears run as separate launches.
 int dual_reserve_sms() {
   static int v = -1;
   if (v < 0) {
     const char* e = std::getenv("IVC_DUAL_RESERVE");
-    v = e ? std::atoi(e) : 20;
+    v = e ? std::atoi(e) : 36;
     if (v < 0) v = 0;
   }
   return v;
@@ -802,7 +805,7 @@ int ivc_vir_route(const void* x, const int32_t* valid_len, int T, int C,
   RouteBufs b;
   carve_route(cv, r, T, b);
   return route_impl(x, valid_len, T, image_offsets, I, r, gate, mask, offsets, nullptr, b, L,
-                    true);
+                    false);
 }
 
 int ivc_route(const float* gate, int T, const int32_t* image_offsets, int I, double rel_q,
@@ -954,7 +957,7 @@ int ivc_flash_compress_routed(const void* x, const int32_t* valid_len, int T, in
   IVC_TRY(launch_ps_stats(static_cast<const bf16*>(x), T, C, f.b1.mean, f.b1.rstd, f.b2.mean,
                           f.b2.rstd, L));
   IVC_TRY(route_impl(x, valid_len, T, image_offsets, I, r, gate, mask, offsets, total, f.br, L,
-                     true));
+                     false));
   const ListBufs& lb = f.lists;
   IVC_TRY(launch_route_lists(mask, offsets, T, lb.list_u, lb.base_u, lb.list_c, lb.base_c,
                              lb.counts, L));

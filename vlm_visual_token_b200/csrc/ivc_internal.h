@@ -181,6 +181,13 @@ int launch_pool_vproj(const float* Z, int T, int D, const bf16* Wv, const bf16* 
 // launches): per 128-token chunk unnormalised sums Zp [T*8*16, D] and their
 // running max / sum (stats: 2 * T*8*16 floats), merged into z [T*16, D];
 // then o = Wv z + bv reads z row (tile*16 + head).
+// The same chunk partials from the tensor-core (tcgen05) form of the
+// attention (ivc_attend_tc.cu), selected inside launch_pool_attend with
+// IVC_ATTEND_TC=1.
+bool attend_tc_wanted();
+int launch_pool_attend_tc(const void* x, const bf16* U2, int Tq, const float* cb,
+                          const int32_t* valid_len, int T, int D, int heads, float* Zp,
+                          float* stats, const Launch& L);
 // combine = false: the chunk partials are left for launch_pool_tail to merge.
 int launch_pool_attend(const void* x, const bf16* U2, int Tq, const float* cb,
                        const int32_t* valid_len, int T, int D, int heads, float* Zp, float* stats,

@@ -840,7 +840,9 @@ int launch_pool_attend(const void* x, const bf16* U2, int Tq, const float* cb,
   const int u2_per_tile = Tq == 1 ? 0 : 1;
   const int cb_stride = Tq == 1 ? 0 : 16;
   int rc;
-  {
+  if (attend_tc_wanted()) {
+    rc = launch_pool_attend_tc(x, U2, Tq, cb, valid_len, T, D, heads, Zp, stats, L);
+  } else {
     TraceScope ts("pool.attend", L.stream);
     // one instantiation per width (the warps' register tiles are sized by it)
     auto run = [&](auto ks) {
