@@ -581,7 +581,8 @@ print("variant ok")
 
 @pytest.mark.parametrize("env", [{"IVC_GEMM_WIDE": "1"}, {"IVC_GEMM_PAIRS": "0"},
                                  {"IVC_ROUTER_FUSED": "1"}, {"IVC_POOL_ATTEND": "0"},
-                                 {"IVC_GATING_FUSED": "1"}, {"IVC_POOL_TAIL": "1"}])
+                                 {"IVC_GATING_FUSED": "1"}, {"IVC_POOL_TAIL": "1"},
+                                 {"IVC_ATTEND_TC": "0"}, {"IVC_GEMM_GRAPH": "0"}])
 def test_flash_kernel_variants(env):
     """The opt-in kernel variants (512-wide pair tiles with split-K, single-CTA
     256-wide tiles, the persistent router inside the dual flow, the pooling as

@@ -8,8 +8,8 @@
 // s_t = x_t . u_h + c_h over the raw features x, and the weighted sum is
 // z_h = sum_t softmax(s)_t x_t (the value projection follows on z_h).
 //
-// One CTA per (tile, chunk of 128 tokens), like the mma.sync form it
-// replaces, with the same outputs: the chunk's unnormalised sums
+// Per (tile, chunk of 128 tokens), like the mma.sync form it replaces, with
+// the same outputs: the chunk's unnormalised sums
 // Zc_h = sum_t exp(s_t - m_h) x_t, its max m_h and sum l_h (pool_combine
 // merges a tile's 8 chunks). Per chunk:
 //   scores   S[128 tokens x 32] = X[128 x D] . U2[32 x D]^T   (M 128, N 32;
@@ -65,17 +65,46 @@ struct AtSmem {
   static constexpr uint32_t TOTAL = 1024 + RING + U2 + AT_P;
 };
 
+// Items are (tile, chunk) pairs, item = tile * 8 + chunk; CTA b takes items
+// b, b + gridDim.x, ... (a grid as wide as the SMs the kernel may use), so
+// that one item's loads and score MMAs overlap the previous item's weighted
+// sums and epilogue. Barriers between the roles, for the k-th item with a
+// valid token (phase k & 1): ufull / uempty (the U2 buffer: loaded /
+// no longer read by the score MMAs), sfull / sfree (S in TMEM: complete /
+// read by the softmax), pfull (P written), zfull / zfree (Z^T in TMEM:
+// complete / drained).
+struct AtItem {
+  int tile, chunk, nvalid;
+};
+
+// `status` is non-null in one thread only: the one that reports a length
+// outside [1, 1024].
+__device__ __forceinline__ AtItem at_item(int item, const int32_t* valid_len, int* status) {
+  AtItem r;
+  r.tile = item / AT_NCH;
+  r.chunk = item % AT_NCH;
+  int n = 1024;
+  if (valid_len != nullptr) {
+    n = valid_len[r.tile];
+    if (n < 1 || n > 1024) {
+      if (r.chunk == 0 && status != nullptr) atomicOr(status, DEV_BAD_VALID_LEN);
+      n = n < 1 ? 1 : 1024;
+    }
+  }
+  r.nvalid = min(AT_TOK, max(0, n - r.chunk * AT_TOK));
+  return r;
+}
+
 template <int NB>
 __global__ void __launch_bounds__(AT_THREADS, 1)
     pool_attend_tc_kernel(const __grid_constant__ CUtensorMap xmap,
                           const __grid_constant__ CUtensorMap umap, int u2_per_tile,
                           const float* __restrict__ cb, int cb_stride,
-                          const int32_t* __restrict__ valid_len, int heads, float* __restrict__ Zp,
-                          float* __restrict__ mstat, float* __restrict__ lstat,
-                          int* __restrict__ status) {
+                          const int32_t* __restrict__ valid_len, int heads, int n_items,
+                          float* __restrict__ Zp, float* __restrict__ mstat,
+                          float* __restrict__ lstat, int* __restrict__ status) {
   using S = AtSmem<NB>;
   constexpr int D = S::D;
-  constexpr int NBOX = 2 * NB;  // x boxes of both passes
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -83,41 +112,22 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   uint8_t* su2 = sm + S::RING;
   uint8_t* sp = su2 + S::U2;
   __shared__ __align__(8) uint64_t full[AT_STAGES], empty[AT_STAGES];
-  __shared__ __align__(8) uint64_t ubar, sbar, pbar, zbar;
+  __shared__ __align__(8) uint64_t ufull, uempty, sfull, sfree, pfull, zfull, zfree;
   __shared__ uint32_t s_tmem;
   __shared__ float red[2][4][16];  // per-warp max, then sum, of each head
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x / AT_NCH, chunk = blockIdx.x % AT_NCH;
-  const int tok0 = chunk * AT_TOK;
-  const size_t row0 = (static_cast<size_t>(tile) * AT_NCH + chunk) * 16;
-  // valid_len is an input of the call
-  int n = 1024;
-  if (valid_len != nullptr) {
-    n = valid_len[tile];
-    if (n < 1 || n > 1024) {
-      if (threadIdx.x == 0 && chunk == 0) atomicOr(status, DEV_BAD_VALID_LEN);
-      n = n < 1 ? 1 : 1024;
-    }
-  }
-  const int nvalid = min(AT_TOK, max(0, n - tok0));
-  if (nvalid == 0) {  // every token of the chunk is padding
-    pdl_wait();
-    pdl_trigger();
-    if (threadIdx.x < 16) {
-      mstat[row0 + threadIdx.x] = -INFINITY;
-      lstat[row0 + threadIdx.x] = 0.f;
-    }
-    return;
-  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < AT_STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(&ubar, 1);
-    mbar_init(&sbar, 1);
-    mbar_init(&pbar, 128);
-    mbar_init(&zbar, 1);
+    mbar_init(&ufull, 1);
+    mbar_init(&uempty, 1);
+    mbar_init(&sfull, 1);
+    mbar_init(&sfree, 128);
+    mbar_init(&pfull, 128);
+    mbar_init(&zfull, 1);
+    mbar_init(&zfree, 128);
     fence_mbar_init();
     tma_prefetch_desc(&xmap);
     tma_prefetch_desc(&umap);
@@ -137,20 +147,32 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
-      // x is an input: its first boxes go out before waiting for the
-      // previous kernel, which writes U2 (the folded query)
-      const int xrow = tile * 1024 + tok0;
-      for (int it = 0; it < NBOX && ok; ++it) {
-        const int s = it % AT_STAGES;
-        const uint32_t ph = (it / AT_STAGES) & 1;
-        if (!mbar_wait(&empty[s], ph ^ 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(&full[s], AT_BOX);
-        tma_load_3d(ring + s * AT_BOX, &xmap, &full[s], 0, xrow, 2 * (it % NB));
-        if (it == (NBOX < AT_STAGES ? NBOX : AT_STAGES) - 1) {
-          pdl_wait();
-          mbar_arrive_expect_tx(&ubar, S::U2);
-          tma_load_3d(su2, &umap, &ubar, 0, u2_per_tile ? tile * 32 : 0, 0);
+      // x is an input: the first item's first boxes go out before waiting for
+      // the previous kernel, which writes U2 (the folded query)
+      int g = 0, k = 0;
+      bool waited = false;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        const AtItem a = at_item(item, valid_len, nullptr);
+        if (a.nvalid == 0) continue;
+        const int xrow = a.tile * 1024 + a.chunk * AT_TOK;
+        if (waited) {  // the U2 buffer is free once the previous item's score MMAs are done
+          if (!mbar_wait(&uempty, (k & 1) ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&ufull, S::U2);
+          tma_load_3d(su2, &umap, &ufull, 0, u2_per_tile ? a.tile * 32 : 0, 0);
         }
+        for (int it = 0; it < 2 * NB; ++it, ++g) {
+          const int s = g % AT_STAGES;
+          if (!mbar_wait(&empty[s], ((g / AT_STAGES) & 1) ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[s], AT_BOX);
+          tma_load_3d(ring + s * AT_BOX, &xmap, &full[s], 0, xrow, 2 * (it % NB));
+          if (!waited && it == (2 * NB < AT_STAGES ? 2 * NB : AT_STAGES) - 1) {
+            pdl_wait();
+            waited = true;
+            mbar_arrive_expect_tx(&ufull, S::U2);
+            tma_load_3d(su2, &umap, &ufull, 0, u2_per_tile ? a.tile * 32 : 0, 0);
+          }
+        }
+        ++k;
       }
     }
   } else if (warp == 1) {
@@ -158,65 +180,96 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       // ------------------------------------------------------------ MMA issuer
       const uint32_t idesc_s = idesc_bf16_f32(AT_TOK, 32);              // A, B K-major
       const uint32_t idesc_z = idesc_bf16_f32(128, 32) | (1u << 15);   // A MN-major
-      if (!mbar_wait(&ubar, 0)) ok = false;
-      tc_fence_after();
-      // scores: S += X_box(chunk j) . U2(chunk 2b + j)^T
-      for (int b = 0; b < NB && ok; ++b) {
-        const int s = b % AT_STAGES;
-        if (!mbar_wait(&full[s], (b / AT_STAGES) & 1)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t xa = smem_u32(ring + s * AT_BOX);
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const uint64_t ad = sw128_kmajor_desc(xa + j * AT_HALF);
-          const uint64_t bd = sw128_kmajor_desc(smem_u32(su2) + (2 * b + j) * 4096);
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16(tmem, ad + 2 * k, bd + 2 * k, idesc_s, (b | j | k) != 0 ? 1u : 0u);
-        }
-        umma_commit(&empty[s]);
-      }
-      if (ok) umma_commit(&sbar);
-      // weighted sums once the softmax weights are in shared memory
-      if (ok && !mbar_wait(&pbar, 0)) ok = false;
-      tc_fence_after();
       const uint32_t pa = smem_u32(sp);
-      for (int b = 0; b < NB && ok; ++b) {
-        const int it = NB + b;
-        const int s = it % AT_STAGES;
-        if (!mbar_wait(&full[s], (it / AT_STAGES) & 1)) { ok = false; break; }
+      int g = 0, k = 0;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        const AtItem a = at_item(item, valid_len, nullptr);
+        if (a.nvalid == 0) continue;
+        const uint32_t ph = k & 1;
+        // scores: S += X_box(chunk j) . U2(chunk 2b + j)^T, once U2 is loaded
+        // and the softmax has read the previous item's S
+        if (!mbar_wait(&ufull, ph) || !mbar_wait(&sfree, ph ^ 1)) { ok = false; break; }
         tc_fence_after();
-        // A = this box read MN-major: 64-channel atoms 16 KB apart, 8-token
-        // groups 1024 B apart; 16 tokens per MMA = 2048 B
-        const uint64_t ad = sw128_mnmajor_desc(smem_u32(ring + s * AT_BOX), AT_HALF);
+        for (int b = 0; b < NB && ok; ++b, ++g) {
+          const int s = g % AT_STAGES;
+          if (!mbar_wait(&full[s], (g / AT_STAGES) & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t xa = smem_u32(ring + s * AT_BOX);
 #pragma unroll
-        for (int k = 0; k < AT_TOK / 16; ++k) {
-          const uint64_t bd = sw128_kmajor_desc(pa + (k >> 2) * 4096) + 2 * (k & 3);
-          umma_bf16(tmem + 32 + 32 * b, ad + ((2048 * k) >> 4), bd, idesc_z, k != 0 ? 1u : 0u);
+          for (int j = 0; j < 2; ++j) {
+            const uint64_t ad = sw128_kmajor_desc(xa + j * AT_HALF);
+            const uint64_t bd = sw128_kmajor_desc(smem_u32(su2) + (2 * b + j) * 4096);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16(tmem, ad + 2 * kk, bd + 2 * kk, idesc_s, (b | j | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
         }
-        umma_commit(&empty[s]);
+        if (!ok) break;
+        umma_commit(&sfull);
+        umma_commit(&uempty);
+        // weighted sums once the softmax weights are in shared memory and the
+        // epilogue has drained the previous item's sums
+        if (!mbar_wait(&pfull, ph) || !mbar_wait(&zfree, ph ^ 1)) { ok = false; break; }
+        tc_fence_after();
+        for (int b = 0; b < NB && ok; ++b, ++g) {
+          const int s = g % AT_STAGES;
+          if (!mbar_wait(&full[s], (g / AT_STAGES) & 1)) { ok = false; break; }
+          tc_fence_after();
+          // A = this box read MN-major: 64-channel atoms 16 KB apart, 8-token
+          // groups 1024 B apart; 16 tokens per MMA = 2048 B
+          const uint64_t ad = sw128_mnmajor_desc(smem_u32(ring + s * AT_BOX), AT_HALF);
+#pragma unroll
+          for (int kk = 0; kk < AT_TOK / 16; ++kk) {
+            const uint64_t bd = sw128_kmajor_desc(pa + (kk >> 2) * 4096) + 2 * (kk & 3);
+            umma_bf16(tmem + 32 + 32 * b, ad + ((2048 * kk) >> 4), bd, idesc_z,
+                      kk != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        umma_commit(&zfull);
+        ++k;
       }
-      if (ok) umma_commit(&zbar);
     }
   } else {
     // -------------------------------------------------------- softmax, epilogue
     const int quad = warp & 3;
     const int t = quad * 32 + lane;  // token of the chunk = TMEM lane
-    const bool valid = t < nvalid;
-    pdl_wait();  // cb is written by the previous kernel
-    float c_h[16];
+    pdl_wait();                      // cb is written by the previous kernel
+    int k = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      const AtItem a = at_item(item, valid_len, (warp == 2 && lane == 0) ? status : nullptr);
+      const size_t row0 = (static_cast<size_t>(a.tile) * AT_NCH + a.chunk) * 16;
+      if (a.nvalid == 0) {  // every token of the chunk is padding: l = 0
+        if (quad == 0 && lane < 16) {
+          mstat[row0 + lane] = -INFINITY;
+          lstat[row0 + lane] = 0.f;
+        }
+        continue;
+      }
+      const uint32_t ph = k & 1;
+      ++k;
+      const bool valid = t < a.nvalid;
+      float c_h[16];
 #pragma unroll
-    for (int h = 0; h < 16; ++h)
-      c_h[h] = h < heads ? cb[static_cast<size_t>(tile) * cb_stride + h] : 0.f;
-    ok = __all_sync(0xffffffffu, mbar_wait(&sbar, 0));
-    float e[16];
-    float M[16], Lh[16];
-    if (ok) {
+      for (int h = 0; h < 16; ++h)
+        c_h[h] = h < heads ? cb[static_cast<size_t>(a.tile) * cb_stride + h] : 0.f;
+      // after a wait that ran out the warps keep their named barriers in step
+      // (two per item) but do no more work
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sfull, ph));
+      if (!ok) {
+        at_epi_sync();
+        at_epi_sync();
+        continue;
+      }
       tc_fence_after();
       uint32_t r[32];
       tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16), r);
       tmem_ld_wait();
-      float sh[16];
+      tc_fence_before();
+      mbar_arrive(&sfree);  // S is read: the next item's scores may overwrite it
+      float sh[16], e[16], M[16];
 #pragma unroll
       for (int h = 0; h < 16; ++h) {
         sh[h] = (valid && h < heads)
@@ -240,52 +293,49 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       }
       // P [32 rows x 128 tokens] bf16, K-major, 128-byte swizzle: row j of
       // token half a at a * 4096 + j * 128, 16-byte unit (t % 64) / 8 XOR j % 8
-      const int a = t >> 6, tt = t & 63;
+      // (the previous item's weighted sums, which read P, are complete: its
+      // Z^T was drained below before this item's softmax)
+      const int ah = t >> 6, tt = t & 63;
 #pragma unroll
       for (int h = 0; h < 16; ++h) {
         const bf16 hi = __float2bfloat16_rn(e[h]);
         const bf16 lo = __float2bfloat16_rn(e[h] - __bfloat162float(hi));
         const int j0 = h, j1 = 16 + h;
-        *reinterpret_cast<bf16*>(sp + a * 4096 + j0 * 128 + ((((tt >> 3) ^ (j0 & 7))) << 4) +
+        *reinterpret_cast<bf16*>(sp + ah * 4096 + j0 * 128 + (((tt >> 3) ^ (j0 & 7)) << 4) +
                                  (tt & 7) * 2) = hi;
-        *reinterpret_cast<bf16*>(sp + a * 4096 + j1 * 128 + ((((tt >> 3) ^ (j1 & 7))) << 4) +
+        *reinterpret_cast<bf16*>(sp + ah * 4096 + j1 * 128 + (((tt >> 3) ^ (j1 & 7)) << 4) +
                                  (tt & 7) * 2) = lo;
       }
       fence_async_shared();
-      mbar_arrive(&pbar);
+      mbar_arrive(&pfull);
       at_epi_sync();
-#pragma unroll
-      for (int h = 0; h < 16; ++h)
-        Lh[h] = (red[1][0][h] + red[1][1][h]) + (red[1][2][h] + red[1][3][h]);
       if (quad == 0 && lane < 16) {
         float mv = 0.f, lv = 0.f;
 #pragma unroll
         for (int h = 0; h < 16; ++h)
           if (h == lane) {
             mv = M[h];
-            lv = Lh[h];
+            lv = (red[1][0][h] + red[1][1][h]) + (red[1][2][h] + red[1][3][h]);
           }
         mstat[row0 + lane] = lane < heads ? mv : -INFINITY;
         lstat[row0 + lane] = lane < heads ? lv : 0.f;
       }
-      ok = __all_sync(0xffffffffu, mbar_wait(&zbar, 0));
-    } else {
-      at_epi_sync();
-      at_epi_sync();
-    }
-    if (ok) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&zfull, ph));
+      if (!ok) continue;
       tc_fence_after();
 #pragma unroll 1
       for (int b = 0; b < NB; ++b) {
-        uint32_t r[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + 32 + 32 * b, r);
+        uint32_t z[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + 32 + 32 * b, z);
         tmem_ld_wait();
         const int c = b * 128 + quad * 32 + lane;  // channel = TMEM lane of block b
 #pragma unroll
         for (int h = 0; h < 16; ++h)
           if (h < heads)
-            Zp[(row0 + h) * D + c] = __uint_as_float(r[h]) + __uint_as_float(r[16 + h]);
+            Zp[(row0 + h) * D + c] = __uint_as_float(z[h]) + __uint_as_float(z[16 + h]);
       }
+      tc_fence_before();
+      mbar_arrive(&zfree);  // Z^T is drained: the next item's sums may overwrite it
     }
   }
   if (!ok && status != nullptr) atomicOr(status, DEV_WAIT_TIMEOUT);
@@ -304,18 +354,24 @@ int launch_attend_tc_nb(const CUtensorMap& xmap, const CUtensorMap& umap, int u2
   using S = AtSmem<NB>;
   if (smem_optin(reinterpret_cast<const void*>(pool_attend_tc_kernel<NB>), S::TOTAL) != IVC_OK)
     return IVC_ECUDA;
-  return launch_k(pool_attend_tc_kernel<NB>, dim3(T * AT_NCH), dim3(AT_THREADS), S::TOTAL,
-                  L.stream, 1, xmap, umap, u2_per_tile, cb, cb_stride, valid_len, heads, Zp, mstat,
-                  lstat, L.status);
+  const int items = T * AT_NCH;
+  int grid = L.sm_budget > 0 ? L.sm_budget : num_sms();
+  if (grid > items) grid = items;
+  return launch_k(pool_attend_tc_kernel<NB>, dim3(grid), dim3(AT_THREADS), S::TOTAL, L.stream, 1,
+                  xmap, umap, u2_per_tile, cb, cb_stride, valid_len, heads, items, Zp, mstat, lstat,
+                  L.status);
 }
 
 }  // namespace
 
+// The attention on tcgen05 unless IVC_ATTEND_TC=0 selects the mma.sync form
+// (ivc_router.cu): measured 0.183 against 0.196 ms per ivc_vir_route on the
+// 13-tile image, the same within noise inside the dual flow.
 bool attend_tc_wanted() {
   static int v = -1;
   if (v < 0) {
     const char* e = std::getenv("IVC_ATTEND_TC");
-    v = (e && e[0] == '1') ? 1 : 0;
+    v = (e && e[0] == '0') ? 0 : 1;
   }
   return v == 1;
 }

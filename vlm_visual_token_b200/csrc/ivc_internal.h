@@ -22,7 +22,8 @@ constexpr int DEV_BAD_PROMPT = IVC_DEV_BAD_PROMPT;
 
 struct Launch {
   cudaStream_t stream;
-  int* status;  // device status word (workspace header)
+  int* status;     // device status word (workspace header)
+  int sm_budget;   // > 0: SMs a persistent kernel may assume free (beside other work); 0: all
 };
 
 // Brackets one kernel launch with CUDA events when tracing is on (ivc_trace.cu).
