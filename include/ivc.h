@@ -114,7 +114,10 @@ typedef struct ivc_mlp {
  * Wout [2, D]. Routing: tile t is compressed iff
  * gate[t,0] > quantile(gate[.,0] over its group, rel_q) and gate[t,0] >= abs_t,
  * quantile by linear interpolation in fp64; group = image (scope 0) or the
- * whole batch (scope 1). */
+ * whole batch (scope 1).
+ * The `fold_*` fields are optional device pointers written by
+ * ivc_router_fold() (folded pooling only); all NULL: every call projects the
+ * first layer's query and applies Wo and the next Wq one after the other. */
 typedef struct ivc_router {
   int D;
   int heads;
@@ -129,6 +132,11 @@ typedef struct ivc_router {
   int pool_mode;      /* IVC_POOL_FOLDED (0) or IVC_POOL_LITERAL (1) */
   int gate_residual;  /* 0: h <- h + LN(u) (the listed block inside the residual);
                          1: h <- LN(h + u) (residual inside the LayerNorm) */
+  const void* fold_u1;      /* bf16 [32, D]: layer 1's key-folded query, u_h = Wk_h^T Q_h / 8
+                               with Q = Wq_1 query + bq_1; rows h hi, 16 + h lo part */
+  const float* fold_c1;     /* fp32 [16]: bk_h . Q_h / 8 */
+  const void* fold_wqo[3];  /* bf16 [D, 2D]: P_l = Wq_{l+2} Wo_{l+1}, row n = hi | lo of P_l[n,:] */
+  const float* fold_bqo[3]; /* fp32 [D]: Wq_{l+2} bo_{l+1} + bq_{l+2} */
 } ivc_router;
 
 /* How CrossAttentionPooling is evaluated; both compute the same function.
@@ -173,6 +181,25 @@ size_t ivc_workspace_size(int op, int T, int C, const ivc_mlp* m, const ivc_mlp*
  * on success m->fold_* point into it. */
 size_t ivc_mlp_fold_size(const ivc_mlp* m);
 int ivc_mlp_fold(ivc_mlp* m, void* dst, size_t dst_bytes, ivc_stream_t stream);
+
+/* Fold the router's weights once per set of weights (folded pooling,
+ * pool_mode = IVC_POOL_FOLDED, only). [VIR] section 2 chains the four pooling
+ * layers with nothing between one layer's output projection and the next
+ * layer's query projection, and starts from a learnable query, so
+ *   layer 1's query Q_1 = Wq_1 query + bq_1 and its key fold u1, c1 depend on
+ *   the weights alone, and
+ *   Wq_{l+1} (Wo_l o + bo_l) + bq_{l+1} = P_l o + (Wq_{l+1} bo_l + bq_{l+1})
+ *   with P_l = Wq_{l+1} Wo_l (l = 1..3),
+ * an exact rewrite that saves five dependent launches per call. P_l is formed
+ * in fp32 and kept as a bf16 hi | lo pair (about 16 significant bits); the
+ * router's vectors stay fp32.
+ * `dst` (device, 256-byte aligned, >= ivc_router_fold_size(r) bytes) receives
+ * the arrays; on success r->fold_* point into it and every later call with `r`
+ * uses them. Returns IVC_EUNSUPPORTED for literal pooling or an unsupported
+ * shape, IVC_EINVAL for missing weights, IVC_EWORKSPACE for a short `dst`.
+ * Asynchronous on `stream`. */
+size_t ivc_router_fold_size(const ivc_router* r);
+int ivc_router_fold(ivc_router* r, void* dst, size_t dst_bytes, ivc_stream_t stream);
 
 /* pixel_shuffle + connector MLP ([PS] "extract_feature() 完整调用链" steps 5-8;
  * [DP] table "三档 Token 规模").

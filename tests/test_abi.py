@@ -172,3 +172,61 @@ def test_route_rejects_bad_arguments_without_touching_the_gpu():
     y = ctypes.c_void_p(1 << 26)
     assert L.ivc_vir_route(x, None, 1, 1024, x, 1, ctypes.byref(r), y, y, y, ws, 1 << 40,
                            None) == -1
+
+
+def _router_struct(ivc, D=1024):
+    r = ivc._CRouter()
+    r.D, r.heads, r.gate_hidden = D, D // 64, 1024
+    r.query = r.gWout = 1 << 28
+    for k in ("Wq", "Wk", "Wv", "Wo", "gW1", "gW2", "gln_g", "gln_b"):
+        arr = getattr(r, k)
+        for l in range(4):
+            arr[l] = 1 << 28
+    return r
+
+
+def test_router_fold_size_and_argument_checks_without_touching_the_gpu():
+    """ivc_router_fold (InternVL3_5-4B-Flash article, section 2: the pooling
+    layers chain with nothing between Wo_l and Wq_{l+1}): its buffer holds the
+    first layer's query (fp32 D), its split key fold (bf16 32 x D) and bias
+    term (fp32 16), and per later layer P = Wq Wo as a bf16 hi | lo pair
+    (D x 2D) with its fp32 bias (D), each piece 256-byte aligned. Every check
+    runs before the GPU is touched."""
+    import vlm_visual_token_b200 as ivc
+    L = ivc.lib()
+    P = ctypes.byref
+    r = _router_struct(ivc)
+
+    def a(n):
+        return (n + 255) // 256 * 256
+
+    D = 1024
+    want = a(4 * D) + a(2 * 32 * D) + a(4 * 16) + 3 * (a(2 * 2 * D * D) + a(4 * D))
+    assert L.ivc_router_fold_size(P(r)) == want
+    lit = _router_struct(ivc)
+    lit.pool_mode = 1
+    assert L.ivc_router_fold_size(P(lit)) == 0
+    dst = ctypes.c_void_p(1 << 30)
+    assert L.ivc_router_fold(P(lit), dst, want, None) == -2
+    assert L.ivc_router_fold(P(r), None, want, None) == -1
+    assert L.ivc_router_fold(P(r), ctypes.c_void_p((1 << 30) + 16), want, None) == -6
+    assert L.ivc_router_fold(P(r), dst, want - 1, None) == -3
+    no_query = _router_struct(ivc)
+    no_query.query = None
+    assert L.ivc_router_fold(P(no_query), dst, want, None) == -1
+    # the fold fields are all or none, and only with folded pooling
+    part = _router_struct(ivc)
+    part.fold_u1 = 1 << 29
+    x = ctypes.c_void_p(1 << 24)
+    y = ctypes.c_void_p(1 << 26)
+    ws = ctypes.c_void_p(1 << 20)
+    assert L.ivc_vir_route(x, None, 1, 1024, x, 1, P(part), y, y, y, ws, 1 << 40, None) == -1
+    full = _router_struct(ivc)
+    full.fold_u1 = full.fold_c1 = 1 << 29
+    for l in range(3):
+        full.fold_wqo[l] = full.fold_bqo[l] = 1 << 29
+    full.pool_mode = 1
+    assert L.ivc_vir_route(x, None, 1, 1024, x, 1, P(full), y, y, y, ws, 1 << 40, None) == -1
+    full.fold_c1 = (1 << 29) + 4
+    full.pool_mode = 0
+    assert L.ivc_vir_route(x, None, 1, 1024, x, 1, P(full), y, y, y, ws, 1 << 40, None) == -6

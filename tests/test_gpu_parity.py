@@ -148,8 +148,8 @@ def _route_check(ivc, inp, gate, mask, offsets, sample=None, scope=0, rel_q=0.1,
     return err
 
 
-@pytest.mark.parametrize("pool_mode", [0, 1])
-def test_vir_route_small_with_padding(pool_mode):
+@pytest.mark.parametrize("pool_mode,fold", [(0, True), (0, False), (1, False)])
+def test_vir_route_small_with_padding(pool_mode, fold):
     ivc = _ivc()
     w = small_workload(C=256, H=128, tiles=(3, 1, 5), var=0.6)
     inp = W.make(w, affine="random")
@@ -157,7 +157,8 @@ def test_vir_route_small_with_padding(pool_mode):
     vl[1] = 1   # a single valid token
     inp["valid_len"] = vl
     inp["x"] = W.features(inp["T"], 256, 1234 + 90, vl)
-    r = ivc.Router(inp["router"], pool_mode=pool_mode)
+    r = ivc.Router(inp["router"], pool_mode=pool_mode, fold=fold)
+    assert (r.folded is not None) == fold
     ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_VIR_ROUTE, inp["T"], 256, r=r))
     gate, mask, offsets = ivc.vir_route(inp["x"].cuda(), vl.cuda(), inp["image_offsets"].cuda(), r,
                                         workspace=ws)
@@ -167,11 +168,11 @@ def test_vir_route_small_with_padding(pool_mode):
     assert to_np(mask)[3] == 0  # the one-tile image is never compressed
 
 
-@pytest.mark.parametrize("pool_mode", [0, 1])
-def test_vir_route_batch_scope(pool_mode):
+@pytest.mark.parametrize("pool_mode,fold", [(0, True), (0, False), (1, False)])
+def test_vir_route_batch_scope(pool_mode, fold):
     ivc = _ivc()
     inp = W.make(small_workload(C=256, H=128, tiles=(4, 4)), affine="random")
-    r = ivc.Router(inp["router"], scope=1, pool_mode=pool_mode)
+    r = ivc.Router(inp["router"], scope=1, pool_mode=pool_mode, fold=fold)
     gate, mask, offsets = ivc.vir_route(inp["x"].cuda(), None, inp["image_offsets"].cuda(), r)
     torch.cuda.synchronize()
     _route_check(ivc, inp, gate, mask, offsets, scope=1)
@@ -280,12 +281,12 @@ def _flash_check(ivc, inp, res, tiles=None, rel_q=0.1, abs_t=0.5):
     return stats
 
 
-@pytest.mark.parametrize("pool_mode", [0, 1])
-def test_flash_compress_small(pool_mode):
+@pytest.mark.parametrize("pool_mode,fold", [(0, True), (0, False), (1, False)])
+def test_flash_compress_small(pool_mode, fold):
     ivc = _ivc()
     inp = W.make(small_workload(C=256, H=192, tiles=(3, 1, 4), var=0.3), affine="random")
     m1, m2 = ivc.Mlp(inp["mlp1"]), ivc.Mlp(inp["mlp2"]).fold()
-    r = ivc.Router(inp["router"], pool_mode=pool_mode)
+    r = ivc.Router(inp["router"], pool_mode=pool_mode, fold=fold)
     ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_FLASH, inp["T"], 256, m1, m2, r))
     res = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(), inp["image_offsets"].cuda(),
                              m1, m2, r, workspace=ws)
@@ -324,13 +325,13 @@ def test_flash_compress_empty():
     assert int(res["total"].item()) == 0 and int(res["offsets"][0].item()) == 0
 
 
-@pytest.mark.parametrize("pool_mode", [0, 1])
-def test_flash_2b_13tiles_full(pool_mode):
+@pytest.mark.parametrize("pool_mode,fold", [(0, True), (0, False), (1, False)])
+def test_flash_2b_13tiles_full(pool_mode, fold):
     """The benchmark workload, every output checked against the oracle."""
     ivc = _ivc()
     inp = W.make("flash_2b_13tiles")
     m1, m2 = ivc.Mlp(inp["mlp1"]).fold(), ivc.Mlp(inp["mlp2"]).fold()
-    r = ivc.Router(inp["router"], pool_mode=pool_mode)
+    r = ivc.Router(inp["router"], pool_mode=pool_mode, fold=fold)
     res = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(), inp["image_offsets"].cuda(),
                              m1, m2, r)
     torch.cuda.synchronize()
@@ -381,12 +382,12 @@ def _routed_vs_dual(ivc, inp, m1, m2, r, routed_res):
     assert same > 0
 
 
-@pytest.mark.parametrize("pool_mode", [0, 1])
-def test_flash_routed_small(pool_mode):
+@pytest.mark.parametrize("pool_mode,fold", [(0, True), (0, False), (1, False)])
+def test_flash_routed_small(pool_mode, fold):
     ivc = _ivc()
     inp = W.make(small_workload(C=256, H=192, tiles=(3, 1, 4), var=0.3), affine="random")
     m1, m2 = ivc.Mlp(inp["mlp1"]), ivc.Mlp(inp["mlp2"]).fold()
-    r = ivc.Router(inp["router"], pool_mode=pool_mode)
+    r = ivc.Router(inp["router"], pool_mode=pool_mode, fold=fold)
     ws = ivc.new_workspace(ivc.workspace_size(ivc.OP_FLASH, inp["T"], 256, m1, m2, r))
     res = ivc.flash_compress(inp["x"].cuda(), inp["valid_len"].cuda(), inp["image_offsets"].cuda(),
                              m1, m2, r, workspace=ws, routed=True)

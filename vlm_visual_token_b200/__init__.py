@@ -52,7 +52,8 @@ class _CRouter(ctypes.Structure):
                 ("gln_g", _vp * 4), ("gln_b", _vp * 4), ("gWout", _vp), ("gbout", _vp),
                 ("rel_q", ctypes.c_double), ("abs_t", ctypes.c_double),
                 ("quantile_scope", ctypes.c_int), ("pool_mode", ctypes.c_int),
-                ("gate_residual", ctypes.c_int)]
+                ("gate_residual", ctypes.c_int),
+                ("fold_u1", _vp), ("fold_c1", _vp), ("fold_wqo", _vp * 3), ("fold_bqo", _vp * 3)]
 
 
 class IvcError(RuntimeError):
@@ -83,6 +84,10 @@ def lib() -> ctypes.CDLL:
         L.ivc_mlp_fold_size.argtypes = [ctypes.POINTER(_CMlp)]
         L.ivc_mlp_fold.restype = ctypes.c_int
         L.ivc_mlp_fold.argtypes = [ctypes.POINTER(_CMlp), _vp, ctypes.c_size_t, _vp]
+        L.ivc_router_fold_size.restype = ctypes.c_size_t
+        L.ivc_router_fold_size.argtypes = [ctypes.POINTER(_CRouter)]
+        L.ivc_router_fold.restype = ctypes.c_int
+        L.ivc_router_fold.argtypes = [ctypes.POINTER(_CRouter), _vp, ctypes.c_size_t, _vp]
         L.ivc_ps_project.restype = ctypes.c_int
         L.ivc_ps_project.argtypes = [_vp, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
                                      ctypes.POINTER(_CMlp), _vp, _vp, ctypes.c_size_t, _vp]
@@ -176,10 +181,13 @@ class Mlp:
 
 
 class Router:
-    """ViR router weights (CrossAttentionPooling + Gating) and thresholds."""
+    """ViR router weights (CrossAttentionPooling + Gating) and thresholds.
+
+    With `fold` (the default) and folded pooling on a CUDA device, the weight
+    folds of ivc_router_fold are formed once here."""
 
     def __init__(self, params: dict, rel_q: float = 0.1, abs_t: float = 0.5, scope: int = 0,
-                 device="cuda", pool_mode: int = 0, gate_residual: int = 0):
+                 device="cuda", pool_mode: int = 0, gate_residual: int = 0, fold: bool = True):
         def dev(t):
             return t.to(device=device, dtype=torch.bfloat16).contiguous()
         self.t = {}
@@ -205,6 +213,19 @@ class Router:
         c.pool_mode = int(pool_mode)
         c.gate_residual = int(gate_residual)
         self.c = c
+        self.folded = None
+        if fold and c.pool_mode == 0 and torch.device(device).type == "cuda":
+            self.fold()
+
+    def fold(self, stream=None) -> "Router":
+        """Form the weight folds once (ivc_router_fold)."""
+        n = lib().ivc_router_fold_size(ctypes.byref(self.c))
+        if n == 0:
+            raise IvcError(-3, "ivc_router_fold_size")
+        self.folded = torch.empty(n, dtype=torch.uint8, device=self.t["query"].device)
+        _check(lib().ivc_router_fold(ctypes.byref(self.c), _ptr(self.folded), n, _stream(stream)),
+               "ivc_router_fold")
+        return self
 
 
 def workspace_size(op: int, T: int, C: int, m: Optional[Mlp] = None, m2: Optional[Mlp] = None,

@@ -73,6 +73,17 @@ int router_shape_ok(const ivc_router* r, int C) {
     return IVC_EUNSUPPORTED;
   if (!r->query || !r->gWout) return IVC_EINVAL;
   if (!aligned16(r->query)) return IVC_EALIGN;
+  {
+    // the folds of ivc_router_fold: all or none, folded pooling only
+    const void* f[8] = {r->fold_u1,     r->fold_c1,     r->fold_wqo[0], r->fold_wqo[1],
+                        r->fold_wqo[2], r->fold_bqo[0], r->fold_bqo[1], r->fold_bqo[2]};
+    int set = 0;
+    for (const void* p : f) {
+      set += p != nullptr;
+      if (!aligned16(p)) return IVC_EALIGN;
+    }
+    if (set != 0 && (set != 8 || r->pool_mode != IVC_POOL_FOLDED)) return IVC_EINVAL;
+  }
   for (int l = 0; l < 4; ++l) {
     const void* ws[6] = {r->Wq[l], r->Wk[l], r->Wv[l], r->Wo[l], r->gW1[l], r->gW2[l]};
     for (const void* w : ws) {
@@ -342,16 +353,21 @@ int gating_and_route(int T, const int32_t* image_offsets, int I, const ivc_route
 // then either the single-pass attention (scores, running softmax and
 // weighted sums per 128-token chunk, chunks merged) or scores = X u^T on the
 // tensor cores, masked softmax, z = p X on the tensor cores; o = Wv z + bv.
-// Q is [T, D], or the shared query (ldq = 0, Tq = 1).
+// Q is [T, D], or the shared query (ldq = 0, Tq = 1). With u1/c1 (layer 1's
+// fold of the shared query, from ivc_router_fold) there is no fold to do.
 int folded_layer(const void* x, const int32_t* valid_len, int T, const ivc_router* r, int l,
-                 const float* Q, long long ldq, const RouteBufs& b, const Launch& L) {
+                 const float* Q, long long ldq, const RouteBufs& b, const Launch& L,
+                 const bf16* u1 = nullptr, const float* c1 = nullptr) {
   const int D = r->D;
-  const int Tq = ldq == 0 ? 1 : T;
-  IVC_TRY(launch_pool_fold_query(Q, ldq, Tq, static_cast<const bf16*>(r->Wk[l]),
-                                 static_cast<const bf16*>(r->bk[l]), D, b.U2, b.cb, L));
+  const int Tq = (ldq == 0 || u1 != nullptr) ? 1 : T;
+  const bf16* U2 = u1 != nullptr ? u1 : b.U2;
+  const float* cb = u1 != nullptr ? c1 : b.cb;
+  if (u1 == nullptr)
+    IVC_TRY(launch_pool_fold_query(Q, ldq, Tq, static_cast<const bf16*>(r->Wk[l]),
+                                   static_cast<const bf16*>(r->bk[l]), D, b.U2, b.cb, L));
   if (pool_attend_wanted()) {
     // chunk partials in Z, their statistics in S, merged sums in z
-    IVC_TRY(launch_pool_attend(x, b.U2, Tq, b.cb, valid_len, T, D, r->heads, b.Z, b.S, b.z, L));
+    IVC_TRY(launch_pool_attend(x, U2, Tq, cb, valid_len, T, D, r->heads, b.Z, b.S, b.z, L));
     return launch_pool_vproj_heads(b.z, T, D, static_cast<const bf16*>(r->Wv[l]),
                                    static_cast<const bf16*>(r->bv[l]), b.O, L);
   }
@@ -363,7 +379,7 @@ int folded_layer(const void* x, const int32_t* valid_len, int T, const ivc_route
   s.N = 32;
   s.K = D;
   s.groups = 1;
-  s.B[0] = b.U2;
+  s.B[0] = U2;
   s.b_mode = B_K3D;
   s.b_batches = Tq;
   s.b_batch_rows = Tq == 1 ? T * 1024 : 1024;
@@ -374,7 +390,7 @@ int folded_layer(const void* x, const int32_t* valid_len, int T, const ivc_route
   s.out_f32 = 1;
   s.ldo = 32;
   IVC_TRY(launch_gemm(s, L));
-  IVC_TRY(launch_pool_softmax(b.S, b.cb, Tq == 1 ? 0 : 16, valid_len, T, r->heads, b.P2, L));
+  IVC_TRY(launch_pool_softmax(b.S, cb, Tq == 1 ? 0 : 16, valid_len, T, r->heads, b.P2, L));
   GemmCall z{};
   z.tag = "pool.wsum";
   z.a_mode = A_PLAIN;
@@ -447,19 +463,31 @@ int route_impl(const void* x, const int32_t* valid_len, int T, const int32_t* im
     return gating_and_route(T, image_offsets, I, r, gate, mask, offsets, total, b, L);
   }
   if (r->pool_mode == IVC_POOL_FOLDED) {
-    IVC_TRY(launch_gemv_bf16x(static_cast<const bf16*>(r->query), D,
-                              static_cast<const bf16*>(r->Wq[0]),
-                              static_cast<const bf16*>(r->bq[0]), D, b.Q1, L));
+    // With the weight folds of ivc_router_fold: layer 1 starts from its
+    // folded query, and each later layer's query comes from the previous
+    // layer's merged head outputs through P_l = Wq_{l+1} Wo_l in one
+    // projection.
+    const bool pre = r->fold_u1 != nullptr;
+    if (!pre)
+      IVC_TRY(launch_gemv_bf16x(static_cast<const bf16*>(r->query), D,
+                                static_cast<const bf16*>(r->Wq[0]),
+                                static_cast<const bf16*>(r->bq[0]), D, b.Q1, L));
     for (int l = 0; l < 4; ++l) {
       if (l == 0) {
-        IVC_TRY(folded_layer(x, valid_len, T, r, 0, b.Q1, 0, b, L));
+        IVC_TRY(folded_layer(x, valid_len, T, r, 0, b.Q1, 0, b, L,
+                             static_cast<const bf16*>(r->fold_u1), r->fold_c1));
       } else {
-        IVC_TRY(launch_gemv(b.q, D, T, D, static_cast<const bf16*>(r->Wq[l]),
-                            static_cast<const bf16*>(r->bq[l]), D, b.Q, D, 0, L));
+        if (!pre)
+          IVC_TRY(launch_gemv(b.q, D, T, D, static_cast<const bf16*>(r->Wq[l]),
+                              static_cast<const bf16*>(r->bq[l]), D, b.Q, D, 0, L));
         IVC_TRY(folded_layer(x, valid_len, T, r, l, b.Q, D, b, L));
       }
-      IVC_TRY(launch_gemv(b.O, D, T, D, static_cast<const bf16*>(r->Wo[l]),
-                          static_cast<const bf16*>(r->bo[l]), D, b.q, D, 0, L));
+      if (pre && l < 3)
+        IVC_TRY(launch_gemv_split(b.O, D, T, D, static_cast<const bf16*>(r->fold_wqo[l]),
+                                  r->fold_bqo[l], D, b.Q, D, L));
+      else
+        IVC_TRY(launch_gemv(b.O, D, T, D, static_cast<const bf16*>(r->Wo[l]),
+                            static_cast<const bf16*>(r->bo[l]), D, b.q, D, 0, L));
     }
     return gating_and_route(T, image_offsets, I, r, gate, mask, offsets, total, b, L);
   }
@@ -744,6 +772,72 @@ int ivc_mlp_fold(ivc_mlp* m, void* dst, size_t dst_bytes, ivc_stream_t stream) {
   m->fold_W0 = W0;
   m->fold_colsum = cs;
   m->fold_bias = fb;
+  return IVC_OK;
+}
+
+// ivc_router_fold: the weights checked as for a call, the fold fields aside.
+static int router_fold_shape(const ivc_router* r) {
+  if (!r) return IVC_EINVAL;
+  ivc_router w = *r;
+  w.fold_u1 = nullptr;
+  w.fold_c1 = nullptr;
+  for (int l = 0; l < 3; ++l) {
+    w.fold_wqo[l] = nullptr;
+    w.fold_bqo[l] = nullptr;
+  }
+  IVC_TRY(router_shape_ok(&w, w.D));
+  if (w.pool_mode != IVC_POOL_FOLDED || w.D % 64 != 0) return IVC_EUNSUPPORTED;
+  return IVC_OK;
+}
+
+size_t ivc_router_fold_size(const ivc_router* r) {
+  if (router_fold_shape(r) != IVC_OK) return 0;
+  const size_t D = static_cast<size_t>(r->D);
+  return align_up(D * sizeof(float)) + align_up(32 * D * sizeof(bf16)) +
+         align_up(16 * sizeof(float)) +
+         3 * (align_up(2 * D * D * sizeof(bf16)) + align_up(D * sizeof(float)));
+}
+
+int ivc_router_fold(ivc_router* r, void* dst, size_t dst_bytes, ivc_stream_t stream) {
+  if (!r || !dst) return IVC_EINVAL;
+  IVC_TRY(router_fold_shape(r));
+  if (reinterpret_cast<uintptr_t>(dst) % kAlign) return IVC_EALIGN;
+  if (dst_bytes < ivc_router_fold_size(r)) return IVC_EWORKSPACE;
+  const int D = r->D;
+  const size_t Dz = static_cast<size_t>(D);
+  char* p = static_cast<char*>(dst);
+  float* q1 = reinterpret_cast<float*>(p);
+  p += align_up(Dz * sizeof(float));
+  bf16* u1 = reinterpret_cast<bf16*>(p);
+  p += align_up(32 * Dz * sizeof(bf16));
+  float* c1 = reinterpret_cast<float*>(p);
+  p += align_up(16 * sizeof(float));
+  bf16* wqo[3];
+  float* bqo[3];
+  for (int l = 0; l < 3; ++l) {
+    wqo[l] = reinterpret_cast<bf16*>(p);
+    p += align_up(2 * Dz * Dz * sizeof(bf16));
+    bqo[l] = reinterpret_cast<float*>(p);
+    p += align_up(Dz * sizeof(float));
+  }
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Launch L{s, nullptr};
+  IVC_TRY(launch_gemv_bf16x(static_cast<const bf16*>(r->query), D,
+                            static_cast<const bf16*>(r->Wq[0]), static_cast<const bf16*>(r->bq[0]),
+                            D, q1, L));
+  IVC_TRY(launch_pool_fold_query(q1, 0, 1, static_cast<const bf16*>(r->Wk[0]),
+                                 static_cast<const bf16*>(r->bk[0]), D, u1, c1, L));
+  for (int l = 0; l < 3; ++l)
+    IVC_TRY(launch_wq_wo_fold(static_cast<const bf16*>(r->Wq[l + 1]),
+                              static_cast<const bf16*>(r->bq[l + 1]),
+                              static_cast<const bf16*>(r->Wo[l]), static_cast<const bf16*>(r->bo[l]),
+                              D, wqo[l], bqo[l], s));
+  r->fold_u1 = u1;
+  r->fold_c1 = c1;
+  for (int l = 0; l < 3; ++l) {
+    r->fold_wqo[l] = wqo[l];
+    r->fold_bqo[l] = bqo[l];
+  }
   return IVC_OK;
 }
 

@@ -162,6 +162,14 @@ size_t splitk_part_floats();
 int launch_gemv(const float* X, long long ldx, int M, int K, const bf16* W, const bf16* b, int N,
                 float* Y, long long ldy, int gelu, const Launch& L);
 // Same with a bf16 input vector broadcast (M = 1).
+// Y = X P^T + c with P an fp32 matrix stored as bf16 hi | lo per row
+// (W2 [N, 2K]) and an fp32 bias c.
+int launch_gemv_split(const float* X, long long ldx, int M, int K, const bf16* W2,
+                      const float* bf, int N, float* Y, long long ldy, const Launch& L);
+// Once per weight set: P = Wq Wo as a bf16 hi | lo pair per row (P2 [D, 2D])
+// and c = Wq bo + bq (fp32 [D]).
+int launch_wq_wo_fold(const bf16* Wq, const bf16* bq, const bf16* Wo, const bf16* bo, int D,
+                      bf16* P2, float* c, cudaStream_t stream);
 int launch_gemv_bf16x(const bf16* x, int K, const bf16* W, const bf16* b, int N, float* Y,
                       const Launch& L);
 // Masked single-query multi-head attention of one pooling layer.

@@ -76,26 +76,36 @@ __device__ __forceinline__ void split2(float2 v, uint32_t& hi, uint32_t& lo) {
 // sums of the single-pass form); h = (first column of the CTA) / 64.
 enum GemvRows { GV_PLAIN = 0, GV_PAIRED = 1, GV_HEADROW = 2 };
 
-template <typename XT, int ROWS>
+template <typename XT, int ROWS, bool WS = false>
 struct GemvLayout {
   // staged input rows (padded by 8 elements), the weight rows (unpadded, one
-  // copy), the warps' partial tiles; after a 16-byte mbarrier slot
+  // copy; with split weights each row holds the hi and then the lo part), the
+  // warps' partial tiles; after a 16-byte mbarrier slot
   __host__ __device__ static size_t x_bytes(int K) {
     return (ROWS == GV_PAIRED ? 2 : 1) * static_cast<size_t>(GEMV_ROWS) * (K + 8) * sizeof(XT);
   }
-  __host__ __device__ static size_t w_bytes(int K) { return static_cast<size_t>(GEMV_COLS) * K * 2; }
+  __host__ __device__ static size_t w_bytes(int K) {
+    return static_cast<size_t>(GEMV_COLS) * K * 2 * (WS ? 2 : 1);
+  }
   __host__ __device__ static size_t total(int K) {
     return 16 + x_bytes(K) + w_bytes(K) + static_cast<size_t>(GEMV_WARPS) * GEMV_ROWS * GEMV_COLS * 4;
   }
 };
 
 // ROWS: see GemvRows (ldx is the row length of Z / z in the pooling modes).
-template <typename XT, int ROWS>
+// WS: the weights are an fp32 matrix split into bf16 hi and lo parts, row n of
+// W = [hi(W[n, 0..K)) | lo(W[n, 0..K))] (fp32 inputs only); the product takes
+// hi.hi + lo.hi + hi.lo of input and weight parts. `bf` (fp32, optional) is a
+// bias used instead of `b`.
+template <typename XT, int ROWS, bool WS = false>
 __global__ void __launch_bounds__(GEMV_THREADS)
     gemv_kernel(const XT* __restrict__ X, long long ldx, int M, int K,
-                const bf16* __restrict__ W, const bf16* __restrict__ b, int N,
-                float* __restrict__ Y, long long ldy, int gelu, int* __restrict__ status) {
-  using Lay = GemvLayout<XT, ROWS>;
+                const bf16* __restrict__ W, const bf16* __restrict__ b,
+                const float* __restrict__ bf, int N, float* __restrict__ Y, long long ldy,
+                int gelu, int* __restrict__ status) {
+  static_assert(!WS || sizeof(XT) == 4, "split weights take fp32 inputs");
+  using Lay = GemvLayout<XT, ROWS, WS>;
+  constexpr int WF = WS ? 2 : 1;  // weight row length in units of K
   constexpr bool PAIRED = ROWS == GV_PAIRED;
   extern __shared__ __align__(16) uint8_t smem[];
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
@@ -115,8 +125,9 @@ __global__ void __launch_bounds__(GEMV_THREADS)
     fence_mbar_init();
     // the weights do not depend on the previous kernel: request them now,
     // with the byte count of the first round of input rows as well
-    mbar_arrive_expect_tx(bar, w_rows * K * 2 + rows0 * xrow * (PAIRED ? 2 : 1));
-    bulk_load(const_cast<bf16*>(sw), W + static_cast<size_t>(c0) * K, w_rows * K * 2, bar);
+    mbar_arrive_expect_tx(bar, w_rows * K * 2 * WF + rows0 * xrow * (PAIRED ? 2 : 1));
+    bulk_load(const_cast<bf16*>(sw), W + static_cast<size_t>(c0) * K * WF, w_rows * K * 2 * WF,
+              bar);
   }
   __syncthreads();  // barrier initialised before anyone waits on it
   pdl_wait();
@@ -141,7 +152,7 @@ __global__ void __launch_bounds__(GEMV_THREADS)
     }
     ok = __syncthreads_and(ok && mbar_wait(bar, round & 1)) != 0;  // uniform decision
     if (!ok) {
-      if (threadIdx.x == 0) atomicOr(status, DEV_WAIT_TIMEOUT);
+      if (threadIdx.x == 0 && status != nullptr) atomicOr(status, DEV_WAIT_TIMEOUT);
       break;
     }
     // rows >= `rows` of the A tile hold stale values; they only reach output
@@ -155,8 +166,9 @@ __global__ void __launch_bounds__(GEMV_THREADS)
       uint32_t bw[GEMV_NT][2];
 #pragma unroll
       for (int j = 0; j < GEMV_NT; ++j) {
-        bw[j][0] = *reinterpret_cast<const uint32_t*>(sw + static_cast<size_t>(wr[j]) * K + k);
-        bw[j][1] = *reinterpret_cast<const uint32_t*>(sw + static_cast<size_t>(wr[j]) * K + k + 8);
+        const bf16* wrow = sw + static_cast<size_t>(wr[j]) * K * WF;
+        bw[j][0] = *reinterpret_cast<const uint32_t*>(wrow + k);
+        bw[j][1] = *reinterpret_cast<const uint32_t*>(wrow + k + 8);
       }
       if constexpr (sizeof(XT) == 2) {
         uint32_t a[4];
@@ -188,6 +200,12 @@ __global__ void __launch_bounds__(GEMV_THREADS)
         for (int j = 0; j < GEMV_NT; ++j) {
           mma_16816(acc[j], ah, bw[j]);
           mma_16816(acc[j], al, bw[j]);
+          if constexpr (WS) {
+            const bf16* wrow = sw + static_cast<size_t>(wr[j]) * K * WF + K;
+            const uint32_t bl[2] = {*reinterpret_cast<const uint32_t*>(wrow + k),
+                                    *reinterpret_cast<const uint32_t*>(wrow + k + 8)};
+            mma_16816(acc[j], ah, bl);
+          }
         }
       }
     }
@@ -206,7 +224,10 @@ __global__ void __launch_bounds__(GEMV_THREADS)
         float y = 0.f;
 #pragma unroll
         for (int w = 0; w < GEMV_WARPS; ++w) y += red[w * GEMV_ROWS * GEMV_COLS + o];
-        if (b != nullptr) y += __bfloat162float(b[c0 + c]);
+        if (bf != nullptr)
+          y += bf[c0 + c];
+        else if (b != nullptr)
+          y += __bfloat162float(b[c0 + c]);
         if (gelu) y = gelu_f(y);
         Y[static_cast<long long>(m0 + r) * ldy + c0 + c] = y;
       }
@@ -215,43 +236,52 @@ __global__ void __launch_bounds__(GEMV_THREADS)
   }
 }
 
-template <typename XT, int ROWS = GV_PLAIN>
+template <typename XT, int ROWS = GV_PLAIN, bool WS = false>
 static int dispatch_gemv(const XT* X, long long ldx, int M, int K, const bf16* W, const bf16* b,
-                         int N, float* Y, long long ldy, int gelu, const Launch& L) {
+                         const float* bf, int N, float* Y, long long ldy, int gelu,
+                         const Launch& L) {
   if (M == 0 || N == 0) return IVC_OK;
   if (K % (16 * GEMV_WARPS) != 0 || K > 2048 || N % 8 != 0) return IVC_EUNSUPPORTED;
   constexpr bool PAIRED = ROWS == GV_PAIRED;
-  if (PAIRED && K > 1024) return IVC_EUNSUPPORTED;
-  const int smem = static_cast<int>(GemvLayout<XT, ROWS>::total(K));
+  constexpr int KMAX = (PAIRED || WS) ? 1024 : 2048;
+  if (K > KMAX) return IVC_EUNSUPPORTED;
+  using Lay = GemvLayout<XT, ROWS, WS>;
+  const int smem = static_cast<int>(Lay::total(K));
   // once per device, for the widest K this instantiation accepts
-  if (smem_optin(reinterpret_cast<const void*>(gemv_kernel<XT, ROWS>),
-                 GemvLayout<XT, ROWS>::total(PAIRED ? 1024 : 2048)) != IVC_OK)
+  if (smem_optin(reinterpret_cast<const void*>(gemv_kernel<XT, ROWS, WS>), Lay::total(KMAX)) !=
+      IVC_OK)
     return IVC_ECUDA;
-  TraceScope ts(ROWS != GV_PLAIN ? "pool.vproj" : (gelu ? "router.gemv_gelu" : "router.gemv"),
+  TraceScope ts(ROWS != GV_PLAIN ? "pool.vproj"
+                                 : (WS ? "pool.wqo" : (gelu ? "router.gemv_gelu" : "router.gemv")),
                 L.stream);
-  return launch_k(gemv_kernel<XT, ROWS>, dim3((N + GEMV_COLS - 1) / GEMV_COLS),
-                  dim3(GEMV_THREADS), smem, L.stream, 1, X, ldx, M, K, W, b, N, Y, ldy, gelu,
+  return launch_k(gemv_kernel<XT, ROWS, WS>, dim3((N + GEMV_COLS - 1) / GEMV_COLS),
+                  dim3(GEMV_THREADS), smem, L.stream, 1, X, ldx, M, K, W, b, bf, N, Y, ldy, gelu,
                   L.status);
 }
 
 int launch_gemv(const float* X, long long ldx, int M, int K, const bf16* W, const bf16* b, int N,
                 float* Y, long long ldy, int gelu, const Launch& L) {
-  return dispatch_gemv<float>(X, ldx, M, K, W, b, N, Y, ldy, gelu, L);
+  return dispatch_gemv<float>(X, ldx, M, K, W, b, nullptr, N, Y, ldy, gelu, L);
+}
+
+int launch_gemv_split(const float* X, long long ldx, int M, int K, const bf16* W2,
+                      const float* bf, int N, float* Y, long long ldy, const Launch& L) {
+  return dispatch_gemv<float, GV_PLAIN, true>(X, ldx, M, K, W2, nullptr, bf, N, Y, ldy, 0, L);
 }
 
 int launch_gemv_bf16x(const bf16* x, int K, const bf16* W, const bf16* b, int N, float* Y,
                       const Launch& L) {
-  return dispatch_gemv<bf16>(x, 0, 1, K, W, b, N, Y, 0, 0, L);
+  return dispatch_gemv<bf16>(x, 0, 1, K, W, b, nullptr, N, Y, 0, 0, L);
 }
 
 int launch_pool_vproj(const float* Z, int T, int D, const bf16* Wv, const bf16* bv, float* O,
                       const Launch& L) {
-  return dispatch_gemv<float, GV_PAIRED>(Z, D, T, D, Wv, bv, D, O, D, 0, L);
+  return dispatch_gemv<float, GV_PAIRED>(Z, D, T, D, Wv, bv, nullptr, D, O, D, 0, L);
 }
 
 int launch_pool_vproj_heads(const float* z, int T, int D, const bf16* Wv, const bf16* bv, float* O,
                             const Launch& L) {
-  return dispatch_gemv<float, GV_HEADROW>(z, D, T, D, Wv, bv, D, O, D, 0, L);
+  return dispatch_gemv<float, GV_HEADROW>(z, D, T, D, Wv, bv, nullptr, D, O, D, 0, L);
 }
 
 // ---------------------------------------------------------------- pooling attention
@@ -405,6 +435,91 @@ __global__ void __launch_bounds__(128) pool_fold_query_kernel(
       cb[(t0 + threadIdx.x) * 16 + h] = acc;
     }
   }
+}
+
+// ---------------------------------------------------------------- weight folds
+// Once per set of router weights: the output projection of pooling layer l
+// and the query projection of layer l+1 follow each other with nothing in
+// between (InternVL3_5-4B-Flash article, section 2: the layers are chained
+// with no residual or norm), so Wq_{l+1} (Wo_l o + bo_l) + bq_{l+1} =
+// P o + (Wq_{l+1} bo_l + bq_{l+1}) with P = Wq_{l+1} Wo_l. P is formed in
+// fp32 (exact bf16 products, fp32 sums) and stored as a bf16 pair, row n =
+// [hi(P[n, :]) | lo(P[n, :])], hi = bf16(P), lo = bf16(P - hi): about 16
+// significant bits, read by the split-weight GEMV.
+constexpr int WF_TILE = 64;  // output tile of the product kernel
+constexpr int WF_KC = 16;    // inner-dimension chunk staged per step
+
+__global__ void __launch_bounds__(256) wq_wo_fold_kernel(const bf16* __restrict__ A,
+                                                         const bf16* __restrict__ B, int D,
+                                                         bf16* __restrict__ P2) {
+  // P[n][k] = sum_j A[n][j] B[j][k], A = Wq (rows n), B = Wo (rows j)
+  __shared__ float sa[WF_KC][WF_TILE + 1];  // sa[j][n]
+  __shared__ float sb[WF_KC][WF_TILE];      // sb[j][k]
+  const int n0 = blockIdx.y * WF_TILE, k0 = blockIdx.x * WF_TILE;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;  // 4 x 4 outputs each
+  float acc[4][4] = {};
+  for (int j0 = 0; j0 < D; j0 += WF_KC) {
+    for (int i = threadIdx.x; i < WF_KC * WF_TILE; i += 256) {
+      const int r = i / WF_KC, c = i % WF_KC;  // A tile: row n0 + r, column j0 + c
+      sa[c][r] = __bfloat162float(A[static_cast<size_t>(n0 + r) * D + j0 + c]);
+      const int rb = i / WF_TILE, cb = i % WF_TILE;  // B tile: row j0 + rb, column k0 + cb
+      sb[rb][cb] = __bfloat162float(B[static_cast<size_t>(j0 + rb) * D + k0 + cb]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < WF_KC; ++j) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[i] = sa[j][ty * 4 + i];
+        b[i] = sb[j][tx * 4 + i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[i][q] = fmaf(a[i], b[q], acc[i][q]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int n = n0 + ty * 4 + i;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int k = k0 + tx * 4 + q;
+      const bf16 hi = __float2bfloat16_rn(acc[i][q]);
+      const bf16 lo = __float2bfloat16_rn(acc[i][q] - __bfloat162float(hi));
+      P2[static_cast<size_t>(n) * 2 * D + k] = hi;
+      P2[static_cast<size_t>(n) * 2 * D + D + k] = lo;
+    }
+  }
+}
+
+// c[n] = sum_j A[n][j] bo[j] + bq[n] (fp32); one warp per row, either bias
+// may be absent (zero).
+__global__ void __launch_bounds__(256) wq_bo_fold_kernel(const bf16* __restrict__ A,
+                                                         const bf16* __restrict__ bo,
+                                                         const bf16* __restrict__ bq, int D,
+                                                         float* __restrict__ c) {
+  const int n = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (n >= D) return;
+  float acc = 0.f;
+  if (bo != nullptr)
+    for (int j = lane; j < D; j += 32)
+      acc = fmaf(__bfloat162float(A[static_cast<size_t>(n) * D + j]), __bfloat162float(bo[j]), acc);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) c[n] = acc + (bq != nullptr ? __bfloat162float(bq[n]) : 0.f);
+}
+
+int launch_wq_wo_fold(const bf16* Wq, const bf16* bq, const bf16* Wo, const bf16* bo, int D,
+                      bf16* P2, float* c, cudaStream_t stream) {
+  if (D % WF_TILE != 0) return IVC_EUNSUPPORTED;
+  wq_wo_fold_kernel<<<dim3(D / WF_TILE, D / WF_TILE), 256, 0, stream>>>(Wq, Wo, D, P2);
+  const int rc = cu_check(cudaGetLastError());
+  if (rc != IVC_OK) return rc;
+  wq_bo_fold_kernel<<<dim3((D + 7) / 8), 256, 0, stream>>>(Wq, bo, bq, D, c);
+  return cu_check(cudaGetLastError());
 }
 
 int launch_pool_fold_query(const float* Q, long long ldq, int Tq, const bf16* Wk, const bf16* bk,
