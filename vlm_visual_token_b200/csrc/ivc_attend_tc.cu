@@ -376,6 +376,12 @@ bool attend_tc_wanted() {
   return v == 1;
 }
 
+int pool_attend_tc_chunks() { return AT_NCH; }
+
+bool pool_attend_tc_supported(int D, int heads) {
+  return D % 128 == 0 && D <= 1024 && heads >= 1 && heads <= 16 && heads * 64 == D;
+}
+
 int launch_pool_attend_tc(const void* x, const bf16* U2, int Tq, const float* cb,
                           const int32_t* valid_len, int T, int D, int heads, float* Zp,
                           float* stats, const Launch& L) {

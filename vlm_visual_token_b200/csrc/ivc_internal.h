@@ -198,9 +198,13 @@ int launch_pool_attend_tc(const void* x, const bf16* U2, int Tq, const float* cb
                           const int32_t* valid_len, int T, int D, int heads, float* Zp,
                           float* stats, const Launch& L);
 // combine = false: the chunk partials are left for launch_pool_tail to merge.
+// allow_tc = false: the mma.sync form even where the tcgen05 one is selected.
 int launch_pool_attend(const void* x, const bf16* U2, int Tq, const float* cb,
                        const int32_t* valid_len, int T, int D, int heads, float* Zp, float* stats,
-                       float* z, const Launch& L, bool combine = true);
+                       float* z, const Launch& L, bool combine = true, bool allow_tc = true);
+// The tcgen05 attention's partials per tile and the shapes it takes.
+int pool_attend_tc_chunks();
+bool pool_attend_tc_supported(int D, int heads);
 // The tail of folded pooling layer l as one cooperative launch of D/64 CTAs
 // (ivc_router_coop.cu): merge of the chunk partials (Zp, stats as left by
 // launch_pool_attend with combine = false), O = Wv z + bv, q = Wo O + bo, and

@@ -878,23 +878,24 @@ __global__ void __launch_bounds__(256, 1)
 
 // Grid (heads, T): z[tile][h] from the tile's ATTN_NCH chunk partials
 // (chunks without a valid token, l = 0, are skipped).
+template <int NCH>
 __global__ void __launch_bounds__(256)
     pool_combine_kernel(const float* __restrict__ Zp, const float* __restrict__ mstat,
                         const float* __restrict__ lstat, int D, float* __restrict__ z) {
   const int h = blockIdx.x, tile = blockIdx.y;
   pdl_wait();
   pdl_trigger();
-  const size_t r0 = static_cast<size_t>(tile) * ATTN_NCH * 16 + h;
-  float w[ATTN_NCH];
+  const size_t r0 = static_cast<size_t>(tile) * NCH * 16 + h;
+  float w[NCH];
   float M = -INFINITY;
 #pragma unroll
-  for (int c = 0; c < ATTN_NCH; ++c) {
+  for (int c = 0; c < NCH; ++c) {
     w[c] = lstat[r0 + 16 * c] > 0.f ? mstat[r0 + 16 * c] : -INFINITY;
     M = fmaxf(M, w[c]);
   }
   float L = 0.f;
 #pragma unroll
-  for (int c = 0; c < ATTN_NCH; ++c) {
+  for (int c = 0; c < NCH; ++c) {
     w[c] = w[c] == -INFINITY ? 0.f : expf(w[c] - M);
     L += w[c] * lstat[r0 + 16 * c];
   }
@@ -902,7 +903,7 @@ __global__ void __launch_bounds__(256)
   for (int c4 = threadIdx.x * 4; c4 < D; c4 += 1024) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int c = 0; c < ATTN_NCH; ++c) {
+    for (int c = 0; c < NCH; ++c) {
       if (w[c] == 0.f) continue;
       const float4 v = __ldg(reinterpret_cast<const float4*>(Zp + (r0 + 16 * c) * D + c4));
       acc.x = fmaf(w[c], v.x, acc.x);
@@ -937,7 +938,7 @@ static int launch_attend_ks(const CUtensorMap& xmap, const bf16* U2, int u2_per_
 
 int launch_pool_attend(const void* x, const bf16* U2, int Tq, const float* cb,
                        const int32_t* valid_len, int T, int D, int heads, float* Zp, float* stats,
-                       float* z, const Launch& L, bool combine) {
+                       float* z, const Launch& L, bool combine, bool allow_tc) {
   if (T == 0) return IVC_OK;
   if (D % 128 != 0 || D > 1024 || heads < 1 || heads > 16 || heads * 64 != D)
     return IVC_EUNSUPPORTED;
@@ -954,8 +955,11 @@ int launch_pool_attend(const void* x, const bf16* U2, int Tq, const float* cb,
   float* lstat = stats + static_cast<size_t>(T) * ATTN_NCH * 16;
   const int u2_per_tile = Tq == 1 ? 0 : 1;
   const int cb_stride = Tq == 1 ? 0 : 16;
+  const bool tc = allow_tc && attend_tc_wanted() && pool_attend_tc_supported(D, heads);
   int rc;
-  if (attend_tc_wanted()) {
+  if (tc) {
+    // 128-token items: the same partials per tile as the mma.sync form
+    if (pool_attend_tc_chunks() != ATTN_NCH) return IVC_EUNSUPPORTED;
     rc = launch_pool_attend_tc(x, U2, Tq, cb, valid_len, T, D, heads, Zp, stats, L);
   } else {
     TraceScope ts("pool.attend", L.stream);
@@ -977,8 +981,8 @@ int launch_pool_attend(const void* x, const bf16* U2, int Tq, const float* cb,
   }
   if (rc != IVC_OK || !combine) return rc;
   TraceScope ts("pool.combine", L.stream);
-  return launch_k(pool_combine_kernel, dim3(heads, T), dim3(256), 0, L.stream, 1, Zp, mstat, lstat,
-                  D, z);
+  return launch_k(pool_combine_kernel<ATTN_NCH>, dim3(heads, T), dim3(256), 0, L.stream, 1, Zp,
+                  mstat, lstat, D, z);
 }
 
 // ---------------------------------------------------------------- residual + LayerNorm
