@@ -1031,9 +1031,22 @@ __global__ void __launch_bounds__(256) residual_ln_kernel(float* __restrict__ h,
   var /= D;
   const float rstd = 1.0f / sqrtf(var + 1e-5f);
   float* hr = h + static_cast<long long>(t) * D;
-  for (int i = threadIdx.x; i < D; i += 256) {
-    const float n = (ur[i] - mean) * rstd * __bfloat162float(gamma[i]) + __bfloat162float(beta[i]);
-    hr[i] = inside ? n : hr[i] + n;
+  // every load before the first store (a store to h could alias gamma or
+  // beta for the compiler, which would serialise the loads behind it)
+  float out[8];  // D <= 2048 over 256 threads
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int i = threadIdx.x + 256 * j;
+    if (i < D) {
+      const float n = (ur[i] - mean) * rstd * __bfloat162float(gamma[i]) +
+                      __bfloat162float(beta[i]);
+      out[j] = inside ? n : hr[i] + n;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int i = threadIdx.x + 256 * j;
+    if (i < D) hr[i] = out[j];
   }
 }
 
