@@ -2,7 +2,8 @@
 // assigned to exactly one CTA pair, each pair's list is increasing, and
 // running the lists (each pair in order, a tile starting only once the row
 // block it reads is complete) finishes every tile: no deadlock, for the
-// connector problem sets of both MLPs and for random ones.
+// connector problem sets of both MLPs and for random ones, with tiles numbered
+// row block by row block or (n_major) column block by column block.
 #include <cstdio>
 #include <cstdlib>
 #include <vector>
@@ -45,7 +46,9 @@ static bool check(const std::vector<SchedProblem>& P, int pairs) {
       const int u = lists[q][pos[q]];
       int p = 0;
       while (u >= ub[p + 1]) ++p;
-      const int m = (u - ub[p]) / P[p].n_tiles;
+      // the row block of a tile id, as the graph kernel derives it
+      const int idx = u - ub[p];
+      const int m = P[p].n_major ? idx % P[p].m_tiles : idx / P[p].n_tiles;
       if (P[p].dep >= 0 && left[P[p].dep][m] != 0) continue;
       --left[p][m];
       ++pos[q];
@@ -64,6 +67,10 @@ int main() {
       {4, 16, 256, -1}, {13, 8, 64, -1}, {4, 8, 64, 0}, {13, 8, 32, 1}, {4, 8, 32, 2}};
   for (int pairs : {1, 7, 64, 74, 80})
     if (!check(flash, pairs)) return 1;
+  // the same with mlp2.fc1 column block by column block
+  flash[0].n_major = 1;
+  for (int pairs : {1, 7, 56, 64, 74, 80})
+    if (!check(flash, pairs)) return 1;
   // one MLP, fc1 then fc2
   if (!check({{3, 4, 64, -1}, {3, 4, 32, 0}}, 74)) return 1;
   // dependencies must point to earlier problems with the same row blocks
@@ -78,7 +85,7 @@ int main() {
     const int mt = 1 + std::rand() % 9;
     for (int i = 0; i < n; ++i) {
       const int dep = i > 0 && std::rand() % 2 ? std::rand() % i : -1;
-      P.push_back({mt, 1 + std::rand() % 12, 1 + std::rand() % 300, dep});
+      P.push_back({mt, 1 + std::rand() % 12, 1 + std::rand() % 300, dep, std::rand() % 2});
     }
     if (!check(P, 1 + std::rand() % 80)) return 1;
   }

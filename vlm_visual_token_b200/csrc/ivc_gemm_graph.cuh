@@ -92,6 +92,8 @@ struct GraphProblem {
   const float* row_rstd;
   void* out;           // bf16 [M, ldo]
   long long ldo;
+  int n_major;         // 1: tiles column block by column block (the row blocks
+                       // of one weight panel run together and share it in L2)
 };
 
 struct alignas(64) GraphMaps {
@@ -119,6 +121,7 @@ __device__ __forceinline__ GraphTile graph_tile(const GraphArgs& g, int u) {
   int p = 0;
   while (p + 1 < g.n_problems && u >= g.unit_begin[p + 1]) ++p;
   const int idx = u - g.unit_begin[p];
+  if (g.p[p].n_major) return {p, idx % g.p[p].m_tiles, idx / g.p[p].m_tiles};
   return {p, idx / g.p[p].n_tiles, idx % g.p[p].n_tiles};
 }
 

@@ -94,6 +94,7 @@ int launch_gemm_graph(const GraphProblemCall* probs, int n, int* done, int reser
     P.row_rstd = c.row_rstd;
     P.out = c.out;
     P.ldo = c.ldo;
+    P.n_major = c.n_major;
     ctr += P.m_tiles;
     int rc;
     if (c.a_mode == A_PLAIN) {
@@ -108,7 +109,7 @@ int launch_gemm_graph(const GraphProblemCall* probs, int n, int* done, int reser
     amap += P.a_views;
     rc = map_rows_2k(&m.b[i], c.B, c.N, c.K);
     if (rc) return rc;
-    sp[i] = {P.m_tiles, P.n_tiles, c.K / GEMM_BK, c.dep};
+    sp[i] = {P.m_tiles, P.n_tiles, c.K / GEMM_BK, c.dep, c.n_major};
   }
   for (int i = 0; i < n; ++i)
     if (g.p[i].dep >= 0) g.p[i].dep_target = 2 * g.p[g.p[i].dep].n_tiles;

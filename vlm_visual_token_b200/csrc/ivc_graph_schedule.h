@@ -22,8 +22,9 @@ namespace ivc {
 struct SchedProblem {
   int m_tiles;
   int n_tiles;
-  int k_steps;  // cost of one tile in the model
-  int dep;      // problem (earlier index) whose row block m a tile of row block m reads, or -1
+  int k_steps;      // cost of one tile in the model
+  int dep;          // problem (earlier index) whose row block m a tile of row block m reads, or -1
+  int n_major = 0;  // 1: tiles numbered column block by column block
 };
 
 // First global tile id of each problem, and the total in the last entry.
@@ -50,8 +51,11 @@ inline bool list_schedule(const std::vector<SchedProblem>& P, int pairs, int epi
   std::vector<double> free_at(pairs, 0.0);
   int id = 0;
   for (size_t p = 0; p < P.size(); ++p) {
-    for (int m = 0; m < P[p].m_tiles; ++m) {
-      for (int n = 0; n < P[p].n_tiles; ++n, ++id) {
+    const int outer = P[p].n_major ? P[p].n_tiles : P[p].m_tiles;
+    const int inner = P[p].n_major ? P[p].m_tiles : P[p].n_tiles;
+    for (int o = 0; o < outer; ++o) {
+      for (int i = 0; i < inner; ++i, ++id) {
+        const int m = P[p].n_major ? i : o;
         int best = 0;
         for (int q = 1; q < pairs; ++q)
           if (free_at[q] < free_at[best]) best = q;

@@ -145,6 +145,7 @@ struct GraphProblemCall {
   void* out;
   long long ldo;
   int dep;
+  int n_major;         // 1: tiles ordered column block by column block
 };
 int launch_gemm_graph(const GraphProblemCall* probs, int n, int* done, int reserve_sms,
                       const Launch& L);
