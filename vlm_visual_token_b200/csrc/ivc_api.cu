@@ -280,6 +280,20 @@ bool gemm_graph_enabled() {
   return v == 1;
 }
 
+// 256 x 512 tiles for an MLP's first Linear in the single launch: with
+// K >= 8192 (mlp2's, K = 16C; the InternViT-6B connector's mlp1, K = 12800)
+// when it has many rounds of tiles (1, the default), never
+// (IVC_GRAPH_WIDE=0), or always, whatever K and size (2: the parity tests of
+// the wide tiles on small shapes).
+int graph_wide_mode() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("IVC_GRAPH_WIDE");
+    v = (e && (e[0] == '0' || e[0] == '2')) ? e[0] - '0' : 1;
+  }
+  return v;
+}
+
 // The Linears of one pixel_shuffle + MLP as graph problems (appended to
 // `probs`; the first reads x through the pixel_shuffle view with the
 // LayerNorm fold, each later one the previous one's output). The weights
@@ -307,6 +321,8 @@ void mlp_problems(const void* x, int T, int C, bool half, int flags, const ivc_m
   c.out = b.h1;
   c.ldo = m->dims[1];
   c.dep = -1;
+  const int wide_mode = graph_wide_mode();
+  c.wide = wide_mode == 2 ? 2 : (wide_mode == 1 && c.K >= 8192 ? 1 : 0);
   probs.push_back(c);
   for (int i = 1; i < m->n_linear; ++i) {
     const bool last = i + 1 == m->n_linear;

@@ -68,7 +68,35 @@ int launch_gemm_graph(const GraphProblemCall* probs, int n, int* done, int reser
   GraphArgs g{};
   g.n_problems = n;
   g.done = done;
+  int max_pairs = (num_sms() - (reserve_sms > 0 ? reserve_sms : 0)) / 2;
+  if (max_pairs > GG_MAX_PAIRS) max_pairs = GG_MAX_PAIRS;
+  if (max_pairs < 1) max_pairs = 1;
+  // 256 x 512 tiles for the problems that allow them (wide == 1) when they
+  // have many rounds of 256-wide tiles (at least 8 per pair), where the 25%
+  // fewer operand bytes per MAC pay; wide == 2 asks for them in any case.
+  bool use_wide = false;
+  std::vector<int> wide(n, 0);
+  for (int i = 0; i < n; ++i) {
+    const GraphProblemCall& c = probs[i];
+    const long long tiles256 = static_cast<long long>((c.M + GG_TILE_M - 1) / GG_TILE_M) *
+                               ((c.N + GG_BN - 1) / GG_BN);
+    wide[i] = c.wide == 2 || (c.wide == 1 && tiles256 >= 8LL * max_pairs) ? 1 : 0;
+    use_wide = use_wide || wide[i];
+  }
   std::vector<SchedProblem> sp(n);
+  int units = 0;
+  for (int i = 0; i < n; ++i) {
+    const GraphProblemCall& c = probs[i];
+    const int w = wide[i];
+    const int mt = (c.M + GG_TILE_M - 1) / GG_TILE_M;
+    const int nt = (c.N + (GG_BN << w) - 1) / (GG_BN << w);
+    // a wide tile's cost in the model: twice the MACs, 1.5 times the bytes
+    sp[i] = {mt, nt, (c.K / GEMM_BK) * (w ? 7 : 4) / 4, c.dep, c.n_major};
+    units += mt * nt;
+  }
+  const int pairs = units < max_pairs ? units : max_pairs;
+  std::vector<std::vector<int>> lists;
+  if (units <= GG_MAX_SCHED && !list_schedule(sp, pairs, 4, lists)) return IVC_EINVAL;
   int amap = 0, ctr = 0;
   GraphMaps m{};
   for (int i = 0; i < n; ++i) {
@@ -81,7 +109,8 @@ int launch_gemm_graph(const GraphProblemCall* probs, int n, int* done, int reser
     P.a_map = amap;
     P.c_blocks = c.C / GEMM_BK;
     P.m_tiles = (c.M + GG_TILE_M - 1) / GG_TILE_M;
-    P.n_tiles = (c.N + GG_BN - 1) / GG_BN;
+    P.wide = wide[i];
+    P.n_tiles = (c.N + (GG_BN << P.wide) - 1) / (GG_BN << P.wide);
     P.epi_mode = c.epi_mode;
     P.gelu = c.gelu;
     P.remap = c.remap;
@@ -109,23 +138,15 @@ int launch_gemm_graph(const GraphProblemCall* probs, int n, int* done, int reser
     amap += P.a_views;
     rc = map_rows_2k(&m.b[i], c.B, c.N, c.K);
     if (rc) return rc;
-    sp[i] = {P.m_tiles, P.n_tiles, c.K / GEMM_BK, c.dep, c.n_major};
   }
   for (int i = 0; i < n; ++i)
     if (g.p[i].dep >= 0) g.p[i].dep_target = 2 * g.p[g.p[i].dep].n_tiles;
   g.n_amaps = amap;
   const std::vector<int> ub = schedule_unit_begin(sp);
   for (int i = 0; i <= n; ++i) g.unit_begin[i] = ub[i];
-  const int units = ub[n];
-  int pairs = (num_sms() - (reserve_sms > 0 ? reserve_sms : 0)) / 2;
-  if (pairs > GG_MAX_PAIRS) pairs = GG_MAX_PAIRS;
-  if (pairs > units) pairs = units;
-  if (pairs < 1) pairs = 1;
   g.n_pairs = pairs;
   g.scheduled = 0;
-  if (units <= GG_MAX_SCHED) {
-    std::vector<std::vector<int>> lists;
-    if (!list_schedule(sp, pairs, 4, lists)) return IVC_EINVAL;
+  if (!lists.empty()) {
     int off = 0;
     for (int q = 0; q < pairs; ++q) {
       g.sched_off[q] = static_cast<unsigned short>(off);
@@ -135,11 +156,11 @@ int launch_gemm_graph(const GraphProblemCall* probs, int n, int* done, int reser
     g.scheduled = 1;
   }
   using S = GraphSmem;
-  if (smem_optin(reinterpret_cast<const void*>(gemm_graph_kernel), S::TOTAL) != IVC_OK)
-    return IVC_ECUDA;
+  auto kern = use_wide ? gemm_graph_kernel<true> : gemm_graph_kernel<false>;
+  if (smem_optin(reinterpret_cast<const void*>(kern), S::TOTAL) != IVC_OK) return IVC_ECUDA;
   TraceScope ts("connector.graph", L.stream);
-  return launch_k(gemm_graph_kernel, dim3(2 * pairs), dim3(GEMM_THREADS), S::TOTAL, L.stream, 2, m,
-                  g, L.status);
+  return launch_k(kern, dim3(2 * pairs), dim3(GEMM_THREADS), S::TOTAL, L.stream, 2, m, g,
+                  L.status);
 }
 
 }  // namespace ivc

@@ -146,6 +146,8 @@ struct GraphProblemCall {
   long long ldo;
   int dep;
   int n_major;         // 1: tiles ordered column block by column block
+  int wide;            // 1: 256 x 512 tiles if the problem has many rounds of
+                       // 256-wide tiles; 2: 256 x 512 tiles
 };
 int launch_gemm_graph(const GraphProblemCall* probs, int n, int* done, int reserve_sms,
                       const Launch& L);
