@@ -143,9 +143,9 @@ def connector_roles(w):
     return GEMM_ROLES if w.path == "flash" else GEMM_ROLES[:2]
 
 
-def image_gen(rank: int, workload: str = DEFAULT_WORKLOAD):
+def image_gen(rank: int, workload: str = DEFAULT_WORKLOAD, n_images=None):
     import workloads as W
-    return W.make(workload, seed_offset=1000 * rank)
+    return W.make(workload, seed_offset=1000 * rank, n_images=n_images)
 
 
 class ClockSampler:
@@ -779,7 +779,7 @@ def run_op(args):
 
     import vlm_visual_token_b200 as ivc
     torch.cuda.set_device(0)
-    inp = image_gen(0, args.workload)
+    inp = image_gen(0, args.workload, args.images)
     w, T = inp["workload"], inp["T"]
     if w.path != "flash" and args.op not in ("ps_half",):
         raise SystemExit(f"--op {args.op} needs a flash workload; {w.name} has mlp1 only")
@@ -870,6 +870,8 @@ def main(argv=None):
                                           "(flash = the full benchmark)")
     ap.add_argument("--trace", action="store_true",
                     help="with --op: also report per-kernel device times (event-bracketed)")
+    ap.add_argument("--images", type=int, default=None,
+                    help="with --op: only the workload's first N images (small profiling cases)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

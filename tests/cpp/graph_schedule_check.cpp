@@ -3,7 +3,7 @@
 // running the lists (each pair in order, a tile starting only once the row
 // block it reads is complete) finishes every tile: no deadlock, for the
 // connector problem sets of both MLPs and for random ones, with tiles numbered
-// row block by row block or (n_major) column block by column block.
+// row block by row block or in groups of row blocks (tile_coords).
 #include <cstdio>
 #include <cstdlib>
 #include <vector>
@@ -47,8 +47,8 @@ static bool check(const std::vector<SchedProblem>& P, int pairs) {
       int p = 0;
       while (u >= ub[p + 1]) ++p;
       // the row block of a tile id, as the graph kernel derives it
-      const int idx = u - ub[p];
-      const int m = P[p].n_major ? idx % P[p].m_tiles : idx / P[p].n_tiles;
+      int m, n;
+      ivc::tile_coords(u - ub[p], P[p].m_tiles, P[p].n_tiles, P[p].group_m, &m, &n);
       if (P[p].dep >= 0 && left[P[p].dep][m] != 0) continue;
       --left[p][m];
       ++pos[q];
@@ -60,15 +60,40 @@ static bool check(const std::vector<SchedProblem>& P, int pairs) {
   return true;
 }
 
+// tile_coords numbers every (row block, column block) exactly once.
+static bool coords_bijective(int mt, int nt, int group) {
+  std::vector<int> seen(mt * nt, 0);
+  for (int idx = 0; idx < mt * nt; ++idx) {
+    int m, n;
+    ivc::tile_coords(idx, mt, nt, group, &m, &n);
+    CHECK(m >= 0 && m < mt && n >= 0 && n < nt);
+    ++seen[m * nt + n];
+  }
+  for (int v : seen) CHECK(v == 1);
+  return true;
+}
+
 int main() {
+  for (int mt = 1; mt <= 20; ++mt)
+    for (int nt = 1; nt <= 7; ++nt)
+      for (int group = 0; group <= 9; ++group)
+        if (!coords_bijective(mt, nt, group)) return 1;
+  // groups of 3 over 7 row blocks: rows 0-2 column by column, then 3-5, then 6
+  {
+    int m, n;
+    ivc::tile_coords(4, 7, 2, 3, &m, &n);  // group 0, column 1, row 1
+    if (m != 1 || n != 1) return 1;
+    ivc::tile_coords(12, 7, 2, 3, &m, &n);  // last group (row 6 only), column 0
+    if (m != 6 || n != 0) return 1;
+  }
   // both MLPs of a 13-tile image in priority order: mlp2.fc1, mlp1.fc1,
   // mlp2.fc2 (reads 0), mlp1.fc2 (reads 1), mlp2.fc3 (reads 2)
   std::vector<SchedProblem> flash = {
       {4, 16, 256, -1}, {13, 8, 64, -1}, {4, 8, 64, 0}, {13, 8, 32, 1}, {4, 8, 32, 2}};
   for (int pairs : {1, 7, 64, 74, 80})
     if (!check(flash, pairs)) return 1;
-  // the same with mlp2.fc1 column block by column block
-  flash[0].n_major = 1;
+  // the same with mlp2.fc1 in one group (column block by column block)
+  flash[0].group_m = 8;
   for (int pairs : {1, 7, 56, 64, 74, 80})
     if (!check(flash, pairs)) return 1;
   // one MLP, fc1 then fc2
@@ -85,7 +110,7 @@ int main() {
     const int mt = 1 + std::rand() % 9;
     for (int i = 0; i < n; ++i) {
       const int dep = i > 0 && std::rand() % 2 ? std::rand() % i : -1;
-      P.push_back({mt, 1 + std::rand() % 12, 1 + std::rand() % 300, dep, std::rand() % 2});
+      P.push_back({mt, 1 + std::rand() % 12, 1 + std::rand() % 300, dep, std::rand() % 4});
     }
     if (!check(P, 1 + std::rand() % 80)) return 1;
   }

@@ -585,13 +585,14 @@ print("variant ok")
                                  {"IVC_GATING_FUSED": "1"}, {"IVC_POOL_TAIL": "1"},
                                  {"IVC_ATTEND_TC": "0"}, {"IVC_GEMM_GRAPH": "0"},
                                  {"IVC_GRAPH_WIDE": "0"}, {"IVC_GRAPH_WIDE": "2"},
-                                 {"IVC_GRAPH_NMAJOR": "0"}])
+                                 {"IVC_GRAPH_GROUP": "0"}])
 def test_flash_kernel_variants(env):
     """The opt-in kernel variants (512-wide pair tiles with split-K, single-CTA
     256-wide tiles, the persistent router inside the dual flow, the pooling as
     tensor-core scores / softmax / weighted-sum kernels; in the single launch
     only 256-wide tiles, 256 x 512 tiles for both first Linears, row-block tile
-    order), each in a fresh process since the switches are read once."""
+    order throughout), each in a fresh process since the switches are read
+    once."""
     import subprocess
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -639,18 +640,21 @@ def test_flash_single_launch_small(tiles):
         _flash_check(ivc, inp, res)
 
 
-def test_single_launch_small_with_wide_tiles():
-    """The single launch's 256 x 512 tiles on the small shapes above (widths
-    of 256 and 384, so a tile's second half is partly or wholly past N, mixed
-    with 256-wide tiles of the later Linears): the same tests in a fresh
-    process with every first Linear forced to wide tiles."""
+@pytest.mark.parametrize("env", [{"IVC_GRAPH_WIDE": "2"}, {"IVC_GRAPH_GROUP": "2"},
+                                 {"IVC_GRAPH_WIDE": "2", "IVC_GRAPH_GROUP": "3"}])
+def test_single_launch_small_tile_forms(env):
+    """The single launch's other tile forms on the small shapes above, in a
+    fresh process: 256 x 512 tiles on every first Linear (widths of 256 and
+    384, so a tile's second half is partly or wholly past N, mixed with the
+    256-wide tiles of the later Linears), and tiles in groups of 2 or 3 row
+    blocks on every Linear (up to 17 row blocks, so the last group is short)."""
     import subprocess
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     out = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider", "-m", "gpu",
                           os.path.join(root, "tests", "test_gpu_parity.py"), "-k",
-                          "single_launch_small and not wide_tiles"],
-                         env={**os.environ, "IVC_GRAPH_WIDE": "2"}, capture_output=True, text=True,
+                          "single_launch_small and not tile_forms"],
+                         env={**os.environ, **env}, capture_output=True, text=True,
                          timeout=600, cwd=root)
     assert out.returncode == 0, out.stdout[-3000:] + out.stderr[-2000:]
     assert " passed" in out.stdout

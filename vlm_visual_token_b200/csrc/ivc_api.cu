@@ -589,16 +589,6 @@ int gating_and_route(int T, const int32_t* image_offsets, int I, const ivc_route
                       offsets, total, L);
 }
 
-// IVC_GRAPH_NMAJOR=0: mlp2's first Linear in row-block order too.
-bool graph_nmajor_enabled() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = std::getenv("IVC_GRAPH_NMAJOR");
-    v = (e && e[0] == '0') ? 0 : 1;
-  }
-  return v == 1;
-}
-
 // Connector GEMMs beside the router in ivc_flash_compress: SMs they leave to
 // the router's small kernels (IVC_DUAL_RESERVE, default 36). With the
 // connector's Linears in one persistent launch the router is the longer of
@@ -1023,10 +1013,6 @@ int ivc_flash_compress(const void* x, const int32_t* valid_len, int T, int C,
     probs[pos2[0]].B = W02;
     probs[pos2[0]].colsum = cs2;
     probs[pos2[0]].fbias = fb2;
-    // mlp2's first Linear (the longest tiles, a weight matrix larger than L2)
-    // column block by column block: the row blocks of a weight panel run at
-    // once and read it from DRAM once
-    if (graph_nmajor_enabled()) probs[pos2[0]].n_major = 1;
     const int n_ctr = graph_counters(probs.data(), static_cast<int>(probs.size()));
     if (rc == IVC_OK) rc = cu_check(cudaMemsetAsync(f.done, 0, sizeof(int) * n_ctr, s));
     if (rc == IVC_OK)

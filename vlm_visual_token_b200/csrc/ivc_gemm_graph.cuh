@@ -61,6 +61,7 @@
 //     matrix and channel chunk c of block (qb, rb) is one box coordinate.
 #pragma once
 #include "ivc_gemm.cuh"
+#include "ivc_graph_schedule.h"
 
 namespace ivc {
 
@@ -104,9 +105,8 @@ struct GraphProblem {
   const float* row_rstd;
   void* out;           // bf16 [M, ldo]
   long long ldo;
-  int n_major;         // 1: tiles column block by column block (the row blocks
-                       // of one weight panel run together and share it in L2)
   int wide;            // 1: 256 x 512 tiles (n_tiles counts 512-column blocks)
+  int group_m;         // > 0: tiles in groups of group_m row blocks (tile_coords)
 };
 
 struct alignas(64) GraphMaps {
@@ -133,9 +133,9 @@ struct GraphTile {
 __device__ __forceinline__ GraphTile graph_tile(const GraphArgs& g, int u) {
   int p = 0;
   while (p + 1 < g.n_problems && u >= g.unit_begin[p + 1]) ++p;
-  const int idx = u - g.unit_begin[p];
-  if (g.p[p].n_major) return {p, idx % g.p[p].m_tiles, idx / g.p[p].m_tiles};
-  return {p, idx / g.p[p].n_tiles, idx % g.p[p].n_tiles};
+  GraphTile t{p, 0, 0};
+  tile_coords(u - g.unit_begin[p], g.p[p].m_tiles, g.p[p].n_tiles, g.p[p].group_m, &t.m, &t.n);
+  return t;
 }
 
 // Bounded acquire poll of a row-block counter (one thread).

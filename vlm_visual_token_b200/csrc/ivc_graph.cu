@@ -3,6 +3,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cstdlib>
+
 #include <vector>
 
 #include "ivc_gemm_graph.cuh"
@@ -61,6 +63,17 @@ int graph_counters(const GraphProblemCall* probs, int n) {
   return c;
 }
 
+// IVC_GRAPH_GROUP: -1 (unset) for the size rule in launch_gemm_graph, else
+// the group height in row blocks for every problem (0: row-block order).
+static int graph_group_override() {
+  static int v = -2;
+  if (v == -2) {
+    const char* e = std::getenv("IVC_GRAPH_GROUP");
+    v = e && e[0] >= '0' && e[0] <= '9' ? std::atoi(e) : -1;
+  }
+  return v;
+}
+
 int launch_gemm_graph(const GraphProblemCall* probs, int n, int* done, int reserve_sms,
                       const Launch& L) {
   if (done == nullptr) return IVC_EINVAL;
@@ -83,6 +96,18 @@ int launch_gemm_graph(const GraphProblemCall* probs, int n, int* done, int reser
     wide[i] = c.wide == 2 || (c.wide == 1 && tiles256 >= 8LL * max_pairs) ? 1 : 0;
     use_wide = use_wide || wide[i];
   }
+  // A weight matrix larger than half of L2 (128 MB for mlp2.fc1, 131 MB for
+  // the InternViT-6B connector's mlp1.fc1) does not stay in L2 while the
+  // rows of A stream past it: its tiles run in groups of 8 row blocks, column
+  // block by column block, so that each panel comes from DRAM once per group
+  // and the group's rows of A (8 x 256 rows) stay in L2 across the panels.
+  // IVC_GRAPH_GROUP=0 keeps row-block order, =g sets groups of g everywhere.
+  const int group_env = graph_group_override();
+  std::vector<int> group(n, 0);
+  for (int i = 0; i < n; ++i) {
+    const double w_bytes = 2.0 * probs[i].N * probs[i].K;
+    group[i] = group_env >= 0 ? group_env : (w_bytes > 64e6 ? 8 : 0);
+  }
   std::vector<SchedProblem> sp(n);
   int units = 0;
   for (int i = 0; i < n; ++i) {
@@ -91,7 +116,7 @@ int launch_gemm_graph(const GraphProblemCall* probs, int n, int* done, int reser
     const int mt = (c.M + GG_TILE_M - 1) / GG_TILE_M;
     const int nt = (c.N + (GG_BN << w) - 1) / (GG_BN << w);
     // a wide tile's cost in the model: twice the MACs, 1.5 times the bytes
-    sp[i] = {mt, nt, (c.K / GEMM_BK) * (w ? 7 : 4) / 4, c.dep, c.n_major};
+    sp[i] = {mt, nt, (c.K / GEMM_BK) * (w ? 7 : 4) / 4, c.dep, group[i]};
     units += mt * nt;
   }
   const int pairs = units < max_pairs ? units : max_pairs;
@@ -123,7 +148,7 @@ int launch_gemm_graph(const GraphProblemCall* probs, int n, int* done, int reser
     P.row_rstd = c.row_rstd;
     P.out = c.out;
     P.ldo = c.ldo;
-    P.n_major = c.n_major;
+    P.group_m = group[i];
     ctr += P.m_tiles;
     int rc;
     if (c.a_mode == A_PLAIN) {

@@ -145,7 +145,6 @@ struct GraphProblemCall {
   void* out;
   long long ldo;
   int dep;
-  int n_major;         // 1: tiles ordered column block by column block
   int wide;            // 1: 256 x 512 tiles if the problem has many rounds of
                        // 256-wide tiles; 2: 256 x 512 tiles
 };
